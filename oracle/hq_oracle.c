@@ -1,0 +1,437 @@
+/*
+ * hq_oracle.c -- plain, slow, single-threaded CPU oracle for dynamic FP8
+ * quantization (amax -> scale -> saturating RNE cast) and the scaled FP8
+ * GEMM it feeds.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call this
+ * file: only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark load it.  It shares no code, header, table or constant with the
+ * CUDA library; every number below is derived here from the format
+ * definitions.
+ *
+ * Sources (web pages this restates; no code is copied from them):
+ *  [HQ]  hip-quant 0.6.0 README, "FP8 Formats" table (E4M3: 1s.4e.3m, bias 7,
+ *        max +-448, NaN only; E5M2: 1s.5e.2m, bias 15, max +-57344, +-Inf and
+ *        NaN) and the sentence after it (OCP round-to-nearest-even);
+ *        "Training-path numerical guards" (quant scales are pre-quant
+ *        multipliers, the reciprocal is the dequant scale; non-finite amax
+ *        samples are ignored); "Scale / amax tracking" (history_len = 16).
+ *  [AS]  AstrAI csrc/kernels/fp8/ops.cu: commit "finalize fp8 scale rings
+ *        inside quantize kernels" (last-block epilogue folds amax into
+ *        hist[idx], reduces the window, publishes the next scale; ring
+ *        packs [hist | scale | counter]), pack_quantize_params (len =
+ *        numel-2, idx = caller's slot, margin from the recipe), mm_fp8
+ *        (out = a @ b^T * (sa*sb), FP32 accumulate).
+ *  [QS]  fuel-ir 0.22.4 src/quant_scale.rs: ScaleGranularity (PerTensor
+ *        f32[1], PerToken f32[n_rows], PerChannel f32[n_cols]) and
+ *        scale_count.
+ *  [PR]  ROCm/aiter PR 6437, "Technical Details": out[M,N] bf16 from XQ[M,K],
+ *        WQ[N,K], x_scale[M], w_scale[N].
+ *  [GG]  megablocks-hip _dev/TODO-gg.md: per-expert Y_e = X_e . W_e^T, the
+ *        output is overwritten, never accumulated.
+ *
+ * Readings where the pages are silent (each also listed in the design doc):
+ *  R1  NaN input encodes to the canonical code 0x7F in both formats.
+ *  R2  The cast saturates: |y| >= fmax (including +-Inf) -> sign | max code.
+ *  R3  amax skips NaN and +-Inf elements.
+ *  R4  amax == 0, or fmax/amax not finite -> multiplier m = 1.
+ *  R5  The exported per-row/column/tensor scale is the dequant scale d = 1/m.
+ *  R6  Delayed ring: after the cast, hist[idx] = amax; win = max(hist);
+ *      if win is finite and > 0 the scale slot becomes ldexp(fmax/win,
+ *      -margin), else it keeps its value; the counter slot is 0 on exit.
+ *  R7  Per-channel reduces over rows (one scale per column), as [QS] says.
+ *
+ * Floating point: f32 steps are single f32 operations (compile with
+ * -ffp-contract=off, no fast-math); everything else is exact integer
+ * arithmetic or fp64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+
+#define HQO_E4M3 0
+#define HQO_E5M2 1
+#define HQO_F32 0
+#define HQO_BF16 1
+#define HQO_F16 2
+#define HQO_PER_TENSOR 0
+#define HQO_PER_TOKEN 1
+#define HQO_PER_CHANNEL 2
+
+/* ---------------------------------------------------------------- formats */
+
+/* Format parameters straight from the [HQ] "FP8 Formats" table. */
+typedef struct {
+  int ebits, mbits, bias;
+  double fmax;    /* largest finite magnitude */
+  uint8_t maxcode; /* code of +fmax */
+} fmt_info;
+
+static fmt_info get_fmt(int fmt) {
+  fmt_info f;
+  if (fmt == HQO_E4M3) {
+    /* 4 exponent bits, 3 mantissa bits, bias 7.  The all-ones exponent is
+       still finite except for mantissa 111 (NaN), so the top finite value is
+       exponent field 15, mantissa 110: (1 + 6/8) * 2^(15-7) = 448. */
+    f.ebits = 4; f.mbits = 3; f.bias = 7;
+    f.fmax = ldexp(1.0 + 6.0 / 8.0, 15 - 7);
+    f.maxcode = (uint8_t)((15 << 3) | 6);
+  } else {
+    /* 5 exponent bits, 2 mantissa bits, bias 15; exponent field 31 is
+       Inf/NaN, so the top finite value is (1 + 3/4) * 2^(30-15) = 57344. */
+    f.ebits = 5; f.mbits = 2; f.bias = 15;
+    f.fmax = ldexp(1.0 + 3.0 / 4.0, 30 - 15);
+    f.maxcode = (uint8_t)((30 << 2) | 3);
+  }
+  return f;
+}
+
+double hqo_fmax(int fmt) { return get_fmt(fmt).fmax; }
+
+/* Decode one code by its bit fields ([HQ] "FP8 Formats"). */
+double hqo_decode(uint8_t c, int fmt) {
+  fmt_info f = get_fmt(fmt);
+  int s = (c >> 7) & 1;
+  int e = (c >> f.mbits) & ((1 << f.ebits) - 1);
+  int m = c & ((1 << f.mbits) - 1);
+  double v;
+  int emin = 1 - f.bias;
+  if (fmt == HQO_E4M3 && (c & 0x7F) == 0x7F) return NAN;
+  if (fmt == HQO_E5M2 && e == 31) {
+    if (m != 0) return NAN;
+    return s ? -INFINITY : INFINITY;
+  }
+  if (e == 0)
+    v = ldexp((double)m, emin - f.mbits); /* subnormal: m * 2^(emin-mbits) */
+  else
+    v = ldexp(1.0 + ldexp((double)m, -f.mbits), e - f.bias);
+  return s ? -v : v;
+}
+
+/* Saturating round-to-nearest-even encode of an f32 value (R1, R2, [HQ]).
+   |y| as a double is exact; scaling by a power of two and nearbyint (the
+   default rounding mode is to-nearest-even) rounds exactly once. */
+uint8_t hqo_encode_sat(float y, int fmt) {
+  fmt_info f = get_fmt(fmt);
+  int emin = 1 - f.bias;
+  uint8_t sign;
+  double a, quantum, r;
+  int e;
+  if (isnan(y)) return 0x7F;
+  sign = signbit(y) ? 0x80 : 0x00;
+  a = fabs((double)y);
+  if (a >= f.fmax) return (uint8_t)(sign | f.maxcode);
+  if (a < ldexp(1.0, emin)) {
+    quantum = ldexp(1.0, emin - f.mbits);
+  } else {
+    frexp(a, &e); /* a = g * 2^e, g in [0.5, 1): binade exponent is e-1 */
+    quantum = ldexp(1.0, (e - 1) - f.mbits);
+  }
+  r = nearbyint(a / quantum) * quantum;
+  if (r == 0.0) return sign;
+  if (r < ldexp(1.0, emin)) {
+    /* subnormal: exponent field 0, mantissa = r / 2^(emin-mbits) */
+    return (uint8_t)(sign | (int)(r / ldexp(1.0, emin - f.mbits)));
+  }
+  frexp(r, &e);
+  {
+    int efield = (e - 1) + f.bias;
+    int mfield = (int)((ldexp(r, -(e - 1)) - 1.0) * (double)(1 << f.mbits));
+    return (uint8_t)(sign | (efield << f.mbits) | mfield);
+  }
+}
+
+/* ------------------------------------------------------------ bf16 / f16 */
+
+float hqo_bf16_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float x;
+  memcpy(&x, &u, 4);
+  return x;
+}
+
+float hqo_f16_to_f32(uint16_t h) {
+  int s = (h >> 15) & 1, e = (h >> 10) & 31, m = h & 1023;
+  double v;
+  if (e == 31) v = m ? NAN : INFINITY;
+  else if (e == 0) v = ldexp((double)m, -24);
+  else v = ldexp(1.0 + m / 1024.0, e - 15);
+  return (float)(s ? -v : v);
+}
+
+/* Round a double to the nearest bf16 (ties to even), once. */
+uint16_t hqo_double_to_bf16(double v) {
+  double a, q, r;
+  int e;
+  float rf;
+  uint32_t u;
+  if (isnan(v)) return 0x7FC0;
+  a = fabs(v);
+  if (a == 0.0 || isinf(v)) {
+    rf = (float)v;
+    memcpy(&u, &rf, 4);
+    return (uint16_t)(u >> 16);
+  }
+  if (a < ldexp(1.0, -126)) {
+    q = ldexp(1.0, -133); /* bf16 subnormal step: 2^(-126-7) */
+  } else {
+    frexp(a, &e);
+    q = ldexp(1.0, (e - 1) - 7);
+  }
+  r = nearbyint(a / q) * q;
+  if (r >= ldexp(1.0, 128)) r = INFINITY;
+  rf = (float)(v < 0 ? -r : r); /* exact: r is on the bf16 grid */
+  memcpy(&u, &rf, 4);
+  return (uint16_t)(u >> 16);
+}
+
+/* Correct bf16 rounding of an unevaluated sum hi + lo with |lo| <= ulp(hi)/2:
+   only an exact bf16 midpoint in hi can be moved by lo. */
+static uint16_t dd_to_bf16(double hi, double lo) {
+  uint16_t r = hqo_double_to_bf16(hi);
+  if (lo != 0.0 && isfinite(hi) && hi != 0.0) {
+    double a = fabs(hi), q, t;
+    int e;
+    if (a < ldexp(1.0, -126)) q = ldexp(1.0, -133);
+    else { frexp(a, &e); q = ldexp(1.0, (e - 1) - 7); }
+    t = a / q;
+    if (t - floor(t) == 0.5) {
+      /* hi is a tie; the true value lies on lo's side of it */
+      double nudged = hi + (lo > 0 ? 1.0 : -1.0) * q * 0.25;
+      r = hqo_double_to_bf16(nudged);
+    }
+  }
+  return r;
+}
+
+/* ------------------------------------------------------------------ amax */
+
+static float load_elem(const void* x, int dtype, int64_t i) {
+  if (dtype == HQO_F32) return ((const float*)x)[i];
+  if (dtype == HQO_BF16) return hqo_bf16_to_f32(((const uint16_t*)x)[i]);
+  return hqo_f16_to_f32(((const uint16_t*)x)[i]);
+}
+
+/* Multiplier m = fl32(fmax / amax) with reading R4. */
+float hqo_multiplier(float amax, int fmt) {
+  float fmax = (float)get_fmt(fmt).fmax;
+  float m;
+  if (!(amax > 0.0f)) return 1.0f;
+  m = fmax / amax; /* one correctly rounded f32 division */
+  if (!isfinite(m)) return 1.0f;
+  return m;
+}
+
+/* scale_count per [QS] ScaleGranularity::scale_count. */
+int64_t hqo_scale_count(int gran, int64_t rows, int64_t cols) {
+  if (gran == HQO_PER_TENSOR) return 1;
+  if (gran == HQO_PER_TOKEN) return rows;
+  if (gran == HQO_PER_CHANNEL) return cols;
+  return -1;
+}
+
+/* amax over the elements that share one scale (R3, R7).  out has
+   scale_count(gran, rows, cols) entries. */
+void hqo_amax(const void* x, int dtype, int64_t rows, int64_t cols, int gran,
+              float* out) {
+  int64_t n = hqo_scale_count(gran, rows, cols), r, c;
+  for (r = 0; r < n; ++r) out[r] = 0.0f;
+  for (r = 0; r < rows; ++r) {
+    for (c = 0; c < cols; ++c) {
+      float v = load_elem(x, dtype, r * cols + c);
+      float a;
+      int64_t slot;
+      if (!isfinite(v)) continue;
+      a = fabsf(v);
+      slot = (gran == HQO_PER_TENSOR) ? 0 : (gran == HQO_PER_TOKEN ? r : c);
+      if (a > out[slot]) out[slot] = a;
+    }
+  }
+}
+
+/* ---------------------------------------------------------------- quantize */
+
+/* Dynamic quantize (ring == NULL) or delayed per-tensor quantize (ring !=
+   NULL, R6).  q: rows*cols codes; scales: dequant scales d = 1/m (R5);
+   amax_out (nullable): the amax array of the input at this granularity.
+   Returns 0, or -1 on an invalid argument. */
+int hqo_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
+                 int gran, uint8_t* q, float* scales, float* amax_out,
+                 float* ring, int ring_len, int ring_idx, int ring_margin) {
+  int64_t n = hqo_scale_count(gran, rows, cols), r, c;
+  float* amax;
+  float* mult;
+  if (n < 0) return -1;
+  if (ring && (gran != HQO_PER_TENSOR || ring_len < 1 || ring_idx < 0 ||
+               ring_idx >= ring_len))
+    return -1;
+  amax = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  mult = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  hqo_amax(x, dtype, rows, cols, gran, amax);
+  if (ring) {
+    mult[0] = ring[ring_len]; /* the scale slot published by the last step */
+  } else {
+    for (r = 0; r < n; ++r) mult[r] = hqo_multiplier(amax[r], fmt);
+  }
+  for (r = 0; r < n; ++r) scales[r] = 1.0f / mult[r];
+  for (r = 0; r < rows; ++r) {
+    for (c = 0; c < cols; ++c) {
+      int64_t slot = (gran == HQO_PER_TENSOR) ? 0 : (gran == HQO_PER_TOKEN ? r : c);
+      float y = load_elem(x, dtype, r * cols + c) * mult[slot]; /* one f32 mul */
+      q[r * cols + c] = hqo_encode_sat(y, fmt);
+    }
+  }
+  if (amax_out)
+    for (r = 0; r < n; ++r) amax_out[r] = amax[r];
+  if (ring) {
+    float win = 0.0f;
+    int i;
+    ring[ring_idx] = amax[0];
+    for (i = 0; i < ring_len; ++i)
+      if (ring[i] > win) win = ring[i];
+    if (isfinite(win) && win > 0.0f) {
+      float fmax = (float)get_fmt(fmt).fmax;
+      float next = ldexpf(fmax / win, -ring_margin);
+      if (isfinite(next) && next > 0.0f) ring[ring_len] = next;
+    }
+    ring[ring_len + 1] = 0.0f; /* counter slot, 0 on exit */
+  }
+  free(amax);
+  free(mult);
+  return 0;
+}
+
+/* --------------------------------------------------------------------- GEMM */
+
+/* Integer numerator of a finite code: value = n * 2^-frac, frac = 9 (E4M3)
+   or 16 (E5M2).  Returns 0 for NaN/Inf codes. */
+static int code_int(uint8_t c, int fmt, int64_t* n) {
+  double v = hqo_decode(c, fmt);
+  if (!isfinite(v)) return 0;
+  *n = (int64_t)ldexp(v, fmt == HQO_E4M3 ? 9 : 16); /* exact */
+  return 1;
+}
+
+/* Exact dot product S = sum_k dec(a[k]) * dec(b[k]) as a double (exact for
+   E4M3, one rounding of an exact integer for E5M2); non-finite operands fall
+   back to IEEE double arithmetic. */
+static double exact_dot(const uint8_t* a, const uint8_t* b, int64_t K, int fmt) {
+  int frac = (fmt == HQO_E4M3) ? 9 : 16;
+  __int128 acc = 0;
+  int64_t k;
+  for (k = 0; k < K; ++k) {
+    int64_t na, nb;
+    if (!code_int(a[k], fmt, &na) || !code_int(b[k], fmt, &nb)) {
+      double s = 0.0;
+      for (k = 0; k < K; ++k) s += hqo_decode(a[k], fmt) * hqo_decode(b[k], fmt);
+      return s;
+    }
+    acc += (__int128)na * (__int128)nb;
+  }
+  return ldexp((double)acc, -2 * frac);
+}
+
+static uint16_t gemm_entry(const uint8_t* xq, const uint8_t* wq, int fmt,
+                           const float* xs, int64_t xs_len, const float* ws,
+                           int64_t ws_len, int64_t K, int64_t m, int64_t n,
+                           double* ref) {
+  double s = exact_dot(xq + m * K, wq + n * K, K, fmt);
+  double sx = (double)xs[xs_len == 1 ? 0 : m];
+  double sw = (double)ws[ws_len == 1 ? 0 : n];
+  double v = sx * sw * s;
+  if (ref) *ref = v;
+  return hqo_double_to_bf16(v);
+}
+
+/* out[m,n] = bf16(x_scale[m'] * w_scale[n'] * sum_k dec(XQ[m,k]) dec(WQ[n,k]))
+   ([PR] Technical Details; [AS] mm_fp8 NT layout).  x_scale has M or 1
+   entries, w_scale N or 1.  ref_out (nullable) receives the unrounded fp64
+   value. */
+void hqo_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, int fmt,
+                   const float* xs, int64_t xs_len, const float* ws,
+                   int64_t ws_len, int64_t M, int64_t N, int64_t K,
+                   uint16_t* out, double* ref_out) {
+  int64_t m, n;
+  for (m = 0; m < M; ++m)
+    for (n = 0; n < N; ++n)
+      out[m * N + n] = gemm_entry(xq, wq, fmt, xs, xs_len, ws, ws_len, K, m, n,
+                                  ref_out ? &ref_out[m * N + n] : NULL);
+}
+
+/* The same entries at sampled (m, n) positions only. */
+void hqo_gemm_a8w8_entries(const uint8_t* xq, const uint8_t* wq, int fmt,
+                           const float* xs, int64_t xs_len, const float* ws,
+                           int64_t ws_len, int64_t K, const int64_t* ms,
+                           const int64_t* ns, int64_t count, uint16_t* out) {
+  int64_t i;
+  for (i = 0; i < count; ++i)
+    out[i] = gemm_entry(xq, wq, fmt, xs, xs_len, ws, ws_len, K, ms[i], ns[i], NULL);
+}
+
+/* Grouped a8w8 GEMM ([GG]): for expert e, rows [off[e], off[e+1]) of XQ times
+   WQ[e]^T with x_scale[row] and w_scale[e, n].  Rows outside every expert's
+   range are not written.  Returns -1 on malformed offsets. */
+int hqo_grouped_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, int fmt,
+                          const float* xs, const float* ws,
+                          const int32_t* off, int32_t E, int64_t M_total,
+                          int64_t N, int64_t K, uint16_t* out) {
+  int32_t e;
+  int64_t m, n;
+  if (off[0] != 0 || off[E] != M_total) return -1;
+  for (e = 0; e < E; ++e) {
+    if (off[e + 1] < off[e]) return -1;
+    for (m = off[e]; m < off[e + 1]; ++m)
+      for (n = 0; n < N; ++n) {
+        double s = exact_dot(xq + m * K, wq + ((int64_t)e * N + n) * K, K, fmt);
+        double v = (double)xs[m] * (double)ws[(int64_t)e * N + n] * s;
+        out[m * N + n] = hqo_double_to_bf16(v);
+      }
+  }
+  return 0;
+}
+
+/* Grouped bf16 GEMM with a wide accumulator: out = bf16(sum_k a*b).  Each
+   bf16*bf16 product is exact in fp64 (8-bit significands); the sum is carried
+   as an unevaluated double-double (Knuth's TwoSum), then rounded once. */
+int hqo_grouped_gemm_bf16(const uint16_t* x, const uint16_t* w,
+                          const int32_t* off, int32_t E, int64_t M_total,
+                          int64_t N, int64_t K, uint16_t* out) {
+  int32_t e;
+  int64_t m, n, k;
+  if (off[0] != 0 || off[E] != M_total) return -1;
+  for (e = 0; e < E; ++e) {
+    if (off[e + 1] < off[e]) return -1;
+    for (m = off[e]; m < off[e + 1]; ++m)
+      for (n = 0; n < N; ++n) {
+        const uint16_t* a = x + m * K;
+        const uint16_t* b = w + ((int64_t)e * N + n) * K;
+        double hi = 0.0, lo = 0.0;
+        for (k = 0; k < K; ++k) {
+          double p = (double)hqo_bf16_to_f32(a[k]) * (double)hqo_bf16_to_f32(b[k]);
+          double s = hi + p;
+          double bb = s - hi;
+          double err = (hi - (s - bb)) + (p - bb);
+          hi = s;
+          lo += err;
+        }
+        {
+          double s = hi + lo; /* renormalise */
+          double err = lo - (s - hi);
+          out[m * N + n] = dd_to_bf16(s, err);
+        }
+      }
+  }
+  return 0;
+}
+
+/* Batch forms of the scalar encode/decode above (same arithmetic). */
+void hqo_encode_sat_array(const float* y, int64_t n, int fmt, uint8_t* out) {
+  int64_t i;
+  for (i = 0; i < n; ++i) out[i] = hqo_encode_sat(y[i], fmt);
+}
+
+void hqo_decode_array(const uint8_t* c, int64_t n, int fmt, double* out) {
+  int64_t i;
+  for (i = 0; i < n; ++i) out[i] = hqo_decode(c[i], fmt);
+}
