@@ -1,0 +1,192 @@
+"""ctypes binding of libhq.so (include/hq.h).
+
+Argument marshalling only: every step of the path runs in the library's
+CUDA kernels.  torch provides device memory and the current stream.  If the
+library is missing this module raises at import time: there is no fallback.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhq.so")
+
+HQ_OK = 0
+STATUS_NAMES = {0: "HQ_OK", 1: "HQ_ERR_INVALID_ARG", 2: "HQ_ERR_MISALIGNED", 3: "HQ_ERR_OVERLAP",
+                4: "HQ_ERR_WRONG_DEVICE", 5: "HQ_ERR_UNSUPPORTED_ARCH", 6: "HQ_ERR_CUDA",
+                7: "HQ_ERR_TIMEOUT", 8: "HQ_ERR_TOO_LARGE"}
+E4M3, E5M2 = 0, 1
+PER_TENSOR, PER_TOKEN, PER_CHANNEL = 0, 1, 2
+F32, BF16, F16 = 0, 1, 2
+
+EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
+            "hq_quantize_fp8", "hq_gemm_a8w8", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
+            "hq_check_device_error", "hq_last_error", "hq_version"]
+
+
+class HQError(RuntimeError):
+    def __init__(self, status, message):
+        self.status = status
+        self.status_name = STATUS_NAMES.get(status, str(status))
+        super().__init__("%s: %s" % (self.status_name, message))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libhq.so is not built (python -m fp8_dynamic_quantization_amax_b200.build); "
+                          "there is no CPU fallback")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int, ctypes.c_size_t
+    L.hq_scale_count.argtypes = [ci, i64, i64]
+    L.hq_scale_count.restype = i64
+    L.hq_granularity_name.argtypes = [ci]
+    L.hq_granularity_name.restype = ctypes.c_char_p
+    L.hq_scale_pair_name.argtypes = [ci, ci, ctypes.c_char_p, sz]
+    L.hq_scale_pair_name.restype = ci
+    L.hq_quantize_workspace_bytes.argtypes = [ci, i64, i64, ci]
+    L.hq_quantize_workspace_bytes.restype = sz
+    L.hq_quantize_fp8.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P, sz, P]
+    L.hq_quantize_fp8.restype = ci
+    L.hq_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
+    L.hq_gemm_a8w8.restype = ci
+    L.hq_grouped_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, P, i32, i64, i64, i64, P, P]
+    L.hq_grouped_gemm_a8w8.restype = ci
+    L.hq_grouped_gemm_bf16.argtypes = [P, P, P, i32, i64, i64, i64, P, P]
+    L.hq_grouped_gemm_bf16.restype = ci
+    L.hq_check_device_error.argtypes = []
+    L.hq_check_device_error.restype = ci
+    L.hq_last_error.argtypes = []
+    L.hq_last_error.restype = ctypes.c_char_p
+    L.hq_version.argtypes = []
+    L.hq_version.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def check(status):
+    if status != HQ_OK:
+        raise HQError(status, lib.hq_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
+_ws_cache = {}
+
+
+def _workspace(device, nbytes):
+    """A zero-filled workspace per (device, size).  The library returns its
+    accumulator words to zero after each call, so calls that run one after
+    another on one stream can share it."""
+    if nbytes == 0:
+        return None
+    key = (device, nbytes)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def hq_scale_count(gran, rows, cols):
+    return lib.hq_scale_count(gran, rows, cols)
+
+
+def hq_granularity_name(gran):
+    r = lib.hq_granularity_name(gran)
+    return None if r is None else r.decode()
+
+
+def hq_scale_pair_name(act, weight):
+    buf = ctypes.create_string_buffer(64)
+    n = lib.hq_scale_pair_name(act, weight, buf, 64)
+    return None if n < 0 else buf.value.decode()
+
+
+def hq_quantize_workspace_bytes(gran, rows, cols, delayed=False):
+    return lib.hq_quantize_workspace_bytes(gran, rows, cols, 1 if delayed else 0)
+
+
+def hq_quantize_fp8(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=None, ring=None,
+                    ring_idx=0, ring_margin=0, workspace=None, stream=None):
+    """Quantize a 2-D CUDA tensor (f32 / bf16 / f16).  Returns (q uint8,
+    dequant scales f32).  With `ring` (f32 [len+2]) this is the delayed
+    per-tensor mode; the ring is updated in place on the device."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32, bfloat16 or float16")
+    x = x.contiguous()
+    rows, cols = x.shape
+    ns = hq_scale_count(gran, rows, cols)
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((max(ns, 0),), dtype=torch.float32, device=x.device)
+    ring_len = 0
+    if ring is not None:
+        ring_len = ring.numel() - 2
+    need = hq_quantize_workspace_bytes(gran, rows, cols, ring is not None)
+    if workspace is None:
+        workspace = _workspace(x.device, need)
+    check(lib.hq_quantize_fp8(_ptr(x), _DT[x.dtype], rows, cols, fmt, gran, _ptr(q), _ptr(scales),
+                              _ptr(amax_out), _ptr(ring), ring_len, ring_idx, ring_margin,
+                              _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                              _stream(stream)))
+    return q, scales
+
+
+def hq_gemm_a8w8(xq, wq, x_scale, w_scale, fmt=E4M3, out=None, stream=None):
+    """out[M,N] bf16 = x_scale[m] * w_scale[n] * sum_k dec(xq[m,k]) dec(wq[n,k])."""
+    xq, wq = xq.contiguous(), wq.contiguous()
+    x_scale, w_scale = x_scale.contiguous(), w_scale.contiguous()
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    check(lib.hq_gemm_a8w8(_ptr(xq), _ptr(wq), fmt, _ptr(x_scale), x_scale.numel(), _ptr(w_scale),
+                           w_scale.numel(), M, N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def hq_grouped_gemm_a8w8(xq, wq, x_scale, w_scale, offsets, fmt=E4M3, out=None, stream=None):
+    """Per-expert a8w8 GEMM: rows [offsets[e], offsets[e+1]) of xq times wq[e]^T."""
+    xq, wq = xq.contiguous(), wq.contiguous()
+    x_scale, w_scale = x_scale.contiguous(), w_scale.contiguous()
+    M, K = xq.shape
+    E, N, _ = wq.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    check(lib.hq_grouped_gemm_a8w8(_ptr(xq), _ptr(wq), fmt, _ptr(x_scale), x_scale.numel(), _ptr(w_scale),
+                                   w_scale.numel(), _ptr(offsets), E, M, N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def hq_grouped_gemm_bf16(x, w, offsets, out=None, stream=None):
+    """Per-expert bf16 GEMM with FP32 accumulation."""
+    x, w = x.contiguous(), w.contiguous()
+    M, K = x.shape
+    E, N, _ = w.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    check(lib.hq_grouped_gemm_bf16(_ptr(x), _ptr(w), _ptr(offsets), E, M, N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def hq_check_device_error():
+    check(lib.hq_check_device_error())
+
+
+def hq_version():
+    return lib.hq_version().decode()

@@ -1,0 +1,324 @@
+// api.cu -- the extern "C" boundary of libhq.so: argument validation,
+// device and architecture checks, dispatch to the kernels, error strings.
+//
+// Validation order follows ROCm/aiter PR 6437 "Technical Details": every
+// argument check runs before any launch and before the architecture check,
+// so invalid arguments always report INVALID_ARG / MISALIGNED / OVERLAP
+// even on an unsupported device, and no output is touched on error.  An
+// empty output returns after validation without a launch.  Operands must be
+// on the current device (the PR's non-current-device rule).
+#include "../../include/hq.h"
+#include "hq_internal.cuh"
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+namespace {
+
+thread_local std::string g_last_error;
+
+hq_status fail(hq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+hq_status ok() {
+  g_last_error.clear();
+  return HQ_OK;
+}
+
+bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Range {
+  const void* p;
+  size_t bytes;
+  const char* name;
+};
+
+bool overlaps(const Range& a, const Range& b) {
+  if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+  return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+// Every output range against every other range listed after it.
+hq_status check_overlaps(const Range* outs, int n_out, const Range* ins, int n_in) {
+  for (int i = 0; i < n_out; ++i) {
+    for (int j = 0; j < n_in; ++j)
+      if (overlaps(outs[i], ins[j]))
+        return fail(HQ_ERR_OVERLAP, "%s overlaps input %s", outs[i].name, ins[j].name);
+    for (int j = i + 1; j < n_out; ++j)
+      if (overlaps(outs[i], outs[j]))
+        return fail(HQ_ERR_OVERLAP, "%s overlaps %s", outs[i].name, outs[j].name);
+  }
+  return HQ_OK;
+}
+
+// Device pointers of the current device only (managed memory included).
+hq_status check_device_ptrs(const Range* rs, int n) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(HQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  for (int i = 0; i < n; ++i) {
+    if (!rs[i].p) continue;
+    cudaPointerAttributes attr;
+    e = cudaPointerGetAttributes(&attr, rs[i].p);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(HQ_ERR_WRONG_DEVICE, "%s: cudaPointerGetAttributes: %s", rs[i].name, cudaGetErrorString(e));
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+      return fail(HQ_ERR_WRONG_DEVICE, "%s is not device memory", rs[i].name);
+    if (attr.device != dev)
+      return fail(HQ_ERR_WRONG_DEVICE, "%s lives on device %d, current device is %d", rs[i].name, attr.device, dev);
+  }
+  return HQ_OK;
+}
+
+// Compute capability 10.0 (B200, sm_100a) only; cached per device.
+hq_status check_arch() {
+  static std::mutex mu;
+  static int cache[64];
+  static bool init = false;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(HQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(mu);
+  if (!init) {
+    for (int& c : cache) c = -1;
+    init = true;
+  }
+  if (dev < 0 || dev >= 64) return fail(HQ_ERR_UNSUPPORTED_ARCH, "device index %d out of range", dev);
+  if (cache[dev] < 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return fail(HQ_ERR_CUDA, "cudaDeviceGetAttribute failed");
+    cache[dev] = major * 10 + minor;
+  }
+  if (cache[dev] != 100)
+    return fail(HQ_ERR_UNSUPPORTED_ARCH, "compute capability %d.%d; this library is built for sm_100a (10.0)",
+                cache[dev] / 10, cache[dev] % 10);
+  return HQ_OK;
+}
+
+hq_status launched(cudaError_t e, const char* what, const std::string& extra = std::string()) {
+  if (e != cudaSuccess)
+    return fail(HQ_ERR_CUDA, "%s: %s%s%s", what, cudaGetErrorString(e), extra.empty() ? "" : " -- ", extra.c_str());
+  return ok();
+}
+
+constexpr int64_t k2p31 = int64_t(1) << 31;
+constexpr int64_t k2p40 = int64_t(1) << 40;
+
+}  // namespace
+
+namespace hq {
+int device_sm_count(int dev) {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+}  // namespace hq
+
+extern "C" {
+
+int64_t hq_scale_count(hq_granularity g, int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return -1;
+  switch (g) {
+    case HQ_PER_TENSOR: return 1;
+    case HQ_PER_TOKEN: return rows;
+    case HQ_PER_CHANNEL: return cols;
+    default: return -1;
+  }
+}
+
+const char* hq_granularity_name(hq_granularity g) {
+  switch (g) {
+    case HQ_PER_TENSOR: return "per_tensor";
+    case HQ_PER_TOKEN: return "per_token";
+    case HQ_PER_CHANNEL: return "per_channel";
+    default: return nullptr;
+  }
+}
+
+int hq_scale_pair_name(hq_granularity act, hq_granularity weight, char* buf, size_t len) {
+  const char* a = hq_granularity_name(act);
+  const char* w = hq_granularity_name(weight);
+  if (!a || !w || !buf) return -1;
+  const int n = snprintf(buf, len, "act_%s_weight_%s", a, w);
+  if (n < 0 || static_cast<size_t>(n) >= len) return -1;
+  return n;
+}
+
+size_t hq_quantize_workspace_bytes(hq_granularity g, int64_t rows, int64_t cols, int delayed) {
+  if (hq_scale_count(g, rows, cols) < 0) return 0;
+  return hq::quantize_workspace_bytes(static_cast<int>(g), rows, cols, delayed);
+}
+
+hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                          hq_granularity g, uint8_t* q, float* scales, float* amax_out, float* ring,
+                          int32_t ring_len, int32_t ring_idx, int32_t ring_margin, void* workspace,
+                          size_t workspace_bytes, hq_stream_t stream) {
+  // ---- arguments
+  if (xt != HQ_F32 && xt != HQ_BF16 && xt != HQ_F16) return fail(HQ_ERR_INVALID_ARG, "invalid dtype %d", (int)xt);
+  if (fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", (int)fmt);
+  if (g != HQ_PER_TENSOR && g != HQ_PER_TOKEN && g != HQ_PER_CHANNEL)
+    return fail(HQ_ERR_INVALID_ARG, "invalid granularity %d", (int)g);
+  if (rows < 0 || cols < 0) return fail(HQ_ERR_INVALID_ARG, "negative shape [%lld, %lld]", (long long)rows, (long long)cols);
+  if (rows >= k2p31 || cols >= k2p31 || (cols > 0 && rows > (k2p40 - 1) / cols))
+    return fail(HQ_ERR_TOO_LARGE, "shape [%lld, %lld] is beyond the supported range", (long long)rows, (long long)cols);
+  if (ring) {
+    if (g != HQ_PER_TENSOR) return fail(HQ_ERR_INVALID_ARG, "a delayed-scaling ring needs per-tensor granularity");
+    if (ring_len < 1 || ring_len > (1 << 20)) return fail(HQ_ERR_INVALID_ARG, "ring_len %d outside [1, 2^20]", ring_len);
+    if (ring_idx < 0 || ring_idx >= ring_len)
+      return fail(HQ_ERR_INVALID_ARG, "ring_idx %d outside [0, %d)", ring_idx, ring_len);
+    if (ring_margin < -126 || ring_margin > 126) return fail(HQ_ERR_INVALID_ARG, "ring_margin %d outside [-126, 126]", ring_margin);
+  }
+  const int64_t ns = hq_scale_count(g, rows, cols);
+  const int64_t n = rows * cols;
+  const size_t esize = (xt == HQ_F32) ? 4 : 2;
+  const size_t need = hq::quantize_workspace_bytes(static_cast<int>(g), rows, cols, ring != nullptr);
+  if (ns == 0) return ok();
+  if (n > 0 && (!x || !q)) return fail(HQ_ERR_INVALID_ARG, "x and q must not be null");
+  if (!scales) return fail(HQ_ERR_INVALID_ARG, "scales must not be null");
+  if (need > 0 && !workspace) return fail(HQ_ERR_INVALID_ARG, "this mode needs a workspace of %zu bytes", need);
+  if (need > 0 && workspace_bytes < need)
+    return fail(HQ_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
+  if (!is_aligned(x, esize)) return fail(HQ_ERR_MISALIGNED, "x is not aligned to its element size");
+  if (!is_aligned(scales, 4) || !is_aligned(amax_out, 4) || !is_aligned(ring, 4))
+    return fail(HQ_ERR_MISALIGNED, "scales, amax_out and ring must be 4-byte aligned");
+  if (need > 0 && !is_aligned(workspace, 256)) return fail(HQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  const Range outs[] = {{q, static_cast<size_t>(n), "q"},
+                        {scales, static_cast<size_t>(ns) * 4, "scales"},
+                        {amax_out, amax_out ? static_cast<size_t>(ns) * 4 : 0, "amax_out"},
+                        {ring, ring ? static_cast<size_t>(ring_len + 2) * 4 : 0, "ring"},
+                        {workspace, need, "workspace"}};
+  const Range ins[] = {{x, static_cast<size_t>(n) * esize, "x"}};
+  hq_status s = check_overlaps(outs, 5, ins, 1);
+  if (s != HQ_OK) return s;
+  // ---- device
+  const Range devs[] = {{n > 0 ? x : nullptr, 0, "x"}, {n > 0 ? q : nullptr, 0, "q"}, {scales, 0, "scales"},
+                        {amax_out, 0, "amax_out"}, {ring, 0, "ring"}, {need > 0 ? workspace : nullptr, 0, "workspace"}};
+  s = check_device_ptrs(devs, 6);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  // ---- launch
+  hq::QuantizeArgs a;
+  a.x = x; a.xt = xt; a.rows = rows; a.cols = cols; a.fmt = fmt; a.gran = g;
+  a.q = q; a.scales = scales; a.amax_out = amax_out;
+  a.ring = ring; a.ring_len = ring_len; a.ring_idx = ring_idx; a.ring_margin = ring_margin;
+  a.ws = workspace;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  return launched(hq::launch_quantize(a), "quantize launch");
+}
+
+namespace {
+
+hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const float* xs, int64_t xs_len,
+                      const float* ws, int64_t ws_len, const int32_t* offsets, int32_t E, int64_t M, int64_t N,
+                      int64_t K, void* out, hq_stream_t stream) {
+  const bool grouped = offsets != nullptr || E != 1 || kind == 1;
+  if (kind == 0 && fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", fmt);
+  if (M < 0 || N < 0 || K < 0) return fail(HQ_ERR_INVALID_ARG, "negative size");
+  if (M >= k2p31 || N >= k2p31 || K >= k2p31) return fail(HQ_ERR_TOO_LARGE, "M, N and K must be below 2^31");
+  if (grouped) {
+    if (E < 1 || E > 1024) return fail(HQ_ERR_INVALID_ARG, "E = %d outside [1, 1024]", E);
+    if (!offsets) return fail(HQ_ERR_INVALID_ARG, "offsets must not be null");
+    if (static_cast<int64_t>(E) * N >= k2p31) return fail(HQ_ERR_TOO_LARGE, "E*N must be below 2^31");
+  }
+  const int esize = kind == 0 ? 1 : 2;
+  if ((K * esize) % 16 != 0)
+    return fail(HQ_ERR_INVALID_ARG, "K = %lld: rows of A and B must be a multiple of 16 bytes", (long long)K);
+  if (N % 8 != 0) return fail(HQ_ERR_INVALID_ARG, "N = %lld must be a multiple of 8 (16-byte output rows)", (long long)N);
+  if (kind == 0) {
+    if (!xs || !ws) return fail(HQ_ERR_INVALID_ARG, "x_scale and w_scale must not be null");
+    if (xs_len != 1 && xs_len != M)
+      return fail(HQ_ERR_INVALID_ARG, "x_scale_len %lld must be 1 or M = %lld", (long long)xs_len, (long long)M);
+    const int64_t wn = grouped ? static_cast<int64_t>(E) * N : N;
+    if (ws_len != 1 && ws_len != wn)
+      return fail(HQ_ERR_INVALID_ARG, "w_scale_len %lld must be 1 or %lld", (long long)ws_len, (long long)wn);
+    if (!is_aligned(xs, 4) || !is_aligned(ws, 4)) return fail(HQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  }
+  if (!a || !b || !out) return fail(HQ_ERR_INVALID_ARG, "operand and output pointers must not be null");
+  if (!is_aligned(out, 16)) return fail(HQ_ERR_MISALIGNED, "out must start on a 16-byte boundary");
+  if (!is_aligned(a, 16) || !is_aligned(b, 16)) return fail(HQ_ERR_MISALIGNED, "A and B must be 16-byte aligned");
+  if (offsets && !is_aligned(offsets, 4)) return fail(HQ_ERR_MISALIGNED, "offsets must be 4-byte aligned");
+  const int64_t ebatch = grouped ? E : 1;
+  const Range outs[] = {{out, static_cast<size_t>(M) * static_cast<size_t>(N) * 2, "out"}};
+  const Range ins[] = {{a, static_cast<size_t>(M * K * esize), "A"},
+                       {b, static_cast<size_t>(ebatch * N * K * esize), "B"},
+                       {xs, kind == 0 ? static_cast<size_t>(xs_len) * 4 : 0, "x_scale"},
+                       {ws, kind == 0 ? static_cast<size_t>(ws_len) * 4 : 0, "w_scale"},
+                       {offsets, offsets ? static_cast<size_t>(E + 1) * 4 : 0, "offsets"}};
+  hq_status s = check_overlaps(outs, 1, ins, 5);
+  if (s != HQ_OK) return s;
+  const Range devs[] = {{a, 0, "A"}, {b, 0, "B"}, {xs, 0, "x_scale"}, {ws, 0, "w_scale"},
+                        {offsets, 0, "offsets"}, {out, 0, "out"}};
+  s = check_device_ptrs(devs, 6);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  if (M == 0 || N == 0) return ok();
+  hq::GemmArgs g;
+  g.kind = kind; g.fmt = fmt; g.a = a; g.b = b;
+  g.x_scale = xs; g.x_scale_len = xs_len; g.w_scale = ws; g.w_scale_len = ws_len;
+  g.offsets = offsets; g.E = grouped ? E : 1;
+  g.M = M; g.N = N; g.K = K; g.out = out;
+  g.stream = reinterpret_cast<cudaStream_t>(stream);
+  std::string msg;
+  return launched(hq::launch_gemm(g, &msg), "gemm launch", msg);
+}
+
+}  // namespace
+
+hq_status hq_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,
+                       int64_t x_scale_len, const float* w_scale, int64_t w_scale_len, int64_t M, int64_t N,
+                       int64_t K, void* out, hq_stream_t stream) {
+  return gemm_common(0, xq, wq, fmt, x_scale, x_scale_len, w_scale, w_scale_len, nullptr, 1, M, N, K, out, stream);
+}
+
+hq_status hq_grouped_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,
+                               int64_t x_scale_len, const float* w_scale, int64_t w_scale_len,
+                               const int32_t* offsets, int32_t E, int64_t M_total, int64_t N, int64_t K, void* out,
+                               hq_stream_t stream) {
+  if (!offsets) return fail(HQ_ERR_INVALID_ARG, "offsets must not be null");
+  return gemm_common(0, xq, wq, fmt, x_scale, x_scale_len, w_scale, w_scale_len, offsets, E, M_total, N, K, out,
+                     stream);
+}
+
+hq_status hq_grouped_gemm_bf16(const void* x, const void* w, const int32_t* offsets, int32_t E, int64_t M_total,
+                               int64_t N, int64_t K, void* out, hq_stream_t stream) {
+  if (!offsets) return fail(HQ_ERR_INVALID_ARG, "offsets must not be null");
+  return gemm_common(1, x, w, 0, nullptr, 0, nullptr, 0, offsets, E, M_total, N, K, out, stream);
+}
+
+hq_status hq_check_device_error(void) {
+  unsigned w = 0;
+  const cudaError_t e = hq::read_and_clear_device_error(&w);
+  if (e != cudaSuccess) return fail(HQ_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
+  if (w & hq::kDevErrTimeout) return fail(HQ_ERR_TIMEOUT, "a kernel's bounded wait gave up");
+  if (w & hq::kDevErrBadOffsets) return fail(HQ_ERR_INVALID_ARG, "grouped GEMM offsets were malformed");
+  return ok();
+}
+
+const char* hq_last_error(void) { return g_last_error.c_str(); }
+
+const char* hq_version(void) { return "hq 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

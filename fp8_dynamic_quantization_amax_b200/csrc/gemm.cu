@@ -1,0 +1,560 @@
+// gemm.cu -- scaled FP8 (and bf16) GEMM on sm_100a tensor cores.
+//
+// out[m, n] = bf16_rn( acc[m, n] * x_scale[m'] * w_scale[n'] ),
+// acc = sum_k A[m, k] * B[n, k] accumulated in FP32 on tcgen05 tensor cores.
+// (ROCm/aiter PR 6437 "Technical Details": XQ[M,K], WQ[N,K], x_scale[M],
+// w_scale[N], caller-owned bf16 out; AstrAI ops.cu mm_fp8: NT layout, FP32
+// accumulate; megablocks-hip TODO-gg.md: the grouped per-expert form, output
+// overwritten.)
+//
+// Design (one persistent CTA per SM, 192 threads, 6 warps):
+//   warp 0      TMA producer: one elected thread streams 128-byte-wide K
+//               slices of A (128 rows) and B (BN rows) into a ring of shared
+//               memory stages (128B swizzle), signalling mbarriers.
+//   warp 1      allocates TMEM (two BN-column FP32 accumulators) and issues
+//               tcgen05.mma (kind::f8f6f4 for FP8, kind::f16 for bf16) from
+//               one thread; tcgen05.commit frees a stage / publishes an
+//               accumulator.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp owns its
+//               32-lane TMEM quadrant), scale, round to bf16, 16-byte stores.
+//               Two accumulators let the epilogue of tile i overlap the
+//               main loop of tile i+1.
+// Every wait is bounded: on a stalled barrier the CTA records an error in a
+// device word, drains what it has in flight and exits instead of hanging.
+#include "hq_internal.cuh"
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <mutex>
+
+namespace hq {
+
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+constexpr int kBM = 128;            // tile rows (MMA M)
+constexpr int kBKBytes = 128;       // K bytes per stage = one 128B swizzle row
+constexpr int kGemmThreads = 192;
+constexpr int kMaxExperts = 1024;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr unsigned long long kDrainLimitNs = 200000000ull;  // 0.2 s
+
+struct Params {
+  int M, N, K;          // M: rows of A (M_total for grouped), K in elements
+  int nkb;              // number of K blocks
+  int n_tiles, m_tiles; // m_tiles: dense only
+  int group_m;          // rasterisation group (dense)
+  int E;                // experts (1 for dense)
+  const int32_t* offsets;
+  const float* xs;
+  int xs_bcast;
+  const float* ws;
+  int ws_bcast;
+  uint16_t* out;
+  uint32_t idesc;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase with the given parity has completed.  Gives up after
+// `limit` ns (recording a timeout) or as soon as another role has aborted.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       unsigned long long limit = kWaitLimitNs) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > limit) {
+        *abort_flag = 1;
+        atomicOr(&g_device_error, kDevErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                 // leading byte offset (16 B; unused here)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;         // stride byte offset: next 8-row group
+  d |= static_cast<uint64_t>(1) << 46;                 // descriptor version for sm_100
+  d |= static_cast<uint64_t>(2) << 61;                 // swizzle mode: 128 B
+  return d;
+}
+
+template <int KIND>
+__device__ __forceinline__ void mma_issue(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  if constexpr (KIND == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  }
+}
+
+// 32 TMEM lanes x 32 columns of 32-bit: thread t of the warp gets lane
+// (quadrant base + t), 32 consecutive columns.  The wait is in the same asm
+// block so the registers are never read before the load has landed.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// ------------------------------------------------------------ tile schedule
+struct Tile {
+  int a_row;   // first A row loaded (global)
+  int b_row;   // first B row loaded (global, in the [E*N, K] view)
+  int row_lo;  // rows [row_lo, row_hi) are written
+  int row_hi;
+  int col0;    // first output column
+  int expert;
+};
+
+template <int BN>
+__device__ __forceinline__ Tile decode_tile(int t, const Params& p, const int* prefix, const int* starts) {
+  Tile T;
+  if (p.offsets == nullptr) {
+    const int per_group = p.group_m * p.n_tiles;
+    const int g = t / per_group;
+    const int within = t - g * per_group;
+    const int gm = min(p.group_m, p.m_tiles - g * p.group_m);
+    const int mt = g * p.group_m + within % gm;
+    const int nt = within / gm;
+    T.row_lo = mt * kBM;
+    T.row_hi = min(p.M, T.row_lo + kBM);
+    T.a_row = T.row_lo;
+    T.col0 = nt * BN;
+    T.b_row = T.col0;
+    T.expert = 0;
+  } else {
+    int lo = 0, hi = p.E;  // find e with prefix[e] <= t < prefix[e+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prefix[mid] <= t) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int local = t - prefix[e];
+    const int mt = local / p.n_tiles;
+    const int nt = local - mt * p.n_tiles;
+    T.row_lo = starts[e] + mt * kBM;
+    T.row_hi = min(starts[e + 1], T.row_lo + kBM);
+    T.a_row = T.row_lo;
+    T.col0 = nt * BN;
+    T.b_row = e * p.N + T.col0;
+    T.expert = e;
+  }
+  return T;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int KIND, int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, const Params p) {
+  constexpr int kABytes = kBM * kBKBytes;
+  constexpr int kBBytes = BN * kBKBytes;
+  constexpr int kStageBytes = kABytes + kBBytes;
+  constexpr int kKElems = (KIND == 0) ? 128 : 64;  // K elements per stage
+  constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t final_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ int tile_prefix[kMaxExperts + 1];
+  __shared__ int row_start[kMaxExperts + 1];
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-byte aligned stages
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kABytes;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 128);
+    }
+    mbar_init(&final_bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (threadIdx.x == 32 && p.offsets != nullptr) {
+    // Clamp the device offsets into [prev, M] and build the tile prefix.
+    bool bad = false;
+    int prev = 0;
+    int acc = 0;
+    for (int e = 0; e <= p.E; ++e) {
+      int o = p.offsets[e];
+      if ((e == 0 && o != 0) || (e == p.E && o != p.M) || o < prev || o > p.M) bad = true;
+      o = min(max(o, prev), p.M);
+      if (e == 0) o = 0;
+      row_start[e] = o;
+      if (e > 0) {
+        const int cnt = o - prev;
+        tile_prefix[e - 1] = acc;
+        acc += ((cnt + kBM - 1) / kBM) * p.n_tiles;
+      }
+      prev = o;
+    }
+    tile_prefix[p.E] = acc;
+    if (bad && blockIdx.x == 0) atomicOr(&g_device_error, kDevErrBadOffsets);
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_b) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  const int total = (p.offsets != nullptr) ? tile_prefix[p.E] : p.m_tiles * p.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed_parity[STAGES];
+      bool armed[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) { armed[s] = false; armed_parity[s] = 0; }
+      bool stop = false;
+      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+        const Tile T = decode_tile<BN>(t, p, tile_prefix, row_start);
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { stop = true; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+          tma_load_2d(sA + stage * kABytes, &tm_a, &full_bar[stage], kb * kKElems, T.a_row);
+          tma_load_2d(sB + stage * kBBytes, &tm_b, &full_bar[stage], kb * kKElems, T.b_row);
+#pragma unroll
+          for (int s = 0; s < STAGES; ++s)
+            if (s == stage) { armed[s] = true; armed_parity[s] = phase; }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (abort_flag) {
+        // drain: every armed stage's last transfer must land before exit
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) {
+          int dummy = 0;
+          if (armed[s]) mbar_wait(&full_bar[s], armed_parity[s], &dummy, kDrainLimitNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    bool issued = false;
+    bool stop = false;
+    int i = 0;
+    for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++i) {
+      const int acc = i & 1;
+      const uint32_t acc_phase = (i >> 1) & 1;
+      if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = 0; kb < p.nkb; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { stop = true; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t ad = smem_desc(smem_u32(sA + stage * kABytes));
+          const uint64_t bd = smem_desc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+          for (int k = 0; k < kBKBytes / 32; ++k)  // 32 bytes of K per instruction
+            mma_issue<KIND>(d_tmem, ad + 2u * k, bd + 2u * k, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&empty_bar[stage]);
+          issued = true;
+        }
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (stop) break;
+      if (lane == 0) tc_commit(&tfull_bar[acc]);
+      __syncwarp();
+    }
+    if (abort_flag && lane == 0 && issued) {
+      int dummy = 0;
+      tc_commit(&final_bar);
+      mbar_wait(&final_bar, 0, &dummy, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------- epilogue
+    const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
+    const int r = quad * 32 + lane;
+    int i = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+      const int acc = i & 1;
+      const uint32_t acc_phase = (i >> 1) & 1;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag)) break;
+      tc_fence_after();
+      const Tile T = decode_tile<BN>(t, p, tile_prefix, row_start);
+      const int row = T.row_lo + r;
+      const bool vrow = row < T.row_hi;
+      float xsv = 1.0f;
+      const float* wsp = nullptr;
+      if (KIND == 0) {
+        if (vrow) xsv = __ldg(p.xs + (p.xs_bcast ? 0 : row));
+        wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
+      }
+      uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN + c), v);
+        const int n0 = T.col0 + c;
+        if (vrow && n0 < p.N) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int nj = n0 + 8 * j;
+            if (nj < p.N) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float a = (p.nkb > 0) ? __uint_as_float(v[8 * j + e]) : 0.0f;
+                if (KIND == 0) {
+                  const float s = xsv * __ldg(wsp + (p.ws_bcast ? 0 : nj + e));
+                  f[e] = a * s;
+                } else {
+                  f[e] = a;
+                }
+              }
+              st_global_v4(orow + nj, pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                           pack_bf16x2(f[6], f[7]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// --------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D row-major [rows, cols] map with a {128-byte, box_rows} box, 128B swizzle.
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, int elem_bytes, uint32_t box_rows,
+              std::string* msg) {
+  auto encode = get_encode_fn();
+  if (!encode) {
+    *msg = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  const CUtensorMapDataType dt = (elem_bytes == 1) ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKBytes / elem_bytes), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (%d) for [%llu, %llu] x %d B", static_cast<int>(r),
+             static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols), elem_bytes);
+    *msg = buf;
+    return false;
+  }
+  return true;
+}
+
+template <int KIND, int BN, int STAGES>
+cudaError_t run(const GemmArgs& a, std::string* msg) {
+  constexpr int kElem = (KIND == 0) ? 1 : 2;
+  constexpr int kSmem = STAGES * (kBM + BN) * kBKBytes + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(k_gemm<KIND, BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  });
+  if (attr_err != cudaSuccess) {
+    *msg = "cudaFuncSetAttribute failed";
+    return attr_err;
+  }
+  const uint64_t kdim = a.K > 0 ? static_cast<uint64_t>(a.K) : 16;  // K == 0: maps are never used
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), kdim, kElem, kBM, msg) ||
+      !make_map(&tb, a.b, static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N), kdim, kElem, BN, msg))
+    return cudaErrorInvalidValue;
+
+  Params p;
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.nkb = static_cast<int>((a.K + (kBKBytes / kElem) - 1) / (kBKBytes / kElem));
+  p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+  p.m_tiles = static_cast<int>((a.M + kBM - 1) / kBM);
+  p.group_m = 16;
+  p.E = a.E;
+  p.offsets = a.offsets;
+  p.xs = a.x_scale;
+  p.xs_bcast = (a.x_scale_len == 1) ? 1 : 0;
+  p.ws = a.w_scale;
+  p.ws_bcast = (a.w_scale_len == 1) ? 1 : 0;
+  p.out = static_cast<uint16_t*>(a.out);
+  const uint32_t ab_fmt = (KIND == 0) ? static_cast<uint32_t>(a.fmt) : 1u;  // E4M3/E5M2, or BF16
+  p.idesc = (1u << 4)                                   // D: FP32
+            | (ab_fmt << 7) | (ab_fmt << 10)            // A and B element types
+            | (static_cast<uint32_t>(BN >> 3) << 17)     // N / 8
+            | (static_cast<uint32_t>(kBM >> 4) << 24);   // M / 16 (A and B K-major)
+
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int sms = device_sm_count(dev);
+  int64_t tiles_bound;
+  if (a.offsets == nullptr)
+    tiles_bound = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  else
+    tiles_bound = (static_cast<int64_t>(p.m_tiles) + a.E) * p.n_tiles;
+  int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
+  if (grid < 1) grid = 1;
+  k_gemm<KIND, BN, STAGES><<<grid, kGemmThreads, kSmem, a.stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
+  // Wide tiles when there is enough work to fill the machine with them.
+  const bool wide = (a.N % 256 == 0) && a.N >= 2048 && a.M >= 256;
+  if (a.kind == 0) {
+    if (wide) return run<0, 256, 4>(a, msg);
+    return run<0, 128, 6>(a, msg);
+  }
+  if (wide) return run<1, 256, 4>(a, msg);
+  return run<1, 128, 6>(a, msg);
+}
+
+cudaError_t read_and_clear_device_error(unsigned* word) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  unsigned w = 0;
+  e = cudaMemcpyFromSymbol(&w, g_device_error, sizeof(w));
+  if (e != cudaSuccess) return e;
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  *word = w;
+  return e;
+}
+
+}  // namespace hq

@@ -1,0 +1,59 @@
+// hq_internal.cuh -- declarations shared by the translation units of
+// libhq.so (api.cu, quantize.cu, gemm.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+#include <string>
+
+namespace hq {
+
+// Format facts (hip-quant README "FP8 Formats"): largest finite magnitude.
+constexpr float kFmaxE4M3 = 448.0f;
+constexpr float kFmaxE5M2 = 57344.0f;
+
+struct QuantizeArgs {
+  const void* x;
+  int xt;            // 0 f32, 1 bf16, 2 f16
+  int64_t rows, cols;
+  int fmt;           // 0 E4M3, 1 E5M2
+  int gran;          // 0 tensor, 1 token, 2 channel
+  uint8_t* q;
+  float* scales;
+  float* amax_out;   // nullable
+  float* ring;       // nullable (delayed mode)
+  int ring_len, ring_idx, ring_margin;
+  void* ws;          // workspace (may be null when none is needed)
+  cudaStream_t stream;
+};
+
+size_t quantize_workspace_bytes(int gran, int64_t rows, int64_t cols, int delayed);
+cudaError_t launch_quantize(const QuantizeArgs& a);
+
+struct GemmArgs {
+  int kind;                 // 0: fp8 a8w8 (kind::f8f6f4), 1: bf16 (kind::f16)
+  int fmt;                  // fp8 format of both operands (kind 0)
+  const void* a;            // [M_total, K]
+  const void* b;            // [E, N, K] (E = 1 for the dense GEMM)
+  const float* x_scale;     // nullable for kind 1
+  int64_t x_scale_len;
+  const float* w_scale;     // nullable for kind 1
+  int64_t w_scale_len;
+  const int32_t* offsets;   // null: dense GEMM (one group of M rows)
+  int E;
+  int64_t M, N, K;
+  void* out;
+  cudaStream_t stream;
+};
+
+// Returns cudaSuccess or the failing call's error; *msg gets a description.
+cudaError_t launch_gemm(const GemmArgs& a, std::string* msg);
+
+// Device error word (set by bounded waits and by offset validation).
+enum : unsigned { kDevErrTimeout = 1u, kDevErrBadOffsets = 2u };
+cudaError_t read_and_clear_device_error(unsigned* word);
+
+int device_sm_count(int dev);
+
+}  // namespace hq

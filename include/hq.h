@@ -1,0 +1,233 @@
+/*
+ * hq.h -- C ABI of the B200 (sm_100a) dynamic-FP8 quantize and scaled FP8
+ * GEMM library (libhq.so).
+ *
+ * The operations restate, in this library's own terms, the problem the
+ * following pages describe:
+ *   - hip-quant 0.6.0 README: "FP8 Formats" (E4M3 / E5M2 facts, OCP
+ *     round-to-nearest-even), "Training-path numerical guards" (scales are
+ *     pre-quant multipliers; the reciprocal is the dequant scale; non-finite
+ *     amax samples are ignored), "Scale / amax tracking", "Memory Safety".
+ *   - AstrAI csrc/kernels/fp8/ops.cu: quantize_bf16 (quantize with fused
+ *     amax), commit "finalize fp8 scale rings inside quantize kernels" (the
+ *     [hist | scale | counter] ring updated by the last block), mm_fp8 and
+ *     linear_forward_fp8 (NT layout: A = XQ[M,K], B = WQ[N,K]).
+ *   - fuel-ir 0.22.4 src/quant_scale.rs: ScaleGranularity, scale_count,
+ *     ScalePair.
+ *   - ROCm/aiter PR 6437 "Technical Details": an a8w8 GEMM that writes a
+ *     caller-owned, contiguous, 16-byte-aligned bf16 out[M,N], validation
+ *     before launch, empty out is a no-op, out must not overlap an input.
+ *   - megablocks-hip _dev/TODO-gg.md: the grouped (per-expert) GEMM; the
+ *     output is overwritten, never accumulated into.
+ *
+ * Conventions common to every entry point:
+ *   - Every buffer pointer is a DEVICE pointer on the current CUDA device,
+ *     owned by the caller.  The library allocates nothing on any call.
+ *   - Buffers are dense and row-major (C order); there are no stride
+ *     arguments.
+ *   - All work is enqueued on `stream` (0 = the legacy default stream).
+ *     Calls are asynchronous: a status of HQ_OK means validation passed and
+ *     the launches were enqueued.
+ *   - Validation runs before any launch.  On any error the call returns a
+ *     status, sets the message returned by hq_last_error(), and writes no
+ *     output buffer.  Argument checks come first, then the device checks
+ *     (pointer attributes), then the architecture check.
+ *   - Device-side failures (a bounded wait that gave up, malformed device
+ *     offsets) are recorded in a device error word that hq_check_device_error()
+ *     reads back.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; no CUDA header is needed. */
+typedef struct CUstream_st* hq_stream_t;
+
+typedef enum {
+  HQ_OK = 0,
+  HQ_ERR_INVALID_ARG = 1,      /* null pointer, bad size, bad enum, bad scale length */
+  HQ_ERR_MISALIGNED = 2,       /* a pointer breaks its alignment rule */
+  HQ_ERR_OVERLAP = 3,          /* an output overlaps an input or another output */
+  HQ_ERR_WRONG_DEVICE = 4,     /* a pointer is not device memory of the current device */
+  HQ_ERR_UNSUPPORTED_ARCH = 5, /* the current device is not compute capability 10.0 */
+  HQ_ERR_CUDA = 6,             /* a CUDA runtime/driver call failed */
+  HQ_ERR_TIMEOUT = 7,          /* a kernel's bounded wait gave up (device error word) */
+  HQ_ERR_TOO_LARGE = 8         /* a size exceeds this library's index range */
+} hq_status;
+
+/* FP8 formats (hip-quant README "FP8 Formats"; AstrAI ops.cu `fmt` 0/1).
+   E4M3: 1 sign, 4 exponent, 3 mantissa bits, bias 7, max +-448, NaN only.
+   E5M2: 1 sign, 5 exponent, 2 mantissa bits, bias 15, max +-57344. */
+typedef enum { HQ_E4M3 = 0, HQ_E5M2 = 1 } hq_fp8_format;
+
+/* Scale granularity of a [rows, cols] tensor (fuel-ir quant_scale.rs
+   ScaleGranularity): one scale for the tensor, one per row, one per column. */
+typedef enum { HQ_PER_TENSOR = 0, HQ_PER_TOKEN = 1, HQ_PER_CHANNEL = 2 } hq_granularity;
+
+/* Element type of a quantize input (hip-quant README: float32, float16 and
+   bfloat16 inputs). */
+typedef enum { HQ_F32 = 0, HQ_BF16 = 1, HQ_F16 = 2 } hq_dtype;
+
+/* Number of f32 scales for a [rows, cols] tensor: 1, rows or cols
+   (quant_scale.rs ScaleGranularity::scale_count).  Returns -1 for an
+   invalid granularity or negative size. */
+int64_t hq_scale_count(hq_granularity g, int64_t rows, int64_t cols);
+
+/* "per_tensor" / "per_token" / "per_channel" (quant_scale.rs as_str), or
+   NULL for an invalid value. */
+const char* hq_granularity_name(hq_granularity g);
+
+/* Writes "act_<g>_weight_<g>" (quant_scale.rs ScalePair Display) into buf
+   (NUL-terminated, at most len bytes).  Returns the string length, or -1
+   on an invalid granularity or a buffer that is too short. */
+int hq_scale_pair_name(hq_granularity act, hq_granularity weight, char* buf, size_t len);
+
+/* Bytes of device workspace hq_quantize_fp8 needs for this shape and mode
+   (delayed != 0: the delayed per-tensor mode).  0 means no workspace.
+   The caller zero-fills a workspace once before its first use; every call
+   returns its accumulator words to zero, so the same workspace can be reused
+   by calls that run one after another on the device.  Two calls that may
+   run at the same time need two workspaces. */
+size_t hq_quantize_workspace_bytes(hq_granularity g, int64_t rows, int64_t cols, int delayed);
+
+/*
+ * Dynamic (or delayed) FP8 quantization of a dense row-major x[rows, cols].
+ *
+ * Computes, per scale group of granularity g (tensor / row / column):
+ *   amax = max |x| over the group's finite elements (NaN and +-Inf skipped)
+ *   m    = fmax / amax in f32 (fmax = 448 or 57344); m = 1 when amax == 0
+ *          or the quotient is not finite
+ *   q    = saturating round-to-nearest-even FP8 code of f32(x) * m:
+ *          |y| >= fmax and +-Inf -> +-max code, NaN -> 0x7F
+ *   scales[i] = 1 / m (f32): the dequant scale the GEMM consumes
+ *   amax_out[i] = amax (optional)
+ * (hip-quant README "FP8 Formats" and "Training-path numerical guards";
+ * AstrAI ops.cu quantize_bf16; quant_scale.rs scale_count.)
+ *
+ * Delayed mode (ring != NULL; only g == HQ_PER_TENSOR): ring is a device f32
+ * buffer of ring_len + 2 words [hist[ring_len] | scale | counter] (AstrAI
+ * ops.cu ring commit and pack_quantize_params).  The kernel quantizes with
+ * m = ring[ring_len], writes scales[0] = 1/m, and its last block then
+ * stores this call's amax in hist[ring_idx], takes win = max(hist) and, if
+ * win is finite and > 0, publishes ring[ring_len] = (fmax / win) * 2^-margin
+ * (kept otherwise).  The counter word must be 0 on entry and is 0 on exit.
+ * A fresh ring is hist = 0, scale = 1, counter = 0; the caller passes
+ * ring_idx = step mod ring_len.
+ *
+ * Arguments:
+ *   x            device, rows*cols elements of type xt
+ *   q            device, rows*cols bytes (uint8 FP8 codes), row-major
+ *   scales       device, hq_scale_count(g, rows, cols) f32
+ *   amax_out     device or NULL, hq_scale_count(g, rows, cols) f32
+ *   workspace    device, >= hq_quantize_workspace_bytes(...) bytes, 256-byte
+ *                aligned, zeroed before first use (NULL if 0 bytes needed)
+ * Errors: HQ_ERR_INVALID_ARG (null, negative size, bad enum, ring with
+ *   g != PER_TENSOR, ring_len < 1, ring_idx outside [0, ring_len), workspace
+ *   too small), HQ_ERR_MISALIGNED (x not aligned to its element size, ring
+ *   or scales not 4-byte aligned, workspace not 256-byte aligned),
+ *   HQ_ERR_OVERLAP (q / scales / amax_out / ring / workspace overlapping
+ *   each other or x), HQ_ERR_WRONG_DEVICE, HQ_ERR_UNSUPPORTED_ARCH,
+ *   HQ_ERR_TOO_LARGE (rows*cols >= 2^40), HQ_ERR_CUDA.
+ * A shape with scale_count == 0 returns HQ_OK without a launch.  rows*cols
+ * == 0 with scale_count > 0 writes scales = 1/m with amax 0 (and updates
+ * the ring with amax 0).
+ */
+hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols,
+                          hq_fp8_format fmt, hq_granularity g,
+                          uint8_t* q, float* scales, float* amax_out,
+                          float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,
+                          void* workspace, size_t workspace_bytes, hq_stream_t stream);
+
+/*
+ * Scaled FP8 GEMM, NT layout, into a caller-owned bf16 buffer:
+ *   out[m, n] = bf16_rn( acc[m, n] * x_scale[m'] * w_scale[n'] ),
+ *   acc[m, n] = sum_k dec(xq[m, k]) * dec(wq[n, k])   (FP32 accumulation)
+ * with m' = m if x_scale_len == M else 0, n' = n if w_scale_len == N else 0
+ * (ROCm/aiter PR 6437 "Technical Details": XQ[M,K], WQ[N,K], x_scale[M],
+ * w_scale[N], bf16 out; AstrAI ops.cu mm_fp8: out = a @ b^T * (sa*sb),
+ * FP32 accumulate).  Both operands use format fmt.
+ *
+ * Arguments:
+ *   xq        device, M*K FP8 codes, row-major [M, K], 16-byte aligned
+ *   wq        device, N*K FP8 codes, row-major [N, K], 16-byte aligned
+ *   x_scale   device f32, x_scale_len in {1, M}
+ *   w_scale   device f32, w_scale_len in {1, N}
+ *   out       device bf16 (uint16 bits), dense row-major [M, N], 16-byte
+ *             aligned start; it may be a view into a larger buffer, and
+ *             nothing outside [out, out + M*N) is written.  Overwritten,
+ *             never accumulated into.
+ * Errors: HQ_ERR_INVALID_ARG (null, negative size, K % 16 != 0, N % 8 != 0,
+ *   bad scale length, bad fmt), HQ_ERR_MISALIGNED (out, xq or wq not 16-byte
+ *   aligned, scales not 4-byte aligned), HQ_ERR_OVERLAP (out overlapping
+ *   any input), HQ_ERR_WRONG_DEVICE, HQ_ERR_UNSUPPORTED_ARCH,
+ *   HQ_ERR_TOO_LARGE (M, N or K >= 2^31), HQ_ERR_CUDA.
+ * M == 0 or N == 0 returns HQ_OK with no launch.  K == 0 writes
+ * bf16(0 * scales).
+ */
+hq_status hq_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt,
+                       const float* x_scale, int64_t x_scale_len,
+                       const float* w_scale, int64_t w_scale_len,
+                       int64_t M, int64_t N, int64_t K, void* out, hq_stream_t stream);
+
+/*
+ * Grouped (per-expert) scaled FP8 GEMM (megablocks-hip TODO-gg.md gmm):
+ * for each expert e and each row r in [offsets[e], offsets[e+1]):
+ *   out[r, n] = bf16_rn( x_scale[r'] * w_scale[e*N + n'] *
+ *                        sum_k dec(xq[r, k]) * dec(wq[e, n, k]) )
+ *
+ * Arguments:
+ *   xq        device [M_total, K] FP8 codes, 16-byte aligned
+ *   wq        device [E, N, K] FP8 codes, 16-byte aligned
+ *   x_scale   device f32, x_scale_len in {1, M_total}
+ *   w_scale   device f32, w_scale_len in {1, E*N}
+ *   offsets   device int32 [E + 1]: offsets[0] = 0, non-decreasing,
+ *             offsets[E] = M_total.  Read on the device only (no host sync).
+ *   out       device bf16 [M_total, N], 16-byte aligned, overwritten.
+ * Rows outside every expert's range are not written.  Malformed offsets
+ * (decreasing, or outside [0, M_total]) never cause an access outside the
+ * buffers: offsets are clamped and the device error word records
+ * HQ_ERR_INVALID_ARG.
+ * Errors as hq_gemm_a8w8, plus E < 1 (HQ_ERR_INVALID_ARG).
+ */
+hq_status hq_grouped_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt,
+                               const float* x_scale, int64_t x_scale_len,
+                               const float* w_scale, int64_t w_scale_len,
+                               const int32_t* offsets, int32_t E,
+                               int64_t M_total, int64_t N, int64_t K,
+                               void* out, hq_stream_t stream);
+
+/*
+ * Grouped bf16 GEMM with FP32 accumulation (megablocks-hip TODO-gg.md: the
+ * per-expert bf16 product, overwritten into out):
+ *   out[r, n] = bf16_rn( sum_k x[r, k] * w[e, n, k] ),  r in expert e's rows
+ * x: device bf16 [M_total, K]; w: device bf16 [E, N, K]; K % 8 == 0.
+ * Other arguments, rules and errors as hq_grouped_gemm_a8w8.
+ */
+hq_status hq_grouped_gemm_bf16(const void* x, const void* w,
+                               const int32_t* offsets, int32_t E,
+                               int64_t M_total, int64_t N, int64_t K,
+                               void* out, hq_stream_t stream);
+
+/* Synchronizes the current device, then reads and clears the device error
+   word: HQ_OK, HQ_ERR_TIMEOUT (a bounded wait in a kernel gave up; that
+   launch's outputs are undefined), HQ_ERR_INVALID_ARG (malformed grouped
+   offsets), or HQ_ERR_CUDA. */
+hq_status hq_check_device_error(void);
+
+/* Message for the last error on this host thread ("" if none). */
+const char* hq_last_error(void);
+
+/* Library version string. */
+const char* hq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

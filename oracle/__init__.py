@@ -60,6 +60,8 @@ def lib():
         L.hqo_encode_sat_array.restype = None
         L.hqo_decode_array.argtypes = [P, i64, ci, P]
         L.hqo_decode_array.restype = None
+        L.hqo_ring_update.argtypes = [ctypes.c_float, ci, P, ci, ci, ci]
+        L.hqo_ring_update.restype = None
         _lib = L
     return _lib
 
@@ -73,7 +75,9 @@ def _dtype_code(x):
         return F32
     if x.dtype == np.uint16:
         return BF16  # bf16 carried as raw uint16 bit patterns
-    raise TypeError("oracle inputs are float32 or bf16 bit patterns (uint16)")
+    if x.dtype == np.float16:
+        return F16
+    raise TypeError("oracle inputs are float32, float16 or bf16 bit patterns (uint16)")
 
 
 def decode(code: int, fmt: int) -> float:
@@ -143,6 +147,12 @@ def quantize(x: np.ndarray, fmt: int, gran: int, ring: np.ndarray = None,
     if rc != 0:
         raise ValueError("oracle quantize: invalid arguments")
     return q, scales, am
+
+
+def ring_update(amax_value: float, fmt: int, ring: np.ndarray, ring_idx: int, ring_margin: int = 0):
+    """One delayed-scaling ring step (in place) given this step's amax."""
+    assert ring.dtype == np.float32 and ring.flags.c_contiguous
+    lib().hqo_ring_update(amax_value, fmt, _p(ring), ring.size - 2, ring_idx, ring_margin)
 
 
 def gemm_a8w8(xq, wq, fmt, x_scale, w_scale, return_ref=False):

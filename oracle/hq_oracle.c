@@ -252,6 +252,25 @@ void hqo_amax(const void* x, int dtype, int64_t rows, int64_t cols, int gran,
 
 /* ---------------------------------------------------------------- quantize */
 
+/* Delayed-scaling ring step (R6; AstrAI ops.cu ring commit): fold this
+   step's amax into hist[idx], reduce the window, publish the next multiplier
+   fmax / max(hist) / 2^margin when that window is finite and > 0, and leave
+   the counter slot at 0. */
+void hqo_ring_update(float amax, int fmt, float* ring, int ring_len, int ring_idx,
+                     int ring_margin) {
+  float win = 0.0f;
+  int i;
+  ring[ring_idx] = amax;
+  for (i = 0; i < ring_len; ++i)
+    if (ring[i] > win) win = ring[i];
+  if (isfinite(win) && win > 0.0f) {
+    float fmax = (float)get_fmt(fmt).fmax;
+    float next = ldexpf(fmax / win, -ring_margin);
+    if (isfinite(next) && next > 0.0f) ring[ring_len] = next;
+  }
+  ring[ring_len + 1] = 0.0f; /* counter slot, 0 on exit */
+}
+
 /* Dynamic quantize (ring == NULL) or delayed per-tensor quantize (ring !=
    NULL, R6).  q: rows*cols codes; scales: dequant scales d = 1/m (R5);
    amax_out (nullable): the amax array of the input at this granularity.
@@ -284,19 +303,7 @@ int hqo_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
   }
   if (amax_out)
     for (r = 0; r < n; ++r) amax_out[r] = amax[r];
-  if (ring) {
-    float win = 0.0f;
-    int i;
-    ring[ring_idx] = amax[0];
-    for (i = 0; i < ring_len; ++i)
-      if (ring[i] > win) win = ring[i];
-    if (isfinite(win) && win > 0.0f) {
-      float fmax = (float)get_fmt(fmt).fmax;
-      float next = ldexpf(fmax / win, -ring_margin);
-      if (isfinite(next) && next > 0.0f) ring[ring_len] = next;
-    }
-    ring[ring_len + 1] = 0.0f; /* counter slot, 0 on exit */
-  }
+  if (ring) hqo_ring_update(amax[0], fmt, ring, ring_len, ring_idx, ring_margin);
   free(amax);
   free(mult);
   return 0;
@@ -305,12 +312,20 @@ int hqo_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
 /* --------------------------------------------------------------------- GEMM */
 
 /* Integer numerator of a finite code: value = n * 2^-frac, frac = 9 (E4M3)
-   or 16 (E5M2).  Returns 0 for NaN/Inf codes. */
-static int code_int(uint8_t c, int fmt, int64_t* n) {
-  double v = hqo_decode(c, fmt);
-  if (!isfinite(v)) return 0;
-  *n = (int64_t)ldexp(v, fmt == HQO_E4M3 ? 9 : 16); /* exact */
-  return 1;
+   or 16 (E5M2).  The 256 numerators of each format are taken once from
+   hqo_decode and cached; finite[] marks the codes that have one. */
+static int64_t num_tbl[2][256];
+static int finite_tbl[2][256];
+static int tbl_ready[2];
+
+static void build_tbl(int fmt) {
+  int c;
+  for (c = 0; c < 256; ++c) {
+    double v = hqo_decode((uint8_t)c, fmt);
+    finite_tbl[fmt][c] = isfinite(v) ? 1 : 0;
+    num_tbl[fmt][c] = isfinite(v) ? (int64_t)ldexp(v, fmt == HQO_E4M3 ? 9 : 16) : 0; /* exact */
+  }
+  tbl_ready[fmt] = 1;
 }
 
 /* Exact dot product S = sum_k dec(a[k]) * dec(b[k]) as a double (exact for
@@ -318,18 +333,34 @@ static int code_int(uint8_t c, int fmt, int64_t* n) {
    back to IEEE double arithmetic. */
 static double exact_dot(const uint8_t* a, const uint8_t* b, int64_t K, int fmt) {
   int frac = (fmt == HQO_E4M3) ? 9 : 16;
-  __int128 acc = 0;
+  const int64_t* nt;
+  const int* ft;
   int64_t k;
-  for (k = 0; k < K; ++k) {
-    int64_t na, nb;
-    if (!code_int(a[k], fmt, &na) || !code_int(b[k], fmt, &nb)) {
-      double s = 0.0;
-      for (k = 0; k < K; ++k) s += hqo_decode(a[k], fmt) * hqo_decode(b[k], fmt);
-      return s;
+  if (!tbl_ready[fmt]) build_tbl(fmt);
+  nt = num_tbl[fmt];
+  ft = finite_tbl[fmt];
+  if (fmt == HQO_E4M3) {
+    /* |n| <= 448 * 2^9 < 2^18: products < 2^36, K < 2^27 terms fit int64 */
+    int64_t acc = 0;
+    for (k = 0; k < K; ++k) {
+      if (!ft[a[k]] || !ft[b[k]]) goto nonfinite;
+      acc += nt[a[k]] * nt[b[k]];
     }
-    acc += (__int128)na * (__int128)nb;
+    return ldexp((double)acc, -2 * frac);
+  } else {
+    __int128 acc = 0;
+    for (k = 0; k < K; ++k) {
+      if (!ft[a[k]] || !ft[b[k]]) goto nonfinite;
+      acc += (__int128)nt[a[k]] * (__int128)nt[b[k]];
+    }
+    return ldexp((double)acc, -2 * frac);
   }
-  return ldexp((double)acc, -2 * frac);
+nonfinite:
+  {
+    double s = 0.0;
+    for (k = 0; k < K; ++k) s += hqo_decode(a[k], fmt) * hqo_decode(b[k], fmt);
+    return s;
+  }
 }
 
 static uint16_t gemm_entry(const uint8_t* xq, const uint8_t* wq, int fmt,

@@ -1,0 +1,160 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/hq.h declares, and rejects invalid arguments with a
+status before any CUDA call (so fake pointer values are never touched).
+
+Contract source: ROCm/aiter PR 6437 "Technical Details" (validation before
+launch, 16-byte-aligned contiguous out, no overlap) and fuel-ir
+quant_scale.rs (scale_count, as_str, ScalePair display strings).
+"""
+import ctypes
+import os
+import re
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+from fp8_dynamic_quantization_amax_b200 import _hq as H  # noqa: E402
+
+L = H.lib
+OK, INVALID, MISALIGNED, OVERLAP, TOO_LARGE = 0, 1, 2, 3, 8
+
+
+def test_every_declared_symbol_is_exported():
+    header = open(os.path.join(ROOT, "include", "hq.h")).read()
+    declared = set(re.findall(r"\b(hq_[a-z0-9_]+)\s*\(", header))
+    assert declared == set(H.EXPORTED)
+    nm = subprocess.run(["nm", "-D", "--defined-only", H.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (hq_[a-z0-9_]+)\b", nm))
+    assert declared <= exported, declared - exported
+    for name in declared:
+        assert hasattr(L, name)
+
+
+def test_library_links_no_torch_and_no_driver_library():
+    ldd = subprocess.run(["ldd", H.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libtorch" not in ldd and "libc10" not in ldd
+    assert "libcuda.so" not in ldd  # driver reached through the runtime's entry-point query
+
+
+def test_scale_count_and_names():
+    # quant_scale.rs: scale_count(100, 200) = 1 / 100 / 200
+    assert H.hq_scale_count(H.PER_TENSOR, 100, 200) == 1
+    assert H.hq_scale_count(H.PER_TOKEN, 100, 200) == 100
+    assert H.hq_scale_count(H.PER_CHANNEL, 100, 200) == 200
+    assert H.hq_scale_count(7, 1, 1) == -1 and H.hq_scale_count(H.PER_TOKEN, -1, 2) == -1
+    assert [H.hq_granularity_name(g) for g in (0, 1, 2)] == ["per_tensor", "per_token", "per_channel"]
+    assert H.hq_granularity_name(3) is None
+    assert H.hq_scale_pair_name(H.PER_TOKEN, H.PER_CHANNEL) == "act_per_token_weight_per_channel"
+    assert H.hq_scale_pair_name(H.PER_TENSOR, H.PER_TENSOR) == "act_per_tensor_weight_per_tensor"
+    buf = ctypes.create_string_buffer(8)
+    assert L.hq_scale_pair_name(1, 2, buf, 8) == -1  # too short
+    assert H.hq_version().startswith("hq ")
+
+
+def test_workspace_sizes():
+    assert H.hq_quantize_workspace_bytes(H.PER_TOKEN, 8192, 8192) == 0
+    assert H.hq_quantize_workspace_bytes(H.PER_TENSOR, 8192, 8192) == 256
+    assert H.hq_quantize_workspace_bytes(H.PER_TENSOR, 10, 10, delayed=True) == 256
+    c = H.hq_quantize_workspace_bytes(H.PER_CHANNEL, 3, 8192)
+    assert c >= 16 + 8 * 8192 and c % 256 == 0
+
+
+# Fake device addresses: validation must reject before dereferencing.
+BASE = 0x7F0000000000
+
+
+def q(x=BASE, xt=H.BF16, rows=4, cols=64, fmt=H.E4M3, g=H.PER_TOKEN, qp=BASE + 0x100000,
+      sc=BASE + 0x200000, am=None, ring=None, rl=0, ri=0, rm=0, ws=None, wsb=0):
+    return L.hq_quantize_fp8(x, xt, rows, cols, fmt, g, qp, sc, am, ring, rl, ri, rm, ws, wsb, None)
+
+
+def test_quantize_rejections():
+    assert q(xt=5) == INVALID
+    assert q(fmt=2) == INVALID
+    assert q(g=3) == INVALID
+    assert q(rows=-1) == INVALID
+    assert q(rows=1 << 31) == TOO_LARGE
+    assert q(rows=1 << 21, cols=1 << 20) == TOO_LARGE
+    assert q(x=None) == INVALID
+    assert q(qp=None) == INVALID
+    assert q(sc=None) == INVALID
+    # ring only with per-tensor; len >= 1; idx in range
+    assert q(ring=BASE + 0x300000, rl=16, g=H.PER_TOKEN) == INVALID
+    assert q(ring=BASE + 0x300000, rl=0, g=H.PER_TENSOR, ws=BASE + 0x400000, wsb=256) == INVALID
+    assert q(ring=BASE + 0x300000, rl=16, ri=16, g=H.PER_TENSOR, ws=BASE + 0x400000, wsb=256) == INVALID
+    assert q(ring=BASE + 0x300000, rl=16, ri=-1, g=H.PER_TENSOR, ws=BASE + 0x400000, wsb=256) == INVALID
+    # workspace required and large enough
+    assert q(g=H.PER_TENSOR) == INVALID
+    assert q(g=H.PER_TENSOR, ws=BASE + 0x400000, wsb=16) == INVALID
+    assert "workspace" in L.hq_last_error().decode()
+    # alignment
+    assert q(x=BASE + 1) == MISALIGNED
+    assert q(xt=H.F32, x=BASE + 2) == MISALIGNED
+    assert q(sc=BASE + 0x200002) == MISALIGNED
+    assert q(g=H.PER_TENSOR, ws=BASE + 0x400010, wsb=512) == MISALIGNED
+    # overlap: outputs with x, and with each other
+    assert q(qp=BASE + 8) == OVERLAP
+    assert q(sc=BASE + 0x100000 + 8) == OVERLAP
+    assert q(am=BASE + 0x200000) == OVERLAP
+    assert "overlaps" in L.hq_last_error().decode()
+    # nothing to do: scale_count == 0 is accepted without touching anything
+    assert q(rows=0, x=None, qp=None, sc=None) == OK
+
+
+def g8(xq=BASE, wq=BASE + 0x1000000, fmt=H.E4M3, xs=BASE + 0x2000000, xsl=64, ws=BASE + 0x3000000, wsl=128,
+       M=64, N=128, K=256, out=BASE + 0x4000000):
+    return L.hq_gemm_a8w8(xq, wq, fmt, xs, xsl, ws, wsl, M, N, K, out, None)
+
+
+def test_gemm_rejections():
+    assert g8(fmt=9) == INVALID
+    assert g8(M=-1) == INVALID
+    assert g8(K=1 << 31) == TOO_LARGE
+    assert g8(K=250) == INVALID          # rows must be whole 16-byte units
+    assert g8(N=100) == INVALID          # 16-byte output rows
+    assert g8(xsl=3) == INVALID and g8(wsl=64) == INVALID
+    assert g8(xs=None) == INVALID and g8(out=None) == INVALID and g8(xq=None) == INVALID
+    assert g8(out=BASE + 0x4000000 + 2) == MISALIGNED   # odd bf16 offset
+    assert g8(out=BASE + 0x4000000 + 8) == MISALIGNED
+    assert g8(xq=BASE + 8) == MISALIGNED
+    assert g8(xs=BASE + 0x2000001) == MISALIGNED
+    assert g8(out=BASE + 0x10) == OVERLAP                # out over XQ
+    assert g8(out=BASE + 0x1000000) == OVERLAP           # out over WQ
+    assert g8(out=BASE + 0x2000000 - 0x10) == OVERLAP    # out runs into x_scale
+
+
+def test_grouped_rejections():
+    gg = L.hq_grouped_gemm_a8w8
+    args = dict(xq=BASE, wq=BASE + 0x1000000, fmt=0, xs=BASE + 0x2000000, xsl=100, ws=BASE + 0x3000000,
+                wsl=4 * 64, off=BASE + 0x5000000, E=4, M=100, N=64, K=128, out=BASE + 0x6000000)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return gg(a["xq"], a["wq"], a["fmt"], a["xs"], a["xsl"], a["ws"], a["wsl"], a["off"], a["E"], a["M"],
+                  a["N"], a["K"], a["out"], None)
+
+    assert call(off=None) == INVALID
+    assert call(E=0) == INVALID and call(E=2000) == INVALID
+    assert call(wsl=64) == INVALID       # must be 1 or E*N
+    assert call(off=BASE + 0x5000002) == MISALIGNED
+    assert call(out=BASE + 0x5000000) == OVERLAP   # out over offsets
+    b16 = L.hq_grouped_gemm_bf16
+    assert b16(BASE, BASE + 0x1000000, None, 4, 100, 64, 128, BASE + 0x6000000, None) == INVALID
+    assert b16(BASE, BASE + 0x1000000, BASE + 0x5000000, 4, 100, 64, 12, BASE + 0x6000000, None) == INVALID
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # A copy of the package without libhq.so must refuse to import: there is
+    # no CPU or library fallback behind the binding.
+    pkg = os.path.join(ROOT, "fp8_dynamic_quantization_amax_b200")
+    dst = tmp_path / "fp8_dynamic_quantization_amax_b200"
+    dst.mkdir()
+    for f in ("__init__.py", "_hq.py"):
+        shutil.copy(os.path.join(pkg, f), dst / f)
+    r = subprocess.run([sys.executable, "-c", "import fp8_dynamic_quantization_amax_b200"], cwd=str(tmp_path),
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "libhq.so is not built" in r.stderr

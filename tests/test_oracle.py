@@ -507,3 +507,23 @@ def test_zipf_counts_recipe():
     cnt = np.diff(off)
     assert off[0] == 0 and off[-1] == 32768 and cnt[7] == 0 and cnt[41] == 0
     assert (cnt == 0).sum() == 2
+
+
+def test_ring_update_matches_quantize_ring_and_f16_input():
+    # ring_update is the ring step of the delayed quantize, exposed alone
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((6, 10)).astype(np.float32) * np.float32(7.0)
+    r1 = np.array([3.0, 0.5, 2.0, 9.0, 100.0, 0.0], np.float32)
+    r2 = r1.copy()
+    O.quantize(x, O.E5M2, O.PER_TENSOR, ring=r1, ring_idx=2, ring_margin=1)
+    O.ring_update(float(np.abs(x).max()), O.E5M2, r2, 2, 1)
+    np.testing.assert_array_equal(r1, r2)
+    # float16 input: values widen exactly; codes equal those of the f32 copy
+    h = (rng.standard_normal((5, 24)) * 30).astype(np.float16)
+    h[0, 0] = np.float16(np.inf)
+    h[1, 1] = np.float16(np.nan)
+    for gran in (O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL):
+        qa, sa, aa = O.quantize(h, O.E4M3, gran)
+        qb, sb, ab = O.quantize(h.astype(np.float32), O.E4M3, gran)
+        np.testing.assert_array_equal(qa, qb)
+        np.testing.assert_array_equal(sa, sb)

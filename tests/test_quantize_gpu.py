@@ -1,0 +1,175 @@
+"""GPU parity of the quantize kernels against the oracle: codes, dequant
+scales and amax must be bit-exact, through the C ABI.
+
+Covers every kernel variant (warp-per-row, CTA-per-row, generic per-token;
+vector and scalar per-tensor / per-channel; delayed ring), all three input
+types, both formats, ragged shapes, special values (NaN, +-Inf, +-0, f32
+subnormals, huge values, all-zero and all-NaN rows), the degenerate empty
+shapes, and the workload sizes of the quantize sweep (bf16 [8192, 8192]).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from fp8_dynamic_quantization_amax_b200 import _hq as H
+from _gpu import dev, dev_bf16, host
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = ["f32", "bf16", "f16"]
+SHAPES = [(1, 1), (3, 5), (7, 40), (33, 257), (64, 256), (130, 1024), (17, 4096), (5, 8200), (2, 30000),
+          (3, 40000)]
+
+
+def make_input(shape, dtype, seed):
+    rows, cols = shape
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(shape).astype(np.float32) * np.float32(rng.uniform(0.1, 30))
+    flat = x.reshape(-1)
+    n = flat.size
+    if n >= 16:
+        idx = rng.choice(n, size=min(n, 12), replace=False)
+        specials = [np.nan, np.inf, -np.inf, -0.0, 0.0, 1e-40, -1e-40, 3e4, -3e4, 1e-7, 60000.0, 2.5e-5]
+        flat[idx] = np.array(specials[:len(idx)], np.float32)
+    if rows >= 4 and cols >= 2:
+        x[1, :] = 0.0
+        x[2, :] = np.nan
+        x[3, :] = -0.0
+    if dtype == "f32":
+        return x, torch.from_numpy(x).cuda()
+    if dtype == "bf16":
+        b = W.f32_to_bf16_bits(x)
+        return b, dev_bf16(b)
+    h = x.astype(np.float16)
+    return h, torch.from_numpy(h).cuda()
+
+
+def run_gpu(xd, fmt, gran, ring=None, ring_idx=0, ring_margin=0):
+    rows, cols = xd.shape
+    ns = H.hq_scale_count(gran, rows, cols)
+    amax = torch.full((max(ns, 1),), -7.0, dtype=torch.float32, device="cuda")[:ns]
+    q, s = H.hq_quantize_fp8(xd, fmt, gran, amax_out=amax, ring=ring, ring_idx=ring_idx, ring_margin=ring_margin)
+    torch.cuda.synchronize()
+    return host(q), host(s), host(amax)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("gran", [O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL])
+@pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
+def test_quantize_bit_exact(dtype, gran, fmt):
+    for i, shape in enumerate(SHAPES):
+        xh, xd = make_input(shape, dtype, seed=1000 * i + 10 * gran + fmt)
+        q, s, a = run_gpu(xd, fmt, gran)
+        qo, so, ao = O.quantize(xh, fmt, gran)
+        np.testing.assert_array_equal(q, qo, err_msg="codes %s %s" % (shape, dtype))
+        np.testing.assert_array_equal(s.view(np.uint32), so.view(np.uint32), err_msg="scales %s" % (shape,))
+        np.testing.assert_array_equal(a.view(np.uint32), ao.view(np.uint32), err_msg="amax %s" % (shape,))
+    H.hq_check_device_error()
+
+
+@pytest.mark.parametrize("gran", [O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL])
+def test_misaligned_input_takes_scalar_path(gran):
+    # x starting 2 bytes into an allocation: no 16-byte vectors possible
+    xh, _ = make_input((9, 72), "bf16", seed=5)
+    buf = torch.zeros(9 * 72 + 8, dtype=torch.bfloat16, device="cuda")
+    buf[1:1 + 9 * 72] = torch.from_numpy(xh.view(np.int16).reshape(-1)).view(torch.bfloat16).cuda()
+    xd = buf[1:1 + 9 * 72].view(9, 72)
+    assert xd.data_ptr() % 16 != 0
+    q, s, a = run_gpu(xd, O.E4M3, gran)
+    qo, so, ao = O.quantize(xh, O.E4M3, gran)
+    np.testing.assert_array_equal(q, qo)
+    np.testing.assert_array_equal(s, so)
+
+
+def test_empty_shapes():
+    # scale_count == 0: nothing happens; numel == 0 with scales: amax 0, m = 1
+    for gran, shape, ns in [(O.PER_TOKEN, (0, 16), 0), (O.PER_CHANNEL, (16, 0), 0),
+                            (O.PER_TENSOR, (0, 16), 1), (O.PER_TOKEN, (4, 0), 4), (O.PER_CHANNEL, (0, 8), 8)]:
+        xd = torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+        q, s, a = run_gpu(xd, O.E4M3, gran)
+        assert s.size == ns
+        assert (s == 1.0).all() and (a == 0.0).all()
+
+
+def test_workspace_returned_to_zero():
+    xh, xd = make_input((300, 520), "bf16", seed=77)
+    for gran in (O.PER_TENSOR, O.PER_CHANNEL):
+        nbytes = H.hq_quantize_workspace_bytes(gran, 300, 520)
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        for _ in range(3):  # repeated calls on one workspace give the same result
+            q, s = H.hq_quantize_fp8(xd, O.E5M2, gran, workspace=ws)
+            qo, so, _ = O.quantize(xh, O.E5M2, gran)
+            np.testing.assert_array_equal(host(q), qo)
+            np.testing.assert_array_equal(host(s), so)
+        w = host(ws).view(np.uint32)
+        if gran == O.PER_TENSOR:
+            assert w[0] == 0 and w[1] == 0      # amax accumulator and counter
+        else:
+            assert w[0] == 0                    # counter
+            c4 = (520 + 3) // 4 * 4
+            assert (w[4:4 + c4] == 0).all()     # per-column amax accumulators
+
+
+def test_ring_golden_trace_on_gpu():
+    # The hand-computed trace of tests/golden/ring_trace.txt, through the GPU.
+    from test_oracle import _parse_ring_golden
+    ring = torch.tensor([0, 0, 1, 0], dtype=torch.float32, device="cuda")
+    for st in _parse_ring_golden():
+        xd = torch.from_numpy(st["x"].reshape(1, 4).copy()).cuda()
+        q, s, a = run_gpu(xd, O.E4M3, O.PER_TENSOR, ring=ring, ring_idx=st["idx"], ring_margin=st["margin"])
+        assert list(q[0]) == st["codes"]
+        assert s[0] == st["scale"]
+        np.testing.assert_array_equal(host(ring), st["ring"])
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
+def test_delayed_ring_steps(dtype, fmt):
+    L = 16
+    ring_o = np.zeros(L + 2, np.float32)
+    ring_o[L] = 1.0
+    ring_d = torch.from_numpy(ring_o.copy()).cuda()
+    for t in range(40):
+        shape = [(64, 1000), (33, 257), (1, 8), (128, 4096)][t % 4]
+        xh, xd = make_input(shape, dtype, seed=500 + t)
+        margin = t % 3
+        q, s, a = run_gpu(xd, fmt, O.PER_TENSOR, ring=ring_d, ring_idx=t % L, ring_margin=margin)
+        qo, so, ao = O.quantize(xh, fmt, O.PER_TENSOR, ring=ring_o, ring_idx=t % L, ring_margin=margin)
+        np.testing.assert_array_equal(q, qo)
+        np.testing.assert_array_equal(s, so)
+        np.testing.assert_array_equal(a, ao)
+        np.testing.assert_array_equal(host(ring_d).view(np.uint32), ring_o.view(np.uint32))
+    H.hq_check_device_error()
+
+
+def test_structured_f32_cast_through_delayed_scale_one():
+    # With the ring's scale slot at 1.0 the delayed mode casts x itself: run
+    # every (sign, exponent, top-7-mantissa) f32 pattern with several tails.
+    from test_oracle import _structured_f32
+    y = _structured_f32().reshape(-1, 640)
+    ring = torch.tensor([0.0, 1.0, 0.0], dtype=torch.float32, device="cuda")
+    for fmt in (O.E4M3, O.E5M2):
+        ring[1] = 1.0
+        q, s, a = run_gpu(torch.from_numpy(y).cuda(), fmt, O.PER_TENSOR, ring=ring, ring_idx=0)
+        np.testing.assert_array_equal(q.reshape(-1), O.encode_sat_array(y.reshape(-1), fmt))
+
+
+@pytest.fixture(scope="module")
+def sweep_input():
+    return W.sweep()  # bf16 [8192, 8192], the quantize-sweep recipe
+
+
+@pytest.mark.parametrize("gran", [O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL])
+@pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
+def test_quantize_sweep_full_size(sweep_input, gran, fmt):
+    xd = dev_bf16(sweep_input)
+    q, s, a = run_gpu(xd, fmt, gran)
+    qo, so, ao = O.quantize(sweep_input, fmt, gran)
+    np.testing.assert_array_equal(s.view(np.uint32), so.view(np.uint32))
+    np.testing.assert_array_equal(a.view(np.uint32), ao.view(np.uint32))
+    assert np.array_equal(q, qo)
+    if gran == O.PER_TOKEN:
+        assert s[4321] == 1.0 and (q[4321] == 0).all()   # the all-zero row
+    H.hq_check_device_error()

@@ -1,0 +1,116 @@
+"""The delayed-scaling linear stack on the GPU, 200 steps: per step,
+quantize X_t, W_up with their rings -> h = GEMM -> quantize h, W_down with
+their rings -> y = GEMM (per-tensor E4M3, ring length 16, margin 0, X_t std
+ramping 0.5 -> 8; AstrAI ops.cu linear_forward_fp8 and the ring commit).
+
+The oracle is never fed a GPU output.  Stages whose inputs come from the
+generator (X_t, W_up, W_down) are compared bit-exactly, rings included, every
+step.  The later stages (h, its ring, y) depend on GEMM outputs that may
+differ from the exact oracle by a bf16 rounding, so they are compared within
+the GEMM tolerance on a reduced-size stack where the oracle runs the whole
+chain, and by properties at full size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from fp8_dynamic_quantization_amax_b200 import _hq as H
+from _gpu import assert_gemm_close, dev_bf16, host, host_bits
+
+pytestmark = pytest.mark.gpu
+L = 16
+
+
+def fresh_ring():
+    r = np.zeros(L + 2, np.float32)
+    r[L] = 1.0
+    return r
+
+
+def q_delayed(xd, ring_d, t):
+    return H.hq_quantize_fp8(xd, H.E4M3, H.PER_TENSOR, ring=ring_d, ring_idx=t % L, ring_margin=0)
+
+
+def test_stack_reduced_size_full_chain():
+    tokens, dim, hidden, steps = 256, 128, 512, 200
+    wu, wd = W.f32_to_bf16_bits(W.normal((hidden, dim), 0.02, 1)), W.f32_to_bf16_bits(W.normal((dim, hidden), 0.02, 2))
+    wu_d, wd_d = dev_bf16(wu), dev_bf16(wd)
+    rings_o = {k: fresh_ring() for k in ("x", "wu", "h", "wd")}
+    rings_d = {k: torch.from_numpy(fresh_ring()).cuda() for k in rings_o}
+    compared = 0
+    for t in range(steps):
+        x = W.delayed_x(t, tokens, dim, steps)
+        # h's multiplier for this step, before the step, on both sides
+        h_scale_same = host(rings_d["h"])[L] == rings_o["h"][L]
+        xq, xs = q_delayed(dev_bf16(x), rings_d["x"], t)
+        wuq, wus = q_delayed(wu_d, rings_d["wu"], t)
+        h = H.hq_gemm_a8w8(xq, wuq, xs, wus, H.E4M3)
+        hq_, hs = q_delayed(h, rings_d["h"], t)
+        wdq, wds = q_delayed(wd_d, rings_d["wd"], t)
+        y = H.hq_gemm_a8w8(hq_, wdq, hs, wds, H.E4M3)
+        torch.cuda.synchronize()
+        # oracle, fed only generator inputs
+        xqo, xso, _ = O.quantize(x, O.E4M3, O.PER_TENSOR, ring=rings_o["x"], ring_idx=t % L)
+        wuqo, wuso, _ = O.quantize(wu, O.E4M3, O.PER_TENSOR, ring=rings_o["wu"], ring_idx=t % L)
+        ho = O.gemm_a8w8(xqo, wuqo, O.E4M3, xso, wuso)
+        hqo, hso, _ = O.quantize(ho, O.E4M3, O.PER_TENSOR, ring=rings_o["h"], ring_idx=t % L)
+        wdqo, wdso, _ = O.quantize(wd, O.E4M3, O.PER_TENSOR, ring=rings_o["wd"], ring_idx=t % L)
+        yo = O.gemm_a8w8(hqo, wdqo, O.E4M3, hso, wdso)
+        for k in ("x", "wu", "wd"):
+            np.testing.assert_array_equal(host(rings_d[k]).view(np.uint32), rings_o[k].view(np.uint32))
+        np.testing.assert_array_equal(host(xq), xqo)
+        np.testing.assert_array_equal(host(wuq), wuqo)
+        np.testing.assert_array_equal(host(wdq), wdqo)
+        assert_gemm_close(host_bits(h), ho)
+        # h's ring holds amax values of h and the multiplier derived from them:
+        # equal up to the bf16 rounding of the largest |h|
+        np.testing.assert_allclose(host(rings_d["h"])[:L + 1], rings_o["h"][:L + 1], rtol=2e-2)
+        if h_scale_same:
+            # same multiplier for h: y within the GEMM tolerance
+            assert_gemm_close(host_bits(y), yo)
+            compared += 1
+    assert compared >= steps * 3 // 4, compared
+    H.hq_check_device_error()
+
+
+def test_stack_full_size():
+    tokens, dim, hidden, steps = 2048, 1024, 4096, 200
+    wu, wd = W.delayed_weights(dim, hidden)
+    wu_d, wd_d = dev_bf16(wu), dev_bf16(wd)
+    rings_o = {k: fresh_ring() for k in ("x", "wu", "wd")}
+    rings_d = {k: torch.from_numpy(fresh_ring()).cuda() for k in ("x", "wu", "h", "wd")}
+    amax_wu = float(O.amax(wu, O.PER_TENSOR)[0])
+    amax_wd = float(O.amax(wd, O.PER_TENSOR)[0])
+    rng = np.random.default_rng(0)
+    for t in range(steps):
+        x = W.delayed_x(t, tokens, dim, steps)
+        before = {k: r.copy() for k, r in rings_o.items()}
+        xq, xs = q_delayed(dev_bf16(x), rings_d["x"], t)
+        wuq, wus = q_delayed(wu_d, rings_d["wu"], t)
+        h = H.hq_gemm_a8w8(xq, wuq, xs, wus, H.E4M3)
+        hq_, hs = q_delayed(h, rings_d["h"], t)
+        wdq, wds = q_delayed(wd_d, rings_d["wd"], t)
+        y = H.hq_gemm_a8w8(hq_, wdq, hs, wds, H.E4M3)
+        # the oracle's ring steps for the generator-fed stages
+        O.ring_update(float(O.amax(x, O.PER_TENSOR)[0]), O.E4M3, rings_o["x"], t % L)
+        O.ring_update(amax_wu, O.E4M3, rings_o["wu"], t % L)
+        O.ring_update(amax_wd, O.E4M3, rings_o["wd"], t % L)
+        torch.cuda.synchronize()
+        for k in ("x", "wu", "wd"):
+            np.testing.assert_array_equal(host(rings_d[k]).view(np.uint32), rings_o[k].view(np.uint32))
+        # property: h's ring recorded max|h| of the h it quantized, exactly
+        hb = host_bits(h)
+        assert host(rings_d["h"])[t % L] == np.abs(W.bf16_bits_to_f32(hb)).max()
+        if t % 40 == 0 or t == steps - 1:
+            xqo, xso, _ = O.quantize(x, O.E4M3, O.PER_TENSOR, ring=before["x"], ring_idx=t % L)
+            wqo, wso, _ = O.quantize(wu, O.E4M3, O.PER_TENSOR, ring=before["wu"], ring_idx=t % L)
+            np.testing.assert_array_equal(host(xq), xqo)
+            np.testing.assert_array_equal(host(wuq), wqo)
+            ms = rng.integers(0, tokens, 512)
+            ns = rng.integers(0, hidden, 512)
+            ref = O.gemm_a8w8_entries(xqo, wqo, O.E4M3, xso, wso, ms, ns)
+            assert_gemm_close(hb[ms, ns], ref)
+            assert np.isfinite(W.bf16_bits_to_f32(host_bits(y))).all()
+    H.hq_check_device_error()
