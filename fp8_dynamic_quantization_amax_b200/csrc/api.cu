@@ -255,7 +255,8 @@ hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const flo
       return fail(HQ_ERR_INVALID_ARG, "w_scale_len %lld must be 1 or %lld", (long long)ws_len, (long long)wn);
     if (!is_aligned(xs, 4) || !is_aligned(ws, 4)) return fail(HQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
   }
-  if (!a || !b || !out) return fail(HQ_ERR_INVALID_ARG, "operand and output pointers must not be null");
+  if (!out || (K > 0 && (!a || !b)))
+    return fail(HQ_ERR_INVALID_ARG, "operand and output pointers must not be null");
   if (!is_aligned(out, 16)) return fail(HQ_ERR_MISALIGNED, "out must start on a 16-byte boundary");
   if (!is_aligned(a, 16) || !is_aligned(b, 16)) return fail(HQ_ERR_MISALIGNED, "A and B must be 16-byte aligned");
   if (offsets && !is_aligned(offsets, 4)) return fail(HQ_ERR_MISALIGNED, "offsets must be 4-byte aligned");

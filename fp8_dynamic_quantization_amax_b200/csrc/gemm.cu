@@ -28,6 +28,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 namespace hq {
@@ -491,11 +492,15 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
     *msg = "cudaFuncSetAttribute failed";
     return attr_err;
   }
-  const uint64_t kdim = a.K > 0 ? static_cast<uint64_t>(a.K) : 16;  // K == 0: maps are never used
   CUtensorMap ta, tb;
-  if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), kdim, kElem, kBM, msg) ||
-      !make_map(&tb, a.b, static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N), kdim, kElem, BN, msg))
-    return cudaErrorInvalidValue;
+  memset(&ta, 0, sizeof(ta));
+  memset(&tb, 0, sizeof(tb));
+  if (a.K > 0) {  // K == 0: no loads are issued and the maps are never read
+    if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kElem, kBM, msg) ||
+        !make_map(&tb, a.b, static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K),
+                  kElem, BN, msg))
+      return cudaErrorInvalidValue;
+  }
 
   Params p;
   p.M = static_cast<int>(a.M);

@@ -224,8 +224,8 @@ __global__ void __launch_bounds__(kThreads) k_token_generic(
 }
 
 // --------------------------------------------------------------- per-tensor
-// Workspace words: [0] amax bits (accumulator, 0 between calls),
-// [1] CTA counter (0 between calls), [2] published multiplier m.
+// Workspace words: [0] amax bits, [1] CTA counter, [2] the multiplier m
+// published by phase 1 for phase 2.  All three are zero between calls.
 constexpr int kUnroll = 4;
 
 template <int DT, bool VECP>
@@ -281,8 +281,9 @@ __global__ void __launch_bounds__(kThreads) k_tensor_amax(
 // Cast with one multiplier; walks the vectors from the end backwards.
 template <int DT, int FMT, bool VECP>
 __global__ void __launch_bounds__(kThreads) k_tensor_cast(
-    const void* __restrict__ x, int64_t n, const uint32_t* __restrict__ ws, uint8_t* __restrict__ q) {
+    const void* __restrict__ x, int64_t n, uint32_t* __restrict__ ws, uint8_t* __restrict__ q) {
   constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
+  __shared__ bool is_last;
   const float m = __uint_as_float(__ldcg(&ws[2]));
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
   const int64_t gstride = static_cast<int64_t>(gridDim.x) * kThreads;
@@ -306,6 +307,14 @@ __global__ void __launch_bounds__(kThreads) k_tensor_cast(
     done = nv * VEC;
   }
   for (int64_t i = done + gtid; i < n; i += gstride) q[i] = cvt1<FMT>(__fmul_rn(Dt<DT>::load1(x, i), m));
+  // Every CTA has read m: the last one returns the workspace to zero.
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(&ws[1], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (is_last && threadIdx.x == 0) {
+    atomicExch(&ws[2], 0u);
+    atomicExch(&ws[1], 0u);
+  }
 }
 
 // -------------------------------------------------------------- per-channel
@@ -376,42 +385,54 @@ __global__ void __launch_bounds__(kThreads) k_channel_amax(
 template <int DT, int FMT, bool VECP>
 __global__ void __launch_bounds__(kThreads) k_channel_cast(
     const void* __restrict__ x, int64_t rows, int64_t cols, int64_t band_rows,
-    const float* __restrict__ ws_m, uint8_t* __restrict__ q) {
+    uint32_t* __restrict__ counter, float* __restrict__ ws_m, uint8_t* __restrict__ q) {
   constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
+  __shared__ bool is_last;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int64_t nvc = cols / VEC;
   const int64_t cv = static_cast<int64_t>(blockIdx.x) * 32 + l;
-  if (cv >= nvc) return;
-  // bands in reverse launch order: the last band read by phase 1 goes first
-  const int64_t band = static_cast<int64_t>(gridDim.y) - 1 - blockIdx.y;
-  const int64_t r0 = band * band_rows;
-  const int64_t r1 = min(rows, r0 + band_rows);
-  float m[VEC];
+  if (cv < nvc) {
+    // bands in reverse launch order: the last band read by phase 1 goes first
+    const int64_t band = static_cast<int64_t>(gridDim.y) - 1 - blockIdx.y;
+    const int64_t r0 = band * band_rows;
+    const int64_t r1 = min(rows, r0 + band_rows);
+    float m[VEC];
 #pragma unroll
-  for (int j = 0; j < VEC; ++j) m[j] = __ldcg(&ws_m[cv * VEC + j]);
-  const int64_t nrows = r1 - r0;
-  for (int64_t i = w; i < nrows; i += kThreads / 32) {
-    const int64_t r = r1 - 1 - i;
-    if (VECP) {
-      const uint4 u = ld_stream(reinterpret_cast<const uint4*>(static_cast<const char*>(x) +
-                                                               (r * cols + cv * VEC) * Dt<DT>::kSize));
-      float f[Dt<DT>::kVec];
-      Dt<DT>::unpack(u, f);
-      if constexpr (Dt<DT>::kVec == 8) {
-        uint2 o;
-        o.x = cvt2<FMT>(__fmul_rn(f[0], m[0]), __fmul_rn(f[1], m[1])) |
+    for (int j = 0; j < VEC; ++j) m[j] = __ldcg(&ws_m[cv * VEC + j]);
+    const int64_t nrows = r1 - r0;
+    for (int64_t i = w; i < nrows; i += kThreads / 32) {
+      const int64_t r = r1 - 1 - i;
+      if (VECP) {
+        const uint4 u = ld_stream(reinterpret_cast<const uint4*>(static_cast<const char*>(x) +
+                                                                 (r * cols + cv * VEC) * Dt<DT>::kSize));
+        float f[Dt<DT>::kVec];
+        Dt<DT>::unpack(u, f);
+        if constexpr (Dt<DT>::kVec == 8) {
+          uint2 o;
+          o.x = cvt2<FMT>(__fmul_rn(f[0], m[0]), __fmul_rn(f[1], m[1])) |
+                (cvt2<FMT>(__fmul_rn(f[2], m[2]), __fmul_rn(f[3], m[3])) << 16);
+          o.y = cvt2<FMT>(__fmul_rn(f[4], m[4]), __fmul_rn(f[5], m[5])) |
+                (cvt2<FMT>(__fmul_rn(f[6], m[6]), __fmul_rn(f[7], m[7])) << 16);
+          *reinterpret_cast<uint2*>(q + r * cols + cv * VEC) = o;
+        } else {
+          *reinterpret_cast<uint32_t*>(q + r * cols + cv * VEC) =
+              cvt2<FMT>(__fmul_rn(f[0], m[0]), __fmul_rn(f[1], m[1])) |
               (cvt2<FMT>(__fmul_rn(f[2], m[2]), __fmul_rn(f[3], m[3])) << 16);
-        o.y = cvt2<FMT>(__fmul_rn(f[4], m[4]), __fmul_rn(f[5], m[5])) |
-              (cvt2<FMT>(__fmul_rn(f[6], m[6]), __fmul_rn(f[7], m[7])) << 16);
-        *reinterpret_cast<uint2*>(q + r * cols + cv * VEC) = o;
+        }
       } else {
-        *reinterpret_cast<uint32_t*>(q + r * cols + cv * VEC) =
-            cvt2<FMT>(__fmul_rn(f[0], m[0]), __fmul_rn(f[1], m[1])) |
-            (cvt2<FMT>(__fmul_rn(f[2], m[2]), __fmul_rn(f[3], m[3])) << 16);
+        q[r * cols + cv] = cvt1<FMT>(__fmul_rn(Dt<DT>::load1(x, r * cols + cv), m[0]));
       }
-    } else {
-      q[r * cols + cv] = cvt1<FMT>(__fmul_rn(Dt<DT>::load1(x, r * cols + cv), m[0]));
     }
+  }
+  // Every CTA has read its multipliers: the last one zeroes them and the
+  // counter, so the whole workspace is zero again when the call ends.
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(counter, 1u) == gridDim.x * gridDim.y - 1;
+  __syncthreads();
+  if (is_last) {
+    for (int64_t c = threadIdx.x; c < cols; c += kThreads) ws_m[c] = 0.0f;
+    __syncthreads();
+    if (threadIdx.x == 0) atomicExch(counter, 0u);
   }
 }
 
@@ -603,9 +624,11 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || n == 0) return e;
   if (row_vec)
-    k_channel_cast<DT, FMT, true><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, ws_m, a.q);
+    k_channel_cast<DT, FMT, true><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, counter, ws_m,
+                                                                   a.q);
   else
-    k_channel_cast<DT, FMT, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, ws_m, a.q);
+    k_channel_cast<DT, FMT, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, counter, ws_m,
+                                                                    a.q);
   return cudaGetLastError();
 }
 

@@ -91,9 +91,9 @@ int hq_scale_pair_name(hq_granularity act, hq_granularity weight, char* buf, siz
 /* Bytes of device workspace hq_quantize_fp8 needs for this shape and mode
    (delayed != 0: the delayed per-tensor mode).  0 means no workspace.
    The caller zero-fills a workspace once before its first use; every call
-   returns its accumulator words to zero, so the same workspace can be reused
-   by calls that run one after another on the device.  Two calls that may
-   run at the same time need two workspaces. */
+   returns the whole workspace to zero, so one workspace can serve calls of
+   any shape and mode that run one after another on the device.  Two calls
+   that may run at the same time need two workspaces. */
 size_t hq_quantize_workspace_bytes(hq_granularity g, int64_t rows, int64_t cols, int delayed);
 
 /*
@@ -155,7 +155,9 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
  *
  * Arguments:
  *   xq        device, M*K FP8 codes, row-major [M, K], 16-byte aligned
+ *             (may be NULL when K == 0)
  *   wq        device, N*K FP8 codes, row-major [N, K], 16-byte aligned
+ *             (may be NULL when K == 0)
  *   x_scale   device f32, x_scale_len in {1, M}
  *   w_scale   device f32, w_scale_len in {1, N}
  *   out       device bf16 (uint16 bits), dense row-major [M, N], 16-byte

