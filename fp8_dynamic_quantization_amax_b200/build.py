@@ -1,6 +1,8 @@
 """Build libhq.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m fp8_dynamic_quantization_amax_b200.build [--force] [-v]
+    python fp8_dynamic_quantization_amax_b200/build.py [--force] [-v]
+
+(run by path: importing the package loads the library being built).
 
 Each .cu under csrc/ is compiled to an object in parallel, then linked into
 fp8_dynamic_quantization_amax_b200/libhq.so.  The CUDA runtime is linked
