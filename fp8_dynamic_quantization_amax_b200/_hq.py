@@ -22,7 +22,8 @@ F32, BF16, F16 = 0, 1, 2
 
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
             "hq_quantize_fp8", "hq_gemm_a8w8", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
-            "hq_check_device_error", "hq_last_error", "hq_version"]
+            "hq_quantize_fp8_noalloc", "hq_check_device_error", "hq_last_error", "hq_version"]
+NOALLOC_SCRATCH_BYTES = 256 * 1024
 
 
 class HQError(RuntimeError):
@@ -34,7 +35,7 @@ class HQError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libhq.so is not built (python -m fp8_dynamic_quantization_amax_b200.build); "
+        raise ImportError("libhq.so is not built (python fp8_dynamic_quantization_amax_b200/build.py); "
                           "there is no CPU fallback")
     L = ctypes.CDLL(LIB_PATH)
     P, i64, i32, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int, ctypes.c_size_t
@@ -48,6 +49,8 @@ def _load():
     L.hq_quantize_workspace_bytes.restype = sz
     L.hq_quantize_fp8.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P, sz, P]
     L.hq_quantize_fp8.restype = ci
+    L.hq_quantize_fp8_noalloc.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P]
+    L.hq_quantize_fp8_noalloc.restype = ci
     L.hq_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
     L.hq_gemm_a8w8.restype = ci
     L.hq_grouped_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, P, i32, i64, i64, i64, P, P]
@@ -144,6 +147,30 @@ def hq_quantize_fp8(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=N
                               _ptr(amax_out), _ptr(ring), ring_len, ring_idx, ring_margin,
                               _ptr(workspace), 0 if workspace is None else workspace.numel(),
                               _stream(stream)))
+    return q, scales
+
+
+def hq_quantize_fp8_noalloc(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=None, ring=None,
+                            ring_idx=0, ring_margin=0, stream=None):
+    """hq_quantize_fp8 for callers that cannot allocate device memory: the
+    library's static scratch replaces the workspace (calls must not overlap
+    on the GPU).  Returns (q, scales)."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32, bfloat16 or float16")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    rows, cols = x.shape
+    ns = hq_scale_count(gran, rows, cols)
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((max(ns, 0),), dtype=torch.float32, device=x.device)
+    ring_len = 0 if ring is None else ring.numel() - 2
+    check(lib.hq_quantize_fp8_noalloc(_ptr(x), _DT[x.dtype], rows, cols, fmt, gran, _ptr(q), _ptr(scales),
+                                      _ptr(amax_out), _ptr(ring), ring_len, ring_idx, ring_margin,
+                                      _stream(stream)))
     return q, scales
 
 

@@ -121,6 +121,16 @@ constexpr int64_t k2p40 = int64_t(1) << 40;
 }  // namespace
 
 namespace hq {
+hq_status set_error(hq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
 int device_sm_count(int dev) {
   static std::mutex mu;
   static int cache[64] = {0};

@@ -3,6 +3,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include "../../include/hq.h"
 #include <cstddef>
 #include <cstdint>
 #include <string>
@@ -55,5 +57,8 @@ enum : unsigned { kDevErrTimeout = 1u, kDevErrBadOffsets = 2u };
 cudaError_t read_and_clear_device_error(unsigned* word);
 
 int device_sm_count(int dev);
+
+// Records a printf-style message for hq_last_error() and returns s.
+hq_status set_error(hq_status s, const char* fmt, ...);
 
 }  // namespace hq

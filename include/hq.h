@@ -216,6 +216,34 @@ hq_status hq_grouped_gemm_bf16(const void* x, const void* w,
                                int64_t M_total, int64_t N, int64_t K,
                                void* out, hq_stream_t stream);
 
+/*
+ * hq_quantize_fp8 without a caller workspace, for callers that cannot
+ * allocate device memory (no cudaMalloc in their context, or no allocator of
+ * their own: they receive only input and output buffers).  No page describes
+ * this entry point; it is this library's addition.
+ *
+ * Same arguments, computation, results and errors as hq_quantize_fp8, minus
+ * `workspace` / `workspace_bytes`.  The per-tensor, per-channel and delayed
+ * modes use one static device array of HQ_NOALLOC_SCRATCH_BYTES (256 KiB)
+ * instead, which every GPU that loads the library holds until the process
+ * exits.  Per-tensor and delayed calls always fit; a per-channel call fits
+ * up to 32,764 columns; a larger one returns HQ_ERR_TOO_LARGE before any
+ * launch.  The call itself allocates nothing.
+ *
+ * The first call on a device that needs the array looks up its device
+ * address and clears it (a synchronous memset on that device); make that
+ * first call before any stream capture.  Every call leaves the array zero
+ * again.  All calls share the one array: two calls that may overlap on the
+ * GPU (different streams, or different host threads) race on it and must be
+ * serialised by the caller.
+ */
+#define HQ_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+hq_status hq_quantize_fp8_noalloc(const void* x, hq_dtype xt, int64_t rows, int64_t cols,
+                                  hq_fp8_format fmt, hq_granularity g,
+                                  uint8_t* q, float* scales, float* amax_out,
+                                  float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,
+                                  hq_stream_t stream);
+
 /* Synchronizes the current device, then reads and clears the device error
    word: HQ_OK, HQ_ERR_TIMEOUT (a bounded wait in a kernel gave up; that
    launch's outputs are undefined), HQ_ERR_INVALID_ARG (malformed grouped
