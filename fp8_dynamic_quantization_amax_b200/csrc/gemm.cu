@@ -22,6 +22,7 @@
 // Every wait is bounded: on a stalled barrier the CTA records an error in a
 // device word, drains what it has in flight and exits instead of hanging.
 #include "hq_internal.cuh"
+#include "ptx.cuh"
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -41,8 +42,7 @@ constexpr int kBM = 128;            // tile rows (MMA M)
 constexpr int kBKBytes = 128;       // K bytes per stage = one 128B swizzle row
 constexpr int kGemmThreads = 192;
 constexpr int kMaxExperts = 1024;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
-constexpr unsigned long long kDrainLimitNs = 200000000ull;  // 0.2 s
+constexpr unsigned long long kDrainLimitNs = ptx::kDrainLimitNs;
 
 struct Params {
   int M, N, K;          // M: rows of A (M_total for grouped), K in elements
@@ -60,54 +60,15 @@ struct Params {
 };
 
 // ------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ unsigned long long globaltimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
+using ptx::smem_u32;
+using ptx::mbar_init;
+using ptx::mbar_arrive_expect_tx;
+using ptx::mbar_arrive;
 
-// Wait until the phase with the given parity has completed.  Gives up after
-// `limit` ns (recording a timeout) or as soon as another role has aborted.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                       unsigned long long limit = kWaitLimitNs) {
-  const uint32_t addr = smem_u32(bar);
-  if (mbar_try_wait(addr, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(addr, parity)) return true;
-    if ((it & 31u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer() - t0 > limit) {
-        *abort_flag = 1;
-        atomicOr(&g_device_error, kDevErrTimeout);
-        return false;
-      }
-    }
-  }
+// Bounded wait; a timeout is recorded in the device error word.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit = ptx::kWaitLimitNs) {
+  return ptx::mbar_wait(bar, parity, abort_flag, &g_device_error, kDevErrTimeout, limit);
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
@@ -269,7 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(&final_bar, 1);
     abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    ptx::fence_mbarrier_init();
   }
   if (threadIdx.x == 32 && p.offsets != nullptr) {
     // Clamp the device offsets into [prev, M] and build the tile prefix.
@@ -548,6 +509,20 @@ cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
   }
   if (wide) return run<1, 256, 4>(a, msg);
   return run<1, 128, 6>(a, msg);
+}
+
+unsigned* device_error_word() {
+  static std::mutex mu;
+  static unsigned* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptrs[dev] = static_cast<unsigned*>(p);
+    else cudaGetLastError();
+  }
+  return ptrs[dev];
 }
 
 cudaError_t read_and_clear_device_error(unsigned* word) {

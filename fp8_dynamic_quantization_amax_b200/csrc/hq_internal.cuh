@@ -55,6 +55,8 @@ cudaError_t launch_gemm(const GemmArgs& a, std::string* msg);
 // Device error word (set by bounded waits and by offset validation).
 enum : unsigned { kDevErrTimeout = 1u, kDevErrBadOffsets = 2u };
 cudaError_t read_and_clear_device_error(unsigned* word);
+// Device address of that word on the current device (nullptr if unavailable).
+unsigned* device_error_word();
 
 int device_sm_count(int dev);
 

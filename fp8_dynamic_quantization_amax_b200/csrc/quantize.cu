@@ -8,10 +8,12 @@
 //   q     = satfinite round-to-nearest-even FP8 code of f32(x) * m
 //   scale = 1 / m (the dequant scale), amax_out = amax
 //
-// Kernel family (all memory bound; 16-byte vector loads, warp-shuffle
-// reductions):
-//   per-token   one pass: a warp (short rows) or a CTA (long rows) holds the
-//               row in registers, reduces its amax, then casts it.
+// Kernel family (memory bound; every kernel keeps several 16-byte loads or
+// bulk copies in flight per thread and no kernel waits on another CTA):
+//   per-token   one pass, persistent CTAs: a ring of shared-memory stages is
+//               filled by 1-D bulk copies (TMA), each stage a group of whole
+//               rows; a stage is reduced and cast while the next ones load.
+//               Unaligned or very long rows take a scalar path.
 //   per-tensor  two launches: phase 1 reduces amax with per-CTA partials and
 //               an atomicMax on the f32 bit pattern; the last CTA (threadfence
 //               + counter election) publishes m.  Phase 2 casts, walking the
@@ -19,9 +21,19 @@
 //   per-channel the same two phases on [column strip x row band] tiles.
 //   delayed     one pass with the multiplier already in the ring; the last
 //               CTA folds amax into hist[idx] and publishes the next scale.
-// No kernel here waits on another CTA: the last-CTA election only counts.
+//
+// Instruction economy (the kernels are ALU-issue bound otherwise):
+//   - amax runs on raw bit patterns: for non-negative floats the unsigned
+//     order of the bits is the numeric order, so |x| is one AND and the max
+//     is one max.u16x2 per two bf16/f16 elements (one max.u32 per f32).
+//   - Inf/NaN have the all-ones exponent, so the raw maximum also tells
+//     whether any non-finite element was seen.  Only then does a thread redo
+//     its range on the exact path (finite-only amax, canonical NaN codes).
+//   - the cast is one FMUL per element plus one cvt.rn.satfinite per pair.
 #include "hq_internal.cuh"
+#include "ptx.cuh"
 
+#include <algorithm>
 #include <cfloat>
 #include <cuda_fp16.h>
 
@@ -29,20 +41,38 @@ namespace hq {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kUnroll = 4;        // delayed kernel (casts and reduces: register bound)
+constexpr int kUnrollFlat = 8;    // per-tensor phases: eight 16-byte loads in flight per thread
+constexpr int kMaxStages = 4;
+constexpr int kRowUnroll = 8;     // per-channel: rows loaded per step
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 
 // ------------------------------------------------------------ element types
-// DT: 0 f32, 1 bf16, 2 f16.  VEC = elements per 16-byte vector.
+// DT: 0 f32, 1 bf16, 2 f16.  kVec = elements per 16-byte vector.  A "raw
+// magnitude word" is a 32-bit word of the input with the sign bits cleared;
+// lmax takes the lane-wise maximum of two such words (2 lanes for 16-bit
+// types, 1 for f32).
 template <int DT> struct Dt;
 template <> struct Dt<0> {
-  static constexpr int kSize = 4, kVec = 4;
+  static constexpr int kSize = 4, kVec = 4, kLanes = 1;
   __device__ static float load1(const void* p, int64_t i) { return __ldg(static_cast<const float*>(p) + i); }
   __device__ static void unpack(const uint4& u, float (&f)[4]) {
     f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
     f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
   }
+  __device__ static uint32_t mag(uint32_t w) { return w & 0x7FFFFFFFu; }
+  __device__ static uint32_t lmax(uint32_t a, uint32_t b) { return max(a, b); }
+  __device__ static bool nonfinite(uint32_t m) { return m >= 0x7F800000u; }
+  __device__ static float lane_value(uint32_t m, int) { return __uint_as_float(m); }
+  __device__ static float value(uint32_t m) { return __uint_as_float(m); }
 };
 template <> struct Dt<1> {
-  static constexpr int kSize = 2, kVec = 8;
+  static constexpr int kSize = 2, kVec = 8, kLanes = 2;
   __device__ static float load1(const void* p, int64_t i) {
     return __uint_as_float(static_cast<uint32_t>(__ldg(static_cast<const unsigned short*>(p) + i)) << 16);
   }
@@ -54,9 +84,17 @@ template <> struct Dt<1> {
       f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   }
+  __device__ static uint32_t mag(uint32_t w) { return w & 0x7FFF7FFFu; }
+  __device__ static uint32_t lmax(uint32_t a, uint32_t b) { return max_u16x2(a, b); }
+  // a lane >= 0x7F80 (exponent all ones) carries into its bit 15
+  __device__ static bool nonfinite(uint32_t m) { return ((m + 0x00800080u) & 0x80008000u) != 0; }
+  __device__ static float lane_value(uint32_t m, int lane) {
+    return __uint_as_float(((m >> (16 * lane)) & 0xFFFFu) << 16);
+  }
+  __device__ static float value(uint32_t m) { return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16); }
 };
 template <> struct Dt<2> {
-  static constexpr int kSize = 2, kVec = 8;
+  static constexpr int kSize = 2, kVec = 8, kLanes = 2;
   __device__ static float load1(const void* p, int64_t i) {
     return __half2float(__ushort_as_half(__ldg(static_cast<const unsigned short*>(p) + i)));
   }
@@ -68,7 +106,24 @@ template <> struct Dt<2> {
       f[2 * i + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] >> 16)));
     }
   }
+  __device__ static uint32_t mag(uint32_t w) { return w & 0x7FFF7FFFu; }
+  __device__ static uint32_t lmax(uint32_t a, uint32_t b) { return max_u16x2(a, b); }
+  // a lane >= 0x7C00 (exponent all ones) carries into its bit 15
+  __device__ static bool nonfinite(uint32_t m) { return ((m + 0x04000400u) & 0x80008000u) != 0; }
+  __device__ static float lane_value(uint32_t m, int lane) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>((m >> (16 * lane)) & 0xFFFFu)));
+  }
+  __device__ static float value(uint32_t m) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(max(m & 0xFFFFu, m >> 16))));
+  }
 };
+
+// Raw magnitude maximum of the elements of one 16-byte vector.
+template <int DT>
+__device__ __forceinline__ uint32_t vec_mag(const uint4& u) {
+  return Dt<DT>::lmax(Dt<DT>::lmax(Dt<DT>::mag(u.x), Dt<DT>::mag(u.y)),
+                      Dt<DT>::lmax(Dt<DT>::mag(u.z), Dt<DT>::mag(u.w)));
+}
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 r;
@@ -81,10 +136,29 @@ template <int FMT> struct Fmt;
 template <> struct Fmt<0> { static constexpr float kMax = kFmaxE4M3; };
 template <> struct Fmt<1> { static constexpr float kMax = kFmaxE5M2; };
 
-// Two f32 values -> two FP8 codes (lo in the low byte), saturating
-// round-to-nearest-even.  A NaN input gives the canonical code 0x7F.
+// Four f32 values -> four FP8 codes in one word (a0 in the low byte),
+// saturating round-to-nearest-even.  Inputs must not be NaN.
 template <int FMT>
-__device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
+__device__ __forceinline__ uint32_t cvt4(float a0, float a1, float a2, float a3) {
+  uint32_t d;
+  if (FMT == 0)
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\t"
+        "mov.b32 %0, {l, h};\n\t}"
+        : "=r"(d) : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  else
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "cvt.rn.satfinite.e5m2x2.f32 l, %2, %1;\n\t"
+        "cvt.rn.satfinite.e5m2x2.f32 h, %4, %3;\n\t"
+        "mov.b32 %0, {l, h};\n\t}"
+        : "=r"(d) : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return d;
+}
+
+// Exact-path conversion of two values: a NaN input gives the canonical 0x7F.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt2_exact(float lo, float hi) {
   unsigned short r;
   if (FMT == 0)
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
@@ -97,8 +171,8 @@ __device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
 }
 
 template <int FMT>
-__device__ __forceinline__ uint8_t cvt1(float y) {
-  return static_cast<uint8_t>(cvt2<FMT>(y, 0.0f) & 0xFFu);
+__device__ __forceinline__ uint8_t cvt1_exact(float y) {
+  return static_cast<uint8_t>(cvt2_exact<FMT>(y, 0.0f) & 0xFFu);
 }
 
 // |v| if finite, else 0 (NaN and +-Inf do not take part in amax).
@@ -108,7 +182,7 @@ __device__ __forceinline__ float finite_abs(float v) {
 }
 
 template <int DT>
-__device__ __forceinline__ float vec_amax(const uint4& u, float acc) {
+__device__ __forceinline__ float vec_amax_exact(const uint4& u, float acc) {
   float f[Dt<DT>::kVec];
   Dt<DT>::unpack(u, f);
 #pragma unroll
@@ -116,22 +190,42 @@ __device__ __forceinline__ float vec_amax(const uint4& u, float acc) {
   return acc;
 }
 
-// Scale the vector by m and store its codes (VEC bytes at dst).
-template <int DT, int FMT>
-__device__ __forceinline__ void vec_store_codes(uint8_t* dst, const uint4& u, float m) {
+// Four f32 codes-to-be (already scaled) -> one word, on the fast (no NaN) or
+// the exact path.
+template <int FMT, bool FAST>
+__device__ __forceinline__ uint32_t pack4(float a0, float a1, float a2, float a3) {
+  if (FAST) return cvt4<FMT>(a0, a1, a2, a3);
+  return cvt2_exact<FMT>(a0, a1) | (cvt2_exact<FMT>(a2, a3) << 16);
+}
+
+// Scale one vector by m and store its codes (kVec bytes at dst).  FAST: the
+// vector holds no NaN (checked by the caller) and m is finite.
+template <int DT, int FMT, bool FAST>
+__device__ __forceinline__ void vec_store(uint8_t* dst, const uint4& u, float m) {
   float f[Dt<DT>::kVec];
   Dt<DT>::unpack(u, f);
+#pragma unroll
+  for (int i = 0; i < Dt<DT>::kVec; ++i) f[i] = __fmul_rn(f[i], m);
   if constexpr (Dt<DT>::kVec == 8) {
-    uint2 o;
-    o.x = cvt2<FMT>(__fmul_rn(f[0], m), __fmul_rn(f[1], m)) |
-          (cvt2<FMT>(__fmul_rn(f[2], m), __fmul_rn(f[3], m)) << 16);
-    o.y = cvt2<FMT>(__fmul_rn(f[4], m), __fmul_rn(f[5], m)) |
-          (cvt2<FMT>(__fmul_rn(f[6], m), __fmul_rn(f[7], m)) << 16);
-    *reinterpret_cast<uint2*>(dst) = o;
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(pack4<FMT, FAST>(f[0], f[1], f[2], f[3]), pack4<FMT, FAST>(f[4], f[5], f[6], f[7]));
   } else {
-    *reinterpret_cast<uint32_t*>(dst) =
-        cvt2<FMT>(__fmul_rn(f[0], m), __fmul_rn(f[1], m)) |
-        (cvt2<FMT>(__fmul_rn(f[2], m), __fmul_rn(f[3], m)) << 16);
+    *reinterpret_cast<uint32_t*>(dst) = pack4<FMT, FAST>(f[0], f[1], f[2], f[3]);
+  }
+}
+
+// The same with one multiplier per element (per-channel).
+template <int DT, int FMT, bool FAST>
+__device__ __forceinline__ void vec_store_m(uint8_t* dst, const uint4& u, const float (&m)[Dt<DT>::kVec]) {
+  float f[Dt<DT>::kVec];
+  Dt<DT>::unpack(u, f);
+#pragma unroll
+  for (int i = 0; i < Dt<DT>::kVec; ++i) f[i] = __fmul_rn(f[i], m[i]);
+  if constexpr (Dt<DT>::kVec == 8) {
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(pack4<FMT, FAST>(f[0], f[1], f[2], f[3]), pack4<FMT, FAST>(f[4], f[5], f[6], f[7]));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack4<FMT, FAST>(f[0], f[1], f[2], f[3]);
   }
 }
 
@@ -141,7 +235,7 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Max over the whole CTA (kThreads threads); every thread gets the result.
+// Max over the whole CTA; every thread gets the result.
 __device__ __forceinline__ float block_max(float v, float* sh) {
   v = warp_max(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -149,8 +243,7 @@ __device__ __forceinline__ float block_max(float v, float* sh) {
   if (l == 0) sh[w] = v;
   __syncthreads();
   float r = (l < kThreads / 32) ? sh[l] : 0.0f;
-  r = warp_max(r);
-  return r;
+  return warp_max(r);
 }
 
 // m = fmax / amax, with m = 1 for amax == 0 or a non-finite quotient.
@@ -161,43 +254,142 @@ __device__ __forceinline__ float multiplier(float amax, float fmax) {
 }
 
 // ---------------------------------------------------------------- per-token
-// Vector path: TPR threads per row (32: a warp per row, 8 rows per CTA;
-// 256: a CTA per row).  Each thread holds up to MAXV 16-byte vectors.
-template <int DT, int FMT, int TPR, int MAXV>
-__global__ void __launch_bounds__(kThreads) k_token_vec(
-    const void* __restrict__ x, int64_t rows, int64_t cols, uint8_t* __restrict__ q,
-    float* __restrict__ scales, float* __restrict__ amax_out) {
+// TMA-staged path.  Persistent CTAs walk groups of R consecutive rows (one
+// bulk copy per group: the rows are contiguous); S stages are in flight.
+// Within a stage each row is owned by 8/R warps (a "team").
+constexpr int kHeld = 4;  // vectors per thread kept in registers between the passes
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kThreads, 4) k_token_tma(
+    const void* __restrict__ x, int64_t rows, int64_t cols, int R, int S, uint8_t* __restrict__ q,
+    float* __restrict__ scales, float* __restrict__ amax_out, unsigned* err) {
   constexpr int VEC = Dt<DT>::kVec;
-  constexpr int RPC = kThreads / TPR;
-  __shared__ float sh[kThreads / 32];
-  const int sub = threadIdx.x / TPR, t = threadIdx.x % TPR;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + sub;
-  const bool active = row < rows;
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ __align__(8) uint64_t full[kMaxStages];
+  __shared__ float red[kThreads / 32];
+  __shared__ int rednf[kThreads / 32];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row_bytes = cols * Dt<DT>::kSize;
+  const int64_t stage_bytes = static_cast<int64_t>(R) * row_bytes;
+  const int64_t ngroups = (rows + R - 1) / R;
+  const int wpr = (kThreads / 32) / R;  // warps per row
+  const int team = warp / wpr;
+  const int tt = threadIdx.x - team * wpr * 32;
+  const int team_threads = wpr * 32;
   const int64_t nv = cols / VEC;
-  const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const char*>(x) +
-                                                   (active ? row : 0) * cols * Dt<DT>::kSize);
-  uint4 buf[MAXV];
-  float amax = 0.0f;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) ptx::mbar_init(&full[s], 1);
+    abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  // Thread 0 tracks which stages have a copy in flight (for the abort drain).
+  uint32_t pend_mask = 0, pend_parity = 0;
+  auto issue = [&](int64_t g, int s, uint32_t parity) {
+    const int64_t r0 = g * R;
+    const int64_t nr = min(static_cast<int64_t>(R), rows - r0);
+    const uint32_t bytes = static_cast<uint32_t>(nr * row_bytes);
+    ptx::mbar_arrive_expect_tx(&full[s], bytes);
+    ptx::bulk_load(stage_mem + s * stage_bytes, static_cast<const char*>(x) + r0 * row_bytes, bytes, &full[s]);
+    pend_mask |= 1u << s;
+    pend_parity = (pend_parity & ~(1u << s)) | (parity << s);
+  };
+  if (threadIdx.x == 0)
+    for (int s = 0; s < S; ++s) {
+      const int64_t g = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
+      if (g < ngroups) issue(g, s, 0);
+    }
+
+  int64_t i = 0;
+  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x, ++i) {
+    const int s = static_cast<int>(i % S);
+    const uint32_t parity = static_cast<uint32_t>((i / S) & 1);
+    // One thread waits on the stage's barrier (spinning warps would take
+    // issue slots from the working ones); the others park at __syncthreads.
+    if (threadIdx.x == 0) {
+      if (ptx::mbar_wait(&full[s], parity, &abort_flag, err, kDevErrTimeout)) pend_mask &= ~(1u << s);
+    }
+    __syncthreads();
+    if (abort_flag) break;
+    const int64_t row = g * R + team;
+    const bool valid = row < rows;
+    const uint4* src = reinterpret_cast<const uint4*>(stage_mem + s * stage_bytes + team * row_bytes);
+    // the first kHeld vectors of this thread stay in registers for the cast
+    uint4 held[kHeld];
+    uint32_t mraw = 0;
+    if (valid) {
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int64_t v = static_cast<int64_t>(i) * TPR + t;
-    if (active && v < nv) {
-      buf[i] = ld_stream(xr + v);
-      amax = vec_amax<DT>(buf[i], amax);
+      for (int k = 0; k < kHeld; ++k) {
+        const int64_t v = tt + static_cast<int64_t>(k) * team_threads;
+        if (v < nv) {
+          held[k] = src[v];
+          mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(held[k]));
+        }
+      }
+      for (int64_t v = tt + static_cast<int64_t>(kHeld) * team_threads; v < nv; v += team_threads)
+        mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(src[v]));
+    }
+    const bool nf = Dt<DT>::nonfinite(mraw);
+    float amax;
+    if (!nf) {
+      amax = Dt<DT>::value(mraw);
+    } else {  // rare: finite-only maximum on the exact path
+      amax = 0.0f;
+      for (int64_t v = tt; v < nv; v += team_threads) amax = vec_amax_exact<DT>(src[v], amax);
+    }
+    amax = warp_max(amax);
+    bool row_nf = __any_sync(0xFFFFFFFFu, nf) != 0;
+    if (wpr > 1) {  // combine the team's warps through shared memory
+      if (lane == 0) {
+        red[warp] = amax;
+        rednf[warp] = row_nf ? 1 : 0;
+      }
+      __syncthreads();
+      amax = red[team * wpr];
+      int any = rednf[team * wpr];
+      for (int k = 1; k < wpr; ++k) {
+        amax = fmaxf(amax, red[team * wpr + k]);
+        any |= rednf[team * wpr + k];
+      }
+      row_nf = any != 0;
+    }
+    const float m = multiplier(amax, Fmt<FMT>::kMax);
+    if (valid) {
+      if (tt == 0) {
+        scales[row] = __fdiv_rn(1.0f, m);
+        if (amax_out) amax_out[row] = amax;
+      }
+      uint8_t* qr = q + row * cols;
+      if (!row_nf) {
+#pragma unroll
+        for (int k = 0; k < kHeld; ++k) {
+          const int64_t v = tt + static_cast<int64_t>(k) * team_threads;
+          if (v < nv) vec_store<DT, FMT, true>(qr + v * VEC, held[k], m);
+        }
+        for (int64_t v = tt + static_cast<int64_t>(kHeld) * team_threads; v < nv; v += team_threads)
+          vec_store<DT, FMT, true>(qr + v * VEC, src[v], m);
+      } else {
+        for (int64_t v = tt; v < nv; v += team_threads) vec_store<DT, FMT, false>(qr + v * VEC, src[v], m);
+      }
+    }
+    __syncthreads();  // stage s fully read; red[] free again
+    if (threadIdx.x == 0) {
+      const int64_t g2 = g + static_cast<int64_t>(S) * gridDim.x;
+      if (g2 < ngroups) {
+        ptx::fence_proxy_async_smem();
+        issue(g2, s, parity ^ 1u);
+      }
     }
   }
-  if (TPR == 32) amax = warp_max(amax);
-  else amax = block_max(amax, sh);
-  const float m = multiplier(amax, Fmt<FMT>::kMax);
-  if (active && t == 0) {
-    scales[row] = __fdiv_rn(1.0f, m);
-    if (amax_out) amax_out[row] = amax;
-  }
-  uint8_t* qr = q + (active ? row : 0) * cols;
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int64_t v = static_cast<int64_t>(i) * TPR + t;
-    if (active && v < nv) vec_store_codes<DT, FMT>(qr + v * VEC, buf[i], m);
+  if (abort_flag && threadIdx.x == 0) {
+    // copies still in flight must land before the CTA's shared memory goes
+    int dummy = 0;
+    for (int s = 0; s < S; ++s)
+      if (pend_mask & (1u << s))
+        ptx::mbar_wait(&full[s], (pend_parity >> s) & 1u, &dummy, nullptr, 0, ptx::kDrainLimitNs);
   }
 }
 
@@ -220,36 +412,50 @@ __global__ void __launch_bounds__(kThreads) k_token_generic(
     if (amax_out) amax_out[row] = amax;
   }
   for (int64_t c = threadIdx.x; c < cols; c += kThreads)
-    q[row * cols + c] = cvt1<FMT>(__fmul_rn(Dt<DT>::load1(x, row * cols + c), m));
+    q[row * cols + c] = cvt1_exact<FMT>(__fmul_rn(Dt<DT>::load1(x, row * cols + c), m));
 }
 
 // --------------------------------------------------------------- per-tensor
 // Workspace words: [0] amax bits, [1] CTA counter, [2] the multiplier m
-// published by phase 1 for phase 2.  All three are zero between calls.
-constexpr int kUnroll = 4;
+// published by phase 1 for phase 2, [3] "a non-finite element was seen".
+// All four are zero between calls.
 
+// This thread's share of a flat amax: vectors gtid, gtid + stride, ... then
+// the scalar tail.  *nf reports a non-finite element.
 template <int DT, bool VECP>
-__device__ __forceinline__ float flat_amax(const void* x, int64_t n) {
+__device__ __forceinline__ float flat_amax(const void* x, int64_t n, bool* nf) {
   constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
   const int64_t gstride = static_cast<int64_t>(gridDim.x) * kThreads;
   float amax = 0.0f;
   int64_t done = 0;
+  *nf = false;
   if (VECP) {
     const uint4* xv = static_cast<const uint4*>(x);
     const int64_t nv = n / VEC;
+    uint32_t mraw = 0;
     int64_t v = gtid;
-    for (; v + (kUnroll - 1) * gstride < nv; v += kUnroll * gstride) {
-      uint4 u[kUnroll];
+    for (; v + (kUnrollFlat - 1) * gstride < nv; v += kUnrollFlat * gstride) {
+      uint4 u[kUnrollFlat];
 #pragma unroll
-      for (int j = 0; j < kUnroll; ++j) u[j] = __ldg(xv + v + j * gstride);
+      for (int j = 0; j < kUnrollFlat; ++j) u[j] = __ldg(xv + v + j * gstride);
 #pragma unroll
-      for (int j = 0; j < kUnroll; ++j) amax = vec_amax<DT>(u[j], amax);
+      for (int j = 0; j < kUnrollFlat; ++j) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(u[j]));
     }
-    for (; v < nv; v += gstride) amax = vec_amax<DT>(__ldg(xv + v), amax);
+    for (; v < nv; v += gstride) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(__ldg(xv + v)));
+    if (!Dt<DT>::nonfinite(mraw)) {
+      amax = Dt<DT>::value(mraw);
+    } else {  // rare: redo this thread's vectors on the exact path
+      *nf = true;
+      for (v = gtid; v < nv; v += gstride) amax = vec_amax_exact<DT>(__ldg(xv + v), amax);
+    }
     done = nv * VEC;
   }
-  for (int64_t i = done + gtid; i < n; i += gstride) amax = fmaxf(amax, finite_abs(Dt<DT>::load1(x, i)));
+  for (int64_t i = done + gtid; i < n; i += gstride) {
+    const float f = Dt<DT>::load1(x, i);
+    if (!(fabsf(f) <= FLT_MAX)) *nf = true;
+    amax = fmaxf(amax, finite_abs(f));
+  }
   return amax;
 }
 
@@ -259,7 +465,9 @@ __global__ void __launch_bounds__(kThreads) k_tensor_amax(
     float* __restrict__ scales, float* __restrict__ amax_out) {
   __shared__ float sh[kThreads / 32];
   __shared__ bool is_last;
-  float amax = flat_amax<DT, VECP>(x, n);
+  bool nf;
+  float amax = flat_amax<DT, VECP>(x, n, &nf);
+  if (__syncthreads_or(nf) && threadIdx.x == 0) atomicOr(&ws[3], 1u);
   amax = block_max(amax, sh);
   if (threadIdx.x == 0) {
     atomicMax(&ws[0], __float_as_uint(amax));  // non-negative: bit order = value order
@@ -279,12 +487,9 @@ __global__ void __launch_bounds__(kThreads) k_tensor_amax(
 }
 
 // Cast with one multiplier; walks the vectors from the end backwards.
-template <int DT, int FMT, bool VECP>
-__global__ void __launch_bounds__(kThreads) k_tensor_cast(
-    const void* __restrict__ x, int64_t n, uint32_t* __restrict__ ws, uint8_t* __restrict__ q) {
+template <int DT, int FMT, bool VECP, bool FAST>
+__device__ __forceinline__ void flat_cast(const void* x, int64_t n, float m, uint8_t* q) {
   constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
-  __shared__ bool is_last;
-  const float m = __uint_as_float(__ldcg(&ws[2]));
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
   const int64_t gstride = static_cast<int64_t>(gridDim.x) * kThreads;
   int64_t done = 0;
@@ -292,43 +497,54 @@ __global__ void __launch_bounds__(kThreads) k_tensor_cast(
     const uint4* xv = static_cast<const uint4*>(x);
     const int64_t nv = n / VEC;
     int64_t i = gtid;
-    for (; i + (kUnroll - 1) * gstride < nv; i += kUnroll * gstride) {
-      uint4 u[kUnroll];
+    for (; i + (kUnrollFlat - 1) * gstride < nv; i += kUnrollFlat * gstride) {
+      uint4 u[kUnrollFlat];
 #pragma unroll
-      for (int j = 0; j < kUnroll; ++j) u[j] = ld_stream(xv + (nv - 1 - (i + j * gstride)));
+      for (int j = 0; j < kUnrollFlat; ++j) u[j] = ld_stream(xv + (nv - 1 - (i + j * gstride)));
 #pragma unroll
-      for (int j = 0; j < kUnroll; ++j)
-        vec_store_codes<DT, FMT>(q + (nv - 1 - (i + j * gstride)) * VEC, u[j], m);
+      for (int j = 0; j < kUnrollFlat; ++j) vec_store<DT, FMT, FAST>(q + (nv - 1 - (i + j * gstride)) * VEC, u[j], m);
     }
     for (; i < nv; i += gstride) {
       const int64_t v = nv - 1 - i;
-      vec_store_codes<DT, FMT>(q + v * VEC, ld_stream(xv + v), m);
+      vec_store<DT, FMT, FAST>(q + v * VEC, ld_stream(xv + v), m);
     }
     done = nv * VEC;
   }
-  for (int64_t i = done + gtid; i < n; i += gstride) q[i] = cvt1<FMT>(__fmul_rn(Dt<DT>::load1(x, i), m));
-  // Every CTA has read m: the last one returns the workspace to zero.
+  for (int64_t i = done + gtid; i < n; i += gstride) q[i] = cvt1_exact<FMT>(__fmul_rn(Dt<DT>::load1(x, i), m));
+}
+
+template <int DT, int FMT, bool VECP>
+__global__ void __launch_bounds__(kThreads) k_tensor_cast(
+    const void* __restrict__ x, int64_t n, uint32_t* __restrict__ ws, uint8_t* __restrict__ q) {
+  __shared__ bool is_last;
+  const float m = __uint_as_float(__ldcg(&ws[2]));
+  const bool any_nf = __ldcg(&ws[3]) != 0u;
+  if (!any_nf) flat_cast<DT, FMT, VECP, true>(x, n, m, q);
+  else flat_cast<DT, FMT, VECP, false>(x, n, m, q);
+  // Every CTA has read m and the flag: the last one returns them to zero.
   __syncthreads();
   if (threadIdx.x == 0) is_last = atomicAdd(&ws[1], 1u) == gridDim.x - 1;
   __syncthreads();
   if (is_last && threadIdx.x == 0) {
     atomicExch(&ws[2], 0u);
+    atomicExch(&ws[3], 0u);
     atomicExch(&ws[1], 0u);
   }
 }
 
 // -------------------------------------------------------------- per-channel
 // Tile: a strip of 32 column vectors (32*VEC columns) x a band of rows.  Warp
-// w of the CTA takes rows w, w+8, ... of the band; lane l owns column vector
-// strip*32 + l.  Workspace: [0] counter, then amax bits[cols] (aligned to
-// 16 bytes), then m[cols].
+// w of the CTA takes rows w, w+8, ... of the band, eight rows per step; lane
+// l owns column vector strip*32 + l.  Workspace: [0] counter, [1] the
+// non-finite flag, then amax bits[cols] (from word 4), then m[cols].
 template <int DT, bool VECP>
 __global__ void __launch_bounds__(kThreads) k_channel_amax(
     const void* __restrict__ x, int64_t rows, int64_t cols, int64_t band_rows,
-    uint32_t* __restrict__ counter, uint32_t* __restrict__ ws_amax, float* __restrict__ ws_m,
+    uint32_t* __restrict__ header, uint32_t* __restrict__ ws_amax, float* __restrict__ ws_m,
     float fmax, float* __restrict__ scales, float* __restrict__ amax_out) {
   constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
-  __shared__ float sh[kThreads / 32][32 * VEC];
+  constexpr int W = kThreads / 32;
+  __shared__ float sh[W][32 * VEC];
   __shared__ bool is_last;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   const int64_t nvc = cols / VEC;
@@ -338,21 +554,56 @@ __global__ void __launch_bounds__(kThreads) k_channel_amax(
   float am[VEC];
 #pragma unroll
   for (int j = 0; j < VEC; ++j) am[j] = 0.0f;
+  bool nf = false;
   if (cv < nvc) {
-    if (VECP) {
-      for (int64_t r = r0 + w; r < r1; r += kThreads / 32) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const char*>(x) +
-                                                             (r * cols + cv * VEC) * Dt<DT>::kSize));
-        float f[Dt<DT>::kVec];
-        Dt<DT>::unpack(u, f);
+    if constexpr (VECP) {
+      const char* base = static_cast<const char*>(x) + cv * VEC * Dt<DT>::kSize;
+      const int64_t rstride = cols * Dt<DT>::kSize;
+      uint32_t acc[4] = {0, 0, 0, 0};  // lane-wise raw maxima of the thread's columns
+      int64_t r = r0 + w;
+      for (; r + (kRowUnroll - 1) * W < r1; r += kRowUnroll * W) {
+        uint4 u[kRowUnroll];
 #pragma unroll
-        for (int j = 0; j < VEC; ++j) am[j] = fmaxf(am[j], finite_abs(f[j]));
+        for (int j = 0; j < kRowUnroll; ++j)
+          u[j] = __ldg(reinterpret_cast<const uint4*>(base + (r + j * W) * rstride));
+#pragma unroll
+        for (int j = 0; j < kRowUnroll; ++j) {
+          acc[0] = Dt<DT>::lmax(acc[0], Dt<DT>::mag(u[j].x));
+          acc[1] = Dt<DT>::lmax(acc[1], Dt<DT>::mag(u[j].y));
+          acc[2] = Dt<DT>::lmax(acc[2], Dt<DT>::mag(u[j].z));
+          acc[3] = Dt<DT>::lmax(acc[3], Dt<DT>::mag(u[j].w));
+        }
+      }
+      for (; r < r1; r += W) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + r * rstride));
+        acc[0] = Dt<DT>::lmax(acc[0], Dt<DT>::mag(u.x));
+        acc[1] = Dt<DT>::lmax(acc[1], Dt<DT>::mag(u.y));
+        acc[2] = Dt<DT>::lmax(acc[2], Dt<DT>::mag(u.z));
+        acc[3] = Dt<DT>::lmax(acc[3], Dt<DT>::mag(u.w));
+      }
+      nf = Dt<DT>::nonfinite(Dt<DT>::lmax(Dt<DT>::lmax(acc[0], acc[1]), Dt<DT>::lmax(acc[2], acc[3])));
+      if (!nf) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int ln = 0; ln < Dt<DT>::kLanes; ++ln) am[k * Dt<DT>::kLanes + ln] = Dt<DT>::lane_value(acc[k], ln);
+      } else {  // rare: exact finite-only maxima
+        for (r = r0 + w; r < r1; r += W) {
+          float f[Dt<DT>::kVec];
+          Dt<DT>::unpack(__ldg(reinterpret_cast<const uint4*>(base + r * rstride)), f);
+#pragma unroll
+          for (int j = 0; j < VEC; ++j) am[j] = fmaxf(am[j], finite_abs(f[j]));
+        }
       }
     } else {
-      for (int64_t r = r0 + w; r < r1; r += kThreads / 32)
-        am[0] = fmaxf(am[0], finite_abs(Dt<DT>::load1(x, r * cols + cv)));
+      for (int64_t r = r0 + w; r < r1; r += W) {
+        const float f = Dt<DT>::load1(x, r * cols + cv);
+        if (!(fabsf(f) <= FLT_MAX)) nf = true;
+        am[0] = fmaxf(am[0], finite_abs(f));
+      }
     }
   }
+  if (__syncthreads_or(nf) && threadIdx.x == 0) atomicOr(&header[1], 1u);
 #pragma unroll
   for (int j = 0; j < VEC; ++j) sh[w][l * VEC + j] = am[j];
   __syncthreads();
@@ -361,13 +612,13 @@ __global__ void __launch_bounds__(kThreads) k_channel_amax(
     if (col < cols) {
       float a = sh[0][c];
 #pragma unroll
-      for (int ww = 1; ww < kThreads / 32; ++ww) a = fmaxf(a, sh[ww][c]);
+      for (int ww = 1; ww < W; ++ww) a = fmaxf(a, sh[ww][c]);
       atomicMax(&ws_amax[col], __float_as_uint(a));
     }
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) is_last = atomicAdd(counter, 1u) == gridDim.x * gridDim.y - 1;
+  if (threadIdx.x == 0) is_last = atomicAdd(&header[0], 1u) == gridDim.x * gridDim.y - 1;
   __syncthreads();
   if (is_last) {
     __threadfence();
@@ -378,66 +629,85 @@ __global__ void __launch_bounds__(kThreads) k_channel_amax(
       scales[c] = __fdiv_rn(1.0f, m);
       if (amax_out) amax_out[c] = a;
     }
-    if (threadIdx.x == 0) atomicExch(counter, 0u);
+    if (threadIdx.x == 0) atomicExch(&header[0], 0u);
+  }
+}
+
+template <int DT, int FMT, bool VECP, bool FAST>
+__device__ __forceinline__ void channel_cast_band(const void* x, int64_t cols, int64_t r0, int64_t r1,
+                                                  int64_t cv, const float* ws_m, uint8_t* q) {
+  constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
+  constexpr int W = kThreads / 32;
+  const int w = threadIdx.x >> 5;
+  const int64_t nrows = r1 - r0;
+  if constexpr (VECP) {
+    float m[Dt<DT>::kVec];
+#pragma unroll
+    for (int j = 0; j < Dt<DT>::kVec; ++j) m[j] = __ldcg(&ws_m[cv * VEC + j]);
+    const char* base = static_cast<const char*>(x) + cv * VEC * Dt<DT>::kSize;
+    const int64_t rstride = cols * Dt<DT>::kSize;
+    int64_t i = w;
+    for (; i + (kRowUnroll - 1) * W < nrows; i += kRowUnroll * W) {  // rows from the band's end backwards
+      uint4 u[kRowUnroll];
+#pragma unroll
+      for (int j = 0; j < kRowUnroll; ++j)
+        u[j] = ld_stream(reinterpret_cast<const uint4*>(base + (r1 - 1 - i - j * W) * rstride));
+#pragma unroll
+      for (int j = 0; j < kRowUnroll; ++j)
+        vec_store_m<DT, FMT, FAST>(q + (r1 - 1 - i - j * W) * cols + cv * VEC, u[j], m);
+    }
+    for (; i < nrows; i += W) {
+      const int64_t r = r1 - 1 - i;
+      vec_store_m<DT, FMT, FAST>(q + r * cols + cv * VEC,
+                                 ld_stream(reinterpret_cast<const uint4*>(base + r * rstride)), m);
+    }
+  } else {
+    const float m0 = __ldcg(&ws_m[cv]);
+    for (int64_t i = w; i < nrows; i += W) {
+      const int64_t r = r1 - 1 - i;
+      q[r * cols + cv] = cvt1_exact<FMT>(__fmul_rn(Dt<DT>::load1(x, r * cols + cv), m0));
+    }
   }
 }
 
 template <int DT, int FMT, bool VECP>
 __global__ void __launch_bounds__(kThreads) k_channel_cast(
     const void* __restrict__ x, int64_t rows, int64_t cols, int64_t band_rows,
-    uint32_t* __restrict__ counter, float* __restrict__ ws_m, uint8_t* __restrict__ q) {
+    uint32_t* __restrict__ header, float* __restrict__ ws_m, uint8_t* __restrict__ q) {
   constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
   __shared__ bool is_last;
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int l = threadIdx.x & 31;
   const int64_t nvc = cols / VEC;
   const int64_t cv = static_cast<int64_t>(blockIdx.x) * 32 + l;
+  const bool any_nf = __ldcg(&header[1]) != 0u;
   if (cv < nvc) {
     // bands in reverse launch order: the last band read by phase 1 goes first
     const int64_t band = static_cast<int64_t>(gridDim.y) - 1 - blockIdx.y;
     const int64_t r0 = band * band_rows;
     const int64_t r1 = min(rows, r0 + band_rows);
-    float m[VEC];
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) m[j] = __ldcg(&ws_m[cv * VEC + j]);
-    const int64_t nrows = r1 - r0;
-    for (int64_t i = w; i < nrows; i += kThreads / 32) {
-      const int64_t r = r1 - 1 - i;
-      if (VECP) {
-        const uint4 u = ld_stream(reinterpret_cast<const uint4*>(static_cast<const char*>(x) +
-                                                                 (r * cols + cv * VEC) * Dt<DT>::kSize));
-        float f[Dt<DT>::kVec];
-        Dt<DT>::unpack(u, f);
-        if constexpr (Dt<DT>::kVec == 8) {
-          uint2 o;
-          o.x = cvt2<FMT>(__fmul_rn(f[0], m[0]), __fmul_rn(f[1], m[1])) |
-                (cvt2<FMT>(__fmul_rn(f[2], m[2]), __fmul_rn(f[3], m[3])) << 16);
-          o.y = cvt2<FMT>(__fmul_rn(f[4], m[4]), __fmul_rn(f[5], m[5])) |
-                (cvt2<FMT>(__fmul_rn(f[6], m[6]), __fmul_rn(f[7], m[7])) << 16);
-          *reinterpret_cast<uint2*>(q + r * cols + cv * VEC) = o;
-        } else {
-          *reinterpret_cast<uint32_t*>(q + r * cols + cv * VEC) =
-              cvt2<FMT>(__fmul_rn(f[0], m[0]), __fmul_rn(f[1], m[1])) |
-              (cvt2<FMT>(__fmul_rn(f[2], m[2]), __fmul_rn(f[3], m[3])) << 16);
-        }
-      } else {
-        q[r * cols + cv] = cvt1<FMT>(__fmul_rn(Dt<DT>::load1(x, r * cols + cv), m[0]));
-      }
-    }
+    if (!any_nf) channel_cast_band<DT, FMT, VECP, true>(x, cols, r0, r1, cv, ws_m, q);
+    else channel_cast_band<DT, FMT, VECP, false>(x, cols, r0, r1, cv, ws_m, q);
   }
-  // Every CTA has read its multipliers: the last one zeroes them and the
-  // counter, so the whole workspace is zero again when the call ends.
+  // Every CTA has read its multipliers: the last one zeroes them, the flag
+  // and the counter, so the whole workspace is zero again when the call ends.
   __syncthreads();
-  if (threadIdx.x == 0) is_last = atomicAdd(counter, 1u) == gridDim.x * gridDim.y - 1;
+  if (threadIdx.x == 0) is_last = atomicAdd(&header[0], 1u) == gridDim.x * gridDim.y - 1;
   __syncthreads();
   if (is_last) {
     for (int64_t c = threadIdx.x; c < cols; c += kThreads) ws_m[c] = 0.0f;
     __syncthreads();
-    if (threadIdx.x == 0) atomicExch(counter, 0u);
+    if (threadIdx.x == 0) {
+      atomicExch(&header[1], 0u);
+      atomicExch(&header[0], 0u);
+    }
   }
 }
 
 // ------------------------------------------------------------------ delayed
 // Ring: [hist[len] | scale | counter].  Workspace word [0]: amax accumulator.
+// One pass: cast with the ring's multiplier while reducing amax.  A thread
+// whose raw maximum shows a non-finite element redoes its vectors on the
+// exact path (finite-only amax, canonical NaN codes).
 template <int DT, int FMT, bool VECP>
 __global__ void __launch_bounds__(kThreads) k_delayed(
     const void* __restrict__ x, int64_t n, uint8_t* __restrict__ q, float* __restrict__ ring,
@@ -447,6 +717,7 @@ __global__ void __launch_bounds__(kThreads) k_delayed(
   __shared__ float sh[kThreads / 32];
   __shared__ bool is_last;
   const float m = __ldcg(&ring[len]);
+  const bool m_finite = fabsf(m) <= FLT_MAX;
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
   const int64_t gstride = static_cast<int64_t>(gridDim.x) * kThreads;
   float amax = 0.0f;
@@ -454,28 +725,40 @@ __global__ void __launch_bounds__(kThreads) k_delayed(
   if (VECP) {
     const uint4* xv = static_cast<const uint4*>(x);
     const int64_t nv = n / VEC;
-    int64_t v = gtid;
-    for (; v + (kUnroll - 1) * gstride < nv; v += kUnroll * gstride) {
-      uint4 u[kUnroll];
+    uint32_t mraw = 0;
+    if (m_finite) {
+      int64_t v = gtid;
+      for (; v + (kUnroll - 1) * gstride < nv; v += kUnroll * gstride) {
+        uint4 u[kUnroll];
 #pragma unroll
-      for (int j = 0; j < kUnroll; ++j) u[j] = ld_stream(xv + v + j * gstride);
+        for (int j = 0; j < kUnroll; ++j) u[j] = ld_stream(xv + v + j * gstride);
 #pragma unroll
-      for (int j = 0; j < kUnroll; ++j) {
-        amax = vec_amax<DT>(u[j], amax);
-        vec_store_codes<DT, FMT>(q + (v + j * gstride) * VEC, u[j], m);
+        for (int j = 0; j < kUnroll; ++j) {
+          mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(u[j]));
+          vec_store<DT, FMT, true>(q + (v + j * gstride) * VEC, u[j], m);
+        }
+      }
+      for (; v < nv; v += gstride) {
+        const uint4 u = ld_stream(xv + v);
+        mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(u));
+        vec_store<DT, FMT, true>(q + v * VEC, u, m);
       }
     }
-    for (; v < nv; v += gstride) {
-      const uint4 u = ld_stream(xv + v);
-      amax = vec_amax<DT>(u, amax);
-      vec_store_codes<DT, FMT>(q + v * VEC, u, m);
+    if (m_finite && !Dt<DT>::nonfinite(mraw)) {
+      amax = Dt<DT>::value(mraw);
+    } else {  // rare: redo this thread's vectors on the exact path
+      for (int64_t v = gtid; v < nv; v += gstride) {
+        const uint4 u = __ldg(xv + v);
+        amax = vec_amax_exact<DT>(u, amax);
+        vec_store<DT, FMT, false>(q + v * VEC, u, m);
+      }
     }
     done = nv * VEC;
   }
   for (int64_t i = done + gtid; i < n; i += gstride) {
     const float f = Dt<DT>::load1(x, i);
     amax = fmaxf(amax, finite_abs(f));
-    q[i] = cvt1<FMT>(__fmul_rn(f, m));
+    q[i] = cvt1_exact<FMT>(__fmul_rn(f, m));
   }
   amax = block_max(amax, sh);
   uint32_t* counter = reinterpret_cast<uint32_t*>(ring + len + 1);
@@ -513,40 +796,13 @@ __global__ void __launch_bounds__(kThreads) k_delayed(
 // ------------------------------------------------------------------- launch
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-inline int flat_grid(int64_t nvec, int dev) {
-  const int64_t per_cta = static_cast<int64_t>(kThreads) * kUnroll;
+inline int flat_grid(int64_t nvec, int dev, int unroll) {
+  const int64_t per_cta = static_cast<int64_t>(kThreads) * unroll;
   int64_t g = (nvec + per_cta - 1) / per_cta;
   const int64_t cap = static_cast<int64_t>(device_sm_count(dev)) * 8;
   if (g > cap) g = cap;
   if (g < 1) g = 1;
   return static_cast<int>(g);
-}
-
-template <int DT, int FMT, int TPR>
-cudaError_t launch_token_vec(const QuantizeArgs& a, int maxv) {
-  const int rpc = kThreads / TPR;
-  const dim3 grid(static_cast<unsigned>((a.rows + rpc - 1) / rpc));
-  switch (maxv) {
-#define HQ_TOKEN_CASE(MV)                                                                   \
-  case MV:                                                                                 \
-    k_token_vec<DT, FMT, TPR, MV><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.q, \
-                                                                  a.scales, a.amax_out);   \
-    break;
-    HQ_TOKEN_CASE(1)
-    HQ_TOKEN_CASE(2)
-    HQ_TOKEN_CASE(4)
-    HQ_TOKEN_CASE(8)
-    HQ_TOKEN_CASE(16)
-#undef HQ_TOKEN_CASE
-    default: return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
-}
-
-inline int pow2_at_least(int64_t v) {
-  int p = 1;
-  while (p < v) p <<= 1;
-  return p;
 }
 
 template <int DT, int FMT>
@@ -561,7 +817,7 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
 
   if (a.ring) {  // delayed per-tensor
     uint32_t* ws = static_cast<uint32_t*>(a.ws);
-    const int grid = flat_grid(flat_vec ? n / VEC : n, dev);
+    const int grid = flat_grid(flat_vec ? n / VEC : n, dev, kUnroll);
     if (flat_vec)
       k_delayed<DT, FMT, true><<<grid, kThreads, 0, a.stream>>>(a.x, n, a.q, a.ring, a.ring_len, a.ring_idx,
                                                                 a.ring_margin, ws, a.scales, a.amax_out);
@@ -572,11 +828,29 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
   }
 
   if (a.gran == 1) {  // per-token
-    if (row_vec) {
-      const int64_t nv = a.cols / VEC;
-      if (nv <= 32 * 8) return launch_token_vec<DT, FMT, 32>(a, pow2_at_least((nv + 31) / 32));
-      if (nv <= static_cast<int64_t>(kThreads) * 16)
-        return launch_token_vec<DT, FMT, kThreads>(a, pow2_at_least((nv + kThreads - 1) / kThreads));
+    if (row_vec && a.cols > 0) {
+      // Stages of at least 32 KB (whole rows), two per CTA, as many CTAs per
+      // SM as shared memory and registers allow (a sweep over stage size,
+      // depth and CTAs per SM on the workload shapes picked this rule).
+      const int64_t row_bytes = a.cols * Dt<DT>::kSize;
+      int R = 1;
+      while (R < 8 && R * row_bytes < 32768) R *= 2;
+      const int64_t stage_bytes = R * row_bytes;
+      const int S = 2;
+      if (S * stage_bytes <= 220 * 1024) {
+        const int smem = static_cast<int>(S * stage_bytes);
+        static cudaError_t attr = cudaFuncSetAttribute(k_token_tma<DT, FMT>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+        if (attr != cudaSuccess) return attr;
+        const int64_t ngroups = (a.rows + R - 1) / R;
+        int per_sm = static_cast<int>(std::min<int64_t>(4, (227 * 1024) / (smem + 1024)));
+        if (per_sm < 1) per_sm = 1;
+        int64_t grid = static_cast<int64_t>(device_sm_count(dev)) * per_sm;
+        if (grid > ngroups) grid = ngroups;
+        k_token_tma<DT, FMT><<<static_cast<unsigned>(grid), kThreads, smem, a.stream>>>(
+            a.x, a.rows, a.cols, R, S, a.q, a.scales, a.amax_out, device_error_word());
+        return cudaGetLastError();
+      }
     }
     k_token_generic<DT, FMT><<<static_cast<unsigned>(a.rows), kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.q,
                                                                                         a.scales, a.amax_out);
@@ -585,13 +859,15 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
 
   if (a.gran == 0) {  // per-tensor, two phases
     uint32_t* ws = static_cast<uint32_t*>(a.ws);
-    const int grid = flat_grid(flat_vec ? n / VEC : n, dev);
+    const int grid = flat_grid(flat_vec ? n / VEC : n, dev, kUnrollFlat);
     if (flat_vec)
       k_tensor_amax<DT, true><<<grid, kThreads, 0, a.stream>>>(a.x, n, ws, fmax, a.scales, a.amax_out);
     else
       k_tensor_amax<DT, false><<<grid, kThreads, 0, a.stream>>>(a.x, n, ws, fmax, a.scales, a.amax_out);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || n == 0) return e;
+    if (e != cudaSuccess) return e;
+    if (n == 0)  // nothing to cast: clear the published multiplier and flag
+      return cudaMemsetAsync(ws + 2, 0, 2 * sizeof(uint32_t), a.stream);
     if (flat_vec)
       k_tensor_cast<DT, FMT, true><<<grid, kThreads, 0, a.stream>>>(a.x, n, ws, a.q);
     else
@@ -603,7 +879,7 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
   const int vec = row_vec ? VEC : 1;
   const int64_t nvc = a.cols / vec;
   const int64_t strips = (nvc + 31) / 32;
-  const int64_t target = static_cast<int64_t>(device_sm_count(dev)) * 4;
+  const int64_t target = static_cast<int64_t>(device_sm_count(dev)) * 8;
   int64_t bands = (target + strips - 1) / strips;
   if (bands > a.rows) bands = a.rows;
   if (bands < 1) bands = 1;
@@ -612,22 +888,27 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
   bands = a.rows > 0 ? (a.rows + band_rows - 1) / band_rows : 1;
   if (strips > 0x7FFFFFFF) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(bands));
-  uint32_t* counter = static_cast<uint32_t*>(a.ws);
-  uint32_t* ws_amax = counter + 4;
+  uint32_t* header = static_cast<uint32_t*>(a.ws);
+  uint32_t* ws_amax = header + 4;
   float* ws_m = reinterpret_cast<float*>(ws_amax + ((a.cols + 3) / 4) * 4);
   if (row_vec)
-    k_channel_amax<DT, true><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, counter, ws_amax,
+    k_channel_amax<DT, true><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, header, ws_amax,
                                                               ws_m, fmax, a.scales, a.amax_out);
   else
-    k_channel_amax<DT, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, counter, ws_amax,
+    k_channel_amax<DT, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, header, ws_amax,
                                                                ws_m, fmax, a.scales, a.amax_out);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || n == 0) return e;
+  if (e != cudaSuccess) return e;
+  if (n == 0) {  // nothing to cast: clear the published multipliers and flag
+    e = cudaMemsetAsync(header + 1, 0, sizeof(uint32_t), a.stream);
+    if (e != cudaSuccess) return e;
+    return cudaMemsetAsync(ws_m, 0, static_cast<size_t>(a.cols) * sizeof(float), a.stream);
+  }
   if (row_vec)
-    k_channel_cast<DT, FMT, true><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, counter, ws_m,
+    k_channel_cast<DT, FMT, true><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, header, ws_m,
                                                                    a.q);
   else
-    k_channel_cast<DT, FMT, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, counter, ws_m,
+    k_channel_cast<DT, FMT, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, header, ws_m,
                                                                     a.q);
   return cudaGetLastError();
 }
@@ -639,7 +920,7 @@ size_t quantize_workspace_bytes(int gran, int64_t rows, int64_t cols, int delaye
   if (delayed) return 256;
   if (gran == 0) return 256;
   if (gran == 1) return 0;
-  // counter (16 bytes), amax bits[cols] padded to 16 bytes, m[cols]
+  // header (16 bytes), amax bits[cols] padded to 16 bytes, m[cols]
   const size_t c4 = static_cast<size_t>((cols + 3) / 4) * 4;
   size_t b = 16 + c4 * 4 + static_cast<size_t>(cols) * 4;
   return (b + 255) / 256 * 256;
