@@ -440,6 +440,29 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, 
   return true;
 }
 
+// bf16 out[M, N] for TMA stores: 32 x 32 boxes, no swizzle.
+bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, std::string* msg) {
+  auto encode = get_encode_fn();
+  if (!encode) {
+    *msg = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[128];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (%d) for the output", static_cast<int>(r));
+    *msg = buf;
+    return false;
+  }
+  return true;
+}
+
 template <int KIND, int BN, int STAGES>
 cudaError_t run(const GemmArgs& a, std::string* msg) {
   constexpr int kElem = (KIND == 0) ? 1 : 2;
@@ -498,11 +521,378 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
   return cudaGetLastError();
 }
 
+// ====================================================== 2-CTA pair kernel
+// Dense GEMM on CTA pairs (a cluster of 2, tcgen05 cta_group::2): the pair
+// computes a 256 x BN tile.  CTA rank r loads A rows [m0 + 128 r, +128) and
+// B rows [n0 + BN/2 r, +BN/2) into its own shared memory; the leader (rank 0)
+// issues one M=256 MMA that reads both CTAs' stages, and each CTA's TMEM
+// holds its own 128 accumulator rows.  Per SM this halves the B bytes per
+// MMA cycle of the 1-CTA 128 x BN tile, which lets six stages fit.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(addr), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA tile load into this CTA's shared memory, completing on an mbarrier that
+// may live in the peer CTA of the pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int c0,
+                                                 int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
+      : "memory");
+}
+// Commit this thread's MMAs to the same barrier offset in both CTAs.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// TMA tile store shared -> global (clipped at the tensor's bounds), and its
+// bulk-group bookkeeping.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one committed group may still be reading shared memory
+__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+template <int KIND>
+__device__ __forceinline__ void mma_issue_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  if constexpr (KIND == 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+  }
+}
+
+template <int KIND, int BN, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    k_gemm2(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+            const __grid_constant__ CUtensorMap tm_out, const Params p) {
+  constexpr int kABytes = 128 * kBKBytes;        // this CTA's 128 rows of A
+  constexpr int kBBytes = (BN / 2) * kBKBytes;   // this CTA's BN/2 rows of B
+  constexpr int kStageBytes = kABytes + kBBytes;
+  constexpr int kKElems = (KIND == 0) ? 128 : 64;
+  constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t final_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kABytes;
+  // epilogue: per warp two 32 x 32 bf16 staging tiles (2 KB each) for TMA
+  // stores, and the tile's BN column scales
+  uint8_t* sOut = smem + STAGES * kStageBytes;
+  float* sWs = reinterpret_cast<float*>(sOut + 4 * 2 * 2048);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);   // leader: its producer's arrive + both CTAs' bytes
+      mbar_init(&empty_bar[s], 1);  // one multicast commit per use
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 8);  // leader: 4 epilogue warps x 2 CTAs
+    }
+    mbar_init(&final_bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_b) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_out) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or copy
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+  const int total = p.m_tiles * p.n_tiles;  // tiles of 256 x BN
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t pend_mask = 0, pend_parity = 0;
+      bool stop = false;
+      for (int t = cluster; t < total && !stop; t += nclusters) {
+        const int per_group = p.group_m * p.n_tiles;
+        const int g = t / per_group;
+        const int within = t - g * per_group;
+        const int gm = min(p.group_m, p.m_tiles - g * p.group_m);
+        const int mt = g * p.group_m + within % gm;
+        const int nt = within / gm;
+        const int a_row = mt * 256 + static_cast<int>(rank) * 128;
+        const int b_row = nt * BN + static_cast<int>(rank) * (BN / 2);
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { stop = true; break; }
+          const uint32_t full_leader = mapa_shared(smem_u32(&full_bar[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
+          tma_load_2d_pair(sA + stage * kABytes, &tm_a, full_leader, kb * kKElems, a_row);
+          tma_load_2d_pair(sB + stage * kBBytes, &tm_b, full_leader, kb * kKElems, b_row);
+          pend_mask |= 1u << stage;
+          pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (abort_flag && leader) {
+        // the leader's full barriers also count the peer's bytes: drain them
+        int dummy = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if (pend_mask & (1u << s)) mbar_wait(&full_bar[s], (pend_parity >> s) & 1u, &dummy, kDrainLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    if (leader) {
+      // ------------------------------------------------------- MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued = false;
+      bool stop = false;
+      int i = 0;
+      for (int t = cluster; t < total && !stop; t += nclusters, ++i) {
+        const int acc = i & 1;
+        const uint32_t acc_phase = (i >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { stop = true; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint64_t ad = smem_desc(smem_u32(sA + stage * kABytes));
+            const uint64_t bd = smem_desc(smem_u32(sB + stage * kBBytes));
+#pragma unroll
+            for (int k = 0; k < kBKBytes / 32; ++k)
+              mma_issue_pair<KIND>(d_tmem, ad + 2u * k, bd + 2u * k, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            tc_commit_pair(&empty_bar[stage]);
+            issued = true;
+          }
+          __syncwarp();
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (stop) break;
+        if (lane == 0) tc_commit_pair(&tfull_bar[acc]);
+        __syncwarp();
+      }
+      if (abort_flag && lane == 0 && issued) {
+        int dummy = 0;
+        tc_commit(&final_bar);
+        mbar_wait(&final_bar, 0, &dummy, kDrainLimitNs);
+      }
+      __syncwarp();
+    }
+  } else {
+    // -------------------------------------------------------- epilogue
+    // Warp e (quadrant `quad` of TMEM) owns 32 rows of this CTA's half of
+    // the tile.  Per 32-column chunk it scales, rounds to bf16, writes the
+    // 32 x 32 chunk to a staging tile and stores it with one TMA store
+    // (clipped at M and N); two staging tiles alternate.
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    uint8_t* stage_out = sOut + ew * 2 * 2048;
+    float* wsh = sWs + ew * BN;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
+    int i = 0;
+    uint32_t chunk = 0;
+    for (int t = cluster; t < total; t += nclusters, ++i) {
+      const int acc = i & 1;
+      const uint32_t acc_phase = (i >> 1) & 1;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag)) break;
+      tc_fence_after();
+      const int per_group = p.group_m * p.n_tiles;
+      const int g = t / per_group;
+      const int within = t - g * per_group;
+      const int gm = min(p.group_m, p.m_tiles - g * p.group_m);
+      const int mt = g * p.group_m + within % gm;
+      const int nt = within / gm;
+      const int row0 = mt * 256 + static_cast<int>(rank) * 128 + quad * 32;  // this warp's first row
+      const int row = row0 + lane;
+      const int col0 = nt * BN;
+      float xsv = 0.0f;
+      if (row < p.M) xsv = (KIND == 0) ? __ldg(p.xs + (p.xs_bcast ? 0 : row)) : 1.0f;
+      if (KIND == 0) {
+        for (int j = lane; j < BN; j += 32) {
+          const int n = col0 + j;
+          wsh[j] = (n < p.N) ? __ldg(p.ws + (p.ws_bcast ? 0 : n)) : 0.0f;
+        }
+      } else {
+        for (int j = lane; j < BN; j += 32) wsh[j] = 1.0f;
+      }
+      __syncwarp();
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32, ++chunk) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN + c), v);
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float4 s2 = make_float4(wsh[c + 2 * j], wsh[c + 2 * j + 1], 0.0f, 0.0f);
+          const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * j]) : 0.0f;
+          const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+          w[j] = pack_bf16x2(a0 * (xsv * s2.x), a1 * (xsv * s2.y));
+        }
+        uint8_t* sb = stage_out + (chunk & 1u) * 2048;
+        if (lane == 0) bulk_wait_read_le1();  // the store issued from sb two chunks ago has read it
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) st_shared_v4(sb + lane * 64 + k * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (row0 < p.M && col0 + c < p.N) tma_store_2d(&tm_out, sb, col0 + c, row0);
+          bulk_commit_group();  // possibly empty: keeps one group per chunk
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+    if (lane == 0) bulk_wait_all();  // stores complete before the CTA's shared memory goes
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+template <int KIND, int BN, int STAGES>
+cudaError_t run2(const GemmArgs& a, std::string* msg) {
+  constexpr int kElem = (KIND == 0) ? 1 : 2;
+  constexpr int kSmem = STAGES * (128 + BN / 2) * kBKBytes + 4 * 2 * 2048 + 4 * BN * 4 + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int max_clusters = 0;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(k_gemm2<KIND, BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(148, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, k_gemm2<KIND, BN, STAGES>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      max_clusters = 0;
+    }
+  });
+  if (attr_err != cudaSuccess) {
+    *msg = "cudaFuncSetAttribute failed";
+    return attr_err;
+  }
+  CUtensorMap ta, tb;
+  memset(&ta, 0, sizeof(ta));
+  memset(&tb, 0, sizeof(tb));
+  if (a.K > 0) {
+    if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kElem, 128, msg) ||
+        !make_map(&tb, a.b, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), kElem, BN / 2, msg))
+      return cudaErrorInvalidValue;
+  }
+  CUtensorMap to;
+  if (!make_out_map(&to, a.out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), msg))
+    return cudaErrorInvalidValue;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.nkb = static_cast<int>((a.K + (kBKBytes / kElem) - 1) / (kBKBytes / kElem));
+  p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+  p.m_tiles = static_cast<int>((a.M + 255) / 256);
+  p.group_m = 8;
+  p.E = 1;
+  p.offsets = nullptr;
+  p.xs = a.x_scale;
+  p.xs_bcast = (a.x_scale_len == 1) ? 1 : 0;
+  p.ws = a.w_scale;
+  p.ws_bcast = (a.w_scale_len == 1) ? 1 : 0;
+  p.out = static_cast<uint16_t*>(a.out);
+  const uint32_t ab_fmt = (KIND == 0) ? static_cast<uint32_t>(a.fmt) : 1u;
+  p.idesc = (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+            (static_cast<uint32_t>(256 >> 4) << 24);  // M = 256 across the pair
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int clusters = device_sm_count(dev) / 2;
+  if (max_clusters > 0 && max_clusters < clusters) clusters = max_clusters;
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  if (tiles < clusters) clusters = static_cast<int>(tiles);
+  if (clusters < 1) clusters = 1;
+  k_gemm2<KIND, BN, STAGES><<<2 * clusters, kGemmThreads, kSmem, a.stream>>>(ta, tb, to, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
   // Wide tiles when there is enough work to fill the machine with them.
   const bool wide = (a.N % 256 == 0) && a.N >= 2048 && a.M >= 256;
+  // Large dense GEMMs run on CTA pairs (256 x 256 tiles).
+  const bool pair = a.offsets == nullptr && a.kind == 0 && (a.N % 256 == 0) && a.N >= 2048 && a.M >= 512;
+  if (pair) return run2<0, 256, 6>(a, msg);
   if (a.kind == 0) {
     if (wide) return run<0, 256, 4>(a, msg);
     return run<0, 128, 6>(a, msg);

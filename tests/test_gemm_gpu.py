@@ -34,7 +34,10 @@ def gemm_gpu(xq, wq, xs, ws, fmt):
 
 
 SHAPES = [(1, 8, 16), (5, 8, 32), (128, 128, 128), (129, 136, 144), (200, 264, 512), (300, 256, 1040),
-          (64, 1024, 256), (257, 2048, 384), (512, 4096, 256)]
+          (64, 1024, 256), (257, 2048, 384), (512, 4096, 256),
+          # CTA-pair path (M >= 512, N % 256 == 0): M not a multiple of 256
+          # (the second CTA's half partly or wholly past M), 9 N tiles, ragged K
+          (600, 2304, 272), (700, 2048, 128), (1024, 2560, 512)]
 
 
 @pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
