@@ -133,6 +133,23 @@ def traffic_from_profile(kernel_file, profile_name):
     return float(m.group(1)) if cur == h.group(1) else None
 
 
+# ------------------------------------------------------------ rank logic
+def max_over_ranks(ms, world, device):
+    """The timed region of a multi-rank run is the slowest rank's."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, steps, world, max_ms):
+    """Whole-job throughput: every rank's work over the slowest rank's time."""
+    return flops_per_step * steps * world / (max_ms / 1e3) / 1e12
+
+
 # ------------------------------------------------------------------ ours
 def run_ours(args, rank, local_rank, world):
     import torch
@@ -199,17 +216,13 @@ def run_ours(args, rank, local_rank, world):
         dist.barrier()
     clk = clocks.stop()
     hq.hq_check_device_error()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     qx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     qw_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     g_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
 
     flops = 2.0 * M * N * K
-    value = flops * args.steps * world / (ms / 1e3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, ms)
     gemm_tflops = flops / (g_ms / 1e3) / 1e12
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     q_bytes_x = M * K * 3 + M * 4  # bf16 read, code write, f32 scale write
@@ -239,12 +252,8 @@ def run_ours(args, rank, local_rank, world):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = whole_job_tflops(flops, e2e_steps, world, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -276,7 +285,7 @@ def run_ours(args, rank, local_rank, world):
                    "parallelism": "dp%d" % world},
         "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp8_peak, 4), "traffic": traffic,
-                     "kernel": "k_gemm<fp8,BN=256> (tcgen05 kind::f8f6f4)",
+                     "kernel": "k_gemm2<fp8, 256x256 CTA pair> (tcgen05 cta_group::2 kind::f8f6f4)",
                      "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal fp8/bf16 dense ratio)" %
                                     (peak_src, peaks["bf16_tflops"], FP8_OVER_BF16)},
         "quantize": {"x_per_token": {"ms": round(qx_ms, 4), "GB/s": round(qx_gbs, 1),

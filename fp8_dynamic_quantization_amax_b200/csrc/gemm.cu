@@ -563,6 +563,12 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+// L2 prefetch of a TMA tile (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // TMA tile store shared -> global (clipped at the tensor's bounds), and its
 // bulk-group bookkeeping.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
@@ -604,6 +610,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   constexpr int kStageBytes = kABytes + kBBytes;
   constexpr int kKElems = (KIND == 0) ? 128 : 64;
   constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+  constexpr int kPrefetch = 2 * STAGES;  // L2 prefetch distance for B, in K blocks
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -681,6 +688,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
           tma_load_2d_pair(sA + stage * kABytes, &tm_a, full_leader, kb * kKElems, a_row);
           tma_load_2d_pair(sB + stage * kBBytes, &tm_b, full_leader, kb * kKElems, b_row);
+          // The clusters that share this B tile run in step, so its DRAM
+          // latency would stall all of them at once: ask L2 for the B tile
+          // kPrefetch blocks ahead.
+          if (kb + kPrefetch < p.nkb) tma_prefetch_2d(&tm_b, (kb + kPrefetch) * kKElems, b_row);
           pend_mask |= 1u << stage;
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
