@@ -40,7 +40,8 @@ namespace {
 
 constexpr int kBM = 128;            // tile rows (MMA M)
 constexpr int kBKBytes = 128;       // K bytes per stage = one 128B swizzle row
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 192;   // CTA-pair kernel: TMA, MMA, 4 epilogue warps
+constexpr int kGemm1Threads = 320;  // 1-CTA kernel: TMA, MMA, 8 epilogue warps
 constexpr int kMaxExperts = 1024;
 constexpr unsigned long long kDrainLimitNs = ptx::kDrainLimitNs;
 
@@ -57,6 +58,7 @@ struct Params {
   int ws_bcast;
   uint16_t* out;
   uint32_t idesc;
+  int prefetch;         // 1: L2-prefetch operands ahead of the TMA loads
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -144,6 +146,29 @@ __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, ui
   asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// L2 prefetch of a TMA tile (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+// TMA tile store shared -> global (clipped at the tensor's bounds), and its
+// bulk-group bookkeeping.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one committed group may still be reading shared memory
+__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_le0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
 // ------------------------------------------------------------ tile schedule
 struct Tile {
   int a_row;   // first A row loaded (global)
@@ -192,13 +217,15 @@ __device__ __forceinline__ Tile decode_tile(int t, const Params& p, const int* p
 
 // ------------------------------------------------------------------ kernel
 template <int KIND, int BN, int STAGES>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, const Params p) {
+__global__ void __launch_bounds__(kGemm1Threads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+           const __grid_constant__ CUtensorMap tm_out, const Params p) {
   constexpr int kABytes = kBM * kBKBytes;
   constexpr int kBBytes = BN * kBKBytes;
   constexpr int kStageBytes = kABytes + kBBytes;
   constexpr int kKElems = (KIND == 0) ? 128 : 64;  // K elements per stage
   constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+  constexpr int kPrefetch = 2 * STAGES;  // L2 prefetch distance, in K blocks
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -215,6 +242,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-byte aligned stages
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kABytes;
+  // epilogue: one 32 x 32 bf16 staging tile (2 KB) per warp for TMA stores,
+  // and each warp's BN/2 column scales
+  uint8_t* sOut = smem + STAGES * kStageBytes;
+  float* sWs = reinterpret_cast<float*>(sOut + 8 * 2048);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -226,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 128);
+      mbar_init(&tempty_bar[a], 8);  // one arrive per epilogue warp
     }
     mbar_init(&final_bar, 1);
     abort_flag = 0;
@@ -256,6 +287,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_b) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_out) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
@@ -286,6 +318,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
           tma_load_2d(sA + stage * kABytes, &tm_a, &full_bar[stage], kb * kKElems, T.a_row);
           tma_load_2d(sB + stage * kBBytes, &tm_b, &full_bar[stage], kb * kKElems, T.b_row);
+          // L2 prefetch of both operands kPrefetch blocks ahead: the ring
+          // alone cannot cover DRAM latency at this tile's byte rate
+          if (p.prefetch && kb + kPrefetch < p.nkb) {
+            tma_prefetch_2d(&tm_a, (kb + kPrefetch) * kKElems, T.a_row);
+            tma_prefetch_2d(&tm_b, (kb + kPrefetch) * kKElems, T.b_row);
+          }
 #pragma unroll
           for (int s = 0; s < STAGES; ++s)
             if (s == stage) { armed[s] = true; armed_parity[s] = phase; }
@@ -341,8 +379,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------- epilogue
-    const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
-    const int r = quad * 32 + lane;
+    // Eight warps: warp w reads TMEM lane quadrant w % 4 (32 rows) and one
+    // half of the BN columns.  Per 32-column chunk it scales, rounds to
+    // bf16 and, when its 32 rows lie inside the tile's valid rows (the
+    // tensor map clips at M and N), writes the chunk through a staging tile
+    // with one TMA store; a 32-row group that straddles an expert boundary
+    // uses masked 16-byte stores instead.
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    const int half = ew >> 2;
+    constexpr int kHalf = BN / 2;
+    uint8_t* sb = sOut + ew * 2048;
+    float* wsh = sWs + ew * kHalf;
     int i = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int acc = i & 1;
@@ -350,45 +398,64 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag)) break;
       tc_fence_after();
       const Tile T = decode_tile<BN>(t, p, tile_prefix, row_start);
-      const int row = T.row_lo + r;
+      const int row0 = T.row_lo + quad * 32;
+      const int row = row0 + lane;
       const bool vrow = row < T.row_hi;
-      float xsv = 1.0f;
-      const float* wsp = nullptr;
+      // rows past M are clipped by the tensor map; rows of another expert are not
+      const bool tma_ok = row0 < T.row_hi && (p.offsets == nullptr || row0 + 32 <= T.row_hi);
+      const int colh = T.col0 + half * kHalf;
+      float xsv = 0.0f;
+      if (vrow) xsv = (KIND == 0) ? __ldg(p.xs + (p.xs_bcast ? 0 : row)) : 1.0f;
       if (KIND == 0) {
-        if (vrow) xsv = __ldg(p.xs + (p.xs_bcast ? 0 : row));
-        wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
+        const float* wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
+        for (int j = lane; j < kHalf; j += 32) {
+          const int n = colh + j;
+          wsh[j] = (n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f;
+        }
+      } else {
+        for (int j = lane; j < kHalf; j += 32) wsh[j] = 1.0f;
       }
+      __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = 0; c < kHalf; c += 32) {
         uint32_t v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN + c), v);
-        const int n0 = T.col0 + c;
-        if (vrow && n0 < p.N) {
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                      static_cast<uint32_t>(acc * BN + half * kHalf + c),
+                  v);
+        const int n0 = colh + c;
+        if (n0 >= p.N) continue;
+        uint32_t w[16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int nj = n0 + 8 * j;
-            if (nj < p.N) {
-              float f[8];
+        for (int j = 0; j < 16; ++j) {
+          const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * j]) : 0.0f;
+          const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+          w[j] = pack_bf16x2(a0 * (xsv * wsh[c + 2 * j]), a1 * (xsv * wsh[c + 2 * j + 1]));
+        }
+        if (tma_ok) {
+          if (lane == 0) bulk_wait_read_le0();  // the previous chunk's store has read the staging tile
+          __syncwarp();
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float a = (p.nkb > 0) ? __uint_as_float(v[8 * j + e]) : 0.0f;
-                if (KIND == 0) {
-                  const float s = xsv * __ldg(wsp + (p.ws_bcast ? 0 : nj + e));
-                  f[e] = a * s;
-                } else {
-                  f[e] = a;
-                }
-              }
-              st_global_v4(orow + nj, pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                           pack_bf16x2(f[6], f[7]));
-            }
+          for (int k = 0; k < 4; ++k)
+            st_shared_v4(sb + lane * 64 + k * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_out, sb, n0, row0);
+            bulk_commit_group();
           }
+        } else if (vrow) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (n0 + 8 * k < p.N) st_global_v4(orow + n0 + 8 * k, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty_bar[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
     }
+    if (lane == 0) bulk_wait_all();  // stores complete before the CTA's shared memory goes
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -466,7 +533,7 @@ bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, st
 template <int KIND, int BN, int STAGES>
 cudaError_t run(const GemmArgs& a, std::string* msg) {
   constexpr int kElem = (KIND == 0) ? 1 : 2;
-  constexpr int kSmem = STAGES * (kBM + BN) * kBKBytes + 1024;
+  constexpr int kSmem = STAGES * (kBM + BN) * kBKBytes + 8 * 2048 + 8 * (BN / 2) * 4 + 1024;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -485,6 +552,9 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
                   kElem, BN, msg))
       return cudaErrorInvalidValue;
   }
+  CUtensorMap to;
+  if (!make_out_map(&to, a.out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), msg))
+    return cudaErrorInvalidValue;
 
   Params p;
   p.M = static_cast<int>(a.M);
@@ -501,6 +571,9 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
   p.ws = a.w_scale;
   p.ws_bcast = (a.w_scale_len == 1) ? 1 : 0;
   p.out = static_cast<uint16_t*>(a.out);
+  // Grouped tiles re-read A and B from L2 at a high byte rate and gain from
+  // the prefetch; the small-M dense stream reads W once and loses by it.
+  p.prefetch = (a.offsets != nullptr) ? 1 : 0;
   const uint32_t ab_fmt = (KIND == 0) ? static_cast<uint32_t>(a.fmt) : 1u;  // E4M3/E5M2, or BF16
   p.idesc = (1u << 4)                                   // D: FP32
             | (ab_fmt << 7) | (ab_fmt << 10)            // A and B element types
@@ -517,7 +590,7 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
     tiles_bound = (static_cast<int64_t>(p.m_tiles) + a.E) * p.n_tiles;
   int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
   if (grid < 1) grid = 1;
-  k_gemm<KIND, BN, STAGES><<<grid, kGemmThreads, kSmem, a.stream>>>(ta, tb, p);
+  k_gemm<KIND, BN, STAGES><<<grid, kGemm1Threads, kSmem, a.stream>>>(ta, tb, to, p);
   return cudaGetLastError();
 }
 
@@ -563,28 +636,6 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
-// L2 prefetch of a TMA tile (no shared-memory destination, no barrier).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(c0), "r"(c1)
-               : "memory");
-}
-
-// TMA tile store shared -> global (clipped at the tensor's bounds), and its
-// bulk-group bookkeeping.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
-               "r"(smem_u32(src)), "r"(c0), "r"(c1)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// at most one committed group may still be reading shared memory
-__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-
 template <int KIND>
 __device__ __forceinline__ void mma_issue_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                uint32_t accumulate) {
@@ -900,7 +951,9 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
 
 cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
   // Wide tiles when there is enough work to fill the machine with them.
-  const bool wide = (a.N % 256 == 0) && a.N >= 2048 && a.M >= 256;
+  // 256-wide tiles halve the A bytes per MMA cycle; worth a ragged last N
+  // tile once N is large enough
+  const bool wide = ((a.N % 256 == 0) && a.N >= 2048 && a.M >= 256) || (a.offsets != nullptr && a.N >= 1024);
   // Large dense GEMMs run on CTA pairs (256 x 256 tiles).
   const bool pair = a.offsets == nullptr && a.kind == 0 && (a.N % 256 == 0) && a.N >= 2048 && a.M >= 512;
   if (pair) return run2<0, 256, 6>(a, msg);
