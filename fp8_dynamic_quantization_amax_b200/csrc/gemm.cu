@@ -216,15 +216,30 @@ __device__ __forceinline__ Tile decode_tile(int t, const Params& p, const int* p
 }
 
 // ------------------------------------------------------------------ kernel
-template <int KIND, int BN, int STAGES>
+// AROWS: rows of A loaded per K block.  128 normally; for small M (decode)
+// only the first AROWS >= M rows are loaded, packed at AROWS-row stride, which
+// leaves room for more of B.  The MMA still reads 128 rows of A from the
+// block start; rows past AROWS then come from the following blocks and only
+// produce accumulator rows >= M, which are never stored.
+// KPS: consecutive K blocks per pipeline stage.  With KPS > 1 each stage asks
+// DRAM for KPS * 128 contiguous bytes of every weight row at once instead of
+// one 128-byte piece per row, so more of each opened DRAM page is used.
+template <int KIND, int BN, int STAGES, int AROWS = kBM, int KPS = 1>
 __global__ void __launch_bounds__(kGemm1Threads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_out, const Params p) {
-  constexpr int kABytes = kBM * kBKBytes;
-  constexpr int kBBytes = BN * kBKBytes;
+  static_assert((STAGES * KPS - 1) * AROWS * kBKBytes + kBM * kBKBytes <= STAGES * KPS * (AROWS + BN) * kBKBytes,
+                "the MMA's 128-row read of the last A block must stay inside shared memory");
+  static_assert(AROWS % 8 == 0 && (AROWS * kBKBytes) % 1024 == 0, "A blocks keep the 1024-byte swizzle atom");
+  static_assert(BN % 16 == 0 && BN >= 64 && BN <= 256, "MMA N (M = 128): a multiple of 16 in [64, 256]");
+  constexpr int kChunks = (BN + 31) / 32;      // 32-column epilogue chunks (the last may hold 16)
+  constexpr int kMyChunks = (kChunks + 1) / 2;  // per epilogue warp (two warps per quadrant)
+  constexpr int kABytes = AROWS * kBKBytes;  // one K block of A
+  constexpr int kBBytes = BN * kBKBytes;     // one K block of B
   constexpr int kStageBytes = kABytes + kBBytes;
   constexpr int kKElems = (KIND == 0) ? 128 : 64;  // K elements per stage
   constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+  constexpr uint32_t kAccStride = (2 * BN <= 256) ? BN : 256u;  // TMEM columns between the two accumulators
   constexpr int kPrefetch = 2 * STAGES;  // L2 prefetch distance, in K blocks
 
   extern __shared__ uint8_t smem_raw[];
@@ -241,10 +256,10 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-byte aligned stages
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * kABytes;
+  uint8_t* sB = smem + STAGES * KPS * kABytes;
   // epilogue: one 32 x 32 bf16 staging tile (2 KB) per warp for TMA stores,
   // and each warp's BN/2 column scales
-  uint8_t* sOut = smem + STAGES * kStageBytes;
+  uint8_t* sOut = smem + STAGES * KPS * kStageBytes;
   float* sWs = reinterpret_cast<float*>(sOut + 8 * 2048);
 
   const int warp = threadIdx.x >> 5;
@@ -313,11 +328,14 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       bool stop = false;
       for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
         const Tile T = decode_tile<BN>(t, p, tile_prefix, row_start);
-        for (int kb = 0; kb < p.nkb; ++kb) {
+        for (int kb = 0; kb < p.nkb; kb += KPS) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { stop = true; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
-          tma_load_2d(sA + stage * kABytes, &tm_a, &full_bar[stage], kb * kKElems, T.a_row);
-          tma_load_2d(sB + stage * kBBytes, &tm_b, &full_bar[stage], kb * kKElems, T.b_row);
+          const int nsub = min(KPS, p.nkb - kb);
+          mbar_arrive_expect_tx(&full_bar[stage], nsub * kStageBytes);
+          for (int u = 0; u < nsub; ++u) {
+            tma_load_2d(sA + (stage * KPS + u) * kABytes, &tm_a, &full_bar[stage], (kb + u) * kKElems, T.a_row);
+            tma_load_2d(sB + (stage * KPS + u) * kBBytes, &tm_b, &full_bar[stage], (kb + u) * kKElems, T.b_row);
+          }
           // L2 prefetch of both operands kPrefetch blocks ahead: the ring
           // alone cannot cover DRAM latency at this tile's byte rate
           if (p.prefetch && kb + kPrefetch < p.nkb) {
@@ -351,16 +369,19 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       const uint32_t acc_phase = (i >> 1) & 1;
       if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) break;
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-      for (int kb = 0; kb < p.nkb; ++kb) {
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
+      for (int kb = 0; kb < p.nkb; kb += KPS) {
         if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { stop = true; break; }
         tc_fence_after();
         if (lane == 0) {
-          const uint64_t ad = smem_desc(smem_u32(sA + stage * kABytes));
-          const uint64_t bd = smem_desc(smem_u32(sB + stage * kBBytes));
+          const int nsub = min(KPS, p.nkb - kb);
+          for (int u = 0; u < nsub; ++u) {
+            const uint64_t ad = smem_desc(smem_u32(sA + (stage * KPS + u) * kABytes));
+            const uint64_t bd = smem_desc(smem_u32(sB + (stage * KPS + u) * kBBytes));
 #pragma unroll
-          for (int k = 0; k < kBKBytes / 32; ++k)  // 32 bytes of K per instruction
-            mma_issue<KIND>(d_tmem, ad + 2u * k, bd + 2u * k, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kBKBytes / 32; ++k)  // 32 bytes of K per instruction
+              mma_issue<KIND>(d_tmem, ad + 2u * k, bd + 2u * k, p.idesc, (kb + u > 0 || k > 0) ? 1u : 0u);
+          }
           tc_commit(&empty_bar[stage]);
           issued = true;
         }
@@ -379,18 +400,17 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------- epilogue
-    // Eight warps: warp w reads TMEM lane quadrant w % 4 (32 rows) and one
-    // half of the BN columns.  Per 32-column chunk it scales, rounds to
-    // bf16 and, when its 32 rows lie inside the tile's valid rows (the
-    // tensor map clips at M and N), writes the chunk through a staging tile
-    // with one TMA store; a 32-row group that straddles an expert boundary
-    // uses masked 16-byte stores instead.
+    // Eight warps: warp w reads TMEM lane quadrant w % 4 (32 rows); the two
+    // warps of a quadrant take alternate 32-column chunks of the BN columns.
+    // Per chunk a warp scales, rounds to bf16 and, when its 32 rows lie
+    // inside the tile's valid rows (the tensor map clips at M and N), writes
+    // the chunk through a staging tile with one TMA store; a 32-row group
+    // that straddles an expert boundary uses masked 16-byte stores instead.
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int half = ew >> 2;
-    constexpr int kHalf = BN / 2;
     uint8_t* sb = sOut + ew * 2048;
-    float* wsh = sWs + ew * kHalf;
+    float* wsh = sWs + ew * kMyChunks * 32;
     int i = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int acc = i & 1;
@@ -403,36 +423,39 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       const bool vrow = row < T.row_hi;
       // rows past M are clipped by the tensor map; rows of another expert are not
       const bool tma_ok = row0 < T.row_hi && (p.offsets == nullptr || row0 + 32 <= T.row_hi);
-      const int colh = T.col0 + half * kHalf;
+      const int ncap = min(p.N, T.col0 + BN);  // end of this tile's columns
       float xsv = 0.0f;
       if (vrow) xsv = (KIND == 0) ? __ldg(p.xs + (p.xs_bcast ? 0 : row)) : 1.0f;
       if (KIND == 0) {
         const float* wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
-        for (int j = lane; j < kHalf; j += 32) {
-          const int n = colh + j;
-          wsh[j] = (n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f;
+        for (int i = 0; half + 2 * i < kChunks; ++i) {
+          const int n = T.col0 + (half + 2 * i) * 32 + lane;
+          wsh[i * 32 + lane] = (n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f;
         }
       } else {
-        for (int j = lane; j < kHalf; j += 32) wsh[j] = 1.0f;
+        for (int i = 0; half + 2 * i < kChunks; ++i) wsh[i * 32 + lane] = 1.0f;
       }
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
 #pragma unroll 1
-      for (int c = 0; c < kHalf; c += 32) {
+      for (int i = 0; half + 2 * i < kChunks; ++i) {
+        const int c = (half + 2 * i) * 32;  // chunk's first column within the tile
         uint32_t v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                      static_cast<uint32_t>(acc * BN + half * kHalf + c),
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride +
+                      static_cast<uint32_t>(c),
                   v);
-        const int n0 = colh + c;
-        if (n0 >= p.N) continue;
+        const int n0 = T.col0 + c;
+        if (n0 >= ncap) continue;
+        const float* sc = wsh + i * 32;
         uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * j]) : 0.0f;
           const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-          w[j] = pack_bf16x2(a0 * (xsv * wsh[c + 2 * j]), a1 * (xsv * wsh[c + 2 * j + 1]));
+          w[j] = pack_bf16x2(a0 * (xsv * sc[2 * j]), a1 * (xsv * sc[2 * j + 1]));
         }
-        if (tma_ok) {
+        // the tensor map clips at N; a 16-column tail chunk inside N is masked
+        if (tma_ok && (BN % 32 == 0 || n0 + 32 <= T.col0 + BN)) {
           if (lane == 0) bulk_wait_read_le0();  // the previous chunk's store has read the staging tile
           __syncwarp();
 #pragma unroll
@@ -447,7 +470,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
         } else if (vrow) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            if (n0 + 8 * k < p.N) st_global_v4(orow + n0 + 8 * k, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            if (n0 + 8 * k < ncap) st_global_v4(orow + n0 + 8 * k, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
       tc_fence_before();
@@ -530,14 +553,16 @@ bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, st
   return true;
 }
 
-template <int KIND, int BN, int STAGES>
+template <int KIND, int BN, int STAGES, int AROWS = kBM, int KPS = 1>
 cudaError_t run(const GemmArgs& a, std::string* msg) {
   constexpr int kElem = (KIND == 0) ? 1 : 2;
-  constexpr int kSmem = STAGES * (kBM + BN) * kBKBytes + 8 * 2048 + 8 * (BN / 2) * 4 + 1024;
+  constexpr int kSmem = STAGES * KPS * (AROWS + BN) * kBKBytes + 8 * 2048 + 8 * (((BN + 31) / 32 + 1) / 2) * 32 * 4 + 1024;
+  static_assert(kSmem + 8352 <= 232448, "shared memory over the 227 KB per-CTA limit");
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_gemm<KIND, BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    attr_err =
+        cudaFuncSetAttribute(k_gemm<KIND, BN, STAGES, AROWS, KPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   });
   if (attr_err != cudaSuccess) {
     *msg = "cudaFuncSetAttribute failed";
@@ -547,7 +572,7 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
   memset(&ta, 0, sizeof(ta));
   memset(&tb, 0, sizeof(tb));
   if (a.K > 0) {  // K == 0: no loads are issued and the maps are never read
-    if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kElem, kBM, msg) ||
+    if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kElem, AROWS, msg) ||
         !make_map(&tb, a.b, static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K),
                   kElem, BN, msg))
       return cudaErrorInvalidValue;
@@ -590,7 +615,7 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
     tiles_bound = (static_cast<int64_t>(p.m_tiles) + a.E) * p.n_tiles;
   int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
   if (grid < 1) grid = 1;
-  k_gemm<KIND, BN, STAGES><<<grid, kGemm1Threads, kSmem, a.stream>>>(ta, tb, to, p);
+  k_gemm<KIND, BN, STAGES, AROWS, KPS><<<grid, kGemm1Threads, kSmem, a.stream>>>(ta, tb, to, p);
   return cudaGetLastError();
 }
 
@@ -661,6 +686,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   constexpr int kStageBytes = kABytes + kBBytes;
   constexpr int kKElems = (KIND == 0) ? 128 : 64;
   constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
+  constexpr uint32_t kAccStride = (2 * BN <= 256) ? BN : 256u;  // TMEM columns between the two accumulators
   constexpr int kPrefetch = 2 * STAGES;  // L2 prefetch distance for B, in K blocks
 
   extern __shared__ uint8_t smem_raw[];
@@ -768,7 +794,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const uint32_t acc_phase = (i >> 1) & 1;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
         for (int kb = 0; kb < p.nkb; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { stop = true; break; }
           tc_fence_after();
@@ -957,6 +983,31 @@ cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
   // Large dense GEMMs run on CTA pairs (256 x 256 tiles).
   const bool pair = a.offsets == nullptr && a.kind == 0 && (a.N % 256 == 0) && a.N >= 2048 && a.M >= 512;
   if (pair) return run2<0, 256, 6>(a, msg);
+  // Small M (decode): the weight stream from HBM is the bound.  Only AROWS
+  // rows of A are loaded per K block, which leaves shared memory for several
+  // K blocks of W per stage (longer runs of each weight row per request).
+  // Tile width: 128 when N/128 tiles fit on the SMs in one round; otherwise
+  // 208 (N <= 208 * SMs, one round with fewer idle SMs than 256-wide tiles
+  // leave), else 256.
+  if (a.offsets == nullptr && a.kind == 0 && a.M <= 128) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int64_t sms = device_sm_count(dev);
+    const int bn = ((a.N + 127) / 128 <= sms) ? 128 : ((a.N + 207) / 208 <= sms) ? 208 : 256;
+    if (a.M <= 16) {
+      if (bn == 128) return run<0, 128, 3, 16, 3>(a, msg);
+      if (bn == 208) return run<0, 208, 3, 16, 2>(a, msg);
+      return run<0, 256, 2, 16, 2>(a, msg);
+    }
+    if (a.M <= 64) {
+      if (bn == 128) return run<0, 128, 2, 64, 4>(a, msg);
+      if (bn == 208) return run<0, 208, 2, 64, 2>(a, msg);
+      return run<0, 256, 2, 64, 2>(a, msg);
+    }
+    if (bn == 128) return run<0, 128, 3, 128, 2>(a, msg);
+    if (bn == 208) return run<0, 208, 4, 128, 1>(a, msg);
+    return run<0, 256, 4>(a, msg);
+  }
   if (a.kind == 0) {
     if (wide) return run<0, 256, 4>(a, msg);
     return run<0, 128, 6>(a, msg);

@@ -36,6 +36,7 @@
 #include <algorithm>
 #include <cfloat>
 #include <cuda_fp16.h>
+#include <type_traits>
 
 namespace hq {
 namespace {
@@ -532,6 +533,194 @@ __global__ void __launch_bounds__(kThreads) k_tensor_cast(
   }
 }
 
+// ------------------------------------------------- per-tensor, one launch
+// The same two phases in one cooperative launch (all CTAs resident, one per
+// SM).  CTA b owns the contiguous vectors [b0, b1).  Phase 1 bulk-copies the
+// first part of its range into shared memory (kept there for phase 2) and
+// streams the rest through registers with an L2 evict_last hint, so that
+// phase 2 finds it in L2; a grid barrier (a counter, bounded wait) publishes
+// the global amax; phase 2 casts the streamed part again, newest lines
+// first, and then the part held in shared memory.  DRAM sees x about once.
+// Workspace words: [0] amax bits, [1] arrivals, [2] departures, [3]
+// non-finite flag; the last CTA to leave returns all four to zero.
+constexpr int kFusedThreads = 512;
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint4 ld_hint(const uint4* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p), "l"(pol));
+  return r;
+}
+__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                               uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          ptx::smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(ptx::smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
+    const void* __restrict__ x, int64_t n, int64_t per_cta, int64_t held_max, uint8_t* __restrict__ q,
+    uint32_t* __restrict__ ws, float fmax, float* __restrict__ scales, float* __restrict__ amax_out,
+    unsigned* __restrict__ err_word) {
+  constexpr int VEC = Dt<DT>::kVec;
+  constexpr int T = kFusedThreads;
+  constexpr int U = kUnrollFlat;
+  extern __shared__ __align__(128) uint4 held[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ float sh[T / 32];
+  __shared__ float s_amax;
+  __shared__ int s_flags;  // bit 0: a non-finite element somewhere, bit 1: abort
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const uint4* xv = static_cast<const uint4*>(x);
+  const int64_t nv = n / VEC;
+  const int64_t b0 = min(nv, static_cast<int64_t>(blockIdx.x) * per_cta);
+  const int64_t b1 = min(nv, b0 + per_cta);
+  const int64_t nheld = min(b1 - b0, held_max);
+  const int64_t s0 = b0 + nheld;  // streamed part [s0, b1)
+  const bool tail_cta = blockIdx.x == gridDim.x - 1;
+
+  if (tid == 0) {
+    abort_flag = 0;
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbarrier_init();
+    if (nheld > 0) {
+      const uint64_t pol = policy_evict_first();
+      const uint32_t bytes = static_cast<uint32_t>(nheld * 16);
+      ptx::mbar_arrive_expect_tx(&bar, bytes);
+      for (uint32_t off = 0; off < bytes; off += 65536u)
+        bulk_load_hint(reinterpret_cast<char*>(held) + off, reinterpret_cast<const char*>(xv + b0) + off,
+                       min(65536u, bytes - off), &bar, pol);
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 1: amax
+  const uint64_t keep = policy_evict_last();
+  uint32_t mraw = 0;
+  int64_t v = s0 + tid;
+  for (; v + (U - 1) * T < b1; v += U * T) {
+    uint4 u[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + v + j * T, keep);
+#pragma unroll
+    for (int j = 0; j < U; ++j) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(u[j]));
+  }
+  for (; v < b1; v += T) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(ld_hint(xv + v, keep)));
+  bool landed = true;
+  if (nheld > 0) {
+    landed = ptx::mbar_wait(&bar, 0, &abort_flag, err_word, kDevErrTimeout);
+    if (landed)
+      for (int64_t i = tid; i < nheld; i += T) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(held[i]));
+  }
+  float amax = 0.0f;
+  bool nf = false;
+  if (!Dt<DT>::nonfinite(mraw)) {
+    amax = Dt<DT>::value(mraw);
+  } else {  // rare: this thread's vectors again on the exact path
+    nf = true;
+    for (v = s0 + tid; v < b1; v += T) amax = vec_amax_exact<DT>(__ldg(xv + v), amax);
+    if (landed)
+      for (int64_t i = tid; i < nheld; i += T) amax = vec_amax_exact<DT>(held[i], amax);
+  }
+  if (tail_cta)
+    for (int64_t i = nv * VEC + tid; i < n; i += T) {
+      const float f = Dt<DT>::load1(x, i);
+      if (!(fabsf(f) <= FLT_MAX)) nf = true;
+      amax = fmaxf(amax, finite_abs(f));
+    }
+  nf = __syncthreads_or(nf);
+  // block_max for T threads
+  amax = warp_max(amax);
+  if ((tid & 31) == 0) sh[tid >> 5] = amax;
+  __syncthreads();
+  if (tid < 32) {
+    float r = (tid < T / 32) ? sh[tid] : 0.0f;
+    r = warp_max(r);
+    if (tid == 0) {
+      if (nf) atomicOr(&ws[3], 1u);
+      atomicMax(&ws[0], __float_as_uint(r));
+      __threadfence();
+      atomicAdd(&ws[1], 1u);
+      // grid barrier: every CTA has published its amax
+      bool ok = !abort_flag;
+      const unsigned long long t0 = ptx::globaltimer();
+      for (uint32_t it = 0; ok; ++it) {
+        if (ld_acquire_u32(&ws[1]) >= gridDim.x) break;
+        if ((it & 15u) == 15u && ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
+          atomicOr(err_word, kDevErrTimeout);
+          ok = false;
+        }
+        __nanosleep(100);
+      }
+      s_amax = __uint_as_float(__ldcg(&ws[0]));
+      s_flags = (__ldcg(&ws[3]) != 0u ? 1 : 0) | (ok ? 0 : 2);
+      __threadfence();
+      // departure: the last CTA to leave clears the workspace
+      if (atomicAdd(&ws[2], 1u) == gridDim.x - 1) {
+        atomicExch(&ws[0], 0u);
+        atomicExch(&ws[3], 0u);
+        atomicExch(&ws[1], 0u);
+        atomicExch(&ws[2], 0u);
+      }
+    }
+  }
+  __syncthreads();
+  if (s_flags & 2) {  // barrier or copy gave up: the error word says so
+    if (tid == 0 && nheld > 0 && !landed) {  // let the copy land before the CTA's shared memory goes
+      int dummy = 0;
+      ptx::mbar_wait(&bar, 0, &dummy, nullptr, 0, ptx::kDrainLimitNs);
+    }
+    return;
+  }
+
+  // ---- phase 2: cast
+  const float a = s_amax;
+  const float m = multiplier(a, fmax);
+  if (blockIdx.x == 0 && tid == 0) {
+    scales[0] = __fdiv_rn(1.0f, m);
+    if (amax_out) amax_out[0] = a;
+  }
+  const uint64_t drop = policy_evict_first();
+  const int64_t ns = b1 - s0;
+  auto cast_range = [&](auto fast) {
+    constexpr bool FAST = decltype(fast)::value;
+    int64_t i = tid;
+    for (; i + (U - 1) * T < ns; i += U * T) {  // streamed part, from its end backwards
+      uint4 u[U];
+#pragma unroll
+      for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + (b1 - 1 - (i + j * T)), drop);
+#pragma unroll
+      for (int j = 0; j < U; ++j) vec_store<DT, FMT, FAST>(q + (b1 - 1 - (i + j * T)) * VEC, u[j], m);
+    }
+    for (; i < ns; i += T) vec_store<DT, FMT, FAST>(q + (b1 - 1 - i) * VEC, ld_hint(xv + (b1 - 1 - i), drop), m);
+    for (int64_t k = tid; k < nheld; k += T) vec_store<DT, FMT, FAST>(q + (b0 + k) * VEC, held[k], m);
+  };
+  if (!(s_flags & 1)) cast_range(std::true_type{});
+  else cast_range(std::false_type{});
+  if (tail_cta)
+    for (int64_t i = nv * VEC + tid; i < n; i += T) q[i] = cvt1_exact<FMT>(__fmul_rn(Dt<DT>::load1(x, i), m));
+}
+
 // -------------------------------------------------------------- per-channel
 // Tile: a strip of 32 column vectors (32*VEC columns) x a band of rows.  Warp
 // w of the CTA takes rows w, w+8, ... of the band, eight rows per step; lane
@@ -805,6 +994,34 @@ inline int flat_grid(int64_t nvec, int dev, int unroll) {
   return static_cast<int>(g);
 }
 
+// Per-tensor in one cooperative launch: one CTA per SM, each holding up to
+// kFusedHeldBytes of its range in shared memory.
+constexpr int64_t kFusedHeldBytes = 208 * 1024;
+constexpr int64_t kFusedMinBytes = 4 << 20;  // smaller tensors: the two-launch path
+
+template <int DT, int FMT>
+cudaError_t launch_tensor_fused(const QuantizeArgs& a, int dev, int64_t n, float fmax) {
+  constexpr int VEC = Dt<DT>::kVec;
+  static cudaError_t attr = cudaFuncSetAttribute(k_tensor_fused<DT, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kFusedHeldBytes));
+  if (attr != cudaSuccess) return attr;
+  const int grid = device_sm_count(dev);
+  const int64_t nv = n / VEC;
+  int64_t per = (nv + grid - 1) / grid;
+  int64_t held_max = std::min<int64_t>(per, kFusedHeldBytes / 16);
+  const size_t smem = static_cast<size_t>(held_max) * 16;
+  const void* x = a.x;
+  uint8_t* q = a.q;
+  uint32_t* ws = static_cast<uint32_t*>(a.ws);
+  float* scales = a.scales;
+  float* amax_out = a.amax_out;
+  unsigned* err = device_error_word();
+  void* args[] = {(void*)&x, (void*)&n, (void*)&per, (void*)&held_max, (void*)&q, (void*)&ws,
+                  (void*)&fmax, (void*)&scales, (void*)&amax_out, (void*)&err};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_tensor_fused<DT, FMT>), dim3(grid),
+                                     dim3(kFusedThreads), args, smem, a.stream);
+}
+
 template <int DT, int FMT>
 cudaError_t launch_typed(const QuantizeArgs& a) {
   constexpr int VEC = Dt<DT>::kVec;
@@ -857,6 +1074,8 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
     return cudaGetLastError();
   }
 
+  if (a.gran == 0 && flat_vec && n * Dt<DT>::kSize >= kFusedMinBytes && device_error_word() != nullptr)
+    return launch_tensor_fused<DT, FMT>(a, dev, n, fmax);
   if (a.gran == 0) {  // per-tensor, two phases
     uint32_t* ws = static_cast<uint32_t*>(a.ws);
     const int grid = flat_grid(flat_vec ? n / VEC : n, dev, kUnrollFlat);

@@ -37,7 +37,14 @@ SHAPES = [(1, 8, 16), (5, 8, 32), (128, 128, 128), (129, 136, 144), (200, 264, 5
           (64, 1024, 256), (257, 2048, 384), (512, 4096, 256),
           # CTA-pair path (M >= 512, N % 256 == 0): M not a multiple of 256
           # (the second CTA's half partly or wholly past M), 9 N tiles, ragged K
-          (600, 2304, 272), (700, 2048, 128), (1024, 2560, 512)]
+          (600, 2304, 272), (700, 2048, 128), (1024, 2560, 512),
+          # small-M (decode) paths with 128-wide tiles (N/128 tiles fit on the SMs)
+          (17, 2048, 384), (33, 520, 160), (24, 18944, 128)]
+
+# Decode paths with wider tiles on a 148-SM B200: 208 columns once N/128
+# tiles exceed the SMs (a ragged last tile, a 16-column tail chunk per
+# tile), 256 beyond 208 x 148 columns; A loaded 16 / 64 / 128 rows per block.
+DECODE_SHAPES = [(40, 19200, 256), (16, 19000, 256), (100, 19200, 128), (8, 30848, 64), (120, 4096, 384)]
 
 
 @pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
@@ -55,6 +62,22 @@ def test_gemm_random_codes(fmt, bcast):
         out = gemm_gpu(xq, wq, xs, ws, fmt)
         ref = O.gemm_a8w8(xq, wq, fmt, xs, ws)
         assert_gemm_close(out, ref)
+    H.hq_check_device_error()
+
+
+@pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
+def test_gemm_decode_tile_widths(fmt):
+    for i, (M, N, K) in enumerate(DECODE_SHAPES):
+        rng = np.random.default_rng(300 + i)
+        xq = rand_codes(rng, (M, K), fmt)
+        wq = rand_codes(rng, (N, K), fmt)
+        xs = rng.uniform(0.001, 0.01, M).astype(np.float32)
+        ws = rng.uniform(0.001, 0.01, N).astype(np.float32)
+        if fmt == O.E5M2:
+            xs *= np.float32(1e-4)
+            ws *= np.float32(1e-4)
+        out = gemm_gpu(xq, wq, xs, ws, fmt)
+        assert_gemm_close(out, O.gemm_a8w8(xq, wq, fmt, xs, ws))
     H.hq_check_device_error()
 
 
