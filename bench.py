@@ -1,7 +1,7 @@
 """Benchmark of the dynamic-FP8 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large|large4096|sweep|moe]
+                    [--workload large|large4096|decode1|decode16|decode128|sweep|moe|moe_bf16]
 
 Default workload (the large a8w8 GEMM layer): X bf16 [16384, 8192] ~N(0,1),
 W bf16 [28672, 8192] ~N(0,0.02).  One step = per-token E4M3 quantize of X,
@@ -52,18 +52,37 @@ def dist_env():
 
 
 # --------------------------------------------------------------- workloads
+# layer: the large a8w8 layer, X and W quantized every step (default).
+# decode: the same layer at small M; W quantized once before timing (weights
+#   are static at inference), the step is quantize X + GEMM.
+# sweep: quantize only, bf16 [8192, 8192]; every granularity x format.
+# moe / moe_bf16: per-token quantize of the routed tokens + grouped a8w8 GEMM
+#   over 64 experts (W quantized once); the bf16 grouped GEMM alone.
 WORKLOADS = {
-    "large": dict(M=16384, N=28672, K=8192),
-    "large4096": dict(M=4096, N=28672, K=8192),
+    "large": dict(kind="layer", M=16384, N=28672, K=8192),
+    "large4096": dict(kind="layer", M=4096, N=28672, K=8192),
+    "decode1": dict(kind="decode", M=1, N=28672, K=8192),
+    "decode16": dict(kind="decode", M=16, N=28672, K=8192),
+    "decode128": dict(kind="decode", M=128, N=28672, K=8192),
+    "sweep": dict(kind="sweep", M=8192, N=0, K=8192),
+    "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
+    "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }
 
 
 def workload_desc(name, cfg):
-    if name.startswith("large"):
-        return ("large a8w8 GEMM layer: X bf16 [%d,%d] ~N(0,1) per-token E4M3, W bf16 [%d,%d] ~N(0,0.02) "
-                "per-output-channel E4M3, out bf16 [%d,%d] (caller-owned)" % (cfg["M"], cfg["K"], cfg["N"],
-                                                                            cfg["K"], cfg["M"], cfg["N"]))
-    return name
+    k = cfg["kind"]
+    if k in ("layer", "decode"):
+        return ("%s a8w8 GEMM layer: X bf16 [%d,%d] ~N(0,1) per-token E4M3, W bf16 [%d,%d] ~N(0,0.02) "
+                "per-output-channel E4M3%s, out bf16 [%d,%d] (caller-owned)" %
+                ("large" if k == "layer" else "decode", cfg["M"], cfg["K"], cfg["N"], cfg["K"],
+                 "" if k == "layer" else " (quantized once: static weights)", cfg["M"], cfg["N"]))
+    if k == "sweep":
+        return ("quantize sweep: bf16 [%d,%d] ~N(0,1), 0.1%% x100 outliers, 0.1%% zeros, one zero row; "
+                "per-tensor / per-token / per-channel x E4M3 / E5M2" % (cfg["M"], cfg["K"]))
+    return ("grouped MoE GEMM: %d experts, K=%d, N=%d, %d tokens by Zipf(1.1) counts (2 experts empty); %s" %
+            (cfg["E"], cfg["K"], cfg["N"], cfg["M"],
+             "per-token E4M3 X + per-expert per-channel E4M3 W, a8w8" if k == "moe" else "bf16 X and W, fp32 acc"))
 
 
 class ClockSampler:
@@ -151,11 +170,193 @@ def whole_job_tflops(flops_per_step, steps, world, max_ms):
 
 
 # ------------------------------------------------------------------ ours
+def q_bytes(rows, cols, nscales, elem=2):
+    """Algorithmic bytes of one quantize call: read x, write codes and scales."""
+    return rows * cols * (elem + 1) + 4 * nscales
+
+
+def build(args, cfg, rank, dev, stream, peaks):
+    """Device inputs and the step's calls for one workload.  Returns a dict:
+    calls [(label, fn, launches)], per_step (flops or bytes), unit, e2e
+    (copies + step), h2d/d2h bytes, roofline(ms_by_label), config extras."""
+    import torch
+    import workloads as W
+    import fp8_dynamic_quantization_amax_b200 as hq
+
+    kind = cfg["kind"]
+    M, N, K = cfg["M"], cfg["N"], cfg["K"]
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+
+    def bf16_host(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    if kind in ("layer", "decode"):
+        x_host = bf16_host(W.large_x(M, K, seed=rank)).view(M, K)
+        w_host = bf16_host(W.large_w(N, K)).view(N, K)
+        x, w = x_host.to(dev), w_host.to(dev)
+        xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        wq = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        xs = torch.empty((M,), dtype=torch.float32, device=dev)
+        ws = torch.empty((N,), dtype=torch.float32, device=dev)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        qx = ("quantize X", lambda: hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TOKEN, q=xq, scales=xs, stream=stream), 1)
+        qw = ("quantize W", lambda: hq.hq_quantize_fp8(w, hq.E4M3, hq.PER_TOKEN, q=wq, scales=ws, stream=stream), 1)
+        gm = ("gemm", lambda: hq.hq_gemm_a8w8(xq, wq, xs, ws, hq.E4M3, out=out, stream=stream), 1)
+        if kind == "decode":
+            qw[1]()  # static weights: quantized once
+        calls = [qx, qw, gm] if kind == "layer" else [qx, gm]
+
+        def e2e():
+            x.copy_(x_host, non_blocking=True)
+            if kind == "layer":
+                w.copy_(w_host, non_blocking=True)
+            for c in calls:
+                c[1]()
+            out_host.copy_(out, non_blocking=True)
+
+        flops = 2.0 * M * N * K
+        h2d = (M * K + (N * K if kind == "layer" else 0)) * 2
+
+        def roofline(ms):
+            g = ms["gemm"]
+            if kind == "layer":
+                a = flops / (g / 1e3) / 1e12
+                traffic = traffic_from_profile("gemm.cu", "gemm_a8w8_large_M16384_N28672_K8192.md") \
+                    if args.workload == "large" else None
+                rf = {"bound": "tensor", "achieved": round(a, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                      "frac": round(a / fp8_peak, 4), "traffic": traffic,
+                      "kernel": "k_gemm2<fp8, 256x256 CTA pair> (tcgen05 cta_group::2 kind::f8f6f4)",
+                      "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal fp8/bf16 dense ratio)" %
+                                     (peaks["_src"], peaks["bf16_tflops"], FP8_OVER_BF16)}
+            else:
+                byts = N * K + M * K + 2 * M * N + 4 * (M + N)
+                a = byts / (g / 1e3) / 1e9
+                traffic = traffic_from_profile("gemm.cu", "gemm_a8w8_decode_M16_N28672_K8192.md") \
+                    if args.workload == "decode16" else None
+                rf = {"bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                      "frac": round(a / peaks["hbm_gbs"], 4), "traffic": traffic,
+                      "kernel": "k_gemm<fp8, small-M tiles> (tcgen05 kind::f8f6f4, weight stream)",
+                      "algorithmic_bytes": byts, "peak_source": "%s copy" % peaks["_src"]}
+            return rf
+
+        def extras(ms):
+            qd = {"x_per_token": {"ms": round(ms["quantize X"], 4)}}
+            qd["x_per_token"]["GB/s"] = round(q_bytes(M, K, M) / (ms["quantize X"] / 1e3) / 1e9, 1)
+            qd["x_per_token"]["frac_hbm"] = round(qd["x_per_token"]["GB/s"] / peaks["hbm_gbs"], 4)
+            if kind == "layer":
+                gb = q_bytes(N, K, N) / (ms["quantize W"] / 1e3) / 1e9
+                qd["w_per_channel"] = {"ms": round(ms["quantize W"], 4), "GB/s": round(gb, 1),
+                                       "frac_hbm": round(gb / peaks["hbm_gbs"], 4)}
+            qd["bytes"] = "algorithmic: 2 B read + 1 B write per element + 4 B per scale"
+            return {"quantize": qd, "gemm_ms": round(ms["gemm"], 4)}
+
+        l2 = "inputs larger than L2 (W %d MB, X %d MB, out %d MB); no flush" % (N * K * 2 >> 20, M * K * 2 >> 20,
+                                                                               M * N * 2 >> 20)
+        return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=h2d, d2h=M * N * 2,
+                    roofline=roofline, extras=extras, l2=l2, flush=None)
+
+    if kind == "sweep":
+        x_host = bf16_host(W.sweep(M, K, seed=rank)).view(M, K)
+        x = x_host.to(dev)
+        flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev).fill_(1)
+        sink = torch.empty((), dtype=torch.uint8, device=dev)
+        calls, outs, per = [], [], 0
+        names = {hq.PER_TENSOR: "tensor", hq.PER_TOKEN: "token", hq.PER_CHANNEL: "channel"}
+        for fmt in (hq.E4M3, hq.E5M2):
+            for g in (hq.PER_TENSOR, hq.PER_TOKEN, hq.PER_CHANNEL):
+                ns = hq.hq_scale_count(g, M, K)
+                q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+                sc = torch.empty((ns,), dtype=torch.float32, device=dev)
+                outs.append((q, sc, torch.empty((M, K), dtype=torch.uint8).pin_memory(),
+                             torch.empty((ns,), dtype=torch.float32).pin_memory()))
+                launches = 1  # at this size every mode is one launch (per-tensor / per-channel: cooperative)
+                calls.append(("%s %s" % (names[g], "e4m3" if fmt == hq.E4M3 else "e5m2"),
+                              (lambda g=g, fmt=fmt, q=q, sc=sc:
+                               hq.hq_quantize_fp8(x, fmt, g, q=q, scales=sc, stream=stream)), launches))
+                per += q_bytes(M, K, ns)
+
+        def e2e():
+            x.copy_(x_host, non_blocking=True)
+            for c, (q, sc, qh, sh) in zip(calls, outs):
+                c[1]()
+                qh.copy_(q, non_blocking=True)
+                sh.copy_(sc, non_blocking=True)
+
+        def roofline(ms):
+            label = max(ms, key=ms.get)
+            ns = {"tensor": 1, "token": M, "channel": K}[label.split()[0]]
+            a = q_bytes(M, K, ns) / (ms[label] / 1e3) / 1e9
+            return {"bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(a / peaks["hbm_gbs"], 4), "traffic": None,
+                    "kernel": "quantize %s (the slowest mode)" % label, "peak_source": "%s copy" % peaks["_src"]}
+
+        def extras(ms):
+            d = {}
+            for label, t in ms.items():
+                ns = {"tensor": 1, "token": M, "channel": K}[label.split()[0]]
+                gb = q_bytes(M, K, ns) / (t / 1e3) / 1e9
+                d[label] = {"ms": round(t, 4), "GB/s": round(gb, 1), "frac_hbm": round(gb / peaks["hbm_gbs"], 4)}
+            return {"quantize": d}
+
+        return dict(calls=calls, per_step=per, unit="GB/s", e2e=e2e, h2d=M * K * 2,
+                    d2h=sum(q.numel() + 4 * sc.numel() for q, sc, _, _ in outs), roofline=roofline,
+                    extras=extras, flush=lambda: torch.amax(flush, dim=0, out=sink),
+                    l2="L2 flushed (512 MB read) before every call; value = bytes / summed call times")
+
+    # moe / moe_bf16
+    E = cfg["E"]
+    xb, wb, off = W.moe_inputs(E, M, N, K, seed=rank)
+    x_host = bf16_host(xb).view(M, K)
+    w_host = bf16_host(wb).view(E, N, K)
+    x, w = x_host.to(dev), w_host.to(dev)
+    offd = torch.from_numpy(off).to(dev)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    flops = 2.0 * M * N * K
+    if kind == "moe":
+        xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        xs = torch.empty((M,), dtype=torch.float32, device=dev)
+        wq, ws = hq.hq_quantize_fp8(w.view(E * N, K), hq.E4M3, hq.PER_TOKEN, stream=stream)  # static weights
+        wq = wq.view(E, N, K)
+        calls = [("quantize X", lambda: hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TOKEN, q=xq, scales=xs, stream=stream), 1),
+                 ("gemm", lambda: hq.hq_grouped_gemm_a8w8(xq, wq, xs, ws, offd, out=out, stream=stream), 1)]
+        peak, dt = fp8_peak, "fp8"
+    else:
+        calls = [("gemm", lambda: hq.hq_grouped_gemm_bf16(x, w, offd, out=out, stream=stream), 1)]
+        peak, dt = peaks["bf16_tflops"], "bf16"
+
+    def e2e():
+        x.copy_(x_host, non_blocking=True)
+        for c in calls:
+            c[1]()
+        out_host.copy_(out, non_blocking=True)
+
+    def roofline(ms):
+        a = flops / (ms["gemm"] / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": round(a, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(a / peak, 4), "traffic": None,
+                "kernel": "k_gemm<%s, grouped 128x256 tiles> (tcgen05)" % dt,
+                "peak_source": "%s bf16 burst%s" % (peaks["_src"], " x 2 (nominal fp8/bf16)" if dt == "fp8" else "")}
+
+    def extras(ms):
+        d = {"gemm_ms": round(ms["gemm"], 4)}
+        if "quantize X" in ms:
+            gb = q_bytes(M, K, M) / (ms["quantize X"] / 1e3) / 1e9
+            d["quantize"] = {"x_per_token": {"ms": round(ms["quantize X"], 4), "GB/s": round(gb, 1),
+                                             "frac_hbm": round(gb / peaks["hbm_gbs"], 4)}}
+        return d
+
+    return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=M * K * 2, d2h=M * N * 2,
+                roofline=roofline, extras=extras, flush=None,
+                l2="inputs larger than L2 (X %d MB, W %d MB, out %d MB); no flush" %
+                   (M * K * 2 >> 20, E * N * K * (1 if kind == "moe" else 2) >> 20, M * N * 2 >> 20))
+
+
 def run_ours(args, rank, local_rank, world):
     import torch
     import torch.distributed as dist
 
-    import workloads as W
     import fp8_dynamic_quantization_amax_b200 as hq
 
     torch.cuda.set_device(local_rank)
@@ -164,35 +365,21 @@ def run_ours(args, rank, local_rank, world):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     cfg = WORKLOADS[args.workload]
-    M, N, K = cfg["M"], cfg["N"], cfg["K"]
     peaks, peak_src = load_peaks()
-
-    # inputs: seeded host generation; tokens differ per rank, weights replicated
-    x_bits = W.large_x(M, K, seed=rank)
-    w_bits = W.large_w(N, K)
-    x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    w_host = torch.from_numpy(w_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    x = x_host.to(dev).view(M, K)
-    w = w_host.to(dev).view(N, K)
-    xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
-    wq = torch.empty((N, K), dtype=torch.uint8, device=dev)
-    xs = torch.empty((M,), dtype=torch.float32, device=dev)
-    ws = torch.empty((N,), dtype=torch.float32, device=dev)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    peaks = dict(peaks, _src=peak_src)
     stream = torch.cuda.current_stream(dev)
+    wl = build(args, cfg, rank, dev, stream, peaks)
+    calls = wl["calls"]
 
     def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TOKEN, q=xq, scales=xs, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        hq.hq_quantize_fp8(w, hq.E4M3, hq.PER_TOKEN, q=wq, scales=ws, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
-        hq.hq_gemm_a8w8(xq, wq, xs, ws, hq.E4M3, out=out, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
+        for j, (_, fn, _) in enumerate(calls):
+            if wl["flush"] is not None:
+                wl["flush"]()
+            if ev is not None:
+                ev[2 * j].record(stream)
+            fn()
+            if ev is not None:
+                ev[2 * j + 1].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -201,7 +388,7 @@ def run_ours(args, rank, local_rank, world):
 
     clocks = ClockSampler(local_rank)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(calls))] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -216,32 +403,18 @@ def run_ours(args, rank, local_rank, world):
         dist.barrier()
     clk = clocks.stop()
     hq.hq_check_device_error()
-    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
-    qx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    qw_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    g_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    ms_by = {c[0]: statistics.mean(e[2 * j].elapsed_time(e[2 * j + 1]) for e in evs) for j, c in enumerate(calls)}
+    region = t0.elapsed_time(t1)
+    if wl["flush"] is not None:  # flushes sit between the calls: time the calls alone
+        region = sum(sum(e[2 * j].elapsed_time(e[2 * j + 1]) for j in range(len(calls))) for e in evs)
+    ms = max_over_ranks(region, world, dev)
+    scale = 1e12 if wl["unit"] == "TFLOP/s" else 1e9
+    value = wl["per_step"] * args.steps * world / (ms / 1e3) / scale
 
-    flops = 2.0 * M * N * K
-    value = whole_job_tflops(flops, args.steps, world, ms)
-    gemm_tflops = flops / (g_ms / 1e3) / 1e12
-    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
-    q_bytes_x = M * K * 3 + M * 4  # bf16 read, code write, f32 scale write
-    q_bytes_w = N * K * 3 + N * 4
-    qx_gbs = q_bytes_x / (qx_ms / 1e3) / 1e9
-    qw_gbs = q_bytes_w / (qw_ms / 1e3) / 1e9
-
-    # end to end through the C ABI with host buffers: H2D of X and W, the
-    # three kernels, D2H of out, every step
-    out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    # end to end through the C ABI with host buffers: the step's H2D copies,
+    # its kernels and the D2H of its results, every step
     e2e_steps = max(1, min(args.steps, 5))
-
-    def e2e_step():
-        x.copy_(x_host, non_blocking=True)
-        w.copy_(w_host, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
-
-    e2e_step()
+    wl["e2e"]()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -249,27 +422,26 @@ def run_ours(args, rank, local_rank, world):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        e2e_step()
+        wl["e2e"]()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_value = whole_job_tflops(flops, e2e_steps, world, e2e_ms)
+    e2e_value = wl["per_step"] * e2e_steps * world / (e2e_ms / 1e3) / scale
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(M, N, K, budget_rows=(256, 4096))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and cfg["kind"] in ("layer", "decode"):
+        mx = min(256, cfg["M"])
+        cpu = cpu_baseline(cfg["M"], cfg["N"], cfg["K"], budget_rows=(mx, min(cfg["N"], 4096 * 256 // mx)))
 
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    traffic = traffic_from_profile("gemm.cu", "gemm_a8w8_large_M16384_N28672_K8192.md") \
-        if args.workload == "large" else None
     line = {
         "metric": METRIC,
         "value": round(value, 2),
-        "unit": "TFLOP/s",
+        "unit": wl["unit"],
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -277,31 +449,19 @@ def run_ours(args, rank, local_rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)",
-        "data": "synthetic (seeded host normals; X seed = rank, W seed 1)",
-        "config": {"workload": workload_desc(args.workload, cfg), "M": M, "N": N, "K": K,
-                   "l2": "inputs larger than L2 (X %d MB, W %d MB, out %d MB); no flush" %
-                         (M * K * 2 >> 20, N * K * 2 >> 20, M * N * 2 >> 20),
-                   "parallelism": "dp%d" % world},
-        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp8_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp8_peak, 4), "traffic": traffic,
-                     "kernel": "k_gemm2<fp8, 256x256 CTA pair> (tcgen05 cta_group::2 kind::f8f6f4)",
-                     "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal fp8/bf16 dense ratio)" %
-                                    (peak_src, peaks["bf16_tflops"], FP8_OVER_BF16)},
-        "quantize": {"x_per_token": {"ms": round(qx_ms, 4), "GB/s": round(qx_gbs, 1),
-                                     "frac_hbm": round(qx_gbs / peaks["hbm_gbs"], 4)},
-                     "w_per_channel": {"ms": round(qw_ms, 4), "GB/s": round(qw_gbs, 1),
-                                       "frac_hbm": round(qw_gbs / peaks["hbm_gbs"], 4)},
-                     "bytes": "algorithmic: 2 B read + 1 B write per element + 4 B per scale",
-                     "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src},
-        "gemm_ms": round(g_ms, 4),
+        "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)" if cfg["kind"] != "moe_bf16" else "bf16 (fp32 accumulate)",
+        "data": "synthetic (seeded host generators; X seed = rank)",
+        "config": {"workload": workload_desc(args.workload, cfg), "M": cfg["M"], "N": cfg["N"], "K": cfg["K"],
+                   "l2": wl["l2"], "parallelism": "dp%d" % world},
+        "roofline": wl["roofline"](ms_by),
+        "call_ms": {k: round(v, 4) for k, v in ms_by.items()},
         "clocks": clk,
-        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": (M * K + N * K) * 2, "d2h_bytes_per_step": M * N * 2,
-                "steps": e2e_steps},
-        "gpu_launches": 3 * args.steps,
+        "e2e": {"value": round(e2e_value, 2), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
+                "d2h_bytes_per_step": wl["d2h"], "steps": e2e_steps},
+        "gpu_launches": sum(c[2] for c in calls) * args.steps,
         "cpu_baseline": cpu,
     }
+    line.update(wl["extras"](ms_by))
     print(json.dumps(line))
 
 
@@ -329,32 +489,59 @@ def cpu_baseline(M, N, K, budget_rows, seed=0):
             "seconds": round(dt, 2)}
 
 
+def cpu_sweep_sample(rows, cols, seed=0):
+    """The oracle quantizing a row sample of the sweep input in every mode;
+    returns (algorithmic bytes, seconds)."""
+    import oracle as O
+    import workloads as W
+    x = W.sweep(rows, cols, seed=seed, zero_row=rows // 2)
+    O.lib()
+    t = time.perf_counter()
+    byts = 0
+    for fmt in (O.E4M3, O.E5M2):
+        for g in (O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL):
+            _, s, _ = O.quantize(x, fmt, g)
+            byts += rows * cols * 3 + 4 * s.size
+    return byts, time.perf_counter() - t
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
     cfg = WORKLOADS[args.workload]
     M, N, K = cfg["M"], cfg["N"], cfg["K"]
-    rows = (8, 512)
-    for _ in range(args.warmup):
-        cpu_baseline(M, N, K, rows)
-    t = time.perf_counter()
-    last = None
-    for i in range(args.steps):
-        last = cpu_baseline(M, N, K, rows, seed=i)
-    dt = time.perf_counter() - t
-    flops = 2.0 * rows[0] * rows[1] * K
-    value = flops * args.steps / dt / 1e12
+    if cfg["kind"] == "sweep":
+        rows = 64
+        for _ in range(args.warmup):
+            cpu_sweep_sample(rows, K)
+        t = time.perf_counter()
+        byts = 0
+        for i in range(args.steps):
+            byts += cpu_sweep_sample(rows, K, seed=i)[0]
+        dt = time.perf_counter() - t
+        value, unit = byts / dt / 1e9, "GB/s"
+        sample = "per step: %d rows x %d cols of the sweep input, all six modes" % (rows, K)
+        dtype = "fp8 codes from bf16, f64 oracle"
+    else:
+        rows = (8, 512)
+        for _ in range(args.warmup):
+            cpu_baseline(M, N, K, rows)
+        t = time.perf_counter()
+        for i in range(args.steps):
+            cpu_baseline(M, N, K, rows, seed=i)
+        dt = time.perf_counter() - t
+        value, unit = 2.0 * rows[0] * rows[1] * K * args.steps / dt / 1e12, "TFLOP/s"
+        sample = "per step: X %d rows x W %d rows (K=%d), per-token quantize + exact GEMM" % (rows[0], rows[1], K)
+        dtype = "fp8_e4m3 codes, exact integer GEMM, f64"
     line = {
         "impl": "reference",
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(args.steps, 1), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 codes, exact integer GEMM, f64",
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype,
         "data": "synthetic", "config": {"workload": workload_desc(args.workload, cfg), "M": M, "N": N, "K": K,
                                         "parallelism": "rank 0 only"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                         "sample": "per step: X %d rows x W %d rows of the workload (K=%d), quantize + exact GEMM"
-                                   % (rows[0], rows[1], K)},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": "the CPU oracle timed as it stands; no reference implementation exists for this hardware",
     }
     print(json.dumps(line))

@@ -543,7 +543,8 @@ __global__ void __launch_bounds__(kThreads) k_tensor_cast(
 // first, and then the part held in shared memory.  DRAM sees x about once.
 // Workspace words: [0] amax bits, [1] arrivals, [2] departures, [3]
 // non-finite flag; the last CTA to leave returns all four to zero.
-constexpr int kFusedThreads = 512;
+constexpr int kFusedThreads = 1024;
+constexpr int kFusedUnroll = 4;  // 16-byte loads in flight per thread (64 registers at 1024 threads)
 
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
@@ -582,7 +583,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
     unsigned* __restrict__ err_word) {
   constexpr int VEC = Dt<DT>::kVec;
   constexpr int T = kFusedThreads;
-  constexpr int U = kUnrollFlat;
+  constexpr int U = kFusedUnroll;
   extern __shared__ __align__(128) uint4 held[];
   __shared__ __align__(8) uint64_t bar;
   __shared__ float sh[T / 32];
@@ -892,6 +893,219 @@ __global__ void __launch_bounds__(kThreads) k_channel_cast(
   }
 }
 
+// ------------------------------------------------ per-channel, one launch
+// Cooperative, one CTA per SM.  The matrix is cut into S column strips of
+// kStripVecs 16-byte column vectors and B row bands (S * B <= SMs); CTA
+// (strip, band) owns that tile.  Thread t owns column vector t % kStripVecs
+// of the strip and rows t / kStripVecs, + kRowLanes, ... of the band.  The
+// band's first rows of the strip are bulk-copied into shared memory and kept;
+// the rest stream through registers with an L2 evict_last hint.  The row
+// lanes' maxima meet in shared memory and one atomicMax per column per CTA
+// folds them into the workspace, B atomics per column.  After a grid barrier
+// each CTA derives its strip's multipliers into shared memory and casts its
+// tile: streamed rows again (newest first, evict_first), then held rows.
+// Workspace: header [0] arrivals, [1] non-finite flag, [2] departures;
+// amax bits[cols].  The last CTA to leave returns them to zero.
+constexpr int kStripVecs = 256;
+constexpr int kRowLanes = kFusedThreads / kStripVecs;
+constexpr int64_t kMaxHeldRows = 128;  // bulk copies per CTA (one per held row)
+
+__device__ __forceinline__ bool grid_barrier(uint32_t* arrivals, unsigned* err_word) {
+  const unsigned long long t0 = ptx::globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire_u32(arrivals) >= gridDim.x) return true;
+    if ((it & 15u) == 15u && ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
+      atomicOr(err_word, kDevErrTimeout);
+      return false;
+    }
+    __nanosleep(100);
+  }
+}
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
+    const void* __restrict__ x, int64_t rows, int64_t cols, int strips, int64_t band_rows, int64_t held_rows,
+    uint8_t* __restrict__ q, uint32_t* __restrict__ header, uint32_t* __restrict__ ws_amax, float fmax,
+    float* __restrict__ scales, float* __restrict__ amax_out, unsigned* __restrict__ err_word) {
+  constexpr int VEC = Dt<DT>::kVec;
+  constexpr int T = kFusedThreads;
+  constexpr int U = kFusedUnroll;
+  constexpr int RL = kRowLanes;
+  constexpr int SC = kStripVecs * VEC;  // columns per strip
+  extern __shared__ __align__(128) uint8_t fsm[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_flags;  // bit 0: non-finite somewhere, bit 1: give up, bit 2: last to leave
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const int lv = tid % kStripVecs;  // column vector within the strip
+  const int rl = tid / kStripVecs;  // row lane
+  const int64_t nvc = cols / VEC;
+  const int strip = static_cast<int>(blockIdx.x % strips);
+  const int64_t band = blockIdx.x / strips;
+  const int64_t c0 = static_cast<int64_t>(strip) * kStripVecs;
+  const int64_t sv = min(static_cast<int64_t>(kStripVecs), nvc - c0);  // vectors in this strip
+  const int64_t r0 = min(rows, band * band_rows);
+  const int64_t r1 = min(rows, r0 + band_rows);
+  const int64_t nh = min(r1 - r0, held_rows);
+  const int64_t rs0 = r0 + nh;  // streamed rows [rs0, r1)
+  float* red = reinterpret_cast<float*>(fsm);  // [RL][SC] row-lane maxima; later the strip's multipliers
+  uint4* held = reinterpret_cast<uint4*>(fsm + RL * SC * 4);  // [nh][sv]
+  const uint4* xv = static_cast<const uint4*>(x);  // row r, column vector c: xv[r * nvc + c]
+
+  if (tid == 0) {
+    abort_flag = 0;
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbarrier_init();
+    if (nh > 0 && sv > 0) {
+      const uint64_t pol = policy_evict_first();
+      const uint32_t row_bytes = static_cast<uint32_t>(sv * 16);
+      ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nh) * row_bytes);
+      for (int64_t i = 0; i < nh; ++i) bulk_load_hint(held + i * sv, xv + (r0 + i) * nvc + c0, row_bytes, &bar, pol);
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 1: column maxima of the tile
+  const uint64_t keep = policy_evict_last();
+  const bool active = lv < sv;
+  const int64_t c = c0 + lv;
+  uint32_t acc[4] = {0u, 0u, 0u, 0u};
+  if (active) {
+    int64_t r = rs0 + rl;
+    for (; r + (U - 1) * RL < r1; r += U * RL) {
+      uint4 u[U];
+#pragma unroll
+      for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + (r + j * RL) * nvc + c, keep);
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        acc[0] = Dt<DT>::lmax(acc[0], Dt<DT>::mag(u[j].x));
+        acc[1] = Dt<DT>::lmax(acc[1], Dt<DT>::mag(u[j].y));
+        acc[2] = Dt<DT>::lmax(acc[2], Dt<DT>::mag(u[j].z));
+        acc[3] = Dt<DT>::lmax(acc[3], Dt<DT>::mag(u[j].w));
+      }
+    }
+    for (; r < r1; r += RL) {
+      const uint4 u = ld_hint(xv + r * nvc + c, keep);
+      acc[0] = Dt<DT>::lmax(acc[0], Dt<DT>::mag(u.x));
+      acc[1] = Dt<DT>::lmax(acc[1], Dt<DT>::mag(u.y));
+      acc[2] = Dt<DT>::lmax(acc[2], Dt<DT>::mag(u.z));
+      acc[3] = Dt<DT>::lmax(acc[3], Dt<DT>::mag(u.w));
+    }
+  }
+  bool landed = true;
+  if (nh > 0 && sv > 0) landed = ptx::mbar_wait(&bar, 0, &abort_flag, err_word, kDevErrTimeout);
+  if (active && landed)
+    for (int64_t i = rl; i < nh; i += RL) {
+      const uint4 u = held[i * sv + lv];
+      acc[0] = Dt<DT>::lmax(acc[0], Dt<DT>::mag(u.x));
+      acc[1] = Dt<DT>::lmax(acc[1], Dt<DT>::mag(u.y));
+      acc[2] = Dt<DT>::lmax(acc[2], Dt<DT>::mag(u.z));
+      acc[3] = Dt<DT>::lmax(acc[3], Dt<DT>::mag(u.w));
+    }
+  float am[VEC];
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) am[j] = 0.0f;
+  bool nf = false;
+  if (active) {
+    if (!Dt<DT>::nonfinite(Dt<DT>::lmax(Dt<DT>::lmax(acc[0], acc[1]), Dt<DT>::lmax(acc[2], acc[3])))) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int ln = 0; ln < Dt<DT>::kLanes; ++ln) am[w * Dt<DT>::kLanes + ln] = Dt<DT>::lane_value(acc[w], ln);
+    } else {  // rare: finite-only maxima of this lane's rows on the exact path
+      nf = true;
+      for (int64_t r = r0 + rl; r < r1; r += RL) {
+        float f[VEC];
+        Dt<DT>::unpack((r < rs0 && landed) ? held[(r - r0) * sv + lv] : __ldg(xv + r * nvc + c), f);
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) am[j] = fmaxf(am[j], finite_abs(f[j]));
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) red[rl * SC + lv * VEC + j] = am[j];
+  nf = __syncthreads_or(nf);
+  for (int64_t e = tid; e < sv * VEC; e += T) {  // one atomicMax per column of the strip
+    float a = red[e];
+#pragma unroll
+    for (int l = 1; l < RL; ++l) a = fmaxf(a, red[l * SC + e]);
+    atomicMax(&ws_amax[c0 * VEC + e], __float_as_uint(a));
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    if (nf) atomicOr(&header[1], 1u);
+    __threadfence();
+    atomicAdd(&header[0], 1u);
+    const bool ok = !abort_flag && grid_barrier(&header[0], err_word);
+    s_flags = (__ldcg(&header[1]) != 0u ? 1 : 0) | (ok ? 0 : 2);
+  }
+  __syncthreads();
+  const bool ok = !(s_flags & 2);
+  // the strip's multipliers; the CTAs of band 0 publish the scales
+  float* m_s = red;
+  if (ok)
+    for (int64_t e = tid; e < sv * VEC; e += T) {
+      const int64_t col = c0 * VEC + e;
+      const float a = __uint_as_float(__ldcg(&ws_amax[col]));
+      const float m = multiplier(a, fmax);
+      m_s[e] = m;
+      if (band == 0) {
+        scales[col] = __fdiv_rn(1.0f, m);
+        if (amax_out) amax_out[col] = a;
+      }
+    }
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const bool last = atomicAdd(&header[2], 1u) == gridDim.x - 1;
+    s_flags |= last ? 4 : 0;
+  }
+  __syncthreads();
+  if (s_flags & 4) {  // every CTA has read the maxima: clear them and the header
+    for (int64_t col = tid; col < cols; col += T) ws_amax[col] = 0u;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      atomicExch(&header[1], 0u);
+      atomicExch(&header[0], 0u);
+      atomicExch(&header[2], 0u);
+    }
+  }
+  if (!ok) {  // the error word says so
+    if (tid == 0 && nh > 0 && sv > 0 && !landed) {
+      int dummy = 0;
+      ptx::mbar_wait(&bar, 0, &dummy, nullptr, 0, ptx::kDrainLimitNs);
+    }
+    return;
+  }
+
+  // ---- phase 2: cast the tile, this lane's streamed rows from the end backwards
+  if (!active) return;
+  const uint64_t drop = policy_evict_first();
+  float m[VEC];
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) m[j] = m_s[lv * VEC + j];
+  auto cast_tile = [&](auto fast) {
+    constexpr bool FAST = decltype(fast)::value;
+    if (r1 - 1 >= rs0 + rl) {
+      int64_t r = rs0 + rl + ((r1 - 1 - rs0 - rl) / RL) * RL;  // this lane's last streamed row
+      for (; r - (U - 1) * RL >= rs0; r -= U * RL) {
+        uint4 u[U];
+#pragma unroll
+        for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + (r - j * RL) * nvc + c, drop);
+#pragma unroll
+        for (int j = 0; j < U; ++j) vec_store_m<DT, FMT, FAST>(q + (r - j * RL) * cols + c * VEC, u[j], m);
+      }
+      for (; r >= rs0; r -= RL) vec_store_m<DT, FMT, FAST>(q + r * cols + c * VEC, ld_hint(xv + r * nvc + c, drop), m);
+    }
+    for (int64_t i = rl; i < nh; i += RL) vec_store_m<DT, FMT, FAST>(q + (r0 + i) * cols + c * VEC, held[i * sv + lv], m);
+  };
+  if (!(s_flags & 1)) cast_tile(std::true_type{});
+  else cast_tile(std::false_type{});
+}
+
 // ------------------------------------------------------------------ delayed
 // Ring: [hist[len] | scale | counter].  Workspace word [0]: amax accumulator.
 // One pass: cast with the ring's multiplier while reducing amax.  A thread
@@ -1092,6 +1306,41 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
     else
       k_tensor_cast<DT, FMT, false><<<grid, kThreads, 0, a.stream>>>(a.x, n, ws, a.q);
     return cudaGetLastError();
+  }
+
+  if (row_vec && n * Dt<DT>::kSize >= kFusedMinBytes && device_error_word() != nullptr) {
+    const int sms = device_sm_count(dev);
+    const int64_t nvc = a.cols / VEC;
+    const int64_t strips = (nvc + kStripVecs - 1) / kStripVecs;
+    if (strips <= sms) {
+      static cudaError_t attr = cudaFuncSetAttribute(k_channel_fused<DT, FMT>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     static_cast<int>(kFusedHeldBytes));
+      if (attr != cudaSuccess) return attr;
+      int64_t bands = std::max<int64_t>(1, std::min<int64_t>(sms / strips, a.rows));
+      int64_t band = (a.rows + bands - 1) / bands;
+      bands = (a.rows + band - 1) / band;
+      const int64_t fixed = static_cast<int64_t>(kRowLanes) * kStripVecs * VEC * 4;
+      const int64_t strip_bytes = std::min<int64_t>(nvc, kStripVecs) * 16;
+      int64_t held = std::min<int64_t>({band, (kFusedHeldBytes - fixed) / strip_bytes, kMaxHeldRows});
+      const size_t smem = static_cast<size_t>(fixed + held * strip_bytes);
+      uint32_t* header = static_cast<uint32_t*>(a.ws);
+      uint32_t* ws_amax = header + 4;
+      const void* x = a.x;
+      int64_t rows = a.rows, cols = a.cols;
+      int nstrips = static_cast<int>(strips);
+      uint8_t* q = a.q;
+      float f = fmax;
+      float* scales = a.scales;
+      float* amax_out = a.amax_out;
+      unsigned* err = device_error_word();
+      void* args[] = {(void*)&x, (void*)&rows, (void*)&cols, (void*)&nstrips, (void*)&band, (void*)&held,
+                      (void*)&q, (void*)&header, (void*)&ws_amax, (void*)&f, (void*)&scales, (void*)&amax_out,
+                      (void*)&err};
+      return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_channel_fused<DT, FMT>),
+                                         dim3(static_cast<unsigned>(strips * bands)), dim3(kFusedThreads), args, smem,
+                                         a.stream);
+    }
   }
 
   // per-channel, two phases

@@ -116,27 +116,33 @@ def test_workspace_returned_to_zero():
         assert (host(ws) == 0).all()
 
 
-# Per-tensor inputs of 4 MB and more take the single-launch kernel (one CTA
-# per SM, part of each CTA's range held in shared memory, a grid barrier
-# between amax and cast).  Ragged element tails, NaN/Inf (exact path) and a
-# finite input (fast path); the workspace is zero again after each call.
-FUSED_CASES = [((1025, 2051), "f32"), ((2048, 1100), "bf16"), ((1501, 1401), "f16")]
+# Per-tensor and per-channel inputs of 4 MB and more take single-launch
+# kernels (one cooperative CTA per SM, part of each CTA's range held in shared
+# memory, a grid barrier between amax and cast).  Ragged element tails
+# (per-tensor), a column-vector count just past one per thread and the widest
+# supported rows (per-channel), fewer rows than SMs, NaN/Inf (exact path) and
+# a finite input (fast path); the workspace is zero again after each call.
+FUSED_CASES = {
+    O.PER_TENSOR: [((1025, 2051), "f32"), ((2048, 1100), "bf16"), ((1501, 1401), "f16")],
+    O.PER_CHANNEL: [((1025, 2052), "f32"), ((2048, 1104), "bf16"), ((1501, 1400), "f16"), ((130, 32768), "bf16")],
+}
 
 
+@pytest.mark.parametrize("gran", [O.PER_TENSOR, O.PER_CHANNEL])
 @pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
-def test_per_tensor_single_launch(fmt):
-    cases = [make_input(shape, dtype, seed=4000 + i) for i, (shape, dtype) in enumerate(FUSED_CASES)]
+def test_single_launch_two_phase(gran, fmt):
+    cases = [make_input(shape, dtype, seed=4000 + i) for i, (shape, dtype) in enumerate(FUSED_CASES[gran])]
     rng = np.random.default_rng(4100 + fmt)
     xf = (rng.standard_normal((2048, 2048)) * 3.0).astype(np.float32)
     b = W.f32_to_bf16_bits(xf)
     cases.append((b, dev_bf16(b)))
     for xh, xd in cases:
         rows, cols = xd.shape
-        ws = torch.zeros(H.hq_quantize_workspace_bytes(O.PER_TENSOR, rows, cols), dtype=torch.uint8, device="cuda")
-        qo, so, ao = O.quantize(xh, fmt, O.PER_TENSOR)
+        ws = torch.zeros(H.hq_quantize_workspace_bytes(gran, rows, cols), dtype=torch.uint8, device="cuda")
+        qo, so, ao = O.quantize(xh, fmt, gran)
         for _ in range(2):
-            a = torch.full((1,), -7.0, dtype=torch.float32, device="cuda")
-            q, s = H.hq_quantize_fp8(xd, fmt, O.PER_TENSOR, amax_out=a, workspace=ws)
+            a = torch.full((so.size,), -7.0, dtype=torch.float32, device="cuda")
+            q, s = H.hq_quantize_fp8(xd, fmt, gran, amax_out=a, workspace=ws)
             torch.cuda.synchronize()
             np.testing.assert_array_equal(host(q), qo, err_msg="codes %s %s" % (xd.shape, xd.dtype))
             np.testing.assert_array_equal(host(s).view(np.uint32), so.view(np.uint32))
