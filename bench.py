@@ -1,7 +1,7 @@
 """Benchmark of the dynamic-FP8 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large|large4096|decode1|decode16|decode128|sweep|moe|moe_bf16]
+                    [--workload large|large4096|large8192|decode1|decode16|decode128|sweep|moe|moe_bf16]
 
 Default workload (the large a8w8 GEMM layer): X bf16 [16384, 8192] ~N(0,1),
 W bf16 [28672, 8192] ~N(0,0.02).  One step = per-token E4M3 quantize of X,
@@ -61,6 +61,7 @@ def dist_env():
 WORKLOADS = {
     "large": dict(kind="layer", M=16384, N=28672, K=8192),
     "large4096": dict(kind="layer", M=4096, N=28672, K=8192),
+    "large8192": dict(kind="layer", M=8192, N=28672, K=8192),
     "decode1": dict(kind="decode", M=1, N=28672, K=8192),
     "decode16": dict(kind="decode", M=16, N=28672, K=8192),
     "decode128": dict(kind="decode", M=128, N=28672, K=8192),
@@ -226,7 +227,8 @@ def build(args, cfg, rank, dev, stream, peaks):
                     if args.workload == "large" else None
                 rf = {"bound": "tensor", "achieved": round(a, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                       "frac": round(a / fp8_peak, 4), "traffic": traffic,
-                      "kernel": "k_gemm2<fp8, 256x256 CTA pair> (tcgen05 cta_group::2 kind::f8f6f4)",
+                      "kernel": "k_gemm2<fp8, %s CTA-pair tile> (tcgen05 cta_group::2 kind::f8f6f4)" %
+                                ("256x512" if M >= 8192 and N % 512 == 0 else "256x256"),
                       "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal fp8/bf16 dense ratio)" %
                                      (peaks["_src"], peaks["bf16_tflops"], FP8_OVER_BF16)}
             else:
@@ -336,7 +338,7 @@ def build(args, cfg, rank, dev, stream, peaks):
         a = flops / (ms["gemm"] / 1e3) / 1e12
         return {"bound": "tensor", "achieved": round(a, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
                 "frac": round(a / peak, 4), "traffic": None,
-                "kernel": "k_gemm<%s, grouped 128x256 tiles> (tcgen05)" % dt,
+                "kernel": "k_gemm2<%s, grouped 256x256 CTA-pair tiles> (tcgen05 cta_group::2)" % dt,
                 "peak_source": "%s bf16 burst%s" % (peaks["_src"], " x 2 (nominal fp8/bf16)" if dt == "fp8" else "")}
 
     def extras(ms):

@@ -40,7 +40,7 @@ namespace {
 
 constexpr int kBM = 128;            // tile rows (MMA M)
 constexpr int kBKBytes = 128;       // K bytes per stage = one 128B swizzle row
-constexpr int kGemmThreads = 192;   // CTA-pair kernel: TMA, MMA, 4 epilogue warps
+constexpr int kGemmThreads = 320;   // CTA-pair kernel: TMA, MMA, 8 epilogue warps
 constexpr int kGemm1Threads = 320;  // 1-CTA kernel: TMA, MMA, 8 epilogue warps
 constexpr int kMaxExperts = 1024;
 constexpr unsigned long long kDrainLimitNs = ptx::kDrainLimitNs;
@@ -154,14 +154,23 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, 
 
 // TMA tile store shared -> global (clipped at the tensor's bounds), and its
 // bulk-group bookkeeping.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
-               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+// The output tile store carries an L2 evict_first policy: nothing reads the
+// output again in this kernel, and letting L2 write it back early (while the
+// main loop leaves DRAM mostly idle) keeps dirty lines from piling up for the
+// next kernel to flush.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int c0, int c1, uint64_t pol) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+                   map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "l"(pol)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// at most one committed group may still be reading shared memory
-__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// every committed group has finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_le0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -179,7 +188,10 @@ struct Tile {
   int expert;
 };
 
-template <int BN>
+// Tile t of the persistent loop -> rows, columns and expert.  Dense: TM-row
+// tiles rasterised in groups of group_m M-tiles.  Grouped: the per-expert
+// tile prefix (built by build_tile_prefix) is searched for t's expert.
+template <int TM, int BN>
 __device__ __forceinline__ Tile decode_tile(int t, const Params& p, const int* prefix, const int* starts) {
   Tile T;
   if (p.offsets == nullptr) {
@@ -189,8 +201,8 @@ __device__ __forceinline__ Tile decode_tile(int t, const Params& p, const int* p
     const int gm = min(p.group_m, p.m_tiles - g * p.group_m);
     const int mt = g * p.group_m + within % gm;
     const int nt = within / gm;
-    T.row_lo = mt * kBM;
-    T.row_hi = min(p.M, T.row_lo + kBM);
+    T.row_lo = mt * TM;
+    T.row_hi = min(p.M, T.row_lo + TM);
     T.a_row = T.row_lo;
     T.col0 = nt * BN;
     T.b_row = T.col0;
@@ -205,14 +217,39 @@ __device__ __forceinline__ Tile decode_tile(int t, const Params& p, const int* p
     const int local = t - prefix[e];
     const int mt = local / p.n_tiles;
     const int nt = local - mt * p.n_tiles;
-    T.row_lo = starts[e] + mt * kBM;
-    T.row_hi = min(starts[e + 1], T.row_lo + kBM);
+    T.row_lo = starts[e] + mt * TM;
+    T.row_hi = min(starts[e + 1], T.row_lo + TM);
     T.a_row = T.row_lo;
     T.col0 = nt * BN;
     T.b_row = e * p.N + T.col0;
     T.expert = e;
   }
   return T;
+}
+
+// One thread: clamp the device offsets into [prev, M], record each expert's
+// first row and the prefix of its TM-row x BN tiles.  Malformed offsets are
+// flagged in the device error word (once per launch).
+template <int TM>
+__device__ void build_tile_prefix(const Params& p, int* prefix, int* starts) {
+  bool bad = false;
+  int prev = 0;
+  int acc = 0;
+  for (int e = 0; e <= p.E; ++e) {
+    int o = p.offsets[e];
+    if ((e == 0 && o != 0) || (e == p.E && o != p.M) || o < prev || o > p.M) bad = true;
+    o = min(max(o, prev), p.M);
+    if (e == 0) o = 0;
+    starts[e] = o;
+    if (e > 0) {
+      const int cnt = o - prev;
+      prefix[e - 1] = acc;
+      acc += ((cnt + TM - 1) / TM) * p.n_tiles;
+    }
+    prev = o;
+  }
+  prefix[p.E] = acc;
+  if (bad && blockIdx.x == 0) atomicOr(&g_device_error, kDevErrBadOffsets);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -278,27 +315,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
-  if (threadIdx.x == 32 && p.offsets != nullptr) {
-    // Clamp the device offsets into [prev, M] and build the tile prefix.
-    bool bad = false;
-    int prev = 0;
-    int acc = 0;
-    for (int e = 0; e <= p.E; ++e) {
-      int o = p.offsets[e];
-      if ((e == 0 && o != 0) || (e == p.E && o != p.M) || o < prev || o > p.M) bad = true;
-      o = min(max(o, prev), p.M);
-      if (e == 0) o = 0;
-      row_start[e] = o;
-      if (e > 0) {
-        const int cnt = o - prev;
-        tile_prefix[e - 1] = acc;
-        acc += ((cnt + kBM - 1) / kBM) * p.n_tiles;
-      }
-      prev = o;
-    }
-    tile_prefix[p.E] = acc;
-    if (bad && blockIdx.x == 0) atomicOr(&g_device_error, kDevErrBadOffsets);
-  }
+  if (threadIdx.x == 32 && p.offsets != nullptr) build_tile_prefix<kBM>(p, tile_prefix, row_start);
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_b) : "memory");
@@ -327,7 +344,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       for (int s = 0; s < STAGES; ++s) { armed[s] = false; armed_parity[s] = 0; }
       bool stop = false;
       for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
-        const Tile T = decode_tile<BN>(t, p, tile_prefix, row_start);
+        const Tile T = decode_tile<kBM, BN>(t, p, tile_prefix, row_start);
         for (int kb = 0; kb < p.nkb; kb += KPS) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { stop = true; break; }
           const int nsub = min(KPS, p.nkb - kb);
@@ -411,13 +428,14 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     const int half = ew >> 2;
     uint8_t* sb = sOut + ew * 2048;
     float* wsh = sWs + ew * kMyChunks * 32;
+    const uint64_t out_pol = l2_evict_first_policy();
     int i = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int acc = i & 1;
       const uint32_t acc_phase = (i >> 1) & 1;
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag)) break;
       tc_fence_after();
-      const Tile T = decode_tile<BN>(t, p, tile_prefix, row_start);
+      const Tile T = decode_tile<kBM, BN>(t, p, tile_prefix, row_start);
       const int row0 = T.row_lo + quad * 32;
       const int row = row0 + lane;
       const bool vrow = row < T.row_hi;
@@ -464,7 +482,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tm_out, sb, n0, row0);
+            tma_store_2d(&tm_out, sb, n0, row0, out_pol);
             bulk_commit_group();
           }
         } else if (vrow) {
@@ -677,35 +695,46 @@ __device__ __forceinline__ void mma_issue_pair(uint32_t d_tmem, uint64_t adesc, 
   }
 }
 
+// BN = 256 * NSUB columns per pair tile.  NSUB = 1: two accumulators, so tile
+// i's epilogue overlaps tile i+1's main loop.  NSUB = 2: each K step issues two
+// N=256 MMAs against the same A stage (a quarter fewer operand bytes per
+// flop) into one 512-column accumulator; the epilogue then does not overlap.
 template <int KIND, int BN, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_gemm2(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
             const __grid_constant__ CUtensorMap tm_out, const Params p) {
-  constexpr int kABytes = 128 * kBKBytes;        // this CTA's 128 rows of A
-  constexpr int kBBytes = (BN / 2) * kBKBytes;   // this CTA's BN/2 rows of B
+  static_assert(BN == 256 || BN == 512, "pair tile width: 256 or 512 columns");
+  constexpr int NSUB = BN / 256;
+  constexpr int kABytes = 128 * kBKBytes;  // this CTA's 128 rows of A
+  constexpr int kBSub = 128 * kBKBytes;    // this CTA's 128 rows of one 256-column sub-tile of B
+  constexpr int kBBytes = NSUB * kBSub;
   constexpr int kStageBytes = kABytes + kBBytes;
   constexpr int kKElems = (KIND == 0) ? 128 : 64;
-  constexpr uint32_t kTmemCols = (2 * BN <= 256) ? 256u : 512u;
-  constexpr uint32_t kAccStride = (2 * BN <= 256) ? BN : 256u;  // TMEM columns between the two accumulators
+  constexpr int kAccs = (NSUB == 1) ? 2 : 1;  // accumulators in TMEM
+  constexpr uint32_t kTmemCols = 512u;
+  constexpr uint32_t kAccStride = 256u;
   constexpr int kPrefetch = 2 * STAGES;  // L2 prefetch distance for B, in K blocks
+  constexpr int kMyChunks = BN / 64;     // 32-column chunks per epilogue warp (two warps per quadrant)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t tfull_bar[2];
-  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t tfull_bar[kAccs];
+  __shared__ __align__(8) uint64_t tempty_bar[kAccs];
   __shared__ __align__(8) uint64_t final_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int tile_prefix[kMaxExperts + 1];
+  __shared__ int row_start[kMaxExperts + 1];
 
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * kABytes;
-  // epilogue: per warp two 32 x 32 bf16 staging tiles (2 KB each) for TMA
-  // stores, and the tile's BN column scales
+  // epilogue: one 32 x 32 bf16 staging tile (2 KB) per warp for TMA stores,
+  // and each warp's column scales
   uint8_t* sOut = smem + STAGES * kStageBytes;
-  float* sWs = reinterpret_cast<float*>(sOut + 4 * 2 * 2048);
+  float* sWs = reinterpret_cast<float*>(sOut + 8 * 2048);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -716,14 +745,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full_bar[s], 1);   // leader: its producer's arrive + both CTAs' bytes
       mbar_init(&empty_bar[s], 1);  // one multicast commit per use
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kAccs; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 8);  // leader: 4 epilogue warps x 2 CTAs
+      mbar_init(&tempty_bar[a], 16);  // leader: 8 epilogue warps x 2 CTAs
     }
     mbar_init(&final_bar, 1);
     abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
+  // each CTA of the pair builds the same tile prefix from the device offsets
+  if (threadIdx.x == 32 && p.offsets != nullptr) build_tile_prefix<256>(p, tile_prefix, row_start);
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_b) : "memory");
@@ -741,7 +772,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = tmem_slot;
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
-  const int total = p.m_tiles * p.n_tiles;  // tiles of 256 x BN
+  const int total = (p.offsets != nullptr) ? tile_prefix[p.E] : p.m_tiles * p.n_tiles;  // tiles of 256 x BN
 
   if (warp == 0) {
     if (lane == 0) {
@@ -751,24 +782,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t pend_mask = 0, pend_parity = 0;
       bool stop = false;
       for (int t = cluster; t < total && !stop; t += nclusters) {
-        const int per_group = p.group_m * p.n_tiles;
-        const int g = t / per_group;
-        const int within = t - g * per_group;
-        const int gm = min(p.group_m, p.m_tiles - g * p.group_m);
-        const int mt = g * p.group_m + within % gm;
-        const int nt = within / gm;
-        const int a_row = mt * 256 + static_cast<int>(rank) * 128;
-        const int b_row = nt * BN + static_cast<int>(rank) * (BN / 2);
+        const Tile T = decode_tile<256, BN>(t, p, tile_prefix, row_start);
+        // rows past the tile's own (another expert's, or past M) only reach
+        // accumulator rows that are never stored
+        const int a_row = T.a_row + static_cast<int>(rank) * 128;
+        const int b_row = T.b_row + static_cast<int>(rank) * 128;  // + 256 per sub-tile
         for (int kb = 0; kb < p.nkb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { stop = true; break; }
           const uint32_t full_leader = mapa_shared(smem_u32(&full_bar[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStageBytes);
           tma_load_2d_pair(sA + stage * kABytes, &tm_a, full_leader, kb * kKElems, a_row);
-          tma_load_2d_pair(sB + stage * kBBytes, &tm_b, full_leader, kb * kKElems, b_row);
+#pragma unroll
+          for (int s = 0; s < NSUB; ++s)
+            tma_load_2d_pair(sB + stage * kBBytes + s * kBSub, &tm_b, full_leader, kb * kKElems, b_row + 256 * s);
           // The clusters that share this B tile run in step, so its DRAM
           // latency would stall all of them at once: ask L2 for the B tile
           // kPrefetch blocks ahead.
-          if (kb + kPrefetch < p.nkb) tma_prefetch_2d(&tm_b, (kb + kPrefetch) * kKElems, b_row);
+          if (kb + kPrefetch < p.nkb) {
+#pragma unroll
+            for (int s = 0; s < NSUB; ++s) tma_prefetch_2d(&tm_b, (kb + kPrefetch) * kKElems, b_row + 256 * s);
+          }
           pend_mask |= 1u << stage;
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -790,8 +823,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       bool stop = false;
       int i = 0;
       for (int t = cluster; t < total && !stop; t += nclusters, ++i) {
-        const int acc = i & 1;
-        const uint32_t acc_phase = (i >> 1) & 1;
+        const int acc = i % kAccs;
+        const uint32_t acc_phase = (i / kAccs) & 1;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
@@ -800,10 +833,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           if (lane == 0) {
             const uint64_t ad = smem_desc(smem_u32(sA + stage * kABytes));
-            const uint64_t bd = smem_desc(smem_u32(sB + stage * kBBytes));
 #pragma unroll
             for (int k = 0; k < kBKBytes / 32; ++k)
-              mma_issue_pair<KIND>(d_tmem, ad + 2u * k, bd + 2u * k, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+              for (int s = 0; s < NSUB; ++s) {
+                const uint64_t bd = smem_desc(smem_u32(sB + stage * kBBytes + s * kBSub));
+                mma_issue_pair<KIND>(d_tmem + 256u * s, ad + 2u * k, bd + 2u * k, p.idesc,
+                                     (kb > 0 || k > 0) ? 1u : 0u);
+              }
             tc_commit_pair(&empty_bar[stage]);
             issued = true;
           }
@@ -823,70 +860,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // -------------------------------------------------------- epilogue
-    // Warp e (quadrant `quad` of TMEM) owns 32 rows of this CTA's half of
-    // the tile.  Per 32-column chunk it scales, rounds to bf16, writes the
-    // 32 x 32 chunk to a staging tile and stores it with one TMA store
-    // (clipped at M and N); two staging tiles alternate.
+    // Eight warps: warp w reads TMEM lane quadrant w % 4 (32 rows of this
+    // CTA's half of the tile); the two warps of a quadrant take alternate
+    // 32-column chunks.  Per chunk a warp scales, rounds to bf16 and stores
+    // through a staging tile with one TMA store (clipped at M and N); a
+    // 32-row group that straddles an expert boundary uses masked 16-byte
+    // stores.
     const int ew = warp - 2;
     const int quad = warp & 3;
-    uint8_t* stage_out = sOut + ew * 2 * 2048;
-    float* wsh = sWs + ew * BN;
-    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
-    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
+    const int half = ew >> 2;
+    uint8_t* sb = sOut + ew * 2048;
+    float* wsh = sWs + ew * kMyChunks * 32;
+    const uint64_t out_pol = l2_evict_first_policy();
+    uint32_t tempty_leader[kAccs];
+#pragma unroll
+    for (int a = 0; a < kAccs; ++a) tempty_leader[a] = mapa_shared(smem_u32(&tempty_bar[a]), 0);
     int i = 0;
-    uint32_t chunk = 0;
     for (int t = cluster; t < total; t += nclusters, ++i) {
-      const int acc = i & 1;
-      const uint32_t acc_phase = (i >> 1) & 1;
+      const int acc = i % kAccs;
+      const uint32_t acc_phase = (i / kAccs) & 1;
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag)) break;
       tc_fence_after();
-      const int per_group = p.group_m * p.n_tiles;
-      const int g = t / per_group;
-      const int within = t - g * per_group;
-      const int gm = min(p.group_m, p.m_tiles - g * p.group_m);
-      const int mt = g * p.group_m + within % gm;
-      const int nt = within / gm;
-      const int row0 = mt * 256 + static_cast<int>(rank) * 128 + quad * 32;  // this warp's first row
+      const Tile T = decode_tile<256, BN>(t, p, tile_prefix, row_start);
+      const int row0 = T.row_lo + static_cast<int>(rank) * 128 + quad * 32;  // this warp's first row
       const int row = row0 + lane;
-      const int col0 = nt * BN;
+      const bool vrow = row < T.row_hi;
+      // rows past M are clipped by the tensor map; rows of another expert are not
+      const bool tma_ok = row0 < T.row_hi && (p.offsets == nullptr || row0 + 32 <= T.row_hi);
       float xsv = 0.0f;
-      if (row < p.M) xsv = (KIND == 0) ? __ldg(p.xs + (p.xs_bcast ? 0 : row)) : 1.0f;
+      if (vrow) xsv = (KIND == 0) ? __ldg(p.xs + (p.xs_bcast ? 0 : row)) : 1.0f;
       if (KIND == 0) {
-        for (int j = lane; j < BN; j += 32) {
-          const int n = col0 + j;
-          wsh[j] = (n < p.N) ? __ldg(p.ws + (p.ws_bcast ? 0 : n)) : 0.0f;
+        const float* wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
+#pragma unroll 1
+        for (int j = 0; j < kMyChunks; ++j) {
+          const int n = T.col0 + (half + 2 * j) * 32 + lane;
+          wsh[j * 32 + lane] = (n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f;
         }
       } else {
-        for (int j = lane; j < BN; j += 32) wsh[j] = 1.0f;
+        for (int j = 0; j < kMyChunks; ++j) wsh[j * 32 + lane] = 1.0f;
       }
       __syncwarp();
+      uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32, ++chunk) {
+      for (int j = 0; j < kMyChunks; ++j) {
+        const int c = (half + 2 * j) * 32;  // chunk's first column within the tile
         uint32_t v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN + c), v);
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride +
+                      static_cast<uint32_t>(c),
+                  v);
+        const int n0 = T.col0 + c;
+        if (n0 >= p.N) continue;
+        const float* sc = wsh + j * 32;
         uint32_t w[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float4 s2 = make_float4(wsh[c + 2 * j], wsh[c + 2 * j + 1], 0.0f, 0.0f);
-          const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * j]) : 0.0f;
-          const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-          w[j] = pack_bf16x2(a0 * (xsv * s2.x), a1 * (xsv * s2.y));
+        for (int q = 0; q < 16; ++q) {
+          const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * q]) : 0.0f;
+          const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * q + 1]) : 0.0f;
+          w[q] = pack_bf16x2(a0 * (xsv * sc[2 * q]), a1 * (xsv * sc[2 * q + 1]));
         }
-        uint8_t* sb = stage_out + (chunk & 1u) * 2048;
-        if (lane == 0) bulk_wait_read_le1();  // the store issued from sb two chunks ago has read it
-        __syncwarp();
+        if (tma_ok) {
+          if (lane == 0) bulk_wait_read_le0();  // the previous chunk's store has read the staging tile
+          __syncwarp();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) st_shared_v4(sb + lane * 64 + k * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (row0 < p.M && col0 + c < p.N) tma_store_2d(&tm_out, sb, col0 + c, row0);
-          bulk_commit_group();  // possibly empty: keeps one group per chunk
+          for (int k = 0; k < 4; ++k)
+            st_shared_v4(sb + lane * 64 + k * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_out, sb, n0, row0, out_pol);
+            bulk_commit_group();
+          }
+        } else if (vrow) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (n0 + 8 * k < p.N) st_global_v4(orow + n0 + 8 * k, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
     }
     if (lane == 0) bulk_wait_all();  // stores complete before the CTA's shared memory goes
     __syncwarp();
@@ -905,7 +957,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 template <int KIND, int BN, int STAGES>
 cudaError_t run2(const GemmArgs& a, std::string* msg) {
   constexpr int kElem = (KIND == 0) ? 1 : 2;
-  constexpr int kSmem = STAGES * (128 + BN / 2) * kBKBytes + 4 * 2 * 2048 + 4 * BN * 4 + 1024;
+  constexpr int kSmem = STAGES * (128 + BN / 2) * kBKBytes + 8 * 2048 + 8 * (BN / 64) * 32 * 4 + 1024;
+  static_assert(kSmem + 8400 <= 232448, "shared memory over the 227 KB per-CTA limit");
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_clusters = 0;
@@ -937,7 +990,8 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
   memset(&tb, 0, sizeof(tb));
   if (a.K > 0) {
     if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kElem, 128, msg) ||
-        !make_map(&tb, a.b, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), kElem, BN / 2, msg))
+        !make_map(&tb, a.b, static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K),
+                  kElem, 128, msg))
       return cudaErrorInvalidValue;
   }
   CUtensorMap to;
@@ -952,21 +1006,22 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.m_tiles = static_cast<int>((a.M + 255) / 256);
   p.group_m = 8;
-  p.E = 1;
-  p.offsets = nullptr;
+  p.E = a.E;
+  p.offsets = a.offsets;
   p.xs = a.x_scale;
   p.xs_bcast = (a.x_scale_len == 1) ? 1 : 0;
   p.ws = a.w_scale;
   p.ws_bcast = (a.w_scale_len == 1) ? 1 : 0;
   p.out = static_cast<uint16_t*>(a.out);
   const uint32_t ab_fmt = (KIND == 0) ? static_cast<uint32_t>(a.fmt) : 1u;
-  p.idesc = (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-            (static_cast<uint32_t>(256 >> 4) << 24);  // M = 256 across the pair
+  p.idesc = (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+            (static_cast<uint32_t>(256 >> 4) << 24);  // one MMA: M = 256 across the pair, N = 256
   int dev = 0;
   cudaGetDevice(&dev);
   int clusters = device_sm_count(dev) / 2;
   if (max_clusters > 0 && max_clusters < clusters) clusters = max_clusters;
-  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  // grouped: the tile count lives on the device; a bound suffices
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles + (a.offsets != nullptr ? a.E : 0)) * p.n_tiles;
   if (tiles < clusters) clusters = static_cast<int>(tiles);
   if (clusters < 1) clusters = 1;
   k_gemm2<KIND, BN, STAGES><<<2 * clusters, kGemmThreads, kSmem, a.stream>>>(ta, tb, to, p);
@@ -982,28 +1037,43 @@ cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
   const bool wide = ((a.N % 256 == 0) && a.N >= 2048 && a.M >= 256) || (a.offsets != nullptr && a.N >= 1024);
   // Large dense GEMMs run on CTA pairs (256 x 256 tiles).
   const bool pair = a.offsets == nullptr && a.kind == 0 && (a.N % 256 == 0) && a.N >= 2048 && a.M >= 512;
+  // 256 x 512 pair tiles read a quarter fewer operand bytes per flop; with
+  // enough M their coarser last round costs little
+  if (pair && a.N % 512 == 0 && a.M >= 8192) return run2<0, 512, 4>(a, msg);
   if (pair) return run2<0, 256, 6>(a, msg);
-  // Small M (decode): the weight stream from HBM is the bound.  Only AROWS
-  // rows of A are loaded per K block, which leaves shared memory for several
-  // K blocks of W per stage (longer runs of each weight row per request).
-  // Tile width: 128 when N/128 tiles fit on the SMs in one round; otherwise
-  // 208 (N <= 208 * SMs, one round with fewer idle SMs than 256-wide tiles
-  // leave), else 256.
+  // Grouped GEMMs with wide experts run on CTA pairs too: 256-row tiles per
+  // expert, one third fewer operand bytes per flop than 128 x 256 tiles.
+  if (a.offsets != nullptr && a.N >= 1024 && a.M >= 512) {
+    if (a.kind == 0) return run2<0, 256, 6>(a, msg);
+    return run2<1, 256, 6>(a, msg);
+  }
+  // Small M (decode): the weight stream from HBM is the bound, and each SM
+  // streams at a roughly fixed rate, so the tile width is the narrowest that
+  // keeps the most SMs busy in one round: 64 when N/64 tiles fit on the SMs,
+  // else 128, else 208 (N <= 208 * SMs), else 256.  Only AROWS rows of A are
+  // loaded per K block, which leaves shared memory for several K blocks of W
+  // per stage (longer runs of each weight row per request).
   if (a.offsets == nullptr && a.kind == 0 && a.M <= 128) {
     int dev = 0;
     cudaGetDevice(&dev);
     const int64_t sms = device_sm_count(dev);
-    const int bn = ((a.N + 127) / 128 <= sms) ? 128 : ((a.N + 207) / 208 <= sms) ? 208 : 256;
+    const int bn = ((a.N + 63) / 64 <= sms)     ? 64
+                   : ((a.N + 127) / 128 <= sms) ? 128
+                   : ((a.N + 207) / 208 <= sms) ? 208
+                                                : 256;
     if (a.M <= 16) {
+      if (bn == 64) return run<0, 64, 2, 16, 8>(a, msg);
       if (bn == 128) return run<0, 128, 3, 16, 3>(a, msg);
       if (bn == 208) return run<0, 208, 3, 16, 2>(a, msg);
       return run<0, 256, 2, 16, 2>(a, msg);
     }
     if (a.M <= 64) {
+      if (bn == 64) return run<0, 64, 3, 64, 4>(a, msg);
       if (bn == 128) return run<0, 128, 2, 64, 4>(a, msg);
       if (bn == 208) return run<0, 208, 2, 64, 2>(a, msg);
       return run<0, 256, 2, 64, 2>(a, msg);
     }
+    if (bn == 64) return run<0, 64, 2, 128, 4>(a, msg);
     if (bn == 128) return run<0, 128, 3, 128, 2>(a, msg);
     if (bn == 208) return run<0, 208, 4, 128, 1>(a, msg);
     return run<0, 256, 4>(a, msg);

@@ -38,13 +38,19 @@ SHAPES = [(1, 8, 16), (5, 8, 32), (128, 128, 128), (129, 136, 144), (200, 264, 5
           # CTA-pair path (M >= 512, N % 256 == 0): M not a multiple of 256
           # (the second CTA's half partly or wholly past M), 9 N tiles, ragged K
           (600, 2304, 272), (700, 2048, 128), (1024, 2560, 512),
-          # small-M (decode) paths with 128-wide tiles (N/128 tiles fit on the SMs)
+          # 256 x 512 CTA-pair tiles (M >= 8192, N % 512 == 0): a partial last M tile
+          (8200, 2560, 32),
+          # small-M (decode) paths: 64-wide tiles (16 / 64 A rows), 128-wide (64 A rows)
           (17, 2048, 384), (33, 520, 160), (24, 18944, 128)]
 
-# Decode paths with wider tiles on a 148-SM B200: 208 columns once N/128
-# tiles exceed the SMs (a ragged last tile, a 16-column tail chunk per
-# tile), 256 beyond 208 x 148 columns; A loaded 16 / 64 / 128 rows per block.
-DECODE_SHAPES = [(40, 19200, 256), (16, 19000, 256), (100, 19200, 128), (8, 30848, 64), (120, 4096, 384)]
+# Decode paths on a 148-SM B200, by tile width: 64 while N/64 tiles fit on
+# the SMs, 128 while N/128 do, 208 up to 208 x 148 columns (a ragged last
+# tile, a 16-column tail chunk per tile), 256 beyond; each with A loaded 16 /
+# 64 / 128 rows per K block.
+DECODE_SHAPES = [(120, 4096, 384),                                      # 64 / 128 rows
+                 (10, 9600, 128), (90, 12000, 128),                     # 128 / 16 and 128 rows
+                 (40, 19200, 256), (16, 19000, 256), (100, 19200, 128),  # 208 / 64, 16, 128 rows
+                 (8, 30848, 64), (50, 30848, 64), (128, 30976, 64)]     # 256 / 16, 64, 128 rows
 
 
 @pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])

@@ -1,7 +1,8 @@
 """GPU parity of the grouped (per-expert) GEMMs against the oracle, through the
 C ABI: the a8w8 form (kind::f8f6f4) and the bf16 form with FP32
 accumulation (kind::f16).  Expert row ranges come from device offsets;
-empty experts, ragged counts that cross 128-row tiles, malformed offsets,
+empty experts, ragged counts that cross 128- and 256-row tiles (the 1-CTA
+and the CTA-pair kernels), malformed offsets,
 and the MoE workload (64 experts, K=2048, N=1408, 32768 tokens with Zipf(1.1)
 counts and two empty experts) are covered.  Output is overwritten, never
 accumulated (megablocks-hip TODO-gg.md).
@@ -31,6 +32,12 @@ CASES = [  # (counts per expert, N, K)
     ([128, 128, 0, 64], 136, 272),
     ([300], 256, 384),
     ([40] * 20, 128, 256),
+    # CTA-pair path (M_total >= 512, N >= 1024): 256-row tiles per expert,
+    # experts of 300 / 257 / 520 rows (a partial second tile, 32-row groups
+    # that straddle an expert boundary), a last N tile of 16 columns whose
+    # second-CTA weight rows belong to the next expert, ragged K
+    ([3, 0, 300, 1, 0, 257, 40], 1024, 256),
+    ([520, 0, 17], 1040, 160),
 ]
 
 
