@@ -1,7 +1,7 @@
 """Benchmark of the dynamic-FP8 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large|large4096|large8192|decode1|decode16|decode128|sweep|moe|moe_bf16]
+                    [--workload large|large4096|large8192|decode1|decode16|decode128|sweep|stack|moe|moe_bf16]
 
 Default workload (the large a8w8 GEMM layer): X bf16 [16384, 8192] ~N(0,1),
 W bf16 [28672, 8192] ~N(0,0.02).  One step = per-token E4M3 quantize of X,
@@ -66,6 +66,7 @@ WORKLOADS = {
     "decode16": dict(kind="decode", M=16, N=28672, K=8192),
     "decode128": dict(kind="decode", M=128, N=28672, K=8192),
     "sweep": dict(kind="sweep", M=8192, N=0, K=8192),
+    "stack": dict(kind="stack", M=2048, N=4096, K=1024, steps_cycle=200, ring=16),
     "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
     "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }
@@ -78,6 +79,10 @@ def workload_desc(name, cfg):
                 "per-output-channel E4M3%s, out bf16 [%d,%d] (caller-owned)" %
                 ("large" if k == "layer" else "decode", cfg["M"], cfg["K"], cfg["N"], cfg["K"],
                  "" if k == "layer" else " (quantized once: static weights)", cfg["M"], cfg["N"]))
+    if k == "stack":
+        return ("delayed-scaling linear stack: X_t bf16 [2048,1024] (std 0.5 -> 8 over 200 steps), W_up bf16 "
+                "[4096,1024], W_down bf16 [1024,4096] ~N(0,0.02); per-tensor E4M3 with four amax-history rings "
+                "(length 16); h = GEMM(q(X), q(W_up)), y = GEMM(q(h), q(W_down)); step replayed as a CUDA graph")
     if k == "sweep":
         return ("quantize sweep: bf16 [%d,%d] ~N(0,1), 0.1%% x100 outliers, 0.1%% zeros, one zero row; "
                 "per-tensor / per-token / per-channel x E4M3 / E5M2" % (cfg["M"], cfg["K"]))
@@ -258,6 +263,101 @@ def build(args, cfg, rank, dev, stream, peaks):
         return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=h2d, d2h=M * N * 2,
                     roofline=roofline, extras=extras, l2=l2, flush=None)
 
+    if kind == "stack":
+        T, D, H, L = M, K, N, cfg["ring"]
+        cyc = cfg["steps_cycle"]
+        xs_host = [bf16_host(W.delayed_x(t, T, D, cyc)).view(T, D) for t in range(cyc)]
+        xs_dev = torch.stack([x.to(dev) for x in xs_host])
+        wu = bf16_host(W.f32_to_bf16_bits(W.normal((H, D), 0.02, 1))).view(H, D).to(dev)
+        wd = bf16_host(W.f32_to_bf16_bits(W.normal((D, H), 0.02, 2))).view(D, H).to(dev)
+        x_stage = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+        rings = {k: torch.zeros(L + 2, dtype=torch.float32, device=dev) for k in ("x", "wu", "h", "wd")}
+        for r in rings.values():
+            r[L] = 1.0
+        def u8(r, c):
+            return torch.empty((r, c), dtype=torch.uint8, device=dev)
+        def f1():
+            return torch.empty((1,), dtype=torch.float32, device=dev)
+        xq, wuq, hq_, wdq = u8(T, D), u8(H, D), u8(T, H), u8(D, H)
+        xsc, wusc, hsc, wdsc = f1(), f1(), f1(), f1()
+        h = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+        y_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
+        ws = {k: torch.zeros(hq.hq_quantize_workspace_bytes(hq.PER_TENSOR, 1, 1, True), dtype=torch.uint8, device=dev)
+              for k in rings}
+
+        def body(idx):
+            def q(x, key, qo, so):
+                hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TENSOR, q=qo, scales=so, ring=rings[key], ring_idx=idx,
+                                   workspace=ws[key], stream=torch.cuda.current_stream(dev))
+            q(x_stage, "x", xq, xsc)
+            q(wu, "wu", wuq, wusc)
+            hq.hq_gemm_a8w8(xq, wuq, xsc, wusc, hq.E4M3, out=h, stream=torch.cuda.current_stream(dev))
+            q(h, "h", hq_, hsc)
+            q(wd, "wd", wdq, wdsc)
+            hq.hq_gemm_a8w8(hq_, wdq, hsc, wdsc, hq.E4M3, out=y, stream=torch.cuda.current_stream(dev))
+
+        # one graph per ring slot (the slot index is a launch argument)
+        for idx in range(L):
+            body(idx)
+        torch.cuda.synchronize()
+        graph_error = None
+        graphs = []
+        try:
+            for idx in range(L):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr):
+                    body(idx)
+                graphs.append(gr)
+        except Exception as exc:  # eager launches instead; the line says so
+            graphs = None
+            graph_error = "%s: %s" % (type(exc).__name__, str(exc).splitlines()[0] if str(exc) else "")
+            torch.cuda.synchronize()
+        for r in rings.values():  # the warm-up and capture passes ran the rings: start fresh
+            r.zero_()
+            r[L] = 1.0
+        counter = [0]
+
+        def step_fn():
+            t = counter[0] % cyc
+            counter[0] += 1
+            x_stage.copy_(xs_dev[t], non_blocking=True)
+            if graphs is not None:
+                graphs[t % L].replay()
+            else:
+                body(t % L)
+
+        def e2e():
+            t = counter[0] % cyc
+            counter[0] += 1
+            x_stage.copy_(xs_host[t], non_blocking=True)
+            if graphs is not None:
+                graphs[t % L].replay()
+            else:
+                body(t % L)
+            y_host.copy_(y, non_blocking=True)
+
+        flops = 2.0 * T * H * D * 2
+
+        def roofline(ms):
+            a = flops / (ms["step"] / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": round(a, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(a / fp8_peak, 4), "traffic": None,
+                    "kernel": "the whole step (2 GEMMs + 4 delayed quantizes) as one CUDA graph replay",
+                    "peak_source": "%s bf16 burst x 2 (nominal fp8/bf16)" % peaks["_src"]}
+
+        def extras(ms):
+            d = {"kernels_per_step": 6, "rings": "4 x [16 hist | scale | counter], updated on the device every step"}
+            if graphs is not None:
+                d["graph_launches_per_step"] = 1
+            else:
+                d["graph_capture"] = "failed (%s); eager launches" % graph_error
+            return d
+
+        return dict(calls=[("step", step_fn, 6)], per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=T * D * 2,
+                    d2h=T * D * 2, roofline=roofline, extras=extras, flush=None, graphs=graphs,
+                    l2="working set (X 4 MB, W 16 MB, h 16 MB) fits L2: a steady-state layer step")
+
     if kind == "sweep":
         x_host = bf16_host(W.sweep(M, K, seed=rank)).view(M, K)
         x = x_host.to(dev)
@@ -435,6 +535,7 @@ def run_ours(args, rank, local_rank, world):
         mx = min(256, cfg["M"])
         cpu = cpu_baseline(cfg["M"], cfg["N"], cfg["K"], budget_rows=(mx, min(cfg["N"], 4096 * 256 // mx)))
 
+    wl.pop("graphs", None)  # release captured graphs before the process group goes
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

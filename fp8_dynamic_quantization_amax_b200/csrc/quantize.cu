@@ -535,14 +535,15 @@ __global__ void __launch_bounds__(kThreads) k_tensor_cast(
 
 // ------------------------------------------------- per-tensor, one launch
 // The same two phases in one cooperative launch (all CTAs resident, one per
-// SM).  CTA b owns the contiguous vectors [b0, b1).  Phase 1 bulk-copies the
-// first part of its range into shared memory (kept there for phase 2) and
-// streams the rest through registers with an L2 evict_last hint, so that
-// phase 2 finds it in L2; a grid barrier (a counter, bounded wait) publishes
-// the global amax; phase 2 casts the streamed part again, newest lines
-// first, and then the part held in shared memory.  DRAM sees x about once.
-// Workspace words: [0] amax bits, [1] arrivals, [2] departures, [3]
-// non-finite flag; the last CTA to leave returns all four to zero.
+// SM).  CTA b owns the contiguous vectors [b0, b1).  Phase 1 keeps the first
+// part of its range on chip -- up to 208 KB bulk-copied into shared memory,
+// then 256 KB parked in tensor memory (TMEM, tcgen05.st) -- and streams the
+// rest through registers with an L2 evict_last hint, so that phase 2 finds it
+// in L2.  A grid barrier (a counter, bounded wait) publishes the global amax;
+// phase 2 casts the L2 part again, newest lines first, then the TMEM and
+// shared-memory parts.  DRAM sees x about once.  Workspace words: [0] amax
+// bits, [1] arrivals, [2] departures, [3] non-finite flag; the last CTA to
+// leave returns all four to zero.
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedUnroll = 4;  // 16-byte loads in flight per thread (64 registers at 1024 threads)
 
@@ -576,6 +577,57 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   return v;
 }
 
+__device__ __forceinline__ bool grid_barrier(uint32_t* arrivals, unsigned* err_word) {
+  const unsigned long long t0 = ptx::globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire_u32(arrivals) >= gridDim.x) return true;
+    if ((it & 15u) == 15u && ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
+      atomicOr(err_word, kDevErrTimeout);
+      return false;
+    }
+    __nanosleep(100);
+  }
+}
+
+// Tensor memory as a staging store: each warp owns 64 of the 512 columns of
+// its 32-lane quadrant; vector j of a thread sits in columns 4j..4j+3 of its
+// lane.  kTmemVecs vectors per thread (256 KB per CTA).
+constexpr int kTmemVecs = 16;
+constexpr uint32_t kTmemCols = 512;
+
+__device__ __forceinline__ void tmem_alloc_warp(uint32_t* slot) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(ptx::smem_u32(slot)),
+               "r"(kTmemCols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_warp(uint32_t base) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(kTmemCols) : "memory");
+}
+__device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// this thread's column base in its warp's quadrant
+__device__ __forceinline__ uint32_t tmem_thread_base(uint32_t base) {
+  const uint32_t w = threadIdx.x >> 5;
+  return base + ((32u * (w & 3u)) << 16) + (w >> 2) * (4u * kTmemVecs);
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint4& u) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(u.x), "r"(u.y),
+               "r"(u.z), "r"(u.w)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ uint4 tmem_ld4(uint32_t taddr) {
+  uint4 u;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+      : "r"(taddr)
+      : "memory");
+  return u;
+}
+
 template <int DT, int FMT>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
     const void* __restrict__ x, int64_t n, int64_t per_cta, int64_t held_max, uint8_t* __restrict__ q,
@@ -590,6 +642,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
   __shared__ float s_amax;
   __shared__ int s_flags;  // bit 0: a non-finite element somewhere, bit 1: abort
   __shared__ int abort_flag;
+  __shared__ uint32_t tmem_slot;
 
   const int tid = threadIdx.x;
   const uint4* xv = static_cast<const uint4*>(x);
@@ -597,7 +650,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
   const int64_t b0 = min(nv, static_cast<int64_t>(blockIdx.x) * per_cta);
   const int64_t b1 = min(nv, b0 + per_cta);
   const int64_t nheld = min(b1 - b0, held_max);
-  const int64_t s0 = b0 + nheld;  // streamed part [s0, b1)
+  const int64_t s0 = b0 + nheld;                               // TMEM part [s0, s1)
+  const int64_t s1 = min(b1, s0 + static_cast<int64_t>(kTmemVecs) * T);  // L2 part [s1, b1)
   const bool tail_cta = blockIdx.x == gridDim.x - 1;
 
   if (tid == 0) {
@@ -613,12 +667,32 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
                        min(65536u, bytes - off), &bar, pol);
     }
   }
+  if (tid < 32) tmem_alloc_warp(&tmem_slot);
+  tc_before_sync();
   __syncthreads();
+  tc_after_sync();
+  const uint32_t tq = tmem_thread_base(tmem_slot);
 
   // ---- phase 1: amax
   const uint64_t keep = policy_evict_last();
+  const uint64_t once = policy_evict_first();
   uint32_t mraw = 0;
-  int64_t v = s0 + tid;
+#pragma unroll
+  for (int j0 = 0; j0 < kTmemVecs; j0 += U) {  // the TMEM part: read once from DRAM
+    uint4 u[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t v = s0 + static_cast<int64_t>(j0 + j) * T + tid;
+      u[j] = (v < s1) ? ld_hint(xv + v, once) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncwarp();  // tcgen05.st is warp-wide
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(u[j]));
+      tmem_st4(tq + 4u * (j0 + j), u[j]);
+    }
+  }
+  int64_t v = s1 + tid;
   for (; v + (U - 1) * T < b1; v += U * T) {
     uint4 u[U];
 #pragma unroll
@@ -633,6 +707,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
     if (landed)
       for (int64_t i = tid; i < nheld; i += T) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(held[i]));
   }
+  tmem_wait_st();
   float amax = 0.0f;
   bool nf = false;
   if (!Dt<DT>::nonfinite(mraw)) {
@@ -650,7 +725,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
       amax = fmaxf(amax, finite_abs(f));
     }
   nf = __syncthreads_or(nf);
-  // block_max for T threads
   amax = warp_max(amax);
   if ((tid & 31) == 0) sh[tid >> 5] = amax;
   __syncthreads();
@@ -663,16 +737,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
       __threadfence();
       atomicAdd(&ws[1], 1u);
       // grid barrier: every CTA has published its amax
-      bool ok = !abort_flag;
-      const unsigned long long t0 = ptx::globaltimer();
-      for (uint32_t it = 0; ok; ++it) {
-        if (ld_acquire_u32(&ws[1]) >= gridDim.x) break;
-        if ((it & 15u) == 15u && ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
-          atomicOr(err_word, kDevErrTimeout);
-          ok = false;
-        }
-        __nanosleep(100);
-      }
+      const bool ok = !abort_flag && grid_barrier(&ws[1], err_word);
       s_amax = __uint_as_float(__ldcg(&ws[0]));
       s_flags = (__ldcg(&ws[3]) != 0u ? 1 : 0) | (ok ? 0 : 2);
       __threadfence();
@@ -686,40 +751,49 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
     }
   }
   __syncthreads();
-  if (s_flags & 2) {  // barrier or copy gave up: the error word says so
-    if (tid == 0 && nheld > 0 && !landed) {  // let the copy land before the CTA's shared memory goes
-      int dummy = 0;
-      ptx::mbar_wait(&bar, 0, &dummy, nullptr, 0, ptx::kDrainLimitNs);
-    }
-    return;
-  }
 
-  // ---- phase 2: cast
-  const float a = s_amax;
-  const float m = multiplier(a, fmax);
-  if (blockIdx.x == 0 && tid == 0) {
-    scales[0] = __fdiv_rn(1.0f, m);
-    if (amax_out) amax_out[0] = a;
-  }
-  const uint64_t drop = policy_evict_first();
-  const int64_t ns = b1 - s0;
-  auto cast_range = [&](auto fast) {
-    constexpr bool FAST = decltype(fast)::value;
-    int64_t i = tid;
-    for (; i + (U - 1) * T < ns; i += U * T) {  // streamed part, from its end backwards
-      uint4 u[U];
-#pragma unroll
-      for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + (b1 - 1 - (i + j * T)), drop);
-#pragma unroll
-      for (int j = 0; j < U; ++j) vec_store<DT, FMT, FAST>(q + (b1 - 1 - (i + j * T)) * VEC, u[j], m);
+  if (!(s_flags & 2)) {
+    // ---- phase 2: cast
+    const float a = s_amax;
+    const float m = multiplier(a, fmax);
+    if (blockIdx.x == 0 && tid == 0) {
+      scales[0] = __fdiv_rn(1.0f, m);
+      if (amax_out) amax_out[0] = a;
     }
-    for (; i < ns; i += T) vec_store<DT, FMT, FAST>(q + (b1 - 1 - i) * VEC, ld_hint(xv + (b1 - 1 - i), drop), m);
-    for (int64_t k = tid; k < nheld; k += T) vec_store<DT, FMT, FAST>(q + (b0 + k) * VEC, held[k], m);
-  };
-  if (!(s_flags & 1)) cast_range(std::true_type{});
-  else cast_range(std::false_type{});
-  if (tail_cta)
-    for (int64_t i = nv * VEC + tid; i < n; i += T) q[i] = cvt1_exact<FMT>(__fmul_rn(Dt<DT>::load1(x, i), m));
+    const uint64_t drop = policy_evict_first();
+    const int64_t ns = b1 - s1;
+    auto cast_range = [&](auto fast) {
+      constexpr bool FAST = decltype(fast)::value;
+      int64_t i = tid;
+      for (; i + (U - 1) * T < ns; i += U * T) {  // the L2 part, from its end backwards
+        uint4 u[U];
+#pragma unroll
+        for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + (b1 - 1 - (i + j * T)), drop);
+#pragma unroll
+        for (int j = 0; j < U; ++j) vec_store<DT, FMT, FAST>(q + (b1 - 1 - (i + j * T)) * VEC, u[j], m);
+      }
+      for (; i < ns; i += T) vec_store<DT, FMT, FAST>(q + (b1 - 1 - i) * VEC, ld_hint(xv + (b1 - 1 - i), drop), m);
+      __syncwarp();  // tcgen05.ld is warp-wide
+#pragma unroll 4
+      for (int j = 0; j < kTmemVecs; ++j) {  // the TMEM part
+        const uint4 u = tmem_ld4(tq + 4u * j);
+        const int64_t vv = s0 + static_cast<int64_t>(j) * T + tid;
+        if (vv < s1) vec_store<DT, FMT, FAST>(q + vv * VEC, u, m);
+      }
+      for (int64_t k = tid; k < nheld; k += T) vec_store<DT, FMT, FAST>(q + (b0 + k) * VEC, held[k], m);
+    };
+    if (!(s_flags & 1)) cast_range(std::true_type{});
+    else cast_range(std::false_type{});
+    if (tail_cta)
+      for (int64_t i = nv * VEC + tid; i < n; i += T) q[i] = cvt1_exact<FMT>(__fmul_rn(Dt<DT>::load1(x, i), m));
+  } else if (tid == 0 && nheld > 0 && !landed) {  // gave up: let the copy land before shared memory goes
+    int dummy = 0;
+    ptx::mbar_wait(&bar, 0, &dummy, nullptr, 0, ptx::kDrainLimitNs);
+  }
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  if (tid < 32) tmem_dealloc_warp(tmem_slot);
 }
 
 // -------------------------------------------------------------- per-channel
@@ -898,8 +972,9 @@ __global__ void __launch_bounds__(kThreads) k_channel_cast(
 // kStripVecs 16-byte column vectors and B row bands (S * B <= SMs); CTA
 // (strip, band) owns that tile.  Thread t owns column vector t % kStripVecs
 // of the strip and rows t / kStripVecs, + kRowLanes, ... of the band.  The
-// band's first rows of the strip are bulk-copied into shared memory and kept;
-// the rest stream through registers with an L2 evict_last hint.  The row
+// band's first rows of the strip are bulk-copied into shared memory and kept,
+// each lane's next kTmemVecs rows are parked in tensor memory, and the rest
+// stream through registers with an L2 evict_last hint.  The row
 // lanes' maxima meet in shared memory and one atomicMax per column per CTA
 // folds them into the workspace, B atomics per column.  After a grid barrier
 // each CTA derives its strip's multipliers into shared memory and casts its
@@ -909,18 +984,6 @@ __global__ void __launch_bounds__(kThreads) k_channel_cast(
 constexpr int kStripVecs = 256;
 constexpr int kRowLanes = kFusedThreads / kStripVecs;
 constexpr int64_t kMaxHeldRows = 128;  // bulk copies per CTA (one per held row)
-
-__device__ __forceinline__ bool grid_barrier(uint32_t* arrivals, unsigned* err_word) {
-  const unsigned long long t0 = ptx::globaltimer();
-  for (uint32_t it = 0;; ++it) {
-    if (ld_acquire_u32(arrivals) >= gridDim.x) return true;
-    if ((it & 15u) == 15u && ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
-      atomicOr(err_word, kDevErrTimeout);
-      return false;
-    }
-    __nanosleep(100);
-  }
-}
 
 template <int DT, int FMT>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
@@ -936,6 +999,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
   __shared__ __align__(8) uint64_t bar;
   __shared__ int s_flags;  // bit 0: non-finite somewhere, bit 1: give up, bit 2: last to leave
   __shared__ int abort_flag;
+  __shared__ uint32_t tmem_slot;
 
   const int tid = threadIdx.x;
   const int lv = tid % kStripVecs;  // column vector within the strip
@@ -948,7 +1012,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
   const int64_t r0 = min(rows, band * band_rows);
   const int64_t r1 = min(rows, r0 + band_rows);
   const int64_t nh = min(r1 - r0, held_rows);
-  const int64_t rs0 = r0 + nh;  // streamed rows [rs0, r1)
+  const int64_t rs0 = r0 + nh;                 // rows [rs0, rs1) go through TMEM,
+  const int64_t rs1 = rs0 + kTmemVecs * RL;    // rows [rs1, r1) through L2
   float* red = reinterpret_cast<float*>(fsm);  // [RL][SC] row-lane maxima; later the strip's multipliers
   uint4* held = reinterpret_cast<uint4*>(fsm + RL * SC * 4);  // [nh][sv]
   const uint4* xv = static_cast<const uint4*>(x);  // row r, column vector c: xv[r * nvc + c]
@@ -964,15 +1029,38 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
       for (int64_t i = 0; i < nh; ++i) bulk_load_hint(held + i * sv, xv + (r0 + i) * nvc + c0, row_bytes, &bar, pol);
     }
   }
+  if (tid < 32) tmem_alloc_warp(&tmem_slot);
+  tc_before_sync();
   __syncthreads();
+  tc_after_sync();
+  const uint32_t tq = tmem_thread_base(tmem_slot);
 
   // ---- phase 1: column maxima of the tile
   const uint64_t keep = policy_evict_last();
+  const uint64_t once = policy_evict_first();
   const bool active = lv < sv;
   const int64_t c = c0 + lv;
   uint32_t acc[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i0 = 0; i0 < kTmemVecs; i0 += U) {  // this lane's first rows: read once, parked in TMEM
+    uint4 u[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t r = rs0 + rl + static_cast<int64_t>(i0 + j) * RL;
+      u[j] = (active && r < r1) ? ld_hint(xv + r * nvc + c, once) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncwarp();  // tcgen05.st is warp-wide
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      acc[0] = Dt<DT>::lmax(acc[0], Dt<DT>::mag(u[j].x));
+      acc[1] = Dt<DT>::lmax(acc[1], Dt<DT>::mag(u[j].y));
+      acc[2] = Dt<DT>::lmax(acc[2], Dt<DT>::mag(u[j].z));
+      acc[3] = Dt<DT>::lmax(acc[3], Dt<DT>::mag(u[j].w));
+      tmem_st4(tq + 4u * (i0 + j), u[j]);
+    }
+  }
   if (active) {
-    int64_t r = rs0 + rl;
+    int64_t r = rs1 + rl;
     for (; r + (U - 1) * RL < r1; r += U * RL) {
       uint4 u[U];
 #pragma unroll
@@ -993,6 +1081,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
       acc[3] = Dt<DT>::lmax(acc[3], Dt<DT>::mag(u.w));
     }
   }
+  tmem_wait_st();
   bool landed = true;
   if (nh > 0 && sv > 0) landed = ptx::mbar_wait(&bar, 0, &abort_flag, err_word, kDevErrTimeout);
   if (active && landed)
@@ -1073,37 +1162,48 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
       atomicExch(&header[2], 0u);
     }
   }
-  if (!ok) {  // the error word says so
-    if (tid == 0 && nh > 0 && sv > 0 && !landed) {
-      int dummy = 0;
-      ptx::mbar_wait(&bar, 0, &dummy, nullptr, 0, ptx::kDrainLimitNs);
-    }
-    return;
-  }
-
-  // ---- phase 2: cast the tile, this lane's streamed rows from the end backwards
-  if (!active) return;
-  const uint64_t drop = policy_evict_first();
-  float m[VEC];
+  if (ok) {
+    // ---- phase 2: cast the tile: this lane's L2 rows from the end backwards,
+    // then its TMEM rows, then the held rows
+    const uint64_t drop = policy_evict_first();
+    float m[VEC];
 #pragma unroll
-  for (int j = 0; j < VEC; ++j) m[j] = m_s[lv * VEC + j];
-  auto cast_tile = [&](auto fast) {
-    constexpr bool FAST = decltype(fast)::value;
-    if (r1 - 1 >= rs0 + rl) {
-      int64_t r = rs0 + rl + ((r1 - 1 - rs0 - rl) / RL) * RL;  // this lane's last streamed row
-      for (; r - (U - 1) * RL >= rs0; r -= U * RL) {
-        uint4 u[U];
+    for (int j = 0; j < VEC; ++j) m[j] = active ? m_s[lv * VEC + j] : 0.0f;
+    auto cast_tile = [&](auto fast) {
+      constexpr bool FAST = decltype(fast)::value;
+      if (active && r1 - 1 >= rs1 + rl) {
+        int64_t r = rs1 + rl + ((r1 - 1 - rs1 - rl) / RL) * RL;  // this lane's last L2 row
+        for (; r - (U - 1) * RL >= rs1; r -= U * RL) {
+          uint4 u[U];
 #pragma unroll
-        for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + (r - j * RL) * nvc + c, drop);
+          for (int j = 0; j < U; ++j) u[j] = ld_hint(xv + (r - j * RL) * nvc + c, drop);
 #pragma unroll
-        for (int j = 0; j < U; ++j) vec_store_m<DT, FMT, FAST>(q + (r - j * RL) * cols + c * VEC, u[j], m);
+          for (int j = 0; j < U; ++j) vec_store_m<DT, FMT, FAST>(q + (r - j * RL) * cols + c * VEC, u[j], m);
+        }
+        for (; r >= rs1; r -= RL)
+          vec_store_m<DT, FMT, FAST>(q + r * cols + c * VEC, ld_hint(xv + r * nvc + c, drop), m);
       }
-      for (; r >= rs0; r -= RL) vec_store_m<DT, FMT, FAST>(q + r * cols + c * VEC, ld_hint(xv + r * nvc + c, drop), m);
-    }
-    for (int64_t i = rl; i < nh; i += RL) vec_store_m<DT, FMT, FAST>(q + (r0 + i) * cols + c * VEC, held[i * sv + lv], m);
-  };
-  if (!(s_flags & 1)) cast_tile(std::true_type{});
-  else cast_tile(std::false_type{});
+      __syncwarp();  // tcgen05.ld is warp-wide
+#pragma unroll 4
+      for (int i = 0; i < kTmemVecs; ++i) {
+        const uint4 u = tmem_ld4(tq + 4u * i);
+        const int64_t r = rs0 + rl + static_cast<int64_t>(i) * RL;
+        if (active && r < r1) vec_store_m<DT, FMT, FAST>(q + r * cols + c * VEC, u, m);
+      }
+      if (active)
+        for (int64_t i = rl; i < nh; i += RL)
+          vec_store_m<DT, FMT, FAST>(q + (r0 + i) * cols + c * VEC, held[i * sv + lv], m);
+    };
+    if (!(s_flags & 1)) cast_tile(std::true_type{});
+    else cast_tile(std::false_type{});
+  } else if (tid == 0 && nh > 0 && sv > 0 && !landed) {  // gave up: let the copy land before shared memory goes
+    int dummy = 0;
+    ptx::mbar_wait(&bar, 0, &dummy, nullptr, 0, ptx::kDrainLimitNs);
+  }
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  if (tid < 32) tmem_dealloc_warp(tmem_slot);
 }
 
 // ------------------------------------------------------------------ delayed
