@@ -50,6 +50,8 @@ def lib():
         L.hqo_quantize.restype = ci
         L.hqo_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
         L.hqo_gemm_a8w8.restype = None
+        L.hqo_gemm_a8w8_bias.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P]
+        L.hqo_gemm_a8w8_bias.restype = None
         L.hqo_gemm_a8w8_entries.argtypes = [P, P, ci, P, i64, P, i64, i64, P, P, i64, P]
         L.hqo_gemm_a8w8_entries.restype = None
         L.hqo_grouped_gemm_a8w8.argtypes = [P, P, ci, P, P, P, i32, i64, i64, i64, P]
@@ -167,6 +169,21 @@ def gemm_a8w8(xq, wq, fmt, x_scale, w_scale, return_ref=False):
     lib().hqo_gemm_a8w8(_p(xq), _p(wq), fmt, _p(xs), xs.size, _p(ws), ws.size,
                         M, N, K, _p(out), _p(ref))
     return (out, ref) if return_ref else out
+
+
+def gemm_a8w8_bias(xq, wq, fmt, x_scale, w_scale, bias_bf16_bits):
+    """bf16 bits of x_scale * w_scale * (XQ . WQ^T) + bias, rounded once."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    xs = np.ascontiguousarray(x_scale, np.float32).reshape(-1)
+    ws = np.ascontiguousarray(w_scale, np.float32).reshape(-1)
+    b = np.ascontiguousarray(bias_bf16_bits, np.uint16).reshape(-1)
+    M, K = xq.shape
+    N = wq.shape[0]
+    assert b.size == N
+    out = np.empty((M, N), np.uint16)
+    lib().hqo_gemm_a8w8_bias(_p(xq), _p(wq), fmt, _p(xs), xs.size, _p(ws), ws.size, _p(b), M, N, K, _p(out))
+    return out
 
 
 def gemm_a8w8_entries(xq, wq, fmt, x_scale, w_scale, ms, ns):

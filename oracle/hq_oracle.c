@@ -390,6 +390,24 @@ void hqo_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, int fmt,
                                   ref_out ? &ref_out[m * N + n] : NULL);
 }
 
+/* out[m,n] = bf16(x_scale[m'] * w_scale[n'] * sum_k dec(XQ) dec(WQ) + bias[n])
+   with bias a bf16 vector of N entries ([AS] linear_forward_fp8: the bias is
+   added in the GEMM epilogue, before the output rounding).  The sum and the
+   scaling are exact or fp64 as in hqo_gemm_a8w8; the bias is added in fp64
+   and the result rounded once to bf16. */
+void hqo_gemm_a8w8_bias(const uint8_t* xq, const uint8_t* wq, int fmt,
+                        const float* xs, int64_t xs_len, const float* ws,
+                        int64_t ws_len, const uint16_t* bias, int64_t M,
+                        int64_t N, int64_t K, uint16_t* out) {
+  int64_t m, n;
+  for (m = 0; m < M; ++m)
+    for (n = 0; n < N; ++n) {
+      double v;
+      gemm_entry(xq, wq, fmt, xs, xs_len, ws, ws_len, K, m, n, &v);
+      out[m * N + n] = hqo_double_to_bf16(v + (double)hqo_bf16_to_f32(bias[n]));
+    }
+}
+
 /* The same entries at sampled (m, n) positions only. */
 void hqo_gemm_a8w8_entries(const uint8_t* xq, const uint8_t* wq, int fmt,
                            const float* xs, int64_t xs_len, const float* ws,

@@ -421,6 +421,49 @@ def test_gemm_identity_like_and_broadcast_scales():
             assert out[m, n] == O.double_to_bf16(v)
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_gemm_bias_vs_exact_fractions(fmt):
+    # out = bf16 of the exact x_scale * w_scale * S + bias (bias a bf16 vector,
+    # added before the single rounding), against exact rationals.
+    rng = np.random.default_rng(31 + fmt)
+    M, N, K = 4, 6, 40
+    xq = _rand_codes(rng, (M, K), fmt)
+    wq = _rand_codes(rng, (N, K), fmt)
+    xs = rng.uniform(0.01, 2, M).astype(np.float32)
+    ws = rng.uniform(0.01, 2, N).astype(np.float32)
+    bias = W.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32) * np.float32(3.0))
+    out = O.gemm_a8w8_bias(xq, wq, fmt, xs, ws, bias)
+    frac = 9 if fmt == O.E4M3 else 16
+    dx = xq.view(ML[fmt]).astype(np.float64)
+    dw = wq.view(ML[fmt]).astype(np.float64)
+    bv = W.bf16_bits_to_f32(bias)
+    for m in range(M):
+        for n in range(N):
+            s = sum(int(a * 2 ** frac) * int(b * 2 ** frac) for a, b in zip(dx[m], dw[n]))
+            exact = Fraction(s, 2 ** (2 * frac)) * Fraction(float(xs[m])) * Fraction(float(ws[n])) + \
+                Fraction(float(bv[n]))
+            assert out[m, n] == _nearest_bf16(exact)
+
+
+def test_gemm_bias_special_cases():
+    rng = np.random.default_rng(32)
+    M, N, K = 3, 8, 16
+    wq = _rand_codes(rng, (N, K), O.E4M3)
+    xs = np.ones(M, np.float32)
+    ws = rng.uniform(0.1, 1, N).astype(np.float32)
+    bias = W.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    bias[0] = 0x8000  # -0.0: -0 + (+0 product) is +0
+    # all-zero activations: the output is the bias itself
+    out = O.gemm_a8w8_bias(np.zeros((M, K), np.uint8), wq, O.E4M3, xs, ws, bias)
+    expect = np.tile(bias, (M, 1))
+    expect[:, 0] = 0
+    np.testing.assert_array_equal(out, expect)
+    # a zero bias gives the plain GEMM
+    xq = _rand_codes(rng, (M, K), O.E4M3)
+    np.testing.assert_array_equal(O.gemm_a8w8_bias(xq, wq, O.E4M3, xs, ws, np.zeros(N, np.uint16)),
+                                  O.gemm_a8w8(xq, wq, O.E4M3, xs, ws))
+
+
 def test_gemm_entries_match_full():
     rng = np.random.default_rng(4)
     M, N, K = 9, 13, 48
