@@ -279,8 +279,8 @@ def build(args, cfg, rank, dev, stream, peaks):
         def f1():
             return torch.empty((1,), dtype=torch.float32, device=dev)
         xq, wuq, hq_, wdq = u8(T, D), u8(H, D), u8(T, H), u8(D, H)
-        xsc, wusc, hsc, wdsc = f1(), f1(), f1(), f1()
         h = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        xsc, wusc, hsc, wdsc = f1(), f1(), f1(), f1()
         y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
         y_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
         ws = {k: torch.zeros(hq.hq_quantize_workspace_bytes(hq.PER_TENSOR, 1, 1, True), dtype=torch.uint8, device=dev)
@@ -292,6 +292,9 @@ def build(args, cfg, rank, dev, stream, peaks):
                                    workspace=ws[key], stream=torch.cuda.current_stream(dev))
             q(x_stage, "x", xq, xsc)
             q(wu, "wu", wuq, wusc)
+            # h stays a bf16 round trip through L2: at K = 1024 the GEMM's
+            # epilogue is its critical path, and the separate quantize of the
+            # 16 MB h (an L2 read) costs less than the FP8-output epilogue
             hq.hq_gemm_a8w8(xq, wuq, xsc, wusc, hq.E4M3, out=h, stream=torch.cuda.current_stream(dev))
             q(h, "h", hq_, hsc)
             q(wd, "wd", wdq, wdsc)

@@ -21,7 +21,7 @@ PER_TENSOR, PER_TOKEN, PER_CHANNEL = 0, 1, 2
 F32, BF16, F16 = 0, 1, 2
 
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
-            "hq_quantize_fp8", "hq_gemm_a8w8", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
+            "hq_quantize_fp8", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
             "hq_quantize_fp8_noalloc", "hq_check_device_error", "hq_last_error", "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
 
@@ -53,6 +53,9 @@ def _load():
     L.hq_quantize_fp8_noalloc.restype = ci
     L.hq_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
     L.hq_gemm_a8w8.restype = ci
+    L.hq_gemm_a8w8_ex.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P, P, ci, P, P, P, i32, i32, i32, P,
+                                  sz, P]
+    L.hq_gemm_a8w8_ex.restype = ci
     L.hq_grouped_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, P, i32, i64, i64, i64, P, P]
     L.hq_grouped_gemm_a8w8.restype = ci
     L.hq_grouped_gemm_bf16.argtypes = [P, P, P, i32, i64, i64, i64, P, P]
@@ -185,6 +188,35 @@ def hq_gemm_a8w8(xq, wq, x_scale, w_scale, fmt=E4M3, out=None, stream=None):
     check(lib.hq_gemm_a8w8(_ptr(xq), _ptr(wq), fmt, _ptr(x_scale), x_scale.numel(), _ptr(w_scale),
                            w_scale.numel(), M, N, K, _ptr(out), _stream(stream)))
     return out
+
+
+def hq_gemm_a8w8_ex(xq, wq, x_scale, w_scale, fmt=E4M3, bias=None, out=None, q_out=None, q_fmt=E4M3,
+                    q_scale=None, q_amax=None, ring=None, ring_idx=0, ring_margin=0, workspace=None, stream=None):
+    """The a8w8 GEMM with the fused epilogues: an optional bf16 bias [N] added
+    before the rounding, and either the bf16 out (default) or, with `ring`,
+    FP8 codes of the bf16 result quantized per tensor with the delayed ring
+    (bit-identical to hq_gemm_a8w8 + hq_quantize_fp8 with that ring).
+    Returns out, or (q_out, q_scale) with a ring."""
+    xq, wq = xq.contiguous(), wq.contiguous()
+    x_scale, w_scale = x_scale.contiguous(), w_scale.contiguous()
+    M, K = xq.shape
+    N = wq.shape[0]
+    ring_len = 0
+    if ring is not None:
+        ring_len = ring.numel() - 2
+        if q_out is None:
+            q_out = torch.empty((M, N), dtype=torch.uint8, device=xq.device)
+        if q_scale is None:
+            q_scale = torch.empty((1,), dtype=torch.float32, device=xq.device)
+        if workspace is None:
+            workspace = _workspace(xq.device, hq_quantize_workspace_bytes(PER_TENSOR, M, N, True))
+    elif out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    check(lib.hq_gemm_a8w8_ex(_ptr(xq), _ptr(wq), fmt, _ptr(x_scale), x_scale.numel(), _ptr(w_scale),
+                              w_scale.numel(), _ptr(bias), M, N, K, _ptr(out), _ptr(q_out), q_fmt, _ptr(q_scale),
+                              _ptr(q_amax), _ptr(ring), ring_len, ring_idx, ring_margin, _ptr(workspace),
+                              0 if workspace is None else workspace.numel(), _stream(stream)))
+    return (q_out, q_scale) if ring is not None else out
 
 
 def hq_grouped_gemm_a8w8(xq, wq, x_scale, w_scale, offsets, fmt=E4M3, out=None, stream=None):

@@ -240,9 +240,26 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
 
 namespace {
 
+// Fused epilogue arguments of hq_gemm_a8w8_ex (dense a8w8 only).
+struct GemmEx {
+  const void* bias;
+  uint8_t* q_out;
+  int q_fmt;
+  float* q_scale;
+  float* q_amax;
+  float* ring;
+  int32_t ring_len, ring_idx, ring_margin;
+  void* workspace;
+  size_t workspace_bytes;
+};
+
 hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const float* xs, int64_t xs_len,
                       const float* ws, int64_t ws_len, const int32_t* offsets, int32_t E, int64_t M, int64_t N,
-                      int64_t K, void* out, hq_stream_t stream) {
+                      int64_t K, void* out, hq_stream_t stream, const GemmEx* ex = nullptr) {
+  // FP8 output: q_out given, or (an empty result has no codes to point at)
+  // a ring with no bf16 out
+  const bool empty = M == 0 || N == 0;
+  const bool fp8o = ex != nullptr && (ex->q_out != nullptr || (empty && ex->ring != nullptr && out == nullptr));
   const bool grouped = offsets != nullptr || E != 1 || kind == 1;
   if (kind == 0 && fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", fmt);
   if (M < 0 || N < 0 || K < 0) return fail(HQ_ERR_INVALID_ARG, "negative size");
@@ -265,26 +282,70 @@ hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const flo
       return fail(HQ_ERR_INVALID_ARG, "w_scale_len %lld must be 1 or %lld", (long long)ws_len, (long long)wn);
     if (!is_aligned(xs, 4) || !is_aligned(ws, 4)) return fail(HQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
   }
-  if (!out || (K > 0 && (!a || !b)))
+  size_t need = 0;
+  if (ex) {
+    if (grouped) return fail(HQ_ERR_INVALID_ARG, "fused epilogues are for the dense GEMM");
+    if (fp8o == (out != nullptr)) return fail(HQ_ERR_INVALID_ARG, "exactly one of out and q_out must be given");
+    if (ex->bias && !is_aligned(ex->bias, 4)) return fail(HQ_ERR_MISALIGNED, "bias must be 4-byte aligned");
+    if (fp8o) {
+      if (ex->q_fmt != HQ_E4M3 && ex->q_fmt != HQ_E5M2)
+        return fail(HQ_ERR_INVALID_ARG, "invalid q_fmt %d", ex->q_fmt);
+      if (!ex->ring) return fail(HQ_ERR_INVALID_ARG, "q_out needs a delayed-scaling ring");
+      if (ex->ring_len < 1 || ex->ring_len > (1 << 20))
+        return fail(HQ_ERR_INVALID_ARG, "ring_len %d outside [1, 2^20]", ex->ring_len);
+      if (ex->ring_idx < 0 || ex->ring_idx >= ex->ring_len)
+        return fail(HQ_ERR_INVALID_ARG, "ring_idx %d outside [0, %d)", ex->ring_idx, ex->ring_len);
+      if (ex->ring_margin < -126 || ex->ring_margin > 126)
+        return fail(HQ_ERR_INVALID_ARG, "ring_margin %d outside [-126, 126]", ex->ring_margin);
+      if (!ex->q_scale) return fail(HQ_ERR_INVALID_ARG, "q_scale must not be null");
+      need = hq::quantize_workspace_bytes(0, M, N, 1);
+      if (!ex->workspace || ex->workspace_bytes < need)
+        return fail(HQ_ERR_INVALID_ARG, "q_out needs a zeroed workspace of %zu bytes", need);
+      if (N % 16 != 0) return fail(HQ_ERR_INVALID_ARG, "N = %lld must be a multiple of 16 with q_out", (long long)N);
+      if (!is_aligned(ex->q_out, 16)) return fail(HQ_ERR_MISALIGNED, "q_out must start on a 16-byte boundary");
+      if (!is_aligned(ex->q_scale, 4) || !is_aligned(ex->q_amax, 4) || !is_aligned(ex->ring, 4))
+        return fail(HQ_ERR_MISALIGNED, "q_scale, q_amax and ring must be 4-byte aligned");
+      if (!is_aligned(ex->workspace, 256)) return fail(HQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+    }
+  }
+  void* dst = fp8o ? static_cast<void*>(ex->q_out) : out;
+  if ((!dst && !(fp8o && empty)) || (K > 0 && ((!a && M > 0) || (!b && N > 0))))
     return fail(HQ_ERR_INVALID_ARG, "operand and output pointers must not be null");
-  if (!is_aligned(out, 16)) return fail(HQ_ERR_MISALIGNED, "out must start on a 16-byte boundary");
+  if (!is_aligned(dst, 16)) return fail(HQ_ERR_MISALIGNED, "out must start on a 16-byte boundary");
   if (!is_aligned(a, 16) || !is_aligned(b, 16)) return fail(HQ_ERR_MISALIGNED, "A and B must be 16-byte aligned");
   if (offsets && !is_aligned(offsets, 4)) return fail(HQ_ERR_MISALIGNED, "offsets must be 4-byte aligned");
   const int64_t ebatch = grouped ? E : 1;
-  const Range outs[] = {{out, static_cast<size_t>(M) * static_cast<size_t>(N) * 2, "out"}};
+  const Range outs[] = {{dst, static_cast<size_t>(M) * static_cast<size_t>(N) * (fp8o ? 1 : 2), fp8o ? "q_out" : "out"},
+                        {fp8o ? ex->q_scale : nullptr, 4, "q_scale"},
+                        {fp8o ? ex->q_amax : nullptr, 4, "q_amax"},
+                        {fp8o ? ex->ring : nullptr, fp8o ? static_cast<size_t>(ex->ring_len + 2) * 4 : 0, "ring"},
+                        {fp8o ? ex->workspace : nullptr, need, "workspace"}};
   const Range ins[] = {{a, static_cast<size_t>(M * K * esize), "A"},
                        {b, static_cast<size_t>(ebatch * N * K * esize), "B"},
                        {xs, kind == 0 ? static_cast<size_t>(xs_len) * 4 : 0, "x_scale"},
                        {ws, kind == 0 ? static_cast<size_t>(ws_len) * 4 : 0, "w_scale"},
-                       {offsets, offsets ? static_cast<size_t>(E + 1) * 4 : 0, "offsets"}};
-  hq_status s = check_overlaps(outs, 1, ins, 5);
+                       {offsets, offsets ? static_cast<size_t>(E + 1) * 4 : 0, "offsets"},
+                       {ex ? ex->bias : nullptr, static_cast<size_t>(N) * 2, "bias"}};
+  hq_status s = check_overlaps(outs, 5, ins, 6);
   if (s != HQ_OK) return s;
   const Range devs[] = {{a, 0, "A"}, {b, 0, "B"}, {xs, 0, "x_scale"}, {ws, 0, "w_scale"},
-                        {offsets, 0, "offsets"}, {out, 0, "out"}};
-  s = check_device_ptrs(devs, 6);
+                        {offsets, 0, "offsets"}, {dst, 0, "out"}, {ex ? ex->bias : nullptr, 0, "bias"},
+                        {fp8o ? ex->q_scale : nullptr, 0, "q_scale"}, {fp8o ? ex->q_amax : nullptr, 0, "q_amax"},
+                        {fp8o ? ex->ring : nullptr, 0, "ring"}, {fp8o ? ex->workspace : nullptr, 0, "workspace"}};
+  s = check_device_ptrs(devs, 11);
   if (s != HQ_OK) return s;
   s = check_arch();
   if (s != HQ_OK) return s;
+  if ((M == 0 || N == 0) && fp8o) {
+    // the delayed quantize of the empty result: amax 0, the ring still steps
+    hq::QuantizeArgs qa;
+    qa.x = ex->workspace; qa.xt = HQ_BF16; qa.rows = M; qa.cols = N; qa.fmt = ex->q_fmt; qa.gran = HQ_PER_TENSOR;
+    qa.q = ex->q_out; qa.scales = ex->q_scale; qa.amax_out = ex->q_amax;
+    qa.ring = ex->ring; qa.ring_len = ex->ring_len; qa.ring_idx = ex->ring_idx; qa.ring_margin = ex->ring_margin;
+    qa.ws = ex->workspace;
+    qa.stream = reinterpret_cast<cudaStream_t>(stream);
+    return launched(hq::launch_quantize(qa), "quantize launch");
+  }
   if (M == 0 || N == 0) return ok();
   hq::GemmArgs g;
   g.kind = kind; g.fmt = fmt; g.a = a; g.b = b;
@@ -292,6 +353,15 @@ hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const flo
   g.offsets = offsets; g.E = grouped ? E : 1;
   g.M = M; g.N = N; g.K = K; g.out = out;
   g.stream = reinterpret_cast<cudaStream_t>(stream);
+  if (ex) {
+    g.bias = ex->bias;
+    if (fp8o) {
+      g.out = nullptr;
+      g.q_out = ex->q_out; g.q_fmt = ex->q_fmt; g.q_scale = ex->q_scale; g.q_amax = ex->q_amax;
+      g.ring = ex->ring; g.ring_len = ex->ring_len; g.ring_idx = ex->ring_idx; g.ring_margin = ex->ring_margin;
+      g.q_ws = static_cast<uint32_t*>(ex->workspace);
+    }
+  }
   std::string msg;
   return launched(hq::launch_gemm(g, &msg), "gemm launch", msg);
 }
@@ -302,6 +372,17 @@ hq_status hq_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, 
                        int64_t x_scale_len, const float* w_scale, int64_t w_scale_len, int64_t M, int64_t N,
                        int64_t K, void* out, hq_stream_t stream) {
   return gemm_common(0, xq, wq, fmt, x_scale, x_scale_len, w_scale, w_scale_len, nullptr, 1, M, N, K, out, stream);
+}
+
+hq_status hq_gemm_a8w8_ex(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,
+                          int64_t x_scale_len, const float* w_scale, int64_t w_scale_len, const void* bias,
+                          int64_t M, int64_t N, int64_t K, void* out, uint8_t* q_out, hq_fp8_format q_fmt,
+                          float* q_scale, float* q_amax, float* ring, int32_t ring_len, int32_t ring_idx,
+                          int32_t ring_margin, void* workspace, size_t workspace_bytes, hq_stream_t stream) {
+  const GemmEx ex{bias, q_out, static_cast<int>(q_fmt), q_scale, q_amax, ring, ring_len, ring_idx, ring_margin,
+                  workspace, workspace_bytes};
+  return gemm_common(0, xq, wq, fmt, x_scale, x_scale_len, w_scale, w_scale_len, nullptr, 1, M, N, K, out, stream,
+                     &ex);
 }
 
 hq_status hq_grouped_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,

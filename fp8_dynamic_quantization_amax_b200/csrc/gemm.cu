@@ -21,6 +21,7 @@
 //               main loop of tile i+1.
 // Every wait is bounded: on a stalled barrier the CTA records an error in a
 // device word, drains what it has in flight and exits instead of hanging.
+#include "fp8_cvt.cuh"
 #include "hq_internal.cuh"
 #include "ptx.cuh"
 
@@ -59,6 +60,16 @@ struct Params {
   uint16_t* out;
   uint32_t idesc;
   int prefetch;         // 1: L2-prefetch operands ahead of the TMA loads
+  // fused epilogues (dense only): bias added before the bf16 rounding; FP8
+  // output = the delayed per-tensor quantize of the bf16 result
+  const uint16_t* bias;  // bf16 [N] or null
+  uint8_t* qout;         // FP8 codes [M, N] or null (then out holds bf16)
+  int qfmt;
+  float* qscale;
+  float* qamax;
+  float* ring;
+  int ring_len, ring_idx, ring_margin;
+  uint32_t* qws;         // amax accumulator word
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -144,6 +155,81 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// One chunk's 32 scaled values of a lane's row, plus the bias, rounded to
+// bf16 pairs: w[j] holds columns n0 + 2j (low half) and n0 + 2j + 1.
+template <int KIND>
+__device__ __forceinline__ void chunk_to_bf16(const Params& p, const uint32_t (&v)[32], float xsv, const float* sc,
+                                              int n0, uint32_t (&w)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * j]) : 0.0f;
+    const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+    if (KIND == 0 && p.bias != nullptr) {
+      const uint32_t bb =
+          (n0 + 2 * j < p.N) ? __ldg(reinterpret_cast<const uint32_t*>(p.bias) + ((n0 >> 1) + j)) : 0u;
+      w[j] = pack_bf16x2(__fmaf_rn(a0, xsv * sc[2 * j], __uint_as_float(bb << 16)),
+                         __fmaf_rn(a1, xsv * sc[2 * j + 1], __uint_as_float(bb & 0xFFFF0000u)));
+    } else {
+      w[j] = pack_bf16x2(a0 * (xsv * sc[2 * j]), a1 * (xsv * sc[2 * j + 1]));
+    }
+  }
+}
+
+// FP8 output of one chunk: codes of f32(bf16 value) * m, saturating RNE (NaN
+// -> 0x7F); the lane's finite-only amax is updated over its valid columns
+// and the chunk's codes are stored at the lane's row.
+__device__ __forceinline__ void chunk_to_fp8(const Params& p, const uint32_t (&w)[16], float qm, bool vrow, int row,
+                                             int n0, float& qam) {
+  uint32_t c4[8];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float lo = __uint_as_float(w[j] << 16);
+    const float hi = __uint_as_float(w[j] & 0xFFFF0000u);
+    if (vrow && n0 + 2 * j < p.N) qam = fmaxf(qam, fmaxf(finite_abs(lo), finite_abs(hi)));
+    const uint32_t c2 = (p.qfmt == 0) ? cvt2_exact<0>(__fmul_rn(lo, qm), __fmul_rn(hi, qm))
+                                      : cvt2_exact<1>(__fmul_rn(lo, qm), __fmul_rn(hi, qm));
+    c4[j >> 1] = (j & 1) ? (c4[j >> 1] | (c2 << 16)) : c2;
+  }
+  if (vrow) {  // N % 16 == 0 and n0 % 32 == 0: 16 or 32 codes of this chunk lie inside the row
+    uint8_t* dst = p.qout + static_cast<int64_t>(row) * p.N + n0;
+    st_global_v4(dst, c4[0], c4[1], c4[2], c4[3]);
+    if (n0 + 32 <= p.N) st_global_v4(dst + 16, c4[4], c4[5], c4[6], c4[7]);
+  }
+}
+
+// End of a kernel with an FP8 output: the CTA's amax joins the workspace
+// word; the last CTA (threadfence + the ring's counter word) folds it into
+// the ring and publishes the next multiplier, as the delayed quantize does.
+template <int NWARPS>
+__device__ void finalize_fp8_out(const Params& p, float qam) {
+  __shared__ float red[NWARPS];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) qam = fmaxf(qam, __shfl_xor_sync(0xFFFFFFFFu, qam, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = qam;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  float a = 0.0f;
+#pragma unroll
+  for (int w = 0; w < NWARPS; ++w) a = fmaxf(a, red[w]);
+  atomicMax(p.qws, __float_as_uint(a));  // non-negative: bit order = value order
+  __threadfence();
+  uint32_t* counter = reinterpret_cast<uint32_t*>(p.ring + p.ring_len + 1);
+  if (atomicAdd(counter, 1u) != gridDim.x - 1) return;
+  __threadfence();
+  const float am = __uint_as_float(atomicExch(p.qws, 0u));
+  const float m = __ldcg(p.ring + p.ring_len);  // the multiplier every CTA used
+  p.ring[p.ring_idx] = am;
+  float win = 0.0f;
+  for (int i = 0; i < p.ring_len; ++i) win = fmaxf(win, __ldcg(p.ring + i));
+  if (win <= FLT_MAX && win > 0.0f) {
+    const float next = ldexpf(__fdiv_rn(p.qfmt == 0 ? kFmaxE4M3 : kFmaxE5M2, win), -p.ring_margin);
+    if (next <= FLT_MAX && next > 0.0f) p.ring[p.ring_len] = next;
+  }
+  p.qscale[0] = __fdiv_rn(1.0f, m);
+  if (p.qamax) p.qamax[0] = am;
+  atomicExch(counter, 0u);
 }
 
 // L2 prefetch of a TMA tile (no shared-memory destination, no barrier).
@@ -332,6 +418,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   const int total = (p.offsets != nullptr) ? tile_prefix[p.E] : p.m_tiles * p.n_tiles;
+  float qam = 0.0f;  // FP8 output: this thread's finite-only amax of the bf16 result
 
   if (warp == 0) {
     if (lane == 0) {
@@ -429,6 +516,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     uint8_t* sb = sOut + ew * 2048;
     float* wsh = sWs + ew * kMyChunks * 32;
     const uint64_t out_pol = l2_evict_first_policy();
+    const float qm = (p.qout != nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
     int i = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int acc = i & 1;
@@ -466,11 +554,10 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
         if (n0 >= ncap) continue;
         const float* sc = wsh + i * 32;
         uint32_t w[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * j]) : 0.0f;
-          const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-          w[j] = pack_bf16x2(a0 * (xsv * sc[2 * j]), a1 * (xsv * sc[2 * j + 1]));
+        chunk_to_bf16<KIND>(p, v, xsv, sc, n0, w);
+        if (KIND == 0 && p.qout != nullptr) {
+          chunk_to_fp8(p, w, qm, vrow, row, n0, qam);
+          continue;
         }
         // the tensor map clips at N; a 16-column tail chunk inside N is masked
         if (tma_ok && (BN % 32 == 0 || n0 + 32 <= T.col0 + BN)) {
@@ -501,6 +588,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemm1Threads / 32>(p, qam);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
@@ -571,6 +659,28 @@ bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, st
   return true;
 }
 
+// The bf16 output's tensor map.  With an FP8 output the kernels store no bf16
+// tile; the map then describes the code buffer (M rows of N bytes) so that it
+// still names memory the call owns.
+bool make_result_map(CUtensorMap* map, const GemmArgs& a, std::string* msg) {
+  if (a.q_out != nullptr)
+    return make_out_map(map, a.q_out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N / 2), msg);
+  return make_out_map(map, a.out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), msg);
+}
+
+void set_fused_epilogue(const GemmArgs& a, Params& p) {
+  p.bias = static_cast<const uint16_t*>(a.bias);
+  p.qout = a.q_out;
+  p.qfmt = a.q_fmt;
+  p.qscale = a.q_scale;
+  p.qamax = a.q_amax;
+  p.ring = a.ring;
+  p.ring_len = a.ring_len;
+  p.ring_idx = a.ring_idx;
+  p.ring_margin = a.ring_margin;
+  p.qws = a.q_ws;
+}
+
 template <int KIND, int BN, int STAGES, int AROWS = kBM, int KPS = 1>
 cudaError_t run(const GemmArgs& a, std::string* msg) {
   constexpr int kElem = (KIND == 0) ? 1 : 2;
@@ -596,8 +706,7 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
       return cudaErrorInvalidValue;
   }
   CUtensorMap to;
-  if (!make_out_map(&to, a.out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), msg))
-    return cudaErrorInvalidValue;
+  if (!make_result_map(&to, a, msg)) return cudaErrorInvalidValue;
 
   Params p;
   p.M = static_cast<int>(a.M);
@@ -617,6 +726,7 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
   // Grouped tiles re-read A and B from L2 at a high byte rate and gain from
   // the prefetch; the small-M dense stream reads W once and loses by it.
   p.prefetch = (a.offsets != nullptr) ? 1 : 0;
+  set_fused_epilogue(a, p);
   const uint32_t ab_fmt = (KIND == 0) ? static_cast<uint32_t>(a.fmt) : 1u;  // E4M3/E5M2, or BF16
   p.idesc = (1u << 4)                                   // D: FP32
             | (ab_fmt << 7) | (ab_fmt << 10)            // A and B element types
@@ -773,6 +883,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
   const int total = (p.offsets != nullptr) ? tile_prefix[p.E] : p.m_tiles * p.n_tiles;  // tiles of 256 x BN
+  float qam = 0.0f;  // FP8 output: this thread's finite-only amax of the bf16 result
 
   if (warp == 0) {
     if (lane == 0) {
@@ -872,6 +983,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint8_t* sb = sOut + ew * 2048;
     float* wsh = sWs + ew * kMyChunks * 32;
     const uint64_t out_pol = l2_evict_first_policy();
+    const float qm = (p.qout != nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
     uint32_t tempty_leader[kAccs];
 #pragma unroll
     for (int a = 0; a < kAccs; ++a) tempty_leader[a] = mapa_shared(smem_u32(&tempty_bar[a]), 0);
@@ -912,11 +1024,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (n0 >= p.N) continue;
         const float* sc = wsh + j * 32;
         uint32_t w[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * q]) : 0.0f;
-          const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * q + 1]) : 0.0f;
-          w[q] = pack_bf16x2(a0 * (xsv * sc[2 * q]), a1 * (xsv * sc[2 * q + 1]));
+        chunk_to_bf16<KIND>(p, v, xsv, sc, n0, w);
+        if (KIND == 0 && p.qout != nullptr) {
+          chunk_to_fp8(p, w, qm, vrow, row, n0, qam);
+          continue;
         }
         if (tma_ok) {
           if (lane == 0) bulk_wait_read_le0();  // the previous chunk's store has read the staging tile
@@ -946,6 +1057,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemmThreads / 32>(p, qam);
   cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
   if (warp == 1) {
     tc_fence_after();
@@ -995,8 +1107,7 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
       return cudaErrorInvalidValue;
   }
   CUtensorMap to;
-  if (!make_out_map(&to, a.out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), msg))
-    return cudaErrorInvalidValue;
+  if (!make_result_map(&to, a, msg)) return cudaErrorInvalidValue;
   Params p;
   memset(&p, 0, sizeof(p));
   p.M = static_cast<int>(a.M);
@@ -1013,6 +1124,7 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
   p.ws = a.w_scale;
   p.ws_bcast = (a.w_scale_len == 1) ? 1 : 0;
   p.out = static_cast<uint16_t*>(a.out);
+  set_fused_epilogue(a, p);
   const uint32_t ab_fmt = (KIND == 0) ? static_cast<uint32_t>(a.fmt) : 1u;
   p.idesc = (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
             (static_cast<uint32_t>(256 >> 4) << 24);  // one MMA: M = 256 across the pair, N = 256

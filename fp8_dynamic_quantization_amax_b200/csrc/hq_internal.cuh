@@ -45,8 +45,17 @@ struct GemmArgs {
   const int32_t* offsets;   // null: dense GEMM (one group of M rows)
   int E;
   int64_t M, N, K;
-  void* out;
+  void* out;                // bf16 [M, N]; null when q_out is set
   cudaStream_t stream;
+  // fused epilogues (dense only)
+  const void* bias = nullptr;   // bf16 [N]
+  uint8_t* q_out = nullptr;     // FP8 codes [M, N]: the delayed per-tensor quantize of the bf16 result
+  int q_fmt = 0;
+  float* q_scale = nullptr;
+  float* q_amax = nullptr;
+  float* ring = nullptr;
+  int ring_len = 0, ring_idx = 0, ring_margin = 0;
+  uint32_t* q_ws = nullptr;     // amax accumulator word (zero between calls)
 };
 
 // Returns cudaSuccess or the failing call's error; *msg gets a description.

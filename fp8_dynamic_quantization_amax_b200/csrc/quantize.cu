@@ -30,6 +30,7 @@
 //     whether any non-finite element was seen.  Only then does a thread redo
 //     its range on the exact path (finite-only amax, canonical NaN codes).
 //   - the cast is one FMUL per element plus one cvt.rn.satfinite per pair.
+#include "fp8_cvt.cuh"
 #include "hq_internal.cuh"
 #include "ptx.cuh"
 
@@ -155,31 +156,6 @@ __device__ __forceinline__ uint32_t cvt4(float a0, float a1, float a2, float a3)
         "mov.b32 %0, {l, h};\n\t}"
         : "=r"(d) : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
   return d;
-}
-
-// Exact-path conversion of two values: a NaN input gives the canonical 0x7F.
-template <int FMT>
-__device__ __forceinline__ uint32_t cvt2_exact(float lo, float hi) {
-  unsigned short r;
-  if (FMT == 0)
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  else
-    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  uint32_t v = r;
-  v = isnan(lo) ? ((v & 0xFF00u) | 0x7Fu) : v;
-  v = isnan(hi) ? ((v & 0x00FFu) | 0x7F00u) : v;
-  return v;
-}
-
-template <int FMT>
-__device__ __forceinline__ uint8_t cvt1_exact(float y) {
-  return static_cast<uint8_t>(cvt2_exact<FMT>(y, 0.0f) & 0xFFu);
-}
-
-// |v| if finite, else 0 (NaN and +-Inf do not take part in amax).
-__device__ __forceinline__ float finite_abs(float v) {
-  const float a = fabsf(v);
-  return (a <= FLT_MAX) ? a : 0.0f;
 }
 
 template <int DT>

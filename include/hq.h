@@ -178,6 +178,52 @@ hq_status hq_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt,
                        int64_t M, int64_t N, int64_t K, void* out, hq_stream_t stream);
 
 /*
+ * The scaled FP8 GEMM with the fused epilogues of AstrAI ops.cu: mm_fp8
+ * ("out_dtype" 1 = an FP8 output with its "out_scale", the output
+ * quantization step) and linear_forward_fp8 (the bias added in the GEMM
+ * epilogue).  Dense GEMMs only.
+ *
+ *   h[m, n] = bf16_rn( acc[m, n] * (x_scale[m'] * w_scale[n']) + bias[n] )
+ *
+ * (one f32 fused multiply-add before the rounding; no bias: as hq_gemm_a8w8).
+ *
+ * q_out == NULL: h is written to out, as hq_gemm_a8w8 does.
+ * q_out != NULL: out must be NULL and h is not written.  Instead h is
+ *   quantized per tensor with the delayed-scaling ring, exactly as
+ *   hq_quantize_fp8(h, PER_TENSOR, q_fmt, ring, ring_idx, ring_margin) would
+ *   quantize it: q = satfinite RNE code of f32(h) * m with m = ring[ring_len]
+ *   on entry; *q_scale = 1/m; *q_amax (nullable) = max |h| over finite
+ *   elements; the last CTA folds that amax into ring[ring_idx] and publishes
+ *   the next multiplier in ring[ring_len] (the ring and workspace rules of
+ *   hq_quantize_fp8's delayed mode).  The result is bit-identical to the two
+ *   calls; the bf16 h never reaches memory.
+ *
+ * Arguments beyond hq_gemm_a8w8's:
+ *   bias      device bf16 (uint16 bits) [N], 4-byte aligned, or NULL
+ *   out       device bf16 [M, N] as in hq_gemm_a8w8, or NULL with q_out
+ *   q_out     device uint8 [M, N] FP8 codes, 16-byte aligned; needs N % 16 == 0.
+ *             NULL is accepted for an empty result (M == 0 or N == 0) with a
+ *             ring and out == NULL: the FP8 mode is then implied
+ *   q_fmt     format of the output codes
+ *   q_scale   device f32 [1]: receives 1/m (the dequant scale of q_out)
+ *   q_amax    device f32 [1] or NULL
+ *   ring, ring_len, ring_idx, ring_margin: as hq_quantize_fp8 (required with q_out)
+ *   workspace device, >= hq_quantize_workspace_bytes(PER_TENSOR, M, N, 1)
+ *             bytes, all zero on entry; zero again on return (required with q_out)
+ * Errors: those of hq_gemm_a8w8, plus HQ_ERR_INVALID_ARG (both or neither
+ *   of out / q_out, q_out without ring / q_scale / workspace, bad ring
+ *   index, N % 16 != 0 with q_out, bad q_fmt), HQ_ERR_MISALIGNED (q_out,
+ *   bias, q_scale, ring, workspace) and HQ_ERR_OVERLAP among all buffers.
+ * M == 0 or N == 0 with q_out runs the delayed quantize of the empty h
+ * (amax 0, the ring updated, *q_scale = 1/m); with out it is a no-op.
+ */
+hq_status hq_gemm_a8w8_ex(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,
+                          int64_t x_scale_len, const float* w_scale, int64_t w_scale_len, const void* bias,
+                          int64_t M, int64_t N, int64_t K, void* out, uint8_t* q_out, hq_fp8_format q_fmt,
+                          float* q_scale, float* q_amax, float* ring, int32_t ring_len, int32_t ring_idx,
+                          int32_t ring_margin, void* workspace, size_t workspace_bytes, hq_stream_t stream);
+
+/*
  * Grouped (per-expert) scaled FP8 GEMM (megablocks-hip TODO-gg.md gmm):
  * for each expert e and each row r in [offsets[e], offsets[e+1]):
  *   out[r, n] = bf16_rn( x_scale[r'] * w_scale[e*N + n'] *

@@ -127,6 +127,33 @@ def test_gemm_rejections():
     assert g8(out=BASE + 0x2000000 - 0x10) == OVERLAP    # out runs into x_scale
 
 
+def gx(out=None, q_out=BASE + 0x4000000, q_fmt=H.E4M3, q_scale=BASE + 0x5000000, q_amax=None,
+       ring=BASE + 0x5001000, ring_len=16, ring_idx=0, margin=0, ws=BASE + 0x5100000, wsb=256, bias=None,
+       M=64, N=128, K=256):
+    return L.hq_gemm_a8w8_ex(BASE, BASE + 0x1000000, H.E4M3, BASE + 0x2000000, 64, BASE + 0x3000000, 128, bias,
+                             M, N, K, out, q_out, q_fmt, q_scale, q_amax, ring, ring_len, ring_idx, margin, ws, wsb,
+                             None)
+
+
+def test_fused_epilogue_rejections():
+    # hq_gemm_a8w8_ex: exactly one output; the FP8 output follows the
+    # delayed-quantize contract (ring, scale, zeroed workspace)
+    assert gx(out=BASE + 0x6000000) == INVALID                 # both outputs
+    assert gx(q_out=None) == INVALID                           # neither
+    assert gx(ring=None) == INVALID and gx(q_scale=None) == INVALID and gx(ws=None) == INVALID
+    assert gx(ring_idx=16) == INVALID and gx(ring_len=0) == INVALID and gx(margin=200) == INVALID
+    assert gx(q_fmt=7) == INVALID and gx(wsb=64) == INVALID
+    assert gx(N=24) == INVALID                                 # codes rows need N % 16 == 0
+    assert gx(q_out=BASE + 0x4000008) == MISALIGNED
+    assert gx(bias=BASE + 0x5200001) == MISALIGNED
+    assert gx(ws=BASE + 0x5100010) == MISALIGNED
+    assert gx(q_out=BASE + 0x10) == OVERLAP                    # codes over XQ
+    assert gx(bias=BASE + 0x4000000) == OVERLAP                # codes over the bias
+    assert gx(ring=BASE + 0x5000000) == OVERLAP                # ring over q_scale
+    # the bf16 output with a bias keeps hq_gemm_a8w8's checks
+    assert gx(out=BASE + 0x6000002, q_out=None, ring=None, ws=None, bias=BASE + 0x5200000) == MISALIGNED
+
+
 def test_grouped_rejections():
     gg = L.hq_grouped_gemm_a8w8
     args = dict(xq=BASE, wq=BASE + 0x1000000, fmt=0, xs=BASE + 0x2000000, xsl=100, ws=BASE + 0x3000000,
