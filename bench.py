@@ -1,7 +1,7 @@
 """Benchmark of the dynamic-FP8 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large|large4096|large8192|decode1|decode16|decode128|sweep|stack|moe|moe_bf16]
+                    [--workload large|large4096|large8192|decode1|decode16|decode128|sweep|stack|backward|moe|moe_bf16]
 
 Default workload (the large a8w8 GEMM layer): X bf16 [16384, 8192] ~N(0,1),
 W bf16 [28672, 8192] ~N(0,0.02).  One step = per-token E4M3 quantize of X,
@@ -67,6 +67,7 @@ WORKLOADS = {
     "decode128": dict(kind="decode", M=128, N=28672, K=8192),
     "sweep": dict(kind="sweep", M=8192, N=0, K=8192),
     "stack": dict(kind="stack", M=2048, N=4096, K=1024, steps_cycle=200, ring=16),
+    "backward": dict(kind="backward", M=16384, N=28672, K=8192, ring=16),
     "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
     "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }
@@ -79,6 +80,11 @@ def workload_desc(name, cfg):
                 "per-output-channel E4M3%s, out bf16 [%d,%d] (caller-owned)" %
                 ("large" if k == "layer" else "decode", cfg["M"], cfg["K"], cfg["N"], cfg["K"],
                  "" if k == "layer" else " (quantized once: static weights)", cfg["M"], cfg["N"]))
+    if k == "backward":
+        return ("backward of the large a8w8 layer: grad g bf16 [%d,%d] ~N(0,1e-3) quantized per tensor with a "
+                "delayed ring into row-major and transposed codes; W bf16 [%d,%d] and X bf16 [%d,%d] re-quantized "
+                "transposed with their forward multipliers; dX = g W [%d,%d], dW = g^T X [%d,%d] on the NT GEMM" %
+                (cfg["M"], cfg["N"], cfg["N"], cfg["K"], cfg["M"], cfg["K"], cfg["M"], cfg["K"], cfg["N"], cfg["K"]))
     if k == "stack":
         return ("delayed-scaling linear stack: X_t bf16 [2048,1024] (std 0.5 -> 8 over 200 steps), W_up bf16 "
                 "[4096,1024], W_down bf16 [1024,4096] ~N(0,0.02); per-tensor E4M3 with four amax-history rings "
@@ -262,6 +268,80 @@ def build(args, cfg, rank, dev, stream, peaks):
                                                                                M * N * 2 >> 20)
         return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=h2d, d2h=M * N * 2,
                     roofline=roofline, extras=extras, l2=l2, flush=None)
+
+    if kind == "backward":
+        Lr = cfg["ring"]
+        g_host = bf16_host(W.f32_to_bf16_bits(W.normal((M, N), 1e-3, 100 + rank))).view(M, N)
+        x_host = bf16_host(W.large_x(M, K, seed=rank)).view(M, K)
+        w_dev = bf16_host(W.large_w(N, K)).view(N, K).to(dev)
+        g, x = g_host.to(dev), x_host.to(dev)
+        ring = torch.zeros(Lr + 2, dtype=torch.float32, device=dev)
+        ring[Lr] = 448.0 / 4e-3  # E4M3 max over an expected gradient amax
+        # the forward's multipliers of W and X (their dynamic per-tensor scales)
+        _, sw0 = hq.hq_quantize_fp8(w_dev, hq.E4M3, hq.PER_TENSOR)
+        _, sx0 = hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TENSOR)
+        mw, mx = 1.0 / sw0, 1.0 / sx0
+        g8 = torch.empty((M, N), dtype=torch.uint8, device=dev)
+        gT8 = torch.empty((N, M), dtype=torch.uint8, device=dev)
+        wT8 = torch.empty((K, N), dtype=torch.uint8, device=dev)
+        xT8 = torch.empty((K, M), dtype=torch.uint8, device=dev)
+        sg, sw, sx = (torch.empty((1,), dtype=torch.float32, device=dev) for _ in range(3))
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        dX_host = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
+        dW_host = torch.empty((N, K), dtype=torch.bfloat16).pin_memory()
+        wsg, wsw, wsx = (torch.zeros(256, dtype=torch.uint8, device=dev) for _ in range(3))
+        lib, P = hq.lib, (lambda t: None if t is None else t.data_ptr())
+        st = stream.cuda_stream
+        counter = [0]
+
+        def qt(src, qo, qt_, scale, mult=None, rg=None, idx=0, ws_=None):
+            rows, cols = src.shape
+            hq.check(lib.hq_quantize_fp8_transpose(P(src), hq.BF16, rows, cols, hq.E4M3, P(qo), P(qt_), P(scale),
+                                                   None, P(mult), P(rg), Lr if rg is not None else 0, idx, 0,
+                                                   P(ws_), ws_.numel(), st))
+
+        def quant():
+            qt(g, g8, gT8, sg, rg=ring, idx=counter[0] % Lr, ws_=wsg)
+            counter[0] += 1
+            qt(w_dev, None, wT8, sw, mult=mw, ws_=wsw)
+            qt(x, None, xT8, sx, mult=mx, ws_=wsx)
+
+        def gemms():
+            hq.hq_gemm_a8w8(g8, wT8, sg, sw, hq.E4M3, out=dX, stream=stream)
+            hq.hq_gemm_a8w8(gT8, xT8, sg, sx, hq.E4M3, out=dW, stream=stream)
+
+        calls = [("quantize g, W^T, X^T", quant, 3), ("dX and dW GEMMs", gemms, 2)]
+
+        def e2e():
+            g.copy_(g_host, non_blocking=True)
+            x.copy_(x_host, non_blocking=True)
+            quant()
+            gemms()
+            dX_host.copy_(dX, non_blocking=True)
+            dW_host.copy_(dW, non_blocking=True)
+
+        flops = 2.0 * 2 * M * N * K
+
+        def roofline(ms):
+            a = flops / (ms["dX and dW GEMMs"] / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": round(a, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(a / fp8_peak, 4), "traffic": None,
+                    "kernel": "k_gemm2<fp8, 256x512 CTA-pair tile> (dX and dW)",
+                    "peak_source": "%s bf16 burst x 2 (nominal fp8/bf16)" % peaks["_src"]}
+
+        def extras(ms):
+            qbytes = (M * N * 2 + 2 * M * N) + (N * K * 2 + N * K) + (M * K * 2 + M * K)
+            gb = qbytes / (ms["quantize g, W^T, X^T"] / 1e3) / 1e9
+            return {"quantize_transpose": {"ms": round(ms["quantize g, W^T, X^T"], 4), "GB/s": round(gb, 1),
+                                           "frac_hbm": round(gb / peaks["hbm_gbs"], 4),
+                                           "bytes": "g: 2 B read + 2 x 1 B codes; W, X: 2 B read + 1 B codes"},
+                    "gemm_ms": round(ms["dX and dW GEMMs"], 4)}
+
+        return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=(M * N + M * K) * 2,
+                    d2h=(M * K + N * K) * 2, roofline=roofline, extras=extras, flush=None,
+                    l2="inputs larger than L2 (g %d MB, X %d MB, W %d MB); no flush" %
+                       (M * N * 2 >> 20, M * K * 2 >> 20, N * K * 2 >> 20))
 
     if kind == "stack":
         T, D, H, L = M, K, N, cfg["ring"]

@@ -21,7 +21,8 @@ PER_TENSOR, PER_TOKEN, PER_CHANNEL = 0, 1, 2
 F32, BF16, F16 = 0, 1, 2
 
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
-            "hq_quantize_fp8", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
+            "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
+            "hq_grouped_gemm_bf16",
             "hq_quantize_fp8_noalloc", "hq_check_device_error", "hq_last_error", "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
 
@@ -51,6 +52,8 @@ def _load():
     L.hq_quantize_fp8.restype = ci
     L.hq_quantize_fp8_noalloc.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P]
     L.hq_quantize_fp8_noalloc.restype = ci
+    L.hq_quantize_fp8_transpose.argtypes = [P, ci, i64, i64, ci, P, P, P, P, P, P, i32, i32, i32, P, sz, P]
+    L.hq_quantize_fp8_transpose.restype = ci
     L.hq_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
     L.hq_gemm_a8w8.restype = ci
     L.hq_gemm_a8w8_ex.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P, P, ci, P, P, P, i32, i32, i32, P,
@@ -151,6 +154,29 @@ def hq_quantize_fp8(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=N
                               _ptr(workspace), 0 if workspace is None else workspace.numel(),
                               _stream(stream)))
     return q, scales
+
+
+def hq_quantize_fp8_transpose(x, fmt=E4M3, q=False, multiplier=None, amax_out=None, ring=None, ring_idx=0,
+                              ring_margin=0, workspace=None, stream=None):
+    """Per-tensor quantize of a 2-D CUDA tensor writing the codes transposed
+    (qt [cols, rows]) and, with q=True, also row-major.  The multiplier is the
+    ring's (delayed, the ring stepped), a caller's device f32 `multiplier`
+    (static), or the tensor's own fmax/amax (dynamic).  Returns (q or None,
+    qt, dequant scale f32[1])."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    x = x.contiguous()
+    rows, cols = x.shape
+    qo = torch.empty((rows, cols), dtype=torch.uint8, device=x.device) if q else None
+    qt = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((1,), dtype=torch.float32, device=x.device)
+    ring_len = 0 if ring is None else ring.numel() - 2
+    if workspace is None:
+        workspace = _workspace(x.device, hq_quantize_workspace_bytes(PER_TENSOR, rows, cols, True))
+    check(lib.hq_quantize_fp8_transpose(_ptr(x), _DT[x.dtype], rows, cols, fmt, _ptr(qo), _ptr(qt), _ptr(scales),
+                                        _ptr(amax_out), _ptr(multiplier), _ptr(ring), ring_len, ring_idx,
+                                        ring_margin, _ptr(workspace), workspace.numel(), _stream(stream)))
+    return qo, qt, scales
 
 
 def hq_quantize_fp8_noalloc(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=None, ring=None,

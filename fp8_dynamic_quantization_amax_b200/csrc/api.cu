@@ -238,6 +238,66 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
   return launched(hq::launch_quantize(a), "quantize launch");
 }
 
+hq_status hq_quantize_fp8_transpose(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                                    uint8_t* q, uint8_t* qt, float* scales, float* amax_out, const float* multiplier,
+                                    float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,
+                                    void* workspace, size_t workspace_bytes, hq_stream_t stream) {
+  // ---- arguments
+  if (xt != HQ_F32 && xt != HQ_BF16 && xt != HQ_F16) return fail(HQ_ERR_INVALID_ARG, "invalid dtype %d", (int)xt);
+  if (fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", (int)fmt);
+  if (rows < 0 || cols < 0) return fail(HQ_ERR_INVALID_ARG, "negative shape [%lld, %lld]", (long long)rows, (long long)cols);
+  if (rows >= k2p31 || cols >= k2p31 || (cols > 0 && rows > (k2p40 - 1) / cols))
+    return fail(HQ_ERR_TOO_LARGE, "shape [%lld, %lld] is beyond the supported range", (long long)rows, (long long)cols);
+  if (rows % 16 != 0 || cols % 16 != 0)
+    return fail(HQ_ERR_INVALID_ARG, "rows and cols must be multiples of 16 (16-byte code rows both ways)");
+  if (multiplier && ring) return fail(HQ_ERR_INVALID_ARG, "give a multiplier or a ring, not both");
+  if (ring) {
+    if (ring_len < 1 || ring_len > (1 << 20)) return fail(HQ_ERR_INVALID_ARG, "ring_len %d outside [1, 2^20]", ring_len);
+    if (ring_idx < 0 || ring_idx >= ring_len)
+      return fail(HQ_ERR_INVALID_ARG, "ring_idx %d outside [0, %d)", ring_idx, ring_len);
+    if (ring_margin < -126 || ring_margin > 126) return fail(HQ_ERR_INVALID_ARG, "ring_margin %d outside [-126, 126]", ring_margin);
+  }
+  const int64_t n = rows * cols;
+  const size_t esize = (xt == HQ_F32) ? 4 : 2;
+  const size_t need = hq::quantize_workspace_bytes(0, rows, cols, 1);
+  if (n > 0 && (!x || !qt)) return fail(HQ_ERR_INVALID_ARG, "x and qt must not be null");
+  if (!scales) return fail(HQ_ERR_INVALID_ARG, "scales must not be null");
+  if (!workspace || workspace_bytes < need)
+    return fail(HQ_ERR_INVALID_ARG, "a zeroed workspace of %zu bytes is needed", need);
+  if (!is_aligned(x, 16) || !is_aligned(q, 16) || !is_aligned(qt, 16))
+    return fail(HQ_ERR_MISALIGNED, "x, q and qt must start on 16-byte boundaries");
+  if (!is_aligned(scales, 4) || !is_aligned(amax_out, 4) || !is_aligned(ring, 4) || !is_aligned(multiplier, 4))
+    return fail(HQ_ERR_MISALIGNED, "scales, amax_out, multiplier and ring must be 4-byte aligned");
+  if (!is_aligned(workspace, 256)) return fail(HQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  const Range outs[] = {{q, q ? static_cast<size_t>(n) : 0, "q"},
+                        {qt, static_cast<size_t>(n), "qt"},
+                        {scales, 4, "scales"},
+                        {amax_out, amax_out ? 4u : 0u, "amax_out"},
+                        {ring, ring ? static_cast<size_t>(ring_len + 2) * 4 : 0, "ring"},
+                        {workspace, need, "workspace"}};
+  const Range ins[] = {{x, static_cast<size_t>(n) * esize, "x"}, {multiplier, multiplier ? 4u : 0u, "multiplier"}};
+  hq_status s = check_overlaps(outs, 6, ins, 2);
+  if (s != HQ_OK) return s;
+  // ---- device
+  const Range devs[] = {{n > 0 ? x : nullptr, 0, "x"}, {q, 0, "q"}, {n > 0 ? qt : nullptr, 0, "qt"},
+                        {scales, 0, "scales"}, {amax_out, 0, "amax_out"}, {multiplier, 0, "multiplier"},
+                        {ring, 0, "ring"}, {workspace, 0, "workspace"}};
+  s = check_device_ptrs(devs, 8);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  // ---- launch
+  hq::QuantizeArgs a;
+  a.x = x; a.xt = xt; a.rows = rows; a.cols = cols; a.fmt = fmt; a.gran = HQ_PER_TENSOR;
+  a.q = q; a.scales = scales; a.amax_out = amax_out;
+  a.ring = ring; a.ring_len = ring_len; a.ring_idx = ring_idx; a.ring_margin = ring_margin;
+  a.ws = workspace;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.qt = qt;
+  a.mult = multiplier;
+  return launched(hq::launch_quantize_transpose(a), "quantize-transpose launch");
+}
+
 namespace {
 
 // Fused epilogue arguments of hq_gemm_a8w8_ex (dense a8w8 only).

@@ -28,10 +28,15 @@ struct QuantizeArgs {
   int ring_len, ring_idx, ring_margin;
   void* ws;          // workspace (may be null when none is needed)
   cudaStream_t stream;
+  uint8_t* qt = nullptr;        // transposed codes [cols, rows] (launch_quantize_transpose)
+  const float* mult = nullptr;  // a caller's multiplier (static per-tensor form)
 };
 
 size_t quantize_workspace_bytes(int gran, int64_t rows, int64_t cols, int delayed);
 cudaError_t launch_quantize(const QuantizeArgs& a);
+// Per-tensor quantize writing the codes row-major (a.q, nullable) and
+// transposed (a.qt); rows % 16 == 0, cols % 16 == 0, x 16-byte aligned.
+cudaError_t launch_quantize_transpose(const QuantizeArgs& a);
 
 struct GemmArgs {
   int kind;                 // 0: fp8 a8w8 (kind::f8f6f4), 1: bf16 (kind::f16)

@@ -1272,6 +1272,116 @@ __global__ void __launch_bounds__(kThreads) k_delayed(
   }
 }
 
+// ----------------------------------------- per-tensor with a transposed copy
+// For the backward GEMMs (AstrAI ops.cu linear_backward_fp8: dX reads the
+// weight codes transposed, dW reads the gradient and activation codes
+// transposed) one pass writes the codes of x [R, C] row-major (optional) and
+// transposed, qt [C, R].  A CTA walks 64 x 64 tiles: thread t quantizes the
+// 16 consecutive elements at tile row t / 4, columns 16 (t % 4) .. + 15,
+// stores them to q and to a shared tile; after a barrier it gathers the 16
+// codes at tile column t / 4, rows 16 (t % 4) .. + 15, and stores them as one
+// 16-byte piece of qt.  Every access of x, q and qt is a 16-byte vector.
+// MODE 0: dynamic, the multiplier published by a k_tensor_amax pass in
+// ws[2] (the last CTA returns ws[1..3] to zero); 1: delayed, the ring's
+// multiplier, the last CTA steps the ring (as k_delayed); 2: a caller's
+// multiplier, the ring-free static form (amax reported, nothing stepped).
+constexpr int kQtTile = 64;
+constexpr int kQtPitch = 68;  // bytes per shared tile row: conflict-light column gathers
+
+template <int FMT>
+__device__ __forceinline__ uint32_t codes4(const float* f, float m) {
+  return cvt2_exact<FMT>(__fmul_rn(f[0], m), __fmul_rn(f[1], m)) |
+         (cvt2_exact<FMT>(__fmul_rn(f[2], m), __fmul_rn(f[3], m)) << 16);
+}
+
+template <int DT, int FMT, int MODE>
+__global__ void __launch_bounds__(kThreads) k_quant_transpose(
+    const void* __restrict__ x, int64_t rows, int64_t cols, uint8_t* __restrict__ q, uint8_t* __restrict__ qt,
+    const float* __restrict__ mult, float* __restrict__ ring, int len, int idx, int margin,
+    uint32_t* __restrict__ ws, float* __restrict__ scales, float* __restrict__ amax_out) {
+  constexpr int VEC = Dt<DT>::kVec;
+  __shared__ __align__(16) uint8_t tile[kQtTile * kQtPitch];
+  __shared__ float sh[kThreads / 32];
+  __shared__ bool is_last;
+  float m;
+  if (MODE == 0) m = __uint_as_float(__ldcg(&ws[2]));
+  else if (MODE == 1) m = __ldcg(&ring[len]);
+  else m = __ldg(mult);
+  const int64_t ntr = (rows + kQtTile - 1) / kQtTile;
+  const int64_t ntc = (cols + kQtTile - 1) / kQtTile;
+  const int t = threadIdx.x;
+  const int lr = t >> 2, seg = (t & 3) * 16;  // quantize: tile row lr, columns seg .. seg + 15
+  float amax = 0.0f;
+  for (int64_t ti = blockIdx.x; ti < ntr * ntc; ti += gridDim.x) {
+    const int64_t r0 = (ti / ntc) * kQtTile, c0 = (ti % ntc) * kQtTile;
+    const int64_t r = r0 + lr, c = c0 + seg;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (r < rows && c < cols) {  // cols % 16 == 0: all 16 elements are inside
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + (r * cols + c) * Dt<DT>::kSize);
+#pragma unroll
+      for (int v = 0; v < 16 / VEC; ++v) {
+        float f[VEC];
+        Dt<DT>::unpack(ld_stream(src + v), f);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) amax = fmaxf(amax, finite_abs(f[i]));
+#pragma unroll
+        for (int k = 0; k < VEC / 4; ++k) w[v * (VEC / 4) + k] = codes4<FMT>(f + 4 * k, m);
+      }
+      if (q != nullptr) *reinterpret_cast<uint4*>(q + r * cols + c) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    uint32_t* trow = reinterpret_cast<uint32_t*>(tile + lr * kQtPitch + seg);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) trow[k] = w[k];
+    __syncthreads();
+    const int jc = t >> 2, rs = (t & 3) * 16;  // gather: tile column jc, rows rs .. rs + 15
+    const int64_t qr = c0 + jc, qc = r0 + rs;
+    if (qr < cols && qc < rows) {  // rows % 16 == 0
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint8_t* col = tile + (rs + 4 * k) * kQtPitch + jc;
+        o[k] = static_cast<uint32_t>(col[0]) | (static_cast<uint32_t>(col[kQtPitch]) << 8) |
+               (static_cast<uint32_t>(col[2 * kQtPitch]) << 16) | (static_cast<uint32_t>(col[3 * kQtPitch]) << 24);
+      }
+      *reinterpret_cast<uint4*>(qt + qr * rows + qc) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    __syncthreads();
+  }
+  amax = block_max(amax, sh);
+  if (MODE == 0) {  // m and the flag were read by every CTA: the last one clears them
+    if (t == 0) is_last = atomicAdd(&ws[1], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (is_last && t == 0) {
+      atomicExch(&ws[2], 0u);
+      atomicExch(&ws[3], 0u);
+      atomicExch(&ws[1], 0u);
+    }
+    return;
+  }
+  uint32_t* counter = (MODE == 1) ? reinterpret_cast<uint32_t*>(ring + len + 1) : &ws[1];
+  if (t == 0) {
+    atomicMax(&ws[0], __float_as_uint(amax));
+    __threadfence();
+    is_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!is_last || t != 0) return;
+  __threadfence();
+  const float a = __uint_as_float(atomicExch(&ws[0], 0u));
+  if (MODE == 1) {
+    ring[idx] = a;  // fold this step's amax into the history slot
+    float win = 0.0f;
+    for (int i = 0; i < len; ++i) win = fmaxf(win, __ldcg(&ring[i]));
+    if (win <= FLT_MAX && win > 0.0f) {
+      const float next = ldexpf(__fdiv_rn(Fmt<FMT>::kMax, win), -margin);
+      if (next <= FLT_MAX && next > 0.0f) ring[len] = next;
+    }
+  }
+  scales[0] = __fdiv_rn(1.0f, m);
+  if (amax_out) amax_out[0] = a;
+  atomicExch(counter, 0u);
+}
+
 // ------------------------------------------------------------------- launch
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -1457,7 +1567,53 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
   return cudaGetLastError();
 }
 
+template <int DT, int FMT>
+cudaError_t launch_transpose_typed(const QuantizeArgs& a) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t n = a.rows * a.cols;
+  const float fmax = Fmt<FMT>::kMax;
+  uint32_t* ws = static_cast<uint32_t*>(a.ws);
+  const int64_t tiles = ((a.rows + kQtTile - 1) / kQtTile) * ((a.cols + kQtTile - 1) / kQtTile);
+  int64_t grid = std::min<int64_t>(tiles, static_cast<int64_t>(device_sm_count(dev)) * 8);
+  if (grid < 1) grid = 1;
+  const unsigned g = static_cast<unsigned>(grid);
+  if (a.ring) {
+    k_quant_transpose<DT, FMT, 1><<<g, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.q, a.qt, nullptr, a.ring,
+                                                                 a.ring_len, a.ring_idx, a.ring_margin, ws, a.scales,
+                                                                 a.amax_out);
+    return cudaGetLastError();
+  }
+  if (a.mult) {
+    k_quant_transpose<DT, FMT, 2><<<g, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.q, a.qt, a.mult, nullptr, 0,
+                                                                 0, 0, ws, a.scales, a.amax_out);
+    return cudaGetLastError();
+  }
+  // dynamic: the per-tensor amax pass publishes m, then the transposing cast
+  const int agrid = flat_grid(n / Dt<DT>::kVec, dev, kUnrollFlat);
+  k_tensor_amax<DT, true><<<agrid, kThreads, 0, a.stream>>>(a.x, n, ws, fmax, a.scales, a.amax_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (n == 0) return cudaMemsetAsync(ws + 2, 0, 2 * sizeof(uint32_t), a.stream);
+  k_quant_transpose<DT, FMT, 0><<<g, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.q, a.qt, nullptr, nullptr, 0, 0,
+                                                               0, ws, a.scales, a.amax_out);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_transpose(const QuantizeArgs& a) {
+  const int key = a.xt * 2 + a.fmt;
+  switch (key) {
+    case 0: return launch_transpose_typed<0, 0>(a);
+    case 1: return launch_transpose_typed<0, 1>(a);
+    case 2: return launch_transpose_typed<1, 0>(a);
+    case 3: return launch_transpose_typed<1, 1>(a);
+    case 4: return launch_transpose_typed<2, 0>(a);
+    case 5: return launch_transpose_typed<2, 1>(a);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 size_t quantize_workspace_bytes(int gran, int64_t rows, int64_t cols, int delayed) {
   (void)rows;

@@ -145,6 +145,43 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
                           void* workspace, size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * Per-tensor FP8 quantize that also writes the codes transposed, for the
+ * backward GEMMs of AstrAI ops.cu linear_backward_fp8: dX = g @ w reads the
+ * weight codes transposed and dW = g^T @ x reads the gradient and activation
+ * codes transposed.  With the codes of x [rows, cols] row-major in q and
+ * transposed in qt [cols, rows], both GEMMs run as the NT hq_gemm_a8w8.
+ *
+ * The codes are those of hq_quantize_fp8 with per-tensor granularity:
+ *   - ring != NULL: the delayed mode (m = ring[ring_len], the ring stepped
+ *     with this call's amax by the last CTA), exactly as hq_quantize_fp8;
+ *   - multiplier != NULL: a caller's multiplier m = *multiplier (device f32),
+ *     the ring-free static form the backward uses for w and x (the forward's
+ *     scales; no ring is stepped); amax_out still receives the amax;
+ *   - neither: the dynamic mode (m = fmax / amax of this call).
+ * scales[0] receives 1/m in every mode.
+ *
+ * Arguments:
+ *   x           device, [rows, cols] row-major, f32 / bf16 / f16 (xt),
+ *               16-byte aligned; rows % 16 == 0 and cols % 16 == 0
+ *   q           device uint8 [rows, cols], 16-byte aligned, or NULL
+ *   qt          device uint8 [cols, rows], 16-byte aligned
+ *   scales      device f32 [1]; amax_out device f32 [1] or NULL
+ *   multiplier  device f32 [1] or NULL (not together with ring)
+ *   ring, ring_len, ring_idx, ring_margin: as hq_quantize_fp8
+ *   workspace   >= hq_quantize_workspace_bytes(PER_TENSOR, rows, cols, 1)
+ *               bytes, zero on entry, zero again on return
+ * Errors: HQ_ERR_INVALID_ARG (null, shape not a multiple of 16, multiplier
+ *   with ring, bad ring index), HQ_ERR_MISALIGNED, HQ_ERR_OVERLAP,
+ *   HQ_ERR_WRONG_DEVICE, HQ_ERR_UNSUPPORTED_ARCH, HQ_ERR_TOO_LARGE,
+ *   HQ_ERR_CUDA.  An empty x (rows or cols 0) still writes scales (and steps
+ *   the ring in the delayed mode).
+ */
+hq_status hq_quantize_fp8_transpose(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                                    uint8_t* q, uint8_t* qt, float* scales, float* amax_out, const float* multiplier,
+                                    float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,
+                                    void* workspace, size_t workspace_bytes, hq_stream_t stream);
+
+/*
  * Scaled FP8 GEMM, NT layout, into a caller-owned bf16 buffer:
  *   out[m, n] = bf16_rn( acc[m, n] * x_scale[m'] * w_scale[n'] ),
  *   acc[m, n] = sum_k dec(xq[m, k]) * dec(wq[n, k])   (FP32 accumulation)

@@ -154,6 +154,26 @@ def test_fused_epilogue_rejections():
     assert gx(out=BASE + 0x6000002, q_out=None, ring=None, ws=None, bias=BASE + 0x5200000) == MISALIGNED
 
 
+def qtr(x=BASE, xt=H.BF16, rows=64, cols=128, fmt=H.E4M3, q=None, qt=BASE + 0x1000000, scales=BASE + 0x2000000,
+        amax=None, mult=None, ring=None, ring_len=16, ring_idx=0, margin=0, ws=BASE + 0x3000000, wsb=256):
+    return L.hq_quantize_fp8_transpose(x, xt, rows, cols, fmt, q, qt, scales, amax, mult, ring, ring_len, ring_idx,
+                                       margin, ws, wsb, None)
+
+
+def test_quantize_transpose_rejections():
+    assert qtr(rows=72, cols=120) == INVALID          # both must be multiples of 16
+    assert qtr(rows=60) == INVALID
+    assert qtr(mult=BASE + 0x4000000, ring=BASE + 0x5000000) == INVALID   # one multiplier source
+    assert qtr(ring=BASE + 0x5000000, ring_idx=16) == INVALID
+    assert qtr(qt=None) == INVALID and qtr(scales=None) == INVALID and qtr(ws=None) == INVALID
+    assert qtr(wsb=16) == INVALID and qtr(xt=7) == INVALID and qtr(fmt=5) == INVALID
+    assert qtr(qt=BASE + 0x1000008) == MISALIGNED and qtr(x=BASE + 4) == MISALIGNED
+    assert qtr(q=BASE + 0x4000004) == MISALIGNED and qtr(mult=BASE + 0x4000002) == MISALIGNED
+    assert qtr(qt=BASE + 0x100) == OVERLAP            # transposed codes over x
+    assert qtr(q=BASE + 0x1000000) == OVERLAP         # the two code buffers
+    assert qtr(scales=BASE + 0x3000000 + 64) == OVERLAP  # scales inside the workspace
+
+
 def test_grouped_rejections():
     gg = L.hq_grouped_gemm_a8w8
     args = dict(xq=BASE, wq=BASE + 0x1000000, fmt=0, xs=BASE + 0x2000000, xsl=100, ws=BASE + 0x3000000,
