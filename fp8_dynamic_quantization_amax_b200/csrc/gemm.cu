@@ -157,45 +157,49 @@ __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, ui
   asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// One chunk's 32 scaled values of a lane's row, plus the bias, rounded to
-// bf16 pairs: w[j] holds columns n0 + 2j (low half) and n0 + 2j + 1.
-template <int KIND>
-__device__ __forceinline__ void chunk_to_bf16(const Params& p, const uint32_t (&v)[32], float xsv, const float* sc,
-                                              int n0, uint32_t (&w)[16]) {
+// One chunk's 32 scaled values of a lane's row, plus the bias (bias != null),
+// rounded to bf16 pairs: w[j] holds columns n0 + 2j (low half) and n0 + 2j + 1.
+// has_acc == false (K == 0) reads the accumulator as zero.
+__device__ __forceinline__ void chunk_to_bf16(const uint32_t (&v)[32], bool has_acc, float xsv, const float* sc,
+                                              const uint16_t* bias, int n0, int N, uint32_t (&w)[16]) {
+  if (bias == nullptr) {
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float a0 = (p.nkb > 0) ? __uint_as_float(v[2 * j]) : 0.0f;
-    const float a1 = (p.nkb > 0) ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-    if (KIND == 0 && p.bias != nullptr) {
-      const uint32_t bb =
-          (n0 + 2 * j < p.N) ? __ldg(reinterpret_cast<const uint32_t*>(p.bias) + ((n0 >> 1) + j)) : 0u;
+    for (int j = 0; j < 16; ++j) {
+      const float a0 = has_acc ? __uint_as_float(v[2 * j]) : 0.0f;
+      const float a1 = has_acc ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+      w[j] = pack_bf16x2(a0 * (xsv * sc[2 * j]), a1 * (xsv * sc[2 * j + 1]));
+    }
+  } else {
+    const uint32_t* bp = reinterpret_cast<const uint32_t*>(bias) + (n0 >> 1);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float a0 = has_acc ? __uint_as_float(v[2 * j]) : 0.0f;
+      const float a1 = has_acc ? __uint_as_float(v[2 * j + 1]) : 0.0f;
+      const uint32_t bb = (n0 + 2 * j < N) ? __ldg(bp + j) : 0u;
       w[j] = pack_bf16x2(__fmaf_rn(a0, xsv * sc[2 * j], __uint_as_float(bb << 16)),
                          __fmaf_rn(a1, xsv * sc[2 * j + 1], __uint_as_float(bb & 0xFFFF0000u)));
-    } else {
-      w[j] = pack_bf16x2(a0 * (xsv * sc[2 * j]), a1 * (xsv * sc[2 * j + 1]));
     }
   }
 }
 
 // FP8 output of one chunk: codes of f32(bf16 value) * m, saturating RNE (NaN
 // -> 0x7F); the lane's finite-only amax is updated over its valid columns
-// and the chunk's codes are stored at the lane's row.
-__device__ __forceinline__ void chunk_to_fp8(const Params& p, const uint32_t (&w)[16], float qm, bool vrow, int row,
-                                             int n0, float& qam) {
+// and the chunk's codes are stored at the lane's row (qout + row * N + n0).
+__device__ __forceinline__ void chunk_to_fp8(const uint32_t (&w)[16], int qfmt, float qm, bool vrow, uint8_t* qrow,
+                                             int n0, int N, float& qam) {
   uint32_t c4[8];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float lo = __uint_as_float(w[j] << 16);
     const float hi = __uint_as_float(w[j] & 0xFFFF0000u);
-    if (vrow && n0 + 2 * j < p.N) qam = fmaxf(qam, fmaxf(finite_abs(lo), finite_abs(hi)));
-    const uint32_t c2 = (p.qfmt == 0) ? cvt2_exact<0>(__fmul_rn(lo, qm), __fmul_rn(hi, qm))
-                                      : cvt2_exact<1>(__fmul_rn(lo, qm), __fmul_rn(hi, qm));
+    if (vrow && n0 + 2 * j < N) qam = fmaxf(qam, fmaxf(finite_abs(lo), finite_abs(hi)));
+    const uint32_t c2 = (qfmt == 0) ? cvt2_exact<0>(__fmul_rn(lo, qm), __fmul_rn(hi, qm))
+                                    : cvt2_exact<1>(__fmul_rn(lo, qm), __fmul_rn(hi, qm));
     c4[j >> 1] = (j & 1) ? (c4[j >> 1] | (c2 << 16)) : c2;
   }
   if (vrow) {  // N % 16 == 0 and n0 % 32 == 0: 16 or 32 codes of this chunk lie inside the row
-    uint8_t* dst = p.qout + static_cast<int64_t>(row) * p.N + n0;
-    st_global_v4(dst, c4[0], c4[1], c4[2], c4[3]);
-    if (n0 + 32 <= p.N) st_global_v4(dst + 16, c4[4], c4[5], c4[6], c4[7]);
+    st_global_v4(qrow + n0, c4[0], c4[1], c4[2], c4[3]);
+    if (n0 + 32 <= N) st_global_v4(qrow + n0 + 16, c4[4], c4[5], c4[6], c4[7]);
   }
 }
 
@@ -203,7 +207,7 @@ __device__ __forceinline__ void chunk_to_fp8(const Params& p, const uint32_t (&w
 // word; the last CTA (threadfence + the ring's counter word) folds it into
 // the ring and publishes the next multiplier, as the delayed quantize does.
 template <int NWARPS>
-__device__ void finalize_fp8_out(const Params& p, float qam) {
+__device__ __forceinline__ void finalize_fp8_out(const Params& p, float qam) {
   __shared__ float red[NWARPS];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) qam = fmaxf(qam, __shfl_xor_sync(0xFFFFFFFFu, qam, o));
@@ -517,6 +521,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     float* wsh = sWs + ew * kMyChunks * 32;
     const uint64_t out_pol = l2_evict_first_policy();
     const float qm = (p.qout != nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
+    const bool has_acc = p.nkb > 0;
+    const uint16_t* bias = (KIND == 0) ? p.bias : nullptr;
     int i = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int acc = i & 1;
@@ -543,6 +549,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       }
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
+      uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
 #pragma unroll 1
       for (int i = 0; half + 2 * i < kChunks; ++i) {
         const int c = (half + 2 * i) * 32;  // chunk's first column within the tile
@@ -554,9 +561,9 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
         if (n0 >= ncap) continue;
         const float* sc = wsh + i * 32;
         uint32_t w[16];
-        chunk_to_bf16<KIND>(p, v, xsv, sc, n0, w);
-        if (KIND == 0 && p.qout != nullptr) {
-          chunk_to_fp8(p, w, qm, vrow, row, n0, qam);
+        chunk_to_bf16(v, has_acc, xsv, sc, bias, n0, p.N, w);
+        if (KIND == 0 && qrow != nullptr) {
+          chunk_to_fp8(w, p.qfmt, qm, vrow, qrow, n0, p.N, qam);
           continue;
         }
         // the tensor map clips at N; a 16-column tail chunk inside N is masked
@@ -984,6 +991,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     float* wsh = sWs + ew * kMyChunks * 32;
     const uint64_t out_pol = l2_evict_first_policy();
     const float qm = (p.qout != nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
+    const bool has_acc = p.nkb > 0;
+    const uint16_t* bias = (KIND == 0) ? p.bias : nullptr;
     uint32_t tempty_leader[kAccs];
 #pragma unroll
     for (int a = 0; a < kAccs; ++a) tempty_leader[a] = mapa_shared(smem_u32(&tempty_bar[a]), 0);
@@ -1013,6 +1022,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
+      uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
 #pragma unroll 1
       for (int j = 0; j < kMyChunks; ++j) {
         const int c = (half + 2 * j) * 32;  // chunk's first column within the tile
@@ -1024,9 +1034,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (n0 >= p.N) continue;
         const float* sc = wsh + j * 32;
         uint32_t w[16];
-        chunk_to_bf16<KIND>(p, v, xsv, sc, n0, w);
-        if (KIND == 0 && p.qout != nullptr) {
-          chunk_to_fp8(p, w, qm, vrow, row, n0, qam);
+        chunk_to_bf16(v, has_acc, xsv, sc, bias, n0, p.N, w);
+        if (KIND == 0 && qrow != nullptr) {
+          chunk_to_fp8(w, p.qfmt, qm, vrow, qrow, n0, p.N, qam);
           continue;
         }
         if (tma_ok) {
