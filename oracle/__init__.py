@@ -50,6 +50,14 @@ def lib():
         L.hqo_quantize.restype = ci
         L.hqo_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
         L.hqo_gemm_a8w8.restype = None
+        L.hqo_splitmix64_next.argtypes = [P]
+        L.hqo_splitmix64_next.restype = ctypes.c_uint64
+        L.hqo_sr_bits.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+        L.hqo_sr_bits.restype = ctypes.c_uint32
+        L.hqo_encode_e5m2_sr.argtypes = [ctypes.c_float, ctypes.c_uint32]
+        L.hqo_encode_e5m2_sr.restype = ctypes.c_uint8
+        L.hqo_quantize_e5m2_sr.argtypes = [P, ci, i64, i64, ci, ctypes.c_uint64, P, P, P]
+        L.hqo_quantize_e5m2_sr.restype = ci
         L.hqo_gemm_a8w8_bias.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P]
         L.hqo_gemm_a8w8_bias.restype = None
         L.hqo_gemm_a8w8_entries.argtypes = [P, P, ci, P, i64, P, i64, i64, P, P, i64, P]
@@ -169,6 +177,38 @@ def gemm_a8w8(xq, wq, fmt, x_scale, w_scale, return_ref=False):
     lib().hqo_gemm_a8w8(_p(xq), _p(wq), fmt, _p(xs), xs.size, _p(ws), ws.size,
                         M, N, K, _p(out), _p(ref))
     return (out, ref) if return_ref else out
+
+
+def splitmix64_outputs(seed, count):
+    """The first `count` outputs of a SplitMix64 generator started at `seed`."""
+    st = ctypes.c_uint64(seed)
+    return [lib().hqo_splitmix64_next(ctypes.byref(st)) for _ in range(count)]
+
+
+def sr_bits(seed, idx):
+    """The 32-bit draw of element index `idx` under `seed` (stochastic rounding)."""
+    return lib().hqo_sr_bits(seed, idx)
+
+
+def encode_e5m2_sr(y, u):
+    """E5M2 code of the f32 value y rounded stochastically with draw u."""
+    return lib().hqo_encode_e5m2_sr(float(np.float32(y)), int(u))
+
+
+def quantize_e5m2_sr(x, gran, seed):
+    """Dynamic E5M2 quantize with stochastic rounding: (codes, dequant scales,
+    amax); amax and scales as quantize(), the draws by flat element index."""
+    x = np.ascontiguousarray(x)
+    dt = _dtype_code(x)
+    rows, cols = x.shape
+    ns = lib().hqo_scale_count(gran, rows, cols)
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty(max(ns, 1), np.float32)[:ns]
+    a = np.empty(max(ns, 1), np.float32)[:ns]
+    rc = lib().hqo_quantize_e5m2_sr(_p(x), dt, rows, cols, gran, seed, _p(q), _p(s), _p(a))
+    if rc != 0:
+        raise ValueError("invalid arguments")
+    return q, s, a
 
 
 def gemm_a8w8_bias(xq, wq, fmt, x_scale, w_scale, bias_bf16_bits):

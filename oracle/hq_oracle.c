@@ -309,6 +309,84 @@ int hqo_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int fmt,
   return 0;
 }
 
+/* ---------------------------------------------------- stochastic E5M2 */
+
+/* SplitMix64 (Steele, Lea and Flood 2014, with the constants of Vigna's
+   reference implementation) as a counter-based generator: the draw for
+   element index i under seed s is the (i+1)-th output of the generator
+   started at state s; its top 32 bits are returned.  hqo_splitmix64_next
+   steps one generator (used to pin the definition against its published
+   outputs). */
+static uint64_t splitmix64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+uint64_t hqo_splitmix64_next(uint64_t* state) {
+  *state += 0x9E3779B97F4A7C15ull;
+  return splitmix64_mix(*state);
+}
+
+uint32_t hqo_sr_bits(uint64_t seed, uint64_t idx) {
+  return (uint32_t)(splitmix64_mix(seed + (idx + 1) * 0x9E3779B97F4A7C15ull) >> 32);
+}
+
+/* Stochastic rounding of an f32 to E5M2 ([HQ] "Stochastic E5M2 Backward
+   Gradients": between the two adjacent E5M2 values, with probability
+   proportional to the distance from the other one).  With g the E5M2 spacing
+   at |y| (2^(e-2) for |y| in [2^e, 2^(e+1)) with e >= -14, else 2^-16),
+   lo = floor(|y| / g) g and frac32 = floor((|y| - lo) / g * 2^32), |y|
+   rounds up to lo + g iff the draw u < frac32, so P(up) = frac32 / 2^32.
+   NaN gives 0x7F; |y| >= 57344 and +-Inf saturate; the sign is kept (a
+   negative value rounded to zero is -0, code 0x80). */
+uint8_t hqo_encode_e5m2_sr(float y, uint32_t u) {
+  double a, g, t, q, fr, v;
+  uint64_t frac32;
+  int e;
+  if (isnan(y)) return 0x7F;
+  a = fabs((double)y);
+  if (a >= 57344.0 || a == 0.0) return hqo_encode_sat(y, HQO_E5M2);
+  frexp(a, &e); /* a = f * 2^e with f in [0.5, 1): |y| in [2^(e-1), 2^e) */
+  e -= 1;
+  g = ldexp(1.0, (e < -14 ? -14 : e) - 2);
+  t = a / g; /* exact: g is a power of two */
+  q = floor(t);
+  fr = t - q; /* exact */
+  frac32 = (uint64_t)floor(ldexp(fr, 32));
+  v = (q + ((uint64_t)u < frac32 ? 1.0 : 0.0)) * g; /* on the E5M2 grid, <= 57344 */
+  return hqo_encode_sat((float)(signbit(y) ? -v : v), HQO_E5M2);
+}
+
+/* Dynamic quantize to E5M2 with stochastic rounding: amax and the multiplier
+   per granularity exactly as hqo_quantize (no ring), the cast of
+   y = f32(x) * m by hqo_encode_e5m2_sr with the draw of the element's flat
+   index r * cols + c under `seed`. */
+int hqo_quantize_e5m2_sr(const void* x, int dtype, int64_t rows, int64_t cols,
+                         int gran, uint64_t seed, uint8_t* q, float* scales,
+                         float* amax_out) {
+  int64_t n = hqo_scale_count(gran, rows, cols), r, c;
+  float* amax;
+  float* mult;
+  if (n < 0) return -1;
+  amax = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  mult = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  hqo_amax(x, dtype, rows, cols, gran, amax);
+  for (r = 0; r < n; ++r) mult[r] = hqo_multiplier(amax[r], HQO_E5M2);
+  for (r = 0; r < n; ++r) scales[r] = 1.0f / mult[r];
+  for (r = 0; r < rows; ++r)
+    for (c = 0; c < cols; ++c) {
+      int64_t slot = (gran == HQO_PER_TENSOR) ? 0 : (gran == HQO_PER_TOKEN ? r : c);
+      float y = load_elem(x, dtype, r * cols + c) * mult[slot]; /* one f32 mul */
+      q[r * cols + c] = hqo_encode_e5m2_sr(y, hqo_sr_bits(seed, (uint64_t)(r * cols + c)));
+    }
+  if (amax_out)
+    for (r = 0; r < n; ++r) amax_out[r] = amax[r];
+  free(amax);
+  free(mult);
+  return 0;
+}
+
 /* --------------------------------------------------------------------- GEMM */
 
 /* Integer numerator of a finite code: value = n * 2^-frac, frac = 9 (E4M3)

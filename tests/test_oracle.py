@@ -570,3 +570,111 @@ def test_ring_update_matches_quantize_ring_and_f16_input():
         qb, sb, ab = O.quantize(h.astype(np.float32), O.E4M3, gran)
         np.testing.assert_array_equal(qa, qb)
         np.testing.assert_array_equal(sa, sb)
+
+
+# ------------------------------------------------------ stochastic E5M2
+def _golden_splitmix():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "splitmix64.txt")):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            seed, idx, out = line.split()
+            rows.append((int(seed), int(idx), int(out, 16)))
+    return rows
+
+
+def test_splitmix64_published_outputs():
+    rows = _golden_splitmix()
+    outs = O.splitmix64_outputs(0, len(rows))
+    for (seed, idx, out), got in zip(rows, outs):
+        assert got == out
+        # the counter form: element idx draws the top half of output idx
+        assert O.sr_bits(seed, idx) == out >> 32
+
+
+def test_sr_grid_values_are_fixed_points():
+    # a value already on the E5M2 grid never moves, whatever the draw
+    for c in range(256):
+        v = O.decode(c, O.E5M2)
+        if not np.isfinite(v):
+            continue
+        for u in (0, 1, 0x7FFFFFFF, 0xFFFFFFFF):
+            assert O.encode_e5m2_sr(v, u) == O.encode_sat(np.float32(v), O.E5M2)
+
+
+def _neighbours(y):
+    """The E5M2 values just below and above |y| (same sign) and the exact
+    fraction of the way from the lower to the upper one."""
+    a = abs(Fraction(float(y)))
+    e = math.floor(math.log2(a))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    g = Fraction(2) ** (max(e, -14) - 2)
+    lo = (a // g) * g
+    return lo, lo + g, (a - lo) / g
+
+
+def test_sr_rounds_between_neighbours_at_the_exact_threshold():
+    rng = np.random.default_rng(5)
+    ys = list((rng.standard_normal(300) * np.exp(rng.uniform(-14, 10, 300))).astype(np.float32))
+    ys += [np.float32(3e-6), np.float32(-1.7e-5), np.float32(6.1e-5), np.float32(1.5), np.float32(-40000.0)]
+    for y in ys:
+        if abs(float(y)) >= 57344 or y == 0:
+            continue
+        lo, hi, frac = _neighbours(y)
+        if frac == 0:
+            continue
+        thr = math.floor(frac * 2 ** 32)  # round up iff u < thr
+        sign = -1 if y < 0 else 1
+        c_lo = O.encode_sat(np.float32(sign * float(lo)), O.E5M2)
+        c_hi = O.encode_sat(np.float32(sign * float(hi)), O.E5M2)
+        assert O.encode_e5m2_sr(y, 0) == (c_hi if thr > 0 else c_lo)
+        if thr > 0:
+            assert O.encode_e5m2_sr(y, thr - 1) == c_hi
+        assert O.encode_e5m2_sr(y, min(thr, 2 ** 32 - 1)) == c_lo
+        assert O.encode_e5m2_sr(y, 2 ** 32 - 1) == c_lo
+
+
+def test_sr_special_values():
+    assert O.encode_e5m2_sr(np.float32(np.nan), 0) == 0x7F
+    for y, u in [(np.inf, 0), (-np.inf, 5), (60000.0, 0), (-57344.0, 1)]:
+        assert O.encode_e5m2_sr(np.float32(y), u) == O.encode_sat(np.float32(y), O.E5M2)
+    assert O.encode_e5m2_sr(np.float32(0.0), 0) == 0x00
+    assert O.encode_e5m2_sr(np.float32(-0.0), 0) == 0x80
+    # a negative value rounded down to zero keeps its sign
+    assert O.encode_e5m2_sr(np.float32(-1e-9), 0xFFFFFFFF) == 0x80
+
+
+def test_sr_frequency_matches_the_fraction():
+    # over many element indices the up-rounding rate is the fraction (5 sigma),
+    # which also makes the rounding unbiased in the mean
+    n = 20000
+    for y in (np.float32(1.3), np.float32(-0.0021), np.float32(2.5e-5)):
+        lo, hi, frac = _neighbours(y)
+        sign = -1 if y < 0 else 1
+        c_hi = O.encode_sat(np.float32(sign * float(hi)), O.E5M2)
+        ups = sum(O.encode_e5m2_sr(y, O.sr_bits(77, i)) == c_hi for i in range(n))
+        p = float(frac)
+        assert abs(ups / n - p) <= 5 * math.sqrt(p * (1 - p) / n) + 1e-9
+        mean = sign * (float(lo) + (ups / n) * float(hi - lo))
+        assert abs(mean - float(y)) <= 5 * math.sqrt(p * (1 - p) / n) * float(hi - lo) + 1e-12
+
+
+def test_sr_quantize_scales_match_and_codes_are_neighbours():
+    rng = np.random.default_rng(8)
+    x = W.f32_to_bf16_bits(rng.standard_normal((24, 96)).astype(np.float32) * np.float32(3.0))
+    for gran in (O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL):
+        q, s, a = O.quantize_e5m2_sr(x, gran, seed=1234)
+        qr, sr_, ar = O.quantize(x, O.E5M2, gran)
+        np.testing.assert_array_equal(s.view(np.uint32), sr_.view(np.uint32))
+        np.testing.assert_array_equal(a.view(np.uint32), ar.view(np.uint32))
+        # the stochastic code is the RNE code or its neighbour on the other side
+        d = O.decode_array(q.reshape(-1), O.E5M2) - O.decode_array(qr.reshape(-1), O.E5M2)
+        assert (q != qr).any() and (q == qr).any()
+        v = O.decode_array(qr.reshape(-1), O.E5M2)
+        assert (np.abs(d) <= np.abs(v) * 0.5 + 2.0 ** -16).all()
+        # reproducible by seed, different under another seed
+        assert np.array_equal(O.quantize_e5m2_sr(x, gran, seed=1234)[0], q)
+        assert not np.array_equal(O.quantize_e5m2_sr(x, gran, seed=99)[0], q)
