@@ -21,7 +21,7 @@ PER_TENSOR, PER_TOKEN, PER_CHANNEL = 0, 1, 2
 F32, BF16, F16 = 0, 1, 2
 
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
-            "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
+            "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
             "hq_grouped_gemm_bf16",
             "hq_quantize_fp8_noalloc", "hq_check_device_error", "hq_last_error", "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
@@ -52,6 +52,8 @@ def _load():
     L.hq_quantize_fp8.restype = ci
     L.hq_quantize_fp8_noalloc.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P]
     L.hq_quantize_fp8_noalloc.restype = ci
+    L.hq_quantize_e5m2_stochastic.argtypes = [P, ci, i64, i64, ci, ctypes.c_uint64, P, P, P, P, sz, P]
+    L.hq_quantize_e5m2_stochastic.restype = ci
     L.hq_quantize_fp8_transpose.argtypes = [P, ci, i64, i64, ci, P, P, P, P, P, P, i32, i32, i32, P, sz, P]
     L.hq_quantize_fp8_transpose.restype = ci
     L.hq_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
@@ -153,6 +155,28 @@ def hq_quantize_fp8(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=N
                               _ptr(amax_out), _ptr(ring), ring_len, ring_idx, ring_margin,
                               _ptr(workspace), 0 if workspace is None else workspace.numel(),
                               _stream(stream)))
+    return q, scales
+
+
+def hq_quantize_e5m2_stochastic(x, gran=PER_TENSOR, seed=0, q=None, scales=None, amax_out=None, workspace=None,
+                                stream=None):
+    """Dynamic E5M2 quantize with stochastic rounding (seeded, reproducible).
+    Returns (q uint8, dequant scales f32)."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    x = x.contiguous()
+    rows, cols = x.shape
+    ns = hq_scale_count(gran, rows, cols)
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((max(ns, 0),), dtype=torch.float32, device=x.device)
+    need = hq_quantize_workspace_bytes(gran, rows, cols, False)
+    if workspace is None and need > 0:
+        workspace = _workspace(x.device, need)
+    check(lib.hq_quantize_e5m2_stochastic(_ptr(x), _DT[x.dtype], rows, cols, gran, seed & ((1 << 64) - 1), _ptr(q),
+                                          _ptr(scales), _ptr(amax_out), _ptr(workspace),
+                                          0 if workspace is None else workspace.numel(), _stream(stream)))
     return q, scales
 
 

@@ -238,6 +238,53 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
   return launched(hq::launch_quantize(a), "quantize launch");
 }
 
+hq_status hq_quantize_e5m2_stochastic(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_granularity g,
+                                      uint64_t seed, uint8_t* q, float* scales, float* amax_out, void* workspace,
+                                      size_t workspace_bytes, hq_stream_t stream) {
+  if (xt != HQ_F32 && xt != HQ_BF16 && xt != HQ_F16) return fail(HQ_ERR_INVALID_ARG, "invalid dtype %d", (int)xt);
+  if (g != HQ_PER_TENSOR && g != HQ_PER_TOKEN && g != HQ_PER_CHANNEL)
+    return fail(HQ_ERR_INVALID_ARG, "invalid granularity %d", (int)g);
+  if (rows < 0 || cols < 0) return fail(HQ_ERR_INVALID_ARG, "negative shape [%lld, %lld]", (long long)rows, (long long)cols);
+  if (rows >= k2p31 || cols >= k2p31 || (cols > 0 && rows > (k2p40 - 1) / cols))
+    return fail(HQ_ERR_TOO_LARGE, "shape [%lld, %lld] is beyond the supported range", (long long)rows, (long long)cols);
+  const int64_t ns = hq_scale_count(g, rows, cols);
+  const int64_t n = rows * cols;
+  const size_t esize = (xt == HQ_F32) ? 4 : 2;
+  const size_t need = hq::quantize_workspace_bytes(static_cast<int>(g), rows, cols, 0);
+  if (ns == 0) return ok();
+  if (n > 0 && (!x || !q)) return fail(HQ_ERR_INVALID_ARG, "x and q must not be null");
+  if (!scales) return fail(HQ_ERR_INVALID_ARG, "scales must not be null");
+  if (g == HQ_PER_CHANNEL && (static_cast<size_t>(cols) * esize) % 16 != 0)
+    return fail(HQ_ERR_INVALID_ARG, "per-channel rows must be whole 16-byte units");
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(HQ_ERR_INVALID_ARG, "this mode needs a zeroed workspace of %zu bytes", need);
+  if (!is_aligned(x, 16) || !is_aligned(q, 16)) return fail(HQ_ERR_MISALIGNED, "x and q must be 16-byte aligned");
+  if (!is_aligned(scales, 4) || !is_aligned(amax_out, 4))
+    return fail(HQ_ERR_MISALIGNED, "scales and amax_out must be 4-byte aligned");
+  if (need > 0 && !is_aligned(workspace, 256)) return fail(HQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  const Range outs[] = {{q, static_cast<size_t>(n), "q"},
+                        {scales, static_cast<size_t>(ns) * 4, "scales"},
+                        {amax_out, amax_out ? static_cast<size_t>(ns) * 4 : 0, "amax_out"},
+                        {need > 0 ? workspace : nullptr, need, "workspace"}};
+  const Range ins[] = {{x, static_cast<size_t>(n) * esize, "x"}};
+  hq_status s = check_overlaps(outs, 4, ins, 1);
+  if (s != HQ_OK) return s;
+  const Range devs[] = {{n > 0 ? x : nullptr, 0, "x"}, {n > 0 ? q : nullptr, 0, "q"}, {scales, 0, "scales"},
+                        {amax_out, 0, "amax_out"}, {need > 0 ? workspace : nullptr, 0, "workspace"}};
+  s = check_device_ptrs(devs, 5);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  hq::QuantizeArgs a;
+  a.x = x; a.xt = xt; a.rows = rows; a.cols = cols; a.fmt = HQ_E5M2; a.gran = g;
+  a.q = q; a.scales = scales; a.amax_out = amax_out;
+  a.ring = nullptr; a.ring_len = 0; a.ring_idx = 0; a.ring_margin = 0;
+  a.ws = workspace;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.seed = seed;
+  return launched(hq::launch_quantize_sr(a), "stochastic quantize launch");
+}
+
 hq_status hq_quantize_fp8_transpose(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
                                     uint8_t* q, uint8_t* qt, float* scales, float* amax_out, const float* multiplier,
                                     float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,

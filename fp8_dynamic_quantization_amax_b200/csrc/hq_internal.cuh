@@ -30,6 +30,7 @@ struct QuantizeArgs {
   cudaStream_t stream;
   uint8_t* qt = nullptr;        // transposed codes [cols, rows] (launch_quantize_transpose)
   const float* mult = nullptr;  // a caller's multiplier (static per-tensor form)
+  uint64_t seed = 0;            // stochastic rounding (launch_quantize_sr)
 };
 
 size_t quantize_workspace_bytes(int gran, int64_t rows, int64_t cols, int delayed);
@@ -37,6 +38,9 @@ cudaError_t launch_quantize(const QuantizeArgs& a);
 // Per-tensor quantize writing the codes row-major (a.q, nullable) and
 // transposed (a.qt); rows % 16 == 0, cols % 16 == 0, x 16-byte aligned.
 cudaError_t launch_quantize_transpose(const QuantizeArgs& a);
+// Dynamic E5M2 quantize with stochastic rounding (a.seed); x 16-byte aligned,
+// cols a multiple of the 16-byte vector for the per-channel form.
+cudaError_t launch_quantize_sr(const QuantizeArgs& a);
 
 struct GemmArgs {
   int kind;                 // 0: fp8 a8w8 (kind::f8f6f4), 1: bf16 (kind::f16)

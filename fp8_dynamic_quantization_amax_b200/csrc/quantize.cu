@@ -1382,6 +1382,143 @@ __global__ void __launch_bounds__(kThreads) k_quant_transpose(
   atomicExch(counter, 0u);
 }
 
+// ---------------------------------------------------- stochastic E5M2
+// Stochastic rounding to E5M2 (hip-quant README "Stochastic E5M2 Backward
+// Gradients"): between the two adjacent E5M2 values, rounding up with
+// probability proportional to the distance from the lower one, from a
+// stateless hash of (seed, element index).  The hash is SplitMix64 used as a
+// counter-based generator: element i draws the top half of the generator's
+// output i + 1 from state `seed`.
+__device__ __forceinline__ uint32_t sr_draw(uint64_t seed, uint64_t idx) {
+  uint64_t z = seed + (idx + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return static_cast<uint32_t>(z >> 32);
+}
+
+// The E5M2 grid value y rounds to: with g the spacing at |y| and
+// lo = floor(|y| / g) g, up to lo + g iff u < floor((|y| - lo) / g * 2^32).
+// Zero, NaN, +-Inf and |y| >= 57344 come back unchanged (the saturating
+// conversion then gives their codes); the sign is kept.
+__device__ __forceinline__ float sr_e5m2(float y, uint32_t u) {
+  const uint32_t b = __float_as_uint(y);
+  const uint32_t a = b & 0x7FFFFFFFu, sgn = b & 0x80000000u;
+  if (a == 0u || a >= 0x47600000u) return y;
+  uint32_t r;
+  if (a >= 0x38800000u) {  // |y| >= 2^-14: g is 2^21 units of the f32 last place
+    const uint32_t d = a & 0x1FFFFFu;
+    r = (a & ~0x1FFFFFu) + ((u < (d << 11)) ? 0x200000u : 0u);
+  } else {  // below 2^-14: g = 2^-16
+    const float t = __uint_as_float(a) * 65536.0f;  // exact
+    float lo = floorf(t);
+    const uint32_t thr = static_cast<uint32_t>((t - lo) * 4294967296.0f);  // exact, < 2^32
+    lo += (u < thr) ? 1.0f : 0.0f;
+    r = __float_as_uint(lo * 1.52587890625e-05f);  // * 2^-16, exact
+  }
+  return __uint_as_float(r | sgn);
+}
+
+template <int DT>
+__device__ __forceinline__ void sr_store_vec(uint8_t* dst, const uint4& u, float m, uint64_t seed, uint64_t idx0) {
+  float f[Dt<DT>::kVec];
+  Dt<DT>::unpack(u, f);
+  uint32_t w[Dt<DT>::kVec / 4];
+#pragma unroll
+  for (int k = 0; k < Dt<DT>::kVec / 4; ++k) {
+    float g[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) g[i] = sr_e5m2(__fmul_rn(f[4 * k + i], m), sr_draw(seed, idx0 + 4 * k + i));
+    w[k] = cvt2_exact<1>(g[0], g[1]) | (cvt2_exact<1>(g[2], g[3]) << 16);
+  }
+  if constexpr (Dt<DT>::kVec == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  else *reinterpret_cast<uint32_t*>(dst) = w[0];
+}
+
+// Per-tensor (GRAN 0, m in ws[2] from k_tensor_amax) or per-channel (GRAN 2,
+// m[col] in ws_m from k_channel_amax): the stochastic cast of every element;
+// the last CTA returns the workspace to zero.
+template <int DT, int GRAN>
+__global__ void __launch_bounds__(kThreads) k_sr_cast(const void* __restrict__ x, int64_t rows, int64_t cols,
+                                                      uint64_t seed, uint8_t* __restrict__ q,
+                                                      uint32_t* __restrict__ header, float* __restrict__ ws_m) {
+  constexpr int VEC = Dt<DT>::kVec;
+  __shared__ bool is_last;
+  const int64_t n = rows * cols;
+  const int64_t nv = n / VEC;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+  const int64_t gstride = static_cast<int64_t>(gridDim.x) * kThreads;
+  const uint4* xv = static_cast<const uint4*>(x);
+  const float mt = (GRAN == 0) ? __uint_as_float(__ldcg(&header[2])) : 0.0f;
+  for (int64_t v = gtid; v < nv; v += gstride) {
+    if (GRAN == 2) {  // cols % VEC == 0: the vector's columns are c0 .. c0 + VEC - 1
+      float mm[VEC];
+      const int64_t c0 = (v * VEC) % cols;
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) mm[i] = __ldcg(&ws_m[c0 + i]);
+      float f[VEC];
+      Dt<DT>::unpack(ld_stream(xv + v), f);
+      uint32_t w[VEC / 4];
+#pragma unroll
+      for (int k = 0; k < VEC / 4; ++k) {
+        float g[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          g[i] = sr_e5m2(__fmul_rn(f[4 * k + i], mm[4 * k + i]), sr_draw(seed, v * VEC + 4 * k + i));
+        w[k] = cvt2_exact<1>(g[0], g[1]) | (cvt2_exact<1>(g[2], g[3]) << 16);
+      }
+      if constexpr (VEC == 8) *reinterpret_cast<uint2*>(q + v * VEC) = make_uint2(w[0], w[1]);
+      else *reinterpret_cast<uint32_t*>(q + v * VEC) = w[0];
+    } else {
+      sr_store_vec<DT>(q + v * VEC, ld_stream(xv + v), mt, seed, static_cast<uint64_t>(v * VEC));
+    }
+  }
+  for (int64_t i = nv * VEC + gtid; i < n; i += gstride) {  // element tail
+    const float m = (GRAN == 0) ? mt : __ldcg(&ws_m[i % cols]);
+    q[i] = cvt1_exact<1>(sr_e5m2(__fmul_rn(Dt<DT>::load1(x, i), m), sr_draw(seed, static_cast<uint64_t>(i))));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(&header[GRAN == 0 ? 1 : 0], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  if (GRAN == 0) {
+    if (threadIdx.x == 0) {
+      atomicExch(&header[2], 0u);
+      atomicExch(&header[3], 0u);
+      atomicExch(&header[1], 0u);
+    }
+  } else {
+    for (int64_t c = threadIdx.x; c < cols; c += kThreads) ws_m[c] = 0.0f;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      atomicExch(&header[1], 0u);
+      atomicExch(&header[0], 0u);
+    }
+  }
+}
+
+// Per-token: one CTA per row; the row's finite amax, m = fmax / amax (as
+// the RNE quantize), then the stochastic cast of the row.
+template <int DT>
+__global__ void __launch_bounds__(kThreads) k_sr_token(const void* __restrict__ x, int64_t rows, int64_t cols,
+                                                       uint64_t seed, uint8_t* __restrict__ q,
+                                                       float* __restrict__ scales, float* __restrict__ amax_out) {
+  __shared__ float sh[kThreads / 32];
+  const int64_t r = blockIdx.x;
+  const int64_t base = r * cols;
+  float amax = 0.0f;
+  for (int64_t c = threadIdx.x; c < cols; c += kThreads) amax = fmaxf(amax, finite_abs(Dt<DT>::load1(x, base + c)));
+  amax = block_max(amax, sh);
+  const float m = multiplier(amax, Fmt<1>::kMax);
+  if (threadIdx.x == 0) {
+    scales[r] = __fdiv_rn(1.0f, m);
+    if (amax_out) amax_out[r] = amax;
+  }
+  for (int64_t c = threadIdx.x; c < cols; c += kThreads)
+    q[base + c] = cvt1_exact<1>(sr_e5m2(__fmul_rn(Dt<DT>::load1(x, base + c), m),
+                                         sr_draw(seed, static_cast<uint64_t>(base + c))));
+}
+
 // ------------------------------------------------------------------- launch
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -1600,7 +1737,65 @@ cudaError_t launch_transpose_typed(const QuantizeArgs& a) {
   return cudaGetLastError();
 }
 
+template <int DT>
+cudaError_t launch_sr_typed(const QuantizeArgs& a) {
+  constexpr int VEC = Dt<DT>::kVec;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t n = a.rows * a.cols;
+  const float fmax = Fmt<1>::kMax;
+  if (a.gran == 1) {
+    if (a.rows == 0) return cudaSuccess;
+    k_sr_token<DT><<<static_cast<unsigned>(a.rows), kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.seed, a.q,
+                                                                             a.scales, a.amax_out);
+    return cudaGetLastError();
+  }
+  const int grid = flat_grid(n / VEC, dev, 1);
+  if (a.gran == 0) {
+    uint32_t* ws = static_cast<uint32_t*>(a.ws);
+    k_tensor_amax<DT, true><<<flat_grid(n / VEC, dev, kUnrollFlat), kThreads, 0, a.stream>>>(a.x, n, ws, fmax,
+                                                                                           a.scales, a.amax_out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (n == 0) return cudaMemsetAsync(ws + 2, 0, 2 * sizeof(uint32_t), a.stream);
+    k_sr_cast<DT, 0><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.seed, a.q, ws, nullptr);
+    return cudaGetLastError();
+  }
+  // per-channel: the two-launch column amax, then the stochastic cast
+  const int64_t nvc = a.cols / VEC;
+  const int64_t strips = (nvc + 31) / 32;
+  const int64_t target = static_cast<int64_t>(device_sm_count(dev)) * 8;
+  int64_t bands = std::max<int64_t>(1, std::min<int64_t>({(target + strips - 1) / std::max<int64_t>(strips, 1),
+                                                          a.rows, 65535}));
+  const int64_t band_rows = a.rows > 0 ? (a.rows + bands - 1) / bands : 1;
+  bands = a.rows > 0 ? (a.rows + band_rows - 1) / band_rows : 1;
+  uint32_t* header = static_cast<uint32_t*>(a.ws);
+  uint32_t* ws_amax = header + 4;
+  float* ws_m = reinterpret_cast<float*>(ws_amax + ((a.cols + 3) / 4) * 4);
+  const dim3 cgrid(static_cast<unsigned>(std::max<int64_t>(strips, 1)), static_cast<unsigned>(bands));
+  k_channel_amax<DT, true><<<cgrid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, band_rows, header, ws_amax, ws_m,
+                                                              fmax, a.scales, a.amax_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (n == 0) {
+    e = cudaMemsetAsync(header + 1, 0, sizeof(uint32_t), a.stream);
+    if (e != cudaSuccess) return e;
+    return cudaMemsetAsync(ws_m, 0, static_cast<size_t>(a.cols) * sizeof(float), a.stream);
+  }
+  k_sr_cast<DT, 2><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, a.seed, a.q, header, ws_m);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_sr(const QuantizeArgs& a) {
+  switch (a.xt) {
+    case 0: return launch_sr_typed<0>(a);
+    case 1: return launch_sr_typed<1>(a);
+    case 2: return launch_sr_typed<2>(a);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_quantize_transpose(const QuantizeArgs& a) {
   const int key = a.xt * 2 + a.fmt;

@@ -145,6 +145,34 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
                           void* workspace, size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * Dynamic quantize to E5M2 with stochastic rounding, for gradients
+ * (hip-quant README "Stochastic E5M2 Backward Gradients": between the two
+ * adjacent E5M2 values, with probability proportional to the distance, from
+ * a stateless per-element hash of (seed, element index)).
+ *
+ * amax, m = 57344 / amax and the exported dequant scales 1/m are exactly
+ * those of hq_quantize_fp8(x, E5M2, g) for granularity g.  The cast: y =
+ * f32(x) * m (one f32 multiply); with s the E5M2 spacing at |y| (2^(e-2)
+ * for |y| in [2^e, 2^(e+1)), e >= -14, else 2^-16) and lo = floor(|y|/s) s,
+ * |y| rounds up to lo + s iff u < floor((|y| - lo) / s * 2^32), where u is
+ * the element's draw: the top 32 bits of SplitMix64's output number i + 1
+ * from state `seed`, i = the element's row-major index.  NaN gives 0x7F,
+ * |y| >= 57344 and +-Inf saturate, the sign is kept.  The same (x, g, seed)
+ * always gives the same codes.
+ *
+ * Arguments: as hq_quantize_fp8 without the ring; x and q 16-byte aligned;
+ * per-channel needs cols * sizeof(element) % 16 == 0; workspace >=
+ * hq_quantize_workspace_bytes(g, rows, cols, 0) bytes, zero on entry and on
+ * return (none for per-token).
+ * Errors: HQ_ERR_INVALID_ARG, HQ_ERR_MISALIGNED, HQ_ERR_OVERLAP,
+ *   HQ_ERR_WRONG_DEVICE, HQ_ERR_UNSUPPORTED_ARCH, HQ_ERR_TOO_LARGE,
+ *   HQ_ERR_CUDA.
+ */
+hq_status hq_quantize_e5m2_stochastic(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_granularity g,
+                                      uint64_t seed, uint8_t* q, float* scales, float* amax_out, void* workspace,
+                                      size_t workspace_bytes, hq_stream_t stream);
+
+/*
  * Per-tensor FP8 quantize that also writes the codes transposed, for the
  * backward GEMMs of AstrAI ops.cu linear_backward_fp8: dX = g @ w reads the
  * weight codes transposed and dW = g^T @ x reads the gradient and activation

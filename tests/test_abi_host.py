@@ -174,6 +174,21 @@ def test_quantize_transpose_rejections():
     assert qtr(scales=BASE + 0x3000000 + 64) == OVERLAP  # scales inside the workspace
 
 
+def test_stochastic_rejections():
+    sr = L.hq_quantize_e5m2_stochastic
+
+    def call(x=BASE, xt=H.BF16, rows=64, cols=128, g=H.PER_TENSOR, q=BASE + 0x1000000, s=BASE + 0x2000000,
+             ws=BASE + 0x3000000, wsb=256):
+        return sr(x, xt, rows, cols, g, 1234, q, s, None, ws, wsb, None)
+
+    assert call(g=5) == INVALID and call(xt=9) == INVALID and call(rows=-1) == INVALID
+    assert call(q=None) == INVALID and call(s=None) == INVALID and call(ws=None) == INVALID
+    assert call(g=H.PER_CHANNEL, cols=100, wsb=1 << 16) == INVALID    # per-channel rows in 16-byte units
+    assert call(x=BASE + 2) == MISALIGNED and call(q=BASE + 0x1000008) == MISALIGNED
+    assert call(q=BASE + 0x40) == OVERLAP
+    assert call(g=H.PER_TOKEN, ws=None, wsb=0, rows=0) == OK        # nothing to do (no scales)
+
+
 def test_grouped_rejections():
     gg = L.hq_grouped_gemm_a8w8
     args = dict(xq=BASE, wq=BASE + 0x1000000, fmt=0, xs=BASE + 0x2000000, xsl=100, ws=BASE + 0x3000000,
