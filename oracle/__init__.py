@@ -58,6 +58,10 @@ def lib():
         L.hqo_encode_e5m2_sr.restype = ctypes.c_uint8
         L.hqo_quantize_e5m2_sr.argtypes = [P, ci, i64, i64, ci, ctypes.c_uint64, P, P, P]
         L.hqo_quantize_e5m2_sr.restype = ci
+        L.hqo_quantize_blockwise.argtypes = [P, ci, i64, i64, ci, i64, ci, ctypes.c_uint64, P, P, P]
+        L.hqo_quantize_blockwise.restype = ci
+        L.hqo_dequantize_blockwise.argtypes = [P, ci, i64, i64, i64, P, ci, P]
+        L.hqo_dequantize_blockwise.restype = ci
         L.hqo_gemm_a8w8_bias.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P]
         L.hqo_gemm_a8w8_bias.restype = None
         L.hqo_gemm_a8w8_entries.argtypes = [P, P, ci, P, i64, P, i64, i64, P, P, i64, P]
@@ -209,6 +213,34 @@ def quantize_e5m2_sr(x, gran, seed):
     if rc != 0:
         raise ValueError("invalid arguments")
     return q, s, a
+
+
+def quantize_blockwise(x, fmt, block, stochastic=False, seed=0):
+    """Block-wise quantize along the last dimension: (codes [rows, cols],
+    dequant scales f32 [rows, ceil(cols/block)], amax of the same shape)."""
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    nb = -(-cols // block)
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty((rows, nb), np.float32)
+    a = np.empty((rows, nb), np.float32)
+    rc = lib().hqo_quantize_blockwise(_p(x), _dtype_code(x), rows, cols, fmt, block, 1 if stochastic else 0, seed,
+                                      _p(q), _p(s), _p(a))
+    if rc != 0:
+        raise ValueError("invalid arguments")
+    return q, s, a
+
+
+def dequantize_blockwise(q, fmt, block, scales, bf16=False):
+    """f32(dec(q) * block scale), or its bf16 bits."""
+    q = np.ascontiguousarray(q, np.uint8)
+    sc = np.ascontiguousarray(scales, np.float32)
+    rows, cols = q.shape
+    out = np.empty((rows, cols), np.uint16 if bf16 else np.float32)
+    rc = lib().hqo_dequantize_blockwise(_p(q), fmt, rows, cols, block, _p(sc), 1 if bf16 else 0, _p(out))
+    if rc != 0:
+        raise ValueError("invalid arguments")
+    return out
 
 
 def gemm_a8w8_bias(xq, wq, fmt, x_scale, w_scale, bias_bf16_bits):

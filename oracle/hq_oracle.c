@@ -387,6 +387,59 @@ int hqo_quantize_e5m2_sr(const void* x, int dtype, int64_t rows, int64_t cols,
   return 0;
 }
 
+/* ------------------------------------------------------------ block-wise */
+
+/* Block-wise quantize ([HQ] "Block-wise FP8 Scaling"): one f32 dequant scale
+   per block of `block` consecutive elements along the last dimension, scales
+   [rows, ceil(cols / block)] (the last block of a row may be shorter).  Per
+   block: amax over the finite |x|, m = fmax / amax (1 when amax is 0 or the
+   quotient is not finite), scale = 1 / m, codes of f32(x) * m, rounded to
+   nearest even or, with stochastic != 0 (E5M2 only), by hqo_encode_e5m2_sr
+   with the draw of the element's flat index under `seed`. */
+int hqo_quantize_blockwise(const void* x, int dtype, int64_t rows, int64_t cols,
+                           int fmt, int64_t block, int stochastic, uint64_t seed,
+                           uint8_t* q, float* scales, float* amax_out) {
+  int64_t nb, r, b, c;
+  if (block < 1 || rows < 0 || cols < 0 || (stochastic && fmt != HQO_E5M2)) return -1;
+  nb = (cols + block - 1) / block;
+  for (r = 0; r < rows; ++r)
+    for (b = 0; b < nb; ++b) {
+      int64_t c0 = b * block, c1 = c0 + block < cols ? c0 + block : cols;
+      float amax = 0.0f, m;
+      for (c = c0; c < c1; ++c) {
+        float v = fabsf(load_elem(x, dtype, r * cols + c));
+        if (isfinite(v) && v > amax) amax = v;
+      }
+      m = hqo_multiplier(amax, fmt);
+      scales[r * nb + b] = 1.0f / m;
+      if (amax_out) amax_out[r * nb + b] = amax;
+      for (c = c0; c < c1; ++c) {
+        float y = load_elem(x, dtype, r * cols + c) * m; /* one f32 mul */
+        q[r * cols + c] = stochastic ? hqo_encode_e5m2_sr(y, hqo_sr_bits(seed, (uint64_t)(r * cols + c)))
+                                     : hqo_encode_sat(y, fmt);
+      }
+    }
+  return 0;
+}
+
+/* Block-wise dequantize: out = f32(dec(q) * scale) of the element's block
+   (real ~= fp8 * block scale), one f32 multiply; bf16_out rounds that to
+   bf16 (nearest even). */
+int hqo_dequantize_blockwise(const uint8_t* q, int fmt, int64_t rows, int64_t cols,
+                             int64_t block, const float* scales, int bf16_out,
+                             void* out) {
+  int64_t nb, r, c;
+  if (block < 1 || rows < 0 || cols < 0) return -1;
+  nb = (cols + block - 1) / block;
+  for (r = 0; r < rows; ++r)
+    for (c = 0; c < cols; ++c) {
+      float v = (float)hqo_decode(q[r * cols + c], fmt) * scales[r * nb + c / block];
+      if (bf16_out) ((uint16_t*)out)[r * cols + c] = hqo_double_to_bf16((double)v);
+      else ((float*)out)[r * cols + c] = v;
+    }
+  return 0;
+}
+
 /* --------------------------------------------------------------------- GEMM */
 
 /* Integer numerator of a finite code: value = n * 2^-frac, frac = 9 (E4M3)

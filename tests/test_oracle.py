@@ -678,3 +678,75 @@ def test_sr_quantize_scales_match_and_codes_are_neighbours():
         # reproducible by seed, different under another seed
         assert np.array_equal(O.quantize_e5m2_sr(x, gran, seed=1234)[0], q)
         assert not np.array_equal(O.quantize_e5m2_sr(x, gran, seed=99)[0], q)
+
+
+# ------------------------------------------------------------ block-wise
+@pytest.mark.parametrize("fmt", FMTS)
+def test_blockwise_reduces_to_per_token_when_one_block_spans_the_row(fmt):
+    rng = np.random.default_rng(61)
+    x = W.f32_to_bf16_bits(rng.standard_normal((9, 96)).astype(np.float32) * np.float32(7.0))
+    q, s, a = O.quantize_blockwise(x, fmt, 96)
+    qt, st, at = O.quantize(x, fmt, O.PER_TOKEN)
+    np.testing.assert_array_equal(q, qt)
+    np.testing.assert_array_equal(s.reshape(-1).view(np.uint32), st.view(np.uint32))
+    np.testing.assert_array_equal(a.reshape(-1).view(np.uint32), at.view(np.uint32))
+    # a block at least as long as the row behaves the same
+    q2, s2, _ = O.quantize_blockwise(x, fmt, 1000)
+    np.testing.assert_array_equal(q2, qt)
+    assert s2.shape == (9, 1)
+
+
+def test_blockwise_blocks_are_independent_row_slices():
+    # each block equals a per-token quantize of that slice alone; the ragged
+    # last block is the short remainder of the row
+    rng = np.random.default_rng(62)
+    x = (rng.standard_normal((5, 100)) * np.exp(rng.uniform(-3, 3, (5, 100)))).astype(np.float32)
+    x[2, 32:64] = 0.0          # an all-zero block: scale 1, codes 0
+    x[3, 7] = np.nan
+    x[4, 99] = np.inf
+    q, s, a = O.quantize_blockwise(x, O.E4M3, 32)
+    assert s.shape == (5, 4)
+    for b, (c0, c1) in enumerate([(0, 32), (32, 64), (64, 96), (96, 100)]):
+        qb, sb, ab = O.quantize(np.ascontiguousarray(x[:, c0:c1]), O.E4M3, O.PER_TOKEN)
+        np.testing.assert_array_equal(q[:, c0:c1], qb)
+        np.testing.assert_array_equal(s[:, b], sb)
+        np.testing.assert_array_equal(a[:, b], ab)
+    assert s[2, 1] == 1.0 and (q[2, 32:64] == 0).all()
+
+
+def test_blockwise_single_element_blocks_hit_the_max_code():
+    # block 1: every finite nonzero element is its own amax, so |y| = fmax
+    x = np.array([[1.5, -0.25, 3e-5, 0.0, 7.0, -900.0, 1e-30, 2.0]], np.float32)
+    q, s, _ = O.quantize_blockwise(x, O.E4M3, 1)
+    assert list(q[0]) == [0x7E, 0xFE, 0x7E, 0x00, 0x7E, 0xFE, 0x7E, 0x7E]
+    assert s[0, 3] == 1.0
+
+
+def test_blockwise_stochastic_matches_the_element_rule():
+    rng = np.random.default_rng(63)
+    x = (rng.standard_normal((3, 64)) * np.float32(5e-3)).astype(np.float32)
+    q, s, _ = O.quantize_blockwise(x, O.E5M2, 16, stochastic=True, seed=9)
+    for r in range(3):
+        for c in range(64):
+            y = np.float32(x[r, c] * np.float32(O.multiplier(float(np.abs(x[r, (c // 16) * 16:(c // 16 + 1) * 16]).max()), O.E5M2)))
+            assert q[r, c] == O.encode_e5m2_sr(y, O.sr_bits(9, r * 64 + c))
+    with pytest.raises(ValueError):
+        O.quantize_blockwise(x, O.E4M3, 16, stochastic=True)
+
+
+def test_blockwise_dequantize_closed_forms():
+    rng = np.random.default_rng(64)
+    q = rng.integers(0, 256, (4, 48), dtype=np.uint8)
+    q[O.decode_array(q.reshape(-1), O.E4M3).reshape(q.shape) != O.decode_array(q.reshape(-1), O.E4M3).reshape(q.shape)] = 0
+    sc = np.array([[0.5, 2.0, 0.125]] * 4, np.float32)
+    out = O.dequantize_blockwise(q, O.E4M3, 16, sc)
+    dec = O.decode_array(q.reshape(-1), O.E4M3).reshape(q.shape)
+    np.testing.assert_array_equal(out, (dec * np.repeat(sc, 16, axis=1)).astype(np.float32))  # powers of two: exact
+    # bf16 output: the f32 product rounded once
+    outb = O.dequantize_blockwise(q, O.E4M3, 16, sc, bf16=True)
+    np.testing.assert_array_equal(outb, W.f32_to_bf16_bits(out))
+    # a round trip through quantize recovers every value to within half a code step
+    x = (rng.standard_normal((4, 48)) * 3).astype(np.float32)
+    qq, ss, _ = O.quantize_blockwise(x, O.E4M3, 16)
+    back = O.dequantize_blockwise(qq, O.E4M3, 16, ss)
+    assert (np.abs(back - x) <= np.abs(x) * 2.0 ** -4 + np.repeat(ss, 16, axis=1) * 2.0 ** -9).all()
