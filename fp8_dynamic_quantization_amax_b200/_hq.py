@@ -21,7 +21,8 @@ PER_TENSOR, PER_TOKEN, PER_CHANNEL = 0, 1, 2
 F32, BF16, F16 = 0, 1, 2
 
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
-            "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
+            "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic",
+            "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
             "hq_grouped_gemm_bf16",
             "hq_quantize_fp8_noalloc", "hq_check_device_error", "hq_last_error", "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
@@ -52,6 +53,10 @@ def _load():
     L.hq_quantize_fp8.restype = ci
     L.hq_quantize_fp8_noalloc.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P]
     L.hq_quantize_fp8_noalloc.restype = ci
+    L.hq_quantize_fp8_blockwise.argtypes = [P, ci, i64, i64, ci, i64, ci, ctypes.c_uint64, P, P, P, P]
+    L.hq_quantize_fp8_blockwise.restype = ci
+    L.hq_dequantize_fp8_blockwise.argtypes = [P, ci, i64, i64, i64, P, ci, P, P]
+    L.hq_dequantize_fp8_blockwise.restype = ci
     L.hq_quantize_e5m2_stochastic.argtypes = [P, ci, i64, i64, ci, ctypes.c_uint64, P, P, P, P, sz, P]
     L.hq_quantize_e5m2_stochastic.restype = ci
     L.hq_quantize_fp8_transpose.argtypes = [P, ci, i64, i64, ci, P, P, P, P, P, P, i32, i32, i32, P, sz, P]
@@ -156,6 +161,30 @@ def hq_quantize_fp8(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=N
                               _ptr(workspace), 0 if workspace is None else workspace.numel(),
                               _stream(stream)))
     return q, scales
+
+
+def hq_quantize_fp8_blockwise(x, fmt=E4M3, block=32, stochastic=False, seed=0, amax_out=None, stream=None):
+    """Block-wise quantize along the last dimension.  Returns (q uint8
+    [rows, cols], dequant scales f32 [rows, ceil(cols / block)])."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    x = x.contiguous()
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows, -(-cols // block)), dtype=torch.float32, device=x.device)
+    check(lib.hq_quantize_fp8_blockwise(_ptr(x), _DT[x.dtype], rows, cols, fmt, block, 1 if stochastic else 0,
+                                        seed & ((1 << 64) - 1), _ptr(q), _ptr(scales), _ptr(amax_out),
+                                        _stream(stream)))
+    return q, scales
+
+
+def hq_dequantize_fp8_blockwise(q, scales, fmt=E4M3, block=32, out_dtype=torch.float32, stream=None):
+    """f32(dec(q) * block scale), as float32 or rounded to bfloat16."""
+    rows, cols = q.shape
+    out = torch.empty((rows, cols), dtype=out_dtype, device=q.device)
+    check(lib.hq_dequantize_fp8_blockwise(_ptr(q.contiguous()), fmt, rows, cols, block, _ptr(scales.contiguous()),
+                                          _DT[out_dtype], _ptr(out), _stream(stream)))
+    return out
 
 
 def hq_quantize_e5m2_stochastic(x, gran=PER_TENSOR, seed=0, q=None, scales=None, amax_out=None, workspace=None,

@@ -238,6 +238,79 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
   return launched(hq::launch_quantize(a), "quantize launch");
 }
 
+hq_status hq_quantize_fp8_blockwise(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                                    int64_t block, int stochastic, uint64_t seed, uint8_t* q, float* scales,
+                                    float* amax_out, hq_stream_t stream) {
+  if (xt != HQ_F32 && xt != HQ_BF16 && xt != HQ_F16) return fail(HQ_ERR_INVALID_ARG, "invalid dtype %d", (int)xt);
+  if (fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", (int)fmt);
+  if (stochastic && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "stochastic rounding is for E5M2");
+  if (rows < 0 || cols < 0) return fail(HQ_ERR_INVALID_ARG, "negative shape [%lld, %lld]", (long long)rows, (long long)cols);
+  if (rows >= k2p31 || cols >= k2p31 || (cols > 0 && rows > (k2p40 - 1) / cols))
+    return fail(HQ_ERR_TOO_LARGE, "shape [%lld, %lld] is beyond the supported range", (long long)rows, (long long)cols);
+  if (block < 16 || block % 16 != 0 || block >= k2p31)
+    return fail(HQ_ERR_INVALID_ARG, "block = %lld must be a positive multiple of 16", (long long)block);
+  if (cols % 16 != 0) return fail(HQ_ERR_INVALID_ARG, "cols must be a multiple of 16");
+  const int64_t n = rows * cols;
+  const int64_t ns = rows * ((cols + block - 1) / block);
+  const size_t esize = (xt == HQ_F32) ? 4 : 2;
+  if (n == 0) return ok();
+  if (!x || !q || !scales) return fail(HQ_ERR_INVALID_ARG, "x, q and scales must not be null");
+  if (!is_aligned(x, 16) || !is_aligned(q, 16)) return fail(HQ_ERR_MISALIGNED, "x and q must be 16-byte aligned");
+  if (!is_aligned(scales, 4) || !is_aligned(amax_out, 4))
+    return fail(HQ_ERR_MISALIGNED, "scales and amax_out must be 4-byte aligned");
+  const Range outs[] = {{q, static_cast<size_t>(n), "q"},
+                        {scales, static_cast<size_t>(ns) * 4, "scales"},
+                        {amax_out, amax_out ? static_cast<size_t>(ns) * 4 : 0, "amax_out"}};
+  const Range ins[] = {{x, static_cast<size_t>(n) * esize, "x"}};
+  hq_status s = check_overlaps(outs, 3, ins, 1);
+  if (s != HQ_OK) return s;
+  const Range devs[] = {{x, 0, "x"}, {q, 0, "q"}, {scales, 0, "scales"}, {amax_out, 0, "amax_out"}};
+  s = check_device_ptrs(devs, 4);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  hq::QuantizeArgs a;
+  a.x = x; a.xt = xt; a.rows = rows; a.cols = cols; a.fmt = fmt; a.gran = HQ_PER_TOKEN;
+  a.q = q; a.scales = scales; a.amax_out = amax_out;
+  a.ring = nullptr; a.ring_len = 0; a.ring_idx = 0; a.ring_margin = 0;
+  a.ws = nullptr;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.seed = seed;
+  return launched(hq::launch_quantize_blockwise(a, block, stochastic != 0), "block-wise quantize launch");
+}
+
+hq_status hq_dequantize_fp8_blockwise(const uint8_t* q, hq_fp8_format fmt, int64_t rows, int64_t cols,
+                                      int64_t block, const float* scales, hq_dtype out_type, void* out,
+                                      hq_stream_t stream) {
+  if (fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", (int)fmt);
+  if (out_type != HQ_F32 && out_type != HQ_BF16) return fail(HQ_ERR_INVALID_ARG, "out_type must be F32 or BF16");
+  if (rows < 0 || cols < 0) return fail(HQ_ERR_INVALID_ARG, "negative shape [%lld, %lld]", (long long)rows, (long long)cols);
+  if (rows >= k2p31 || cols >= k2p31 || (cols > 0 && rows > (k2p40 - 1) / cols))
+    return fail(HQ_ERR_TOO_LARGE, "shape [%lld, %lld] is beyond the supported range", (long long)rows, (long long)cols);
+  if (block < 16 || block % 16 != 0 || block >= k2p31)
+    return fail(HQ_ERR_INVALID_ARG, "block = %lld must be a positive multiple of 16", (long long)block);
+  if (cols % 16 != 0) return fail(HQ_ERR_INVALID_ARG, "cols must be a multiple of 16");
+  const int64_t n = rows * cols;
+  const int64_t ns = rows * ((cols + block - 1) / block);
+  if (n == 0) return ok();
+  if (!q || !scales || !out) return fail(HQ_ERR_INVALID_ARG, "q, scales and out must not be null");
+  if (!is_aligned(q, 16) || !is_aligned(out, 16)) return fail(HQ_ERR_MISALIGNED, "q and out must be 16-byte aligned");
+  if (!is_aligned(scales, 4)) return fail(HQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  const size_t osize = out_type == HQ_F32 ? 4 : 2;
+  const Range outs[] = {{out, static_cast<size_t>(n) * osize, "out"}};
+  const Range ins[] = {{q, static_cast<size_t>(n), "q"}, {scales, static_cast<size_t>(ns) * 4, "scales"}};
+  hq_status s = check_overlaps(outs, 1, ins, 2);
+  if (s != HQ_OK) return s;
+  const Range devs[] = {{q, 0, "q"}, {scales, 0, "scales"}, {out, 0, "out"}};
+  s = check_device_ptrs(devs, 3);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  return launched(hq::launch_dequantize_blockwise(q, fmt, rows, cols, block, scales, out_type == HQ_BF16, out,
+                                                  reinterpret_cast<cudaStream_t>(stream)),
+                  "block-wise dequantize launch");
+}
+
 hq_status hq_quantize_e5m2_stochastic(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_granularity g,
                                       uint64_t seed, uint8_t* q, float* scales, float* amax_out, void* workspace,
                                       size_t workspace_bytes, hq_stream_t stream) {

@@ -41,6 +41,11 @@ cudaError_t launch_quantize_transpose(const QuantizeArgs& a);
 // Dynamic E5M2 quantize with stochastic rounding (a.seed); x 16-byte aligned,
 // cols a multiple of the 16-byte vector for the per-channel form.
 cudaError_t launch_quantize_sr(const QuantizeArgs& a);
+// Block-wise quantize (scales [rows, ceil(cols / block)]) and dequantize;
+// block % 16 == 0, cols % 16 == 0, 16-byte aligned buffers.
+cudaError_t launch_quantize_blockwise(const QuantizeArgs& a, int64_t block, bool stochastic);
+cudaError_t launch_dequantize_blockwise(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int64_t block,
+                                        const float* scales, bool bf16_out, void* out, cudaStream_t stream);
 
 struct GemmArgs {
   int kind;                 // 0: fp8 a8w8 (kind::f8f6f4), 1: bf16 (kind::f16)

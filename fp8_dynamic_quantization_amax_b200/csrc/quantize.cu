@@ -36,6 +36,7 @@
 
 #include <algorithm>
 #include <cfloat>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <type_traits>
 
@@ -1519,6 +1520,96 @@ __global__ void __launch_bounds__(kThreads) k_sr_token(const void* __restrict__ 
                                          sr_draw(seed, static_cast<uint64_t>(base + c))));
 }
 
+// ---------------------------------------------------------------- block-wise
+// Block-wise FP8 (hip-quant README "Block-wise FP8 Scaling"): one f32 dequant
+// scale per block of `block` consecutive elements along the last dimension,
+// scales [rows, ceil(cols / block)] (the last block of a row may be short).
+// One thread per block, consecutive threads on consecutive blocks: the block
+// is read with 16-byte loads for its finite amax (raw bits, exact redo when
+// a non-finite element shows), then again (from L1) for the cast, rounded
+// to nearest even or, SR, stochastically (E5M2).  block % 16 == 0 and
+// cols % 16 == 0.
+template <int DT, int FMT, bool SR>
+__global__ void __launch_bounds__(kThreads) k_block_quant(const void* __restrict__ x, int64_t rows, int64_t cols,
+                                                          int64_t block, uint64_t seed, uint8_t* __restrict__ q,
+                                                          float* __restrict__ scales, float* __restrict__ amax_out) {
+  constexpr int VEC = Dt<DT>::kVec;
+  const int64_t nb = (cols + block - 1) / block;
+  const int64_t total = rows * nb;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t r = t / nb, b = t - r * nb;
+    const int64_t c0 = b * block;
+    const int nvec = static_cast<int>((min(cols, c0 + block) - c0) / VEC);
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(x) + (r * cols + c0) * Dt<DT>::kSize);
+    uint32_t mraw = 0;
+    for (int v = 0; v < nvec; ++v) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(__ldg(src + v)));
+    float amax = 0.0f;
+    if (!Dt<DT>::nonfinite(mraw)) {
+      amax = Dt<DT>::value(mraw);
+    } else {
+      for (int v = 0; v < nvec; ++v) amax = vec_amax_exact<DT>(__ldg(src + v), amax);
+    }
+    const float m = multiplier(amax, Fmt<FMT>::kMax);
+    scales[t] = __fdiv_rn(1.0f, m);
+    if (amax_out) amax_out[t] = amax;
+    uint8_t* dst = q + r * cols + c0;
+    for (int v = 0; v < nvec; ++v) {
+      const uint4 u = __ldg(src + v);
+      if constexpr (SR) sr_store_vec<DT>(dst + v * VEC, u, m, seed, static_cast<uint64_t>(r * cols + c0 + v * VEC));
+      else vec_store<DT, FMT, false>(dst + v * VEC, u, m);
+    }
+  }
+}
+
+// Block-wise dequantize: out = f32(dec(q) * block scale), or that rounded to
+// bf16.  The codes decode exactly through cvt to f16 pairs.  One thread per
+// 16 codes.
+template <int FMT, bool BF16_OUT>
+__global__ void __launch_bounds__(kThreads) k_block_dequant(const uint8_t* __restrict__ q, int64_t rows, int64_t cols,
+                                                            int64_t block, const float* __restrict__ scales,
+                                                            void* __restrict__ out) {
+  const int64_t nb = (cols + block - 1) / block;
+  const int64_t n16 = rows * cols / 16;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; t < n16;
+       t += static_cast<int64_t>(gridDim.x) * kThreads) {
+    const int64_t e0 = t * 16;
+    const int64_t r = e0 / cols, c = e0 - r * cols;  // cols % 16 == 0: the 16 codes share a row
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(q) + t);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float f[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const unsigned short pair = static_cast<unsigned short>(w[k] >> (16 * h));
+        uint32_t hh;
+        if (FMT == 0) asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"(pair));
+        else asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(hh) : "h"(pair));
+        f[4 * k + 2 * h] = __half2float(__ushort_as_half(static_cast<unsigned short>(hh & 0xFFFFu)));
+        f[4 * k + 2 * h + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(hh >> 16)));
+      }
+    // block % 16 == 0 and c % 16 == 0: the 16 codes also share one block
+    const float sc = __ldg(scales + r * nb + c / block);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], sc);
+    if constexpr (BF16_OUT) {
+      uint32_t o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        o[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * i]))) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * i + 1]))) << 16);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + e0);
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    } else {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + e0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+    }
+  }
+}
+
 // ------------------------------------------------------------------- launch
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -1786,7 +1877,46 @@ cudaError_t launch_sr_typed(const QuantizeArgs& a) {
   return cudaGetLastError();
 }
 
+template <int DT>
+cudaError_t launch_block_typed(const QuantizeArgs& a, int64_t block, bool sr) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t nb = (a.cols + block - 1) / block;
+  const int grid = flat_grid(a.rows * nb, dev, 1);
+  if (sr)
+    k_block_quant<DT, 1, true><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, block, a.seed, a.q, a.scales,
+                                                                 a.amax_out);
+  else if (a.fmt == 0)
+    k_block_quant<DT, 0, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, block, 0, a.q, a.scales,
+                                                                  a.amax_out);
+  else
+    k_block_quant<DT, 1, false><<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, a.cols, block, 0, a.q, a.scales,
+                                                                  a.amax_out);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_blockwise(const QuantizeArgs& a, int64_t block, bool stochastic) {
+  switch (a.xt) {
+    case 0: return launch_block_typed<0>(a, block, stochastic);
+    case 1: return launch_block_typed<1>(a, block, stochastic);
+    case 2: return launch_block_typed<2>(a, block, stochastic);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_dequantize_blockwise(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int64_t block,
+                                        const float* scales, bool bf16_out, void* out, cudaStream_t stream) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int grid = flat_grid(rows * cols / 16, dev, 1);
+  if (fmt == 0 && bf16_out) k_block_dequant<0, true><<<grid, kThreads, 0, stream>>>(q, rows, cols, block, scales, out);
+  else if (fmt == 0) k_block_dequant<0, false><<<grid, kThreads, 0, stream>>>(q, rows, cols, block, scales, out);
+  else if (bf16_out) k_block_dequant<1, true><<<grid, kThreads, 0, stream>>>(q, rows, cols, block, scales, out);
+  else k_block_dequant<1, false><<<grid, kThreads, 0, stream>>>(q, rows, cols, block, scales, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_sr(const QuantizeArgs& a) {
   switch (a.xt) {

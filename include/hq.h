@@ -145,6 +145,38 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
                           void* workspace, size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * Block-wise FP8 (hip-quant README "Block-wise FP8 Scaling"): the codes of x
+ * [rows, cols] plus one f32 dequant scale per block of `block` consecutive
+ * elements along the last dimension, scales [rows, ceil(cols / block)] (the
+ * last block of a row may be shorter), real value ~= fp8 * block scale.  Per
+ * block: amax over the finite |x|, m = fmax / amax (1 when amax is 0 or the
+ * quotient is not finite), scale = 1/m, codes of f32(x) * m rounded to
+ * nearest even, or, with stochastic != 0 (E5M2 only), rounded as
+ * hq_quantize_e5m2_stochastic rounds (draws by row-major element index under
+ * `seed`).  With block >= cols this is the per-token quantize.
+ *
+ * Arguments: x device [rows, cols] f32 / bf16 / f16 (xt), q device uint8
+ *   [rows, cols], both 16-byte aligned; cols % 16 == 0; block % 16 == 0;
+ *   scales device f32 [rows * ceil(cols / block)]; amax_out the same or NULL.
+ * Errors: HQ_ERR_INVALID_ARG, HQ_ERR_MISALIGNED, HQ_ERR_OVERLAP,
+ *   HQ_ERR_WRONG_DEVICE, HQ_ERR_UNSUPPORTED_ARCH, HQ_ERR_TOO_LARGE,
+ *   HQ_ERR_CUDA.
+ */
+hq_status hq_quantize_fp8_blockwise(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                                    int64_t block, int stochastic, uint64_t seed, uint8_t* q, float* scales,
+                                    float* amax_out, hq_stream_t stream);
+
+/*
+ * Block-wise dequantize: out[r, c] = f32(dec(q[r, c]) * scales[r, c / block])
+ * (one f32 multiply), written as f32 (out_type HQ_F32) or rounded to bf16
+ * (HQ_BF16).  Same layout rules as hq_quantize_fp8_blockwise; out 16-byte
+ * aligned.
+ */
+hq_status hq_dequantize_fp8_blockwise(const uint8_t* q, hq_fp8_format fmt, int64_t rows, int64_t cols,
+                                      int64_t block, const float* scales, hq_dtype out_type, void* out,
+                                      hq_stream_t stream);
+
+/*
  * Dynamic quantize to E5M2 with stochastic rounding, for gradients
  * (hip-quant README "Stochastic E5M2 Backward Gradients": between the two
  * adjacent E5M2 values, with probability proportional to the distance, from

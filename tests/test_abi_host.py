@@ -220,3 +220,31 @@ def test_missing_library_fails_loudly(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import fp8_dynamic_quantization_amax_b200"], cwd=str(tmp_path),
                        capture_output=True, text=True)
     assert r.returncode != 0 and "libhq.so is not built" in r.stderr
+
+
+def test_blockwise_rejections():
+    bq = L.hq_quantize_fp8_blockwise
+
+    def call(x=BASE, xt=H.BF16, rows=64, cols=128, fmt=H.E4M3, block=32, sr=0, q=BASE + 0x1000000,
+             s=BASE + 0x2000000, a=None):
+        return bq(x, xt, rows, cols, fmt, block, sr, 7, q, s, a, None)
+
+    assert call(block=24) == INVALID and call(block=0) == INVALID and call(cols=120) == INVALID
+    assert call(sr=1) == INVALID                      # stochastic rounding is E5M2-only
+    assert call(xt=9) == INVALID and call(fmt=3) == INVALID and call(rows=-2) == INVALID
+    assert call(q=None) == INVALID and call(s=None) == INVALID
+    assert call(x=BASE + 2) == MISALIGNED and call(q=BASE + 0x1000008) == MISALIGNED
+    assert call(s=BASE + 0x2000002) == MISALIGNED
+    assert call(s=BASE + 0x100) == OVERLAP and call(a=BASE + 0x2000010) == OVERLAP
+    assert call(rows=0, x=None, q=None, s=None) == OK
+    dq = L.hq_dequantize_fp8_blockwise
+
+    def dcall(q=BASE, fmt=H.E5M2, rows=64, cols=128, block=64, s=BASE + 0x1000000, ot=H.F32,
+              out=BASE + 0x2000000):
+        return dq(q, fmt, rows, cols, block, s, ot, out, None)
+
+    assert dcall(ot=H.F16) == INVALID and dcall(block=8) == INVALID and dcall(cols=72) == INVALID
+    assert dcall(out=None) == INVALID and dcall(s=None) == INVALID
+    assert dcall(out=BASE + 0x2000004) == MISALIGNED and dcall(q=BASE + 8) == MISALIGNED
+    assert dcall(out=BASE + 0x40) == OVERLAP and dcall(out=BASE + 0x1000000 - 0x100) == OVERLAP
+    assert dcall(cols=0, q=None, s=None, out=None) == OK
