@@ -56,6 +56,8 @@ def dist_env():
 # decode: the same layer at small M; W quantized once before timing (weights
 #   are static at inference), the step is quantize X + GEMM.
 # sweep: quantize only, bf16 [8192, 8192]; every granularity x format.
+# blockwise: block-wise quantize of the sweep input along its rows (E4M3 at
+#   blocks of 128 and 32, stochastic E5M2 at 128) and the bf16 dequantize.
 # moe / moe_bf16: per-token quantize of the routed tokens + grouped a8w8 GEMM
 #   over 64 experts (W quantized once); the bf16 grouped GEMM alone.
 WORKLOADS = {
@@ -68,6 +70,7 @@ WORKLOADS = {
     "sweep": dict(kind="sweep", M=8192, N=0, K=8192),
     "stack": dict(kind="stack", M=2048, N=4096, K=1024, steps_cycle=200, ring=16),
     "backward": dict(kind="backward", M=16384, N=28672, K=8192, ring=16),
+    "blockwise": dict(kind="blockwise", M=8192, N=0, K=8192),
     "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
     "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }
@@ -92,6 +95,10 @@ def workload_desc(name, cfg):
     if k == "sweep":
         return ("quantize sweep: bf16 [%d,%d] ~N(0,1), 0.1%% x100 outliers, 0.1%% zeros, one zero row; "
                 "per-tensor / per-token / per-channel x E4M3 / E5M2" % (cfg["M"], cfg["K"]))
+    if k == "blockwise":
+        return ("block-wise quantize: bf16 [%d,%d] ~N(0,1) with the sweep's outliers and zeros, scales per block "
+                "along the rows: E4M3 blocks of 128 and 32, stochastic E5M2 blocks of 128, and the bf16 "
+                "dequantize of the E4M3 block-128 codes" % (cfg["M"], cfg["K"]))
     return ("grouped MoE GEMM: %d experts, K=%d, N=%d, %d tokens by Zipf(1.1) counts (2 experts empty); %s" %
             (cfg["E"], cfg["K"], cfg["N"], cfg["M"],
              "per-token E4M3 X + per-expert per-channel E4M3 W, a8w8" if k == "moe" else "bf16 X and W, fp32 acc"))
@@ -489,6 +496,61 @@ def build(args, cfg, rank, dev, stream, peaks):
                     extras=extras, flush=lambda: torch.amax(flush, dim=0, out=sink),
                     l2="L2 flushed (512 MB read) before every call; value = bytes / summed call times")
 
+    if kind == "blockwise":
+        x_host = bf16_host(W.sweep(M, K, seed=rank)).view(M, K)
+        x = x_host.to(dev)
+        flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev).fill_(1)
+        sink = torch.empty((), dtype=torch.uint8, device=dev)
+        lib, P, st = hq.lib, (lambda t: t.data_ptr()), stream.cuda_stream
+        modes = [("e4m3 b128", hq.E4M3, 128, 0), ("e4m3 b32", hq.E4M3, 32, 0), ("e5m2 sr b128", hq.E5M2, 128, 1)]
+        calls, outs, per, bytes_of = [], [], 0, {}
+        for label, fmt, blk, sr in modes:
+            q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+            sc = torch.empty((M, -(-K // blk)), dtype=torch.float32, device=dev)
+            outs.append((q, sc, torch.empty((M, K), dtype=torch.uint8).pin_memory(),
+                         torch.empty(tuple(sc.shape), dtype=torch.float32).pin_memory()))
+            calls.append(("quantize " + label,
+                          (lambda fmt=fmt, blk=blk, sr=sr, q=q, sc=sc:
+                           hq.check(lib.hq_quantize_fp8_blockwise(P(x), hq.BF16, M, K, fmt, blk, sr, 2024, P(q),
+                                                                  P(sc), None, st))), 1))
+            bytes_of["quantize " + label] = q_bytes(M, K, sc.numel())
+        q128, s128 = outs[0][0], outs[0][1]
+        deq = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        deq_host = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
+        calls.append(("dequantize e4m3 b128 -> bf16",
+                      lambda: hq.check(lib.hq_dequantize_fp8_blockwise(P(q128), hq.E4M3, M, K, 128, P(s128), hq.BF16,
+                                                                       P(deq), st)), 1))
+        bytes_of["dequantize e4m3 b128 -> bf16"] = M * K * 3 + 4 * s128.numel()
+        per = sum(bytes_of.values())
+
+        def e2e():
+            x.copy_(x_host, non_blocking=True)
+            for c, (q, sc, qh, sh) in zip(calls, outs):
+                c[1]()
+                qh.copy_(q, non_blocking=True)
+                sh.copy_(sc, non_blocking=True)
+            calls[-1][1]()
+            deq_host.copy_(deq, non_blocking=True)
+
+        def roofline(ms):
+            label = "quantize e4m3 b128"
+            a = bytes_of[label] / (ms[label] / 1e3) / 1e9
+            return {"bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(a / peaks["hbm_gbs"], 4), "traffic": None,
+                    "kernel": "k_block_quant_warp (E4M3, blocks of 128)", "peak_source": "%s copy" % peaks["_src"]}
+
+        def extras(ms):
+            d = {}
+            for label, t in ms.items():
+                gb = bytes_of[label] / (t / 1e3) / 1e9
+                d[label] = {"ms": round(t, 4), "GB/s": round(gb, 1), "frac_hbm": round(gb / peaks["hbm_gbs"], 4)}
+            return {"blockwise": d}
+
+        return dict(calls=calls, per_step=per, unit="GB/s", e2e=e2e, h2d=M * K * 2,
+                    d2h=sum(q.numel() + 4 * sc.numel() for q, sc, _, _ in outs) + M * K * 2, roofline=roofline,
+                    extras=extras, flush=lambda: torch.amax(flush, dim=0, out=sink),
+                    l2="L2 flushed (512 MB read) before every call; value = bytes / summed call times")
+
     # moe / moe_bf16
     E = cfg["E"]
     xb, wb, off = W.moe_inputs(E, M, N, K, seed=rank)
@@ -617,6 +679,13 @@ def run_ours(args, rank, local_rank, world):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and cfg["kind"] in ("layer", "decode"):
         mx = min(256, cfg["M"])
         cpu = cpu_baseline(cfg["M"], cfg["N"], cfg["K"], budget_rows=(mx, min(cfg["N"], 4096 * 256 // mx)))
+    elif rank == 0 and world == 1 and not args.no_cpu_baseline and cfg["kind"] in ("sweep", "blockwise"):
+        rows = 256
+        fn = cpu_sweep_sample if cfg["kind"] == "sweep" else cpu_blockwise_sample
+        byts, dt = fn(rows, cfg["K"])
+        cpu = {"value": byts / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": "%d rows x %d cols of the workload's input, every call of the step, %.1f s"
+                         % (rows, cfg["K"], dt), "seconds": round(dt, 2)}
 
     wl.pop("graphs", None)  # release captured graphs before the process group goes
     if world > 1:
@@ -635,7 +704,8 @@ def run_ours(args, rank, local_rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)" if cfg["kind"] != "moe_bf16" else "bf16 (fp32 accumulate)",
+        "dtype": ("bf16 -> fp8 codes + f32 scales" if cfg["kind"] in ("sweep", "blockwise") else
+                  "fp8_e4m3 (fp32 accumulate, bf16 out)" if cfg["kind"] != "moe_bf16" else "bf16 (fp32 accumulate)"),
         "data": "synthetic (seeded host generators; X seed = rank)",
         "config": {"workload": workload_desc(args.workload, cfg), "M": cfg["M"], "N": cfg["N"], "K": cfg["K"],
                    "l2": wl["l2"], "parallelism": "dp%d" % world},
@@ -691,22 +761,43 @@ def cpu_sweep_sample(rows, cols, seed=0):
     return byts, time.perf_counter() - t
 
 
+def cpu_blockwise_sample(rows, cols, seed=0):
+    """The oracle on a row sample of the block-wise workload; returns
+    (algorithmic bytes, seconds)."""
+    import oracle as O
+    import workloads as W
+    x = W.sweep(rows, cols, seed=seed, zero_row=rows // 2)
+    O.lib()
+    t = time.perf_counter()
+    byts = 0
+    for fmt, blk, sr in ((O.E4M3, 128, False), (O.E4M3, 32, False), (O.E5M2, 128, True)):
+        q, s, _ = O.quantize_blockwise(x, fmt, blk, stochastic=sr, seed=2024)
+        byts += rows * cols * 3 + 4 * s.size
+        if blk == 128 and fmt == O.E4M3:
+            q128, s128 = q, s
+    O.dequantize_blockwise(q128, O.E4M3, 128, s128, bf16=True)
+    byts += rows * cols * 3 + 4 * s128.size
+    return byts, time.perf_counter() - t
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
     cfg = WORKLOADS[args.workload]
     M, N, K = cfg["M"], cfg["N"], cfg["K"]
-    if cfg["kind"] == "sweep":
+    if cfg["kind"] in ("sweep", "blockwise"):
         rows = 64
+        fn = cpu_sweep_sample if cfg["kind"] == "sweep" else cpu_blockwise_sample
         for _ in range(args.warmup):
-            cpu_sweep_sample(rows, K)
+            fn(rows, K)
         t = time.perf_counter()
         byts = 0
         for i in range(args.steps):
-            byts += cpu_sweep_sample(rows, K, seed=i)[0]
+            byts += fn(rows, K, seed=i)[0]
         dt = time.perf_counter() - t
         value, unit = byts / dt / 1e9, "GB/s"
-        sample = "per step: %d rows x %d cols of the sweep input, all six modes" % (rows, K)
+        sample = ("per step: %d rows x %d cols of the sweep input, %s" %
+                  (rows, K, "all six modes" if cfg["kind"] == "sweep" else "the four block-wise calls"))
         dtype = "fp8 codes from bf16, f64 oracle"
     else:
         rows = (8, 512)

@@ -1562,50 +1562,153 @@ __global__ void __launch_bounds__(kThreads) k_block_quant(const void* __restrict
   }
 }
 
+// Block-wise quantize, warp-cooperative, for power-of-two blocks.  A warp
+// takes chunks of UNR units of U = 32 * kVec * NV consecutive elements of one
+// row; lane l holds vectors l, l + 32, ... of each unit, so every load
+// instruction of the warp reads 512 contiguous bytes.  With NV == 1 a unit
+// holds U / block whole blocks, each on block / kVec adjacent lanes (a power
+// of two dividing 32) that reduce their raw magnitude by xor shuffles; with
+// NV > 1 the unit is one block.  Index arithmetic is one division per chunk;
+// within a row it is 32-bit, and the block index is a shift.  The codes equal
+// k_block_quant's.
+template <int DT, int FMT, bool SR, int NV>
+__global__ void __launch_bounds__(kThreads) k_block_quant_warp(const void* __restrict__ x, int64_t rows, int cols,
+                                                               int log2_block, uint64_t seed,
+                                                               uint8_t* __restrict__ q, float* __restrict__ scales,
+                                                               float* __restrict__ amax_out) {
+  constexpr int VEC = Dt<DT>::kVec;
+  constexpr int U = 32 * VEC * NV;
+  constexpr int UNR = NV == 1 ? 4 : (NV == 2 ? 2 : 1);
+  constexpr int CH = U * UNR;
+  const int lane = threadIdx.x & 31;
+  const int cpr = (cols + CH - 1) / CH;  // chunks per row
+  const int64_t chunks = rows * cpr;
+  const int nb = ((cols - 1) >> log2_block) + 1;
+  const int lpb = NV == 1 ? (1 << log2_block) / VEC : 32;
+  const uint4* xv = static_cast<const uint4*>(x);
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  const bool narrow = chunks <= 0xFFFFFFFFll;
+  for (int64_t ch = warp0; ch < chunks; ch += nwarps) {
+    int64_t r;
+    int cc;
+    if (narrow) {
+      const uint32_t c32 = static_cast<uint32_t>(ch), rr = c32 / static_cast<uint32_t>(cpr);
+      r = rr;
+      cc = static_cast<int>(c32 - rr * static_cast<uint32_t>(cpr)) * CH;
+    } else {
+      r = ch / cpr;
+      cc = static_cast<int>(ch - r * cpr) * CH;
+    }
+    const int64_t rbase = r * cols;
+    uint4 v[UNR][NV];
+#pragma unroll
+    for (int j = 0; j < UNR; ++j)
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int c = cc + j * U + (k * 32 + lane) * VEC;
+        v[j][k] = c < cols ? ld_stream(xv + (rbase + c) / VEC) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+    for (int j = 0; j < UNR; ++j) {
+      const int cu = cc + j * U;
+      if (cu >= cols) break;  // warp-uniform: the rest of the chunk is past the row
+      uint32_t mr = 0;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) mr = Dt<DT>::lmax(mr, vec_mag<DT>(v[j][k]));
+      for (int o = lpb >> 1; o > 0; o >>= 1) mr = Dt<DT>::lmax(mr, __shfl_xor_sync(0xFFFFFFFFu, mr, o));
+      const bool special = __any_sync(0xFFFFFFFFu, Dt<DT>::nonfinite(mr));
+      float amax;
+      if (!special) {
+        amax = Dt<DT>::value(mr);
+      } else {  // warp-uniform: every lane takes the exact amax of its block
+        amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) amax = vec_amax_exact<DT>(v[j][k], amax);
+        for (int o = lpb >> 1; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      }
+      const float m = multiplier(amax, Fmt<FMT>::kMax);
+      const int c0 = cu + lane * VEC;
+      if ((lane & (lpb - 1)) == 0 && c0 < cols) {
+        const int64_t t = r * nb + (c0 >> log2_block);
+        scales[t] = __fdiv_rn(1.0f, m);
+        if (amax_out) amax_out[t] = amax;
+      }
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int c = c0 + k * 32 * VEC;
+        if (c >= cols) continue;
+        if constexpr (SR) sr_store_vec<DT>(q + rbase + c, v[j][k], m, seed, static_cast<uint64_t>(rbase + c));
+        else if (!special) vec_store<DT, FMT, true>(q + rbase + c, v[j][k], m);
+        else vec_store<DT, FMT, false>(q + rbase + c, v[j][k], m);
+      }
+    }
+  }
+}
+
 // Block-wise dequantize: out = f32(dec(q) * block scale), or that rounded to
-// bf16.  The codes decode exactly through cvt to f16 pairs.  One thread per
-// 16 codes.
+// bf16.  The codes decode exactly through cvt to f16 pairs.
+template <int FMT, bool BF16_OUT>
+__device__ __forceinline__ void dequant16(const uint4& u, float sc, void* __restrict__ out, int64_t e0) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  float f[16];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const unsigned short pair = static_cast<unsigned short>(w[k] >> (16 * h));
+      uint32_t hh;
+      if (FMT == 0) asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"(pair));
+      else asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(hh) : "h"(pair));
+      f[4 * k + 2 * h] = __half2float(__ushort_as_half(static_cast<unsigned short>(hh & 0xFFFFu)));
+      f[4 * k + 2 * h + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(hh >> 16)));
+    }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], sc);
+  if constexpr (BF16_OUT) {
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      o[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * i]))) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * i + 1]))) << 16);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + e0);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  } else {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + e0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+  }
+}
+
+// One thread per 16 codes (cols % 16 == 0 and block % 16 == 0: the 16 share a
+// row and a block); kDequantUnroll groups are loaded before any is written.
+constexpr int kDequantUnroll = 4;
 template <int FMT, bool BF16_OUT>
 __global__ void __launch_bounds__(kThreads) k_block_dequant(const uint8_t* __restrict__ q, int64_t rows, int64_t cols,
                                                             int64_t block, const float* __restrict__ scales,
                                                             void* __restrict__ out) {
   const int64_t nb = (cols + block - 1) / block;
   const int64_t n16 = rows * cols / 16;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; t < n16;
-       t += static_cast<int64_t>(gridDim.x) * kThreads) {
-    const int64_t e0 = t * 16;
-    const int64_t r = e0 / cols, c = e0 - r * cols;  // cols % 16 == 0: the 16 codes share a row
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(q) + t);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    float f[16];
+  const int64_t gs = static_cast<int64_t>(gridDim.x) * kThreads;
+  const uint4* qv = reinterpret_cast<const uint4*>(q);
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; t0 < n16;
+       t0 += gs * kDequantUnroll) {
+    uint4 u[kDequantUnroll];
+    float sc[kDequantUnroll];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const unsigned short pair = static_cast<unsigned short>(w[k] >> (16 * h));
-        uint32_t hh;
-        if (FMT == 0) asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hh) : "h"(pair));
-        else asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(hh) : "h"(pair));
-        f[4 * k + 2 * h] = __half2float(__ushort_as_half(static_cast<unsigned short>(hh & 0xFFFFu)));
-        f[4 * k + 2 * h + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(hh >> 16)));
+    for (int j = 0; j < kDequantUnroll; ++j) {
+      const int64_t t = t0 + j * gs;
+      if (t < n16) {
+        const int64_t r = (t * 16) / cols, c = t * 16 - r * cols;
+        u[j] = ld_stream(qv + t);
+        sc[j] = __ldg(scales + r * nb + c / block);
       }
-    // block % 16 == 0 and c % 16 == 0: the 16 codes also share one block
-    const float sc = __ldg(scales + r * nb + c / block);
+    }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], sc);
-    if constexpr (BF16_OUT) {
-      uint32_t o[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        o[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * i]))) |
-               (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f[2 * i + 1]))) << 16);
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + e0);
-      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-    } else {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + e0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+    for (int j = 0; j < kDequantUnroll; ++j) {
+      const int64_t t = t0 + j * gs;
+      if (t < n16) dequant16<FMT, BF16_OUT>(u[j], sc[j], out, t * 16);
     }
   }
 }
@@ -1877,10 +1980,38 @@ cudaError_t launch_sr_typed(const QuantizeArgs& a) {
   return cudaGetLastError();
 }
 
+template <int DT, int NV>
+cudaError_t launch_block_warp(const QuantizeArgs& a, int64_t block, bool sr, int dev) {
+  constexpr int64_t CH = 32 * Dt<DT>::kVec * NV * (NV == 1 ? 4 : (NV == 2 ? 2 : 1));
+  const int64_t warps = a.rows * ((a.cols + CH - 1) / CH);  // one chunk per warp and pass
+  const int64_t g = (warps + kThreads / 32 - 1) / (kThreads / 32);
+  int log2_block = 0;
+  while ((int64_t{1} << log2_block) < block) ++log2_block;
+  auto kern = sr ? k_block_quant_warp<DT, 1, true, NV>
+                 : (a.fmt == 0 ? k_block_quant_warp<DT, 0, false, NV> : k_block_quant_warp<DT, 1, false, NV>);
+  // one resident wave: the warps stride over the units
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
+  if (e != cudaSuccess) return e;
+  const int64_t cap = static_cast<int64_t>(device_sm_count(dev)) * (per_sm > 0 ? per_sm : 1);
+  const int grid = static_cast<int>(g < 1 ? 1 : (g > cap ? cap : g));
+  kern<<<grid, kThreads, 0, a.stream>>>(a.x, a.rows, static_cast<int>(a.cols), log2_block, sr ? a.seed : 0, a.q,
+                                        a.scales, a.amax_out);
+  return cudaGetLastError();
+}
+
 template <int DT>
 cudaError_t launch_block_typed(const QuantizeArgs& a, int64_t block, bool sr) {
   int dev = 0;
   cudaGetDevice(&dev);
+  // Power-of-two blocks go to the warp-cooperative kernel: block / kVec lanes
+  // per block (2..32), or one block per unit of 2, 4 or 8 warp-wide vectors.
+  constexpr int64_t W = 32 * Dt<DT>::kVec;
+  const bool pow2 = (block & (block - 1)) == 0;
+  if (pow2 && block <= W) return launch_block_warp<DT, 1>(a, block, sr, dev);
+  if (pow2 && block == 2 * W) return launch_block_warp<DT, 2>(a, block, sr, dev);
+  if (pow2 && block == 4 * W) return launch_block_warp<DT, 4>(a, block, sr, dev);
+  if (pow2 && block == 8 * W) return launch_block_warp<DT, 8>(a, block, sr, dev);
   const int64_t nb = (a.cols + block - 1) / block;
   const int grid = flat_grid(a.rows * nb, dev, 1);
   if (sr)
@@ -1910,7 +2041,7 @@ cudaError_t launch_dequantize_blockwise(const uint8_t* q, int fmt, int64_t rows,
                                         const float* scales, bool bf16_out, void* out, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
-  const int grid = flat_grid(rows * cols / 16, dev, 1);
+  const int grid = flat_grid(rows * cols / 16, dev, kDequantUnroll);
   if (fmt == 0 && bf16_out) k_block_dequant<0, true><<<grid, kThreads, 0, stream>>>(q, rows, cols, block, scales, out);
   else if (fmt == 0) k_block_dequant<0, false><<<grid, kThreads, 0, stream>>>(q, rows, cols, block, scales, out);
   else if (bf16_out) k_block_dequant<1, true><<<grid, kThreads, 0, stream>>>(q, rows, cols, block, scales, out);

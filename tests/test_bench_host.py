@@ -59,18 +59,19 @@ def test_reference_leg_prints_the_contract_line():
     assert r.returncode == 0 and r.stdout.strip() == ""
 
 
-def test_sweep_reference_leg_reports_gbs():
+@pytest.mark.parametrize("workload,word", [("sweep", "sweep"), ("blockwise", "block-wise")])
+def test_quantize_reference_legs_report_gbs(workload, word):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
-                        "sweep", "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300)
+                        workload, "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     line = json.loads(r.stdout.strip().splitlines()[-1])
-    assert line["unit"] == "GB/s" and line["value"] > 0 and "sweep" in line["config"]["workload"]
+    assert line["unit"] == "GB/s" and line["value"] > 0 and word in line["config"]["workload"]
 
 
 def test_every_workload_is_described_and_sized():
     for name, cfg in bench.WORKLOADS.items():
         d = bench.workload_desc(name, cfg)
         assert isinstance(d, str) and len(d) > 20
-        assert cfg["kind"] in ("layer", "decode", "sweep", "stack", "backward", "moe", "moe_bf16")
+        assert cfg["kind"] in ("layer", "decode", "sweep", "stack", "backward", "blockwise", "moe", "moe_bf16")
     # one quantize call's algorithmic bytes: bf16 read + code write + f32 scales
     assert bench.q_bytes(4, 8, 4) == 4 * 8 * 3 + 16
