@@ -1646,6 +1646,212 @@ __global__ void __launch_bounds__(kThreads) k_block_quant_warp(const void* __res
   }
 }
 
+// Stage pipeline of the block-wise kernels (the per-token one): persistent
+// CTAs; S stages of R whole rows, each filled by one 1-D bulk copy while the
+// other stages are worked on.  work(stage, r0, nr) runs on every thread once
+// rows [r0, r0 + nr) have landed in `stage`; a barrier separates it from the
+// refill of that stage.  A stage that does not land within the time limit
+// sets the error word and ends the kernel after the copies in flight drain.
+template <class Work>
+__device__ __forceinline__ void row_stage_pipeline(const void* __restrict__ x, int64_t rows, int64_t row_bytes, int R,
+                                                   int S, unsigned* err, Work&& work) {
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ __align__(8) uint64_t full[kMaxStages];
+  __shared__ int abort_flag;
+  const int64_t stage_bytes = static_cast<int64_t>(R) * row_bytes;
+  const int64_t ngroups = (rows + R - 1) / R;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) ptx::mbar_init(&full[s], 1);
+    abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  __syncthreads();
+  uint32_t pend_mask = 0, pend_parity = 0;  // thread 0: stages with a copy in flight
+  auto issue = [&](int64_t g, int s, uint32_t parity) {
+    const int64_t r0 = g * R;
+    const int64_t nr = min(static_cast<int64_t>(R), rows - r0);
+    const uint32_t bytes = static_cast<uint32_t>(nr * row_bytes);
+    ptx::mbar_arrive_expect_tx(&full[s], bytes);
+    ptx::bulk_load(stage_mem + s * stage_bytes, static_cast<const char*>(x) + r0 * row_bytes, bytes, &full[s]);
+    pend_mask |= 1u << s;
+    pend_parity = (pend_parity & ~(1u << s)) | (parity << s);
+  };
+  if (threadIdx.x == 0)
+    for (int s = 0; s < S; ++s) {
+      const int64_t g = blockIdx.x + static_cast<int64_t>(s) * gridDim.x;
+      if (g < ngroups) issue(g, s, 0);
+    }
+  int64_t i = 0;
+  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x, ++i) {
+    const int s = static_cast<int>(i % S);
+    const uint32_t parity = static_cast<uint32_t>((i / S) & 1);
+    if (threadIdx.x == 0) {
+      if (ptx::mbar_wait(&full[s], parity, &abort_flag, err, kDevErrTimeout)) pend_mask &= ~(1u << s);
+    }
+    __syncthreads();
+    if (abort_flag) break;
+    const int64_t r0 = g * R;
+    work(stage_mem + s * stage_bytes, r0, static_cast<int>(min(static_cast<int64_t>(R), rows - r0)));
+    __syncthreads();  // stage s fully read
+    if (threadIdx.x == 0) {
+      const int64_t g2 = g + static_cast<int64_t>(S) * gridDim.x;
+      if (g2 < ngroups) {
+        ptx::fence_proxy_async_smem();
+        issue(g2, s, parity ^ 1u);
+      }
+    }
+  }
+  if (abort_flag && threadIdx.x == 0) {
+    int dummy = 0;
+    for (int s = 0; s < S; ++s)
+      if (pend_mask & (1u << s))
+        ptx::mbar_wait(&full[s], (pend_parity >> s) & 1u, &dummy, nullptr, 0, ptx::kDrainLimitNs);
+  }
+}
+
+// Block-wise, staged, blocks of at least one warp-wide vector span (NV = block
+// / (32 kVec) vectors per lane): a warp reduces one block per unit with xor
+// shuffles over all 32 lanes.  A stage's units go to the warps round-robin.
+template <int DT, int FMT, bool SR, int NV>
+__global__ void __launch_bounds__(kThreads, 1) k_block_tma(
+    const void* __restrict__ x, int64_t rows, int cols, int log2_block, int R, int S, uint64_t seed,
+    uint8_t* __restrict__ q, float* __restrict__ scales, float* __restrict__ amax_out, unsigned* err) {
+  constexpr int VEC = Dt<DT>::kVec;
+  constexpr int U = 32 * VEC * NV;
+  constexpr int kWarps = kThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int upr = (cols + U - 1) / U;
+  const int nb = ((cols - 1) >> log2_block) + 1;
+  row_stage_pipeline(x, rows, static_cast<int64_t>(cols) * Dt<DT>::kSize, R, S, err,
+                     [&](const uint8_t* stage, int64_t r0, int nr) {
+    const uint4* st = reinterpret_cast<const uint4*>(stage);
+    const int units = nr * upr;
+    int rl = 0, uu = warp;  // this warp's unit: row rl of the stage, unit uu of the row
+    while (uu >= upr) { uu -= upr; ++rl; }
+    for (int u = warp; u < units; u += kWarps) {  // warp-uniform bounds
+      const int cu = uu * U;
+      uint4 v[NV];
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int c = cu + (k * 32 + lane) * VEC;
+        v[k] = c < cols ? st[(rl * cols + c) / VEC] : make_uint4(0u, 0u, 0u, 0u);
+      }
+      uint32_t mr = 0;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) mr = Dt<DT>::lmax(mr, vec_mag<DT>(v[k]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mr = Dt<DT>::lmax(mr, __shfl_xor_sync(0xFFFFFFFFu, mr, o));
+      const bool special = Dt<DT>::nonfinite(mr);  // uniform: mr is the whole block's
+      float amax;
+      if (!special) {
+        amax = Dt<DT>::value(mr);
+      } else {
+        amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) amax = vec_amax_exact<DT>(v[k], amax);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      }
+      const float m = multiplier(amax, Fmt<FMT>::kMax);
+      const int64_t row = r0 + rl;
+      if (lane == 0) {
+        const int64_t t = row * nb + (cu >> log2_block);
+        scales[t] = __fdiv_rn(1.0f, m);
+        if (amax_out) amax_out[t] = amax;
+      }
+      const int64_t rbase = row * cols;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int c = cu + (k * 32 + lane) * VEC;
+        if (c >= cols) continue;
+        if constexpr (SR) sr_store_vec<DT>(q + rbase + c, v[k], m, seed, static_cast<uint64_t>(rbase + c));
+        else if (!special) vec_store<DT, FMT, true>(q + rbase + c, v[k], m);
+        else vec_store<DT, FMT, false>(q + rbase + c, v[k], m);
+      }
+      uu += kWarps;
+      while (uu >= upr) { uu -= upr; ++rl; }
+    }
+  });
+}
+
+// Block-wise, staged, blocks narrower than a warp-wide vector span (2 .. 16
+// vectors of kVec elements).  A warp task is 32 consecutive blocks of a row:
+// pass 1, lane l alone reduces block l (its vectors visited from a lane-
+// rotated start, so that the strided shared-memory reads do not pile onto the
+// same banks), takes the block's multiplier and dequant scale (one division
+// each for 32 blocks at once) and writes the scales coalesced; pass 2 casts
+// the task's vectors in coalesced order, each fetching its block's multiplier
+// from the owning lane by a shuffle (negated when the block holds a
+// non-finite element, which selects the exact cast).  The codes equal
+// k_block_quant's.
+template <int DT, int FMT, bool SR>
+__global__ void __launch_bounds__(kThreads, 1) k_block_tma_narrow(
+    const void* __restrict__ x, int64_t rows, int cols, int log2_block, int R, int S, uint64_t seed,
+    uint8_t* __restrict__ q, float* __restrict__ scales, float* __restrict__ amax_out, unsigned* err) {
+  constexpr int VEC = Dt<DT>::kVec;
+  constexpr int kLog2Vec = VEC == 8 ? 3 : 2;
+  constexpr int kWarps = kThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int log2_bpv = log2_block - kLog2Vec;  // vectors per block: 1 << log2_bpv
+  const int bpv = 1 << log2_bpv;
+  const int vpr = cols / VEC;                   // vectors per row (cols % 16 == 0)
+  const int nb = ((cols - 1) >> log2_block) + 1;
+  const int ntask = (nb + 31) >> 5;             // tasks per row
+  row_stage_pipeline(x, rows, static_cast<int64_t>(cols) * Dt<DT>::kSize, R, S, err,
+                     [&](const uint8_t* stage, int64_t r0, int nr) {
+    const uint4* st = reinterpret_cast<const uint4*>(stage);
+    const int tasks = nr * ntask;
+    int rl = 0, tk = warp;
+    while (tk >= ntask) { tk -= ntask; ++rl; }
+    for (int t = warp; t < tasks; t += kWarps) {  // warp-uniform bounds
+      const int64_t row = r0 + rl;
+      const uint4* rs = st + rl * vpr;
+      const int v0 = (tk * 32) << log2_bpv;      // the task's first vector in the row
+      // pass 1: block b = tk * 32 + lane, vectors [vb, vb + bpv) of the row
+      const int b = tk * 32 + lane;
+      const int vb = v0 + (lane << log2_bpv);
+      float ms = 1.0f;
+      if (b < nb) {
+        const int nvalid = min(bpv, vpr - vb);
+        uint32_t mr = 0;
+        for (int i = 0; i < bpv; ++i) {
+          const int j = (i + lane) & (bpv - 1);
+          if (j < nvalid) mr = Dt<DT>::lmax(mr, vec_mag<DT>(rs[vb + j]));
+        }
+        const bool special = Dt<DT>::nonfinite(mr);
+        float amax;
+        if (!special) {
+          amax = Dt<DT>::value(mr);
+        } else {
+          amax = 0.0f;
+          for (int j = 0; j < nvalid; ++j) amax = vec_amax_exact<DT>(rs[vb + j], amax);
+        }
+        const float m = multiplier(amax, Fmt<FMT>::kMax);
+        const int64_t ti = row * nb + b;
+        scales[ti] = __fdiv_rn(1.0f, m);
+        if (amax_out) amax_out[ti] = amax;
+        ms = special ? -m : m;
+      }
+      // pass 2: the task's vectors, lane-contiguous
+      const int64_t rbase = row * cols;
+      for (int i = 0; i < bpv; ++i) {
+        const int vl = lane + 32 * i;            // vector within the task
+        const float mv = __shfl_sync(0xFFFFFFFFu, ms, vl >> log2_bpv);
+        const int v = v0 + vl;
+        if (v < vpr) {
+          const uint4 u = rs[v];
+          uint8_t* dst = q + rbase + static_cast<int64_t>(v) * VEC;
+          if constexpr (SR) sr_store_vec<DT>(dst, u, fabsf(mv), seed, static_cast<uint64_t>(rbase + v * VEC));
+          else if (mv > 0.0f) vec_store<DT, FMT, true>(dst, u, mv);
+          else vec_store<DT, FMT, false>(dst, u, -mv);
+        }
+      }
+      tk += kWarps;
+      while (tk >= ntask) { tk -= ntask; ++rl; }
+    }
+  });
+}
+
 // Block-wise dequantize: out = f32(dec(q) * block scale), or that rounded to
 // bf16.  The codes decode exactly through cvt to f16 pairs.
 template <int FMT, bool BF16_OUT>
@@ -1980,6 +2186,50 @@ cudaError_t launch_sr_typed(const QuantizeArgs& a) {
   return cudaGetLastError();
 }
 
+// Staged block-wise launch: two stages of R whole rows, R doubled (up to 8)
+// until a stage holds at least 32 KB and four warp tasks, while the stage
+// pair stays within kBlockStageMax; as many CTAs per SM as shared memory
+// allows (at most 3).  A sweep over the rule on [8192|16384, 8192] and
+// [4096, 28672] bf16 with blocks of 16 .. 128 picked it: asking for a task per
+// warp doubles the stage at blocks of 128, leaving one CTA per SM and 20-35 %
+// less bandwidth.  Returns cudaErrorNotSupported when one row pair does
+// not fit.  NV = 0 selects the narrow-block kernel.
+constexpr int64_t kBlockStageMax = 200 * 1024;
+template <int DT, int NV>
+cudaError_t launch_block_tma(const QuantizeArgs& a, int log2_block, bool sr, int dev) {
+  constexpr int VEC = Dt<DT>::kVec;
+  const int64_t row_bytes = a.cols * Dt<DT>::kSize;
+  const int S = 2;
+  unsigned* err = device_error_word();
+  if (S * row_bytes > kBlockStageMax || err == nullptr) return cudaErrorNotSupported;
+  const int64_t nb = (a.cols + (int64_t{1} << log2_block) - 1) >> log2_block;
+  const int64_t tasks_per_row = NV == 0 ? (nb + 31) / 32 : (a.cols + 32 * VEC * NV - 1) / (32 * VEC * NV);
+  int R = 1;
+  while (R < 8 && (R * row_bytes < 32768 || R * tasks_per_row < 4) &&
+         S * 2 * R * row_bytes <= kBlockStageMax)
+    R *= 2;
+  const int smem = static_cast<int>(S * R * row_bytes);
+  void (*kern)(const void*, int64_t, int, int, int, int, uint64_t, uint8_t*, float*, float*, unsigned*);
+  if constexpr (NV == 0)
+    kern = sr ? k_block_tma_narrow<DT, 1, true>
+              : (a.fmt == 0 ? k_block_tma_narrow<DT, 0, false> : k_block_tma_narrow<DT, 1, false>);
+  else
+    kern = sr ? k_block_tma<DT, 1, true, NV>
+              : (a.fmt == 0 ? k_block_tma<DT, 0, false, NV> : k_block_tma<DT, 1, false, NV>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kBlockStageMax));
+  if (e != cudaSuccess) return e;
+  const int64_t ngroups = (a.rows + R - 1) / R;
+  int per_sm = static_cast<int>(std::min<int64_t>(3, (227 * 1024) / (smem + 1024)));
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = static_cast<int64_t>(device_sm_count(dev)) * per_sm;
+  if (grid > ngroups) grid = ngroups;
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, a.stream>>>(a.x, a.rows, static_cast<int>(a.cols), log2_block,
+                                                                   R, S, sr ? a.seed : 0, a.q, a.scales, a.amax_out,
+                                                                   err);
+  return cudaGetLastError();
+}
+
 template <int DT, int NV>
 cudaError_t launch_block_warp(const QuantizeArgs& a, int64_t block, bool sr, int dev) {
   constexpr int64_t CH = 32 * Dt<DT>::kVec * NV * (NV == 1 ? 4 : (NV == 2 ? 2 : 1));
@@ -2008,6 +2258,16 @@ cudaError_t launch_block_typed(const QuantizeArgs& a, int64_t block, bool sr) {
   // per block (2..32), or one block per unit of 2, 4 or 8 warp-wide vectors.
   constexpr int64_t W = 32 * Dt<DT>::kVec;
   const bool pow2 = (block & (block - 1)) == 0;
+  int log2_block = 0;
+  while ((int64_t{1} << log2_block) < block) ++log2_block;
+  // rows that fit a stage pair go through the bulk-copy pipeline
+  if (pow2 && block <= 4 * W && a.rows > 0) {
+    cudaError_t e = block < W        ? launch_block_tma<DT, 0>(a, log2_block, sr, dev)
+                    : block == W     ? launch_block_tma<DT, 1>(a, log2_block, sr, dev)
+                    : block == 2 * W ? launch_block_tma<DT, 2>(a, log2_block, sr, dev)
+                                     : launch_block_tma<DT, 4>(a, log2_block, sr, dev);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if (pow2 && block <= W) return launch_block_warp<DT, 1>(a, block, sr, dev);
   if (pow2 && block == 2 * W) return launch_block_warp<DT, 2>(a, block, sr, dev);
   if (pow2 && block == 4 * W) return launch_block_warp<DT, 4>(a, block, sr, dev);

@@ -20,10 +20,10 @@ from _gpu import dev, dev_bf16, host, host_bits
 pytestmark = pytest.mark.gpu
 # (rows, cols, block): blocks dividing the row, ragged last blocks, a block
 # wider than the row (the per-token case), a single row of 16; power-of-two
-# blocks of 16 .. 2048 (one to eight warp-wide vectors per block) and blocks
-# of 48 and 80 elements.
+# blocks of 16 .. 2048 (one to eight warp-wide vectors per block), blocks of
+# 48 and 80 elements, and rows too long for a shared-memory stage pair.
 CASES = [(1, 16, 16), (7, 48, 32), (33, 272, 128), (130, 1024, 128), (5, 8208, 64), (9, 96, 256), (64, 4096, 32),
-         (6, 192, 48), (3, 480, 80), (4, 2064, 512), (3, 3008, 1024), (2, 4608, 2048)]
+         (6, 192, 48), (3, 480, 80), (4, 2064, 512), (3, 3008, 1024), (2, 4608, 2048), (3, 40000, 128)]
 
 
 def make(shape, dtype, seed, specials=True):
