@@ -64,6 +64,10 @@ def lib():
         L.hqo_dequantize_blockwise.restype = ci
         L.hqo_gemm_a8w8_bias.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P]
         L.hqo_gemm_a8w8_bias.restype = None
+        L.hqo_gemm_blockscaled.argtypes = [P, P, ci, P, P, i64, P, i64, i64, i64, P, P]
+        L.hqo_gemm_blockscaled.restype = None
+        L.hqo_gemm_blockscaled_entries.argtypes = [P, P, ci, P, P, i64, P, i64, P, P, i64, P]
+        L.hqo_gemm_blockscaled_entries.restype = None
         L.hqo_gemm_a8w8_entries.argtypes = [P, P, ci, P, i64, P, i64, i64, P, P, i64, P]
         L.hqo_gemm_a8w8_entries.restype = None
         L.hqo_grouped_gemm_a8w8.argtypes = [P, P, ci, P, P, P, i32, i64, i64, i64, P]
@@ -255,6 +259,38 @@ def gemm_a8w8_bias(xq, wq, fmt, x_scale, w_scale, bias_bf16_bits):
     assert b.size == N
     out = np.empty((M, N), np.uint16)
     lib().hqo_gemm_a8w8_bias(_p(xq), _p(wq), fmt, _p(xs), xs.size, _p(ws), ws.size, _p(b), M, N, K, _p(out))
+    return out
+
+
+def gemm_blockscaled(xq, wq, fmt, x_scales, w_scales, block, bias_bf16_bits=None, return_ref=False):
+    """bf16 bits of sum_b xs[m,b] ws[n,b] S_b[m,n] (+ bias[n]), one rounding;
+    x_scales [M, ceil(K/block)], w_scales [N, ceil(K/block)]."""
+    xq = np.ascontiguousarray(xq, np.uint8)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    nb = -(-K // block)
+    xs = np.ascontiguousarray(x_scales, np.float32).reshape(M, nb)
+    ws = np.ascontiguousarray(w_scales, np.float32).reshape(N, nb)
+    b = None if bias_bf16_bits is None else np.ascontiguousarray(bias_bf16_bits, np.uint16).reshape(N)
+    out = np.empty((M, N), np.uint16)
+    ref = np.empty((M, N), np.float64) if return_ref else None
+    lib().hqo_gemm_blockscaled(_p(xq), _p(wq), fmt, _p(xs), _p(ws), block, _p(b), M, N, K, _p(out), _p(ref))
+    return (out, ref) if return_ref else out
+
+
+def gemm_blockscaled_entries(xq, wq, fmt, x_scales, w_scales, block, ms, ns, bias_bf16_bits=None):
+    xq = np.ascontiguousarray(xq, np.uint8)
+    wq = np.ascontiguousarray(wq, np.uint8)
+    K = xq.shape[1]
+    xs = np.ascontiguousarray(x_scales, np.float32)
+    ws = np.ascontiguousarray(w_scales, np.float32)
+    b = None if bias_bf16_bits is None else np.ascontiguousarray(bias_bf16_bits, np.uint16)
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    out = np.empty(ms.size, np.uint16)
+    lib().hqo_gemm_blockscaled_entries(_p(xq), _p(wq), fmt, _p(xs), _p(ws), block, _p(b), K, _p(ms), _p(ns),
+                                       ms.size, _p(out))
     return out
 
 

@@ -539,6 +539,57 @@ void hqo_gemm_a8w8_bias(const uint8_t* xq, const uint8_t* wq, int fmt,
     }
 }
 
+/* Block-scaled GEMM ([HQ] "Block-scaled Linear and Adafactor Kernel Helpers":
+   the pre-quantized linear consumes the FP8 bytes and FP32 per-block scales of
+   both operands; [HQ] "Block-wise FP8 Scaling" fixes the layout: one dequant
+   scale per block of `block` consecutive elements along K, xs [M, nb],
+   ws [N, nb], nb = ceil(K / block), the last block the short remainder).
+     out[m,n] = bf16( sum_b xs[m,b] * ws[n,b] * S_b[m,n]  (+ bias[n]) )
+   with S_b the exact dot product of the codes over block b.  Each block's
+   term is sx * sw * S_b in fp64 (sx * sw exact), the terms and the bias are
+   summed in fp64 in block order, and the result is rounded once.  bias
+   (bf16, N entries) is nullable. */
+static double blockscaled_entry(const uint8_t* xq, const uint8_t* wq, int fmt,
+                                const float* xs, const float* ws, int64_t block,
+                                int64_t K, int64_t m, int64_t n) {
+  int64_t nb = (K + block - 1) / block, b;
+  double v = 0.0;
+  for (b = 0; b < nb; ++b) {
+    int64_t k0 = b * block, len = (K - k0 < block) ? K - k0 : block;
+    double s = exact_dot(xq + m * K + k0, wq + n * K + k0, len, fmt);
+    v += (double)xs[m * nb + b] * (double)ws[n * nb + b] * s;
+  }
+  return v;
+}
+
+void hqo_gemm_blockscaled(const uint8_t* xq, const uint8_t* wq, int fmt,
+                          const float* xs, const float* ws, int64_t block,
+                          const uint16_t* bias, int64_t M, int64_t N, int64_t K,
+                          uint16_t* out, double* ref_out) {
+  int64_t m, n;
+  for (m = 0; m < M; ++m)
+    for (n = 0; n < N; ++n) {
+      double v = blockscaled_entry(xq, wq, fmt, xs, ws, block, K, m, n);
+      if (bias) v += (double)hqo_bf16_to_f32(bias[n]);
+      if (ref_out) ref_out[m * N + n] = v;
+      out[m * N + n] = hqo_double_to_bf16(v);
+    }
+}
+
+/* The same at sampled (m, n) positions. */
+void hqo_gemm_blockscaled_entries(const uint8_t* xq, const uint8_t* wq, int fmt,
+                                  const float* xs, const float* ws, int64_t block,
+                                  const uint16_t* bias, int64_t K,
+                                  const int64_t* ms, const int64_t* ns,
+                                  int64_t count, uint16_t* out) {
+  int64_t i;
+  for (i = 0; i < count; ++i) {
+    double v = blockscaled_entry(xq, wq, fmt, xs, ws, block, K, ms[i], ns[i]);
+    if (bias) v += (double)hqo_bf16_to_f32(bias[ns[i]]);
+    out[i] = hqo_double_to_bf16(v);
+  }
+}
+
 /* The same entries at sampled (m, n) positions only. */
 void hqo_gemm_a8w8_entries(const uint8_t* xq, const uint8_t* wq, int fmt,
                            const float* xs, int64_t xs_len, const float* ws,

@@ -750,3 +750,101 @@ def test_blockwise_dequantize_closed_forms():
     qq, ss, _ = O.quantize_blockwise(x, O.E4M3, 16)
     back = O.dequantize_blockwise(qq, O.E4M3, 16, ss)
     assert (np.abs(back - x) <= np.abs(x) * 2.0 ** -4 + np.repeat(ss, 16, axis=1) * 2.0 ** -9).all()
+
+
+# ------------------------------------------------------- block-scaled GEMM
+def _exact_block_dot(xq, wq, fmt, k0, k1):
+    frac = 9 if fmt == O.E4M3 else 16
+    dx = xq.view(ML[fmt]).astype(np.float64)
+    dw = wq.view(ML[fmt]).astype(np.float64)
+    return Fraction(sum(int(a * 2 ** frac) * int(b * 2 ** frac) for a, b in zip(dx[k0:k1], dw[k0:k1])),
+                    2 ** (2 * frac))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("block", [16, 32, 48])
+def test_blockscaled_gemm_vs_fractions(fmt, block):
+    # sum over blocks of xs[m,b] ws[n,b] S_b in exact rationals, the last block
+    # the short remainder of K (K = 80), one round to nearest-even bf16
+    rng = np.random.default_rng(70 + block + fmt)
+    M, N, K = 5, 7, 80
+    nb = -(-K // block)
+    xq = _rand_codes(rng, (M, K), fmt)
+    wq = _rand_codes(rng, (N, K), fmt)
+    xs = rng.uniform(1e-3, 4, (M, nb)).astype(np.float32)
+    ws = rng.uniform(1e-3, 4, (N, nb)).astype(np.float32)
+    bias = W.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    out = O.gemm_blockscaled(xq, wq, fmt, xs, ws, block)
+    outb = O.gemm_blockscaled(xq, wq, fmt, xs, ws, block, bias)
+    bv = W.bf16_bits_to_f32(bias)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(xs[m, b])) * Fraction(float(ws[n, b])) *
+                        _exact_block_dot(xq[m], wq[n], fmt, b * block, min(K, (b + 1) * block)) for b in range(nb))
+            assert out[m, n] == _nearest_bf16(exact)
+            assert outb[m, n] == _nearest_bf16(exact + Fraction(float(bv[n])))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_blockscaled_gemm_one_block_is_the_scaled_gemm(fmt):
+    # a block spanning K leaves one scale per row and per column: the per-row /
+    # per-column scaled GEMM (and its bias form), bit for bit
+    rng = np.random.default_rng(75)
+    M, N, K = 6, 9, 64
+    xq = _rand_codes(rng, (M, K), fmt)
+    wq = _rand_codes(rng, (N, K), fmt)
+    xs = rng.uniform(0.01, 3, (M, 1)).astype(np.float32)
+    ws = rng.uniform(0.01, 3, (N, 1)).astype(np.float32)
+    bias = W.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    for block in (64, 128, 4096):
+        assert np.array_equal(O.gemm_blockscaled(xq, wq, fmt, xs, ws, block), O.gemm_a8w8(xq, wq, fmt, xs, ws))
+        assert np.array_equal(O.gemm_blockscaled(xq, wq, fmt, xs, ws, block, bias),
+                              O.gemm_a8w8_bias(xq, wq, fmt, xs, ws, bias))
+
+
+def test_blockscaled_gemm_uniform_power_of_two_scales():
+    # with the same power-of-two scale in every block of a row (and of a
+    # column) every step is exact, so the blocks sum to the unblocked GEMM
+    rng = np.random.default_rng(76)
+    M, N, K, block = 8, 12, 96, 32
+    xq = _rand_codes(rng, (M, K), O.E4M3)
+    wq = _rand_codes(rng, (N, K), O.E4M3)
+    xs1 = (2.0 ** rng.integers(-6, 6, M)).astype(np.float32)
+    ws1 = (2.0 ** rng.integers(-6, 6, N)).astype(np.float32)
+    xs = np.repeat(xs1[:, None], K // block, axis=1)
+    ws = np.repeat(ws1[:, None], K // block, axis=1)
+    assert np.array_equal(O.gemm_blockscaled(xq, wq, O.E4M3, xs, ws, block), O.gemm_a8w8(xq, wq, O.E4M3, xs1, ws1))
+
+
+def test_blockscaled_gemm_blocks_are_separate_terms():
+    # codes zero outside block 1 leave only that block's term; doubling the
+    # x scale of a block whose codes are all zero changes nothing
+    rng = np.random.default_rng(77)
+    M, N, K, block = 4, 5, 96, 32
+    xq = _rand_codes(rng, (M, K), O.E4M3)
+    wq = _rand_codes(rng, (N, K), O.E4M3)
+    xq[:, :block] = 0
+    xq[:, 2 * block:] = 0
+    xs = rng.uniform(0.1, 2, (M, 3)).astype(np.float32)
+    ws = rng.uniform(0.1, 2, (N, 3)).astype(np.float32)
+    got = O.gemm_blockscaled(xq, wq, O.E4M3, xs, ws, block)
+    one = O.gemm_a8w8(np.ascontiguousarray(xq[:, block:2 * block]), np.ascontiguousarray(wq[:, block:2 * block]),
+                      O.E4M3, xs[:, 1], ws[:, 1])
+    assert np.array_equal(got, one)
+    xs2 = xs.copy()
+    xs2[:, 0] *= 2
+    assert np.array_equal(O.gemm_blockscaled(xq, wq, O.E4M3, xs2, ws, block), got)
+
+
+def test_blockscaled_gemm_entries_equal_the_full_product():
+    rng = np.random.default_rng(78)
+    M, N, K, block = 9, 11, 144, 64
+    xq = _rand_codes(rng, (M, K), O.E5M2)
+    wq = _rand_codes(rng, (N, K), O.E5M2)
+    xs = rng.uniform(0.1, 2, (M, 3)).astype(np.float32)
+    ws = rng.uniform(0.1, 2, (N, 3)).astype(np.float32)
+    bias = W.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    full = O.gemm_blockscaled(xq, wq, O.E5M2, xs, ws, block, bias)
+    ms = rng.integers(0, M, 30)
+    ns = rng.integers(0, N, 30)
+    assert np.array_equal(O.gemm_blockscaled_entries(xq, wq, O.E5M2, xs, ws, block, ms, ns, bias), full[ms, ns])
