@@ -537,7 +537,7 @@ def build(args, cfg, rank, dev, stream, peaks):
             a = bytes_of[label] / (ms[label] / 1e3) / 1e9
             return {"bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(a / peaks["hbm_gbs"], 4), "traffic": None,
-                    "kernel": "k_block_quant_warp (E4M3, blocks of 128)", "peak_source": "%s copy" % peaks["_src"]}
+                    "kernel": "k_block_tma_narrow (E4M3, blocks of 128)", "peak_source": "%s copy" % peaks["_src"]}
 
         def extras(ms):
             d = {}

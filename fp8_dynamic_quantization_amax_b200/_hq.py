@@ -22,7 +22,7 @@ F32, BF16, F16 = 0, 1, 2
 
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
             "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic",
-            "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
+            "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_blockscaled", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
             "hq_grouped_gemm_bf16",
             "hq_quantize_fp8_noalloc", "hq_check_device_error", "hq_last_error", "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
@@ -53,6 +53,8 @@ def _load():
     L.hq_quantize_fp8.restype = ci
     L.hq_quantize_fp8_noalloc.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P]
     L.hq_quantize_fp8_noalloc.restype = ci
+    L.hq_gemm_blockscaled.argtypes = [P, P, ci, P, P, i64, P, i64, i64, i64, P, P]
+    L.hq_gemm_blockscaled.restype = ci
     L.hq_quantize_fp8_blockwise.argtypes = [P, ci, i64, i64, ci, i64, ci, ctypes.c_uint64, P, P, P, P]
     L.hq_quantize_fp8_blockwise.restype = ci
     L.hq_dequantize_fp8_blockwise.argtypes = [P, ci, i64, i64, i64, P, ci, P, P]
@@ -176,6 +178,19 @@ def hq_quantize_fp8_blockwise(x, fmt=E4M3, block=32, stochastic=False, seed=0, a
                                         seed & ((1 << 64) - 1), _ptr(q), _ptr(scales), _ptr(amax_out),
                                         _stream(stream)))
     return q, scales
+
+
+def hq_gemm_blockscaled(xq, wq, x_scales, w_scales, fmt=E4M3, block=32, bias=None, out=None, stream=None):
+    """bf16 [M, N] = sum over K blocks of x_scales[m,b] w_scales[n,b] (XQ . WQ^T
+    over block b) (+ bias)."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    check(lib.hq_gemm_blockscaled(_ptr(xq.contiguous()), _ptr(wq.contiguous()), fmt, _ptr(x_scales.contiguous()),
+                                  _ptr(w_scales.contiguous()), block, _ptr(bias), M, N, K, _ptr(out),
+                                  _stream(stream)))
+    return out
 
 
 def hq_dequantize_fp8_blockwise(q, scales, fmt=E4M3, block=32, out_dtype=torch.float32, stream=None):

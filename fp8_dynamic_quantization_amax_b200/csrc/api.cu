@@ -565,6 +565,45 @@ hq_status hq_gemm_a8w8_ex(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fm
                      &ex);
 }
 
+hq_status hq_gemm_blockscaled(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scales,
+                              const float* w_scales, int64_t block, const void* bias, int64_t M, int64_t N, int64_t K,
+                              void* out, hq_stream_t stream) {
+  if (fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", (int)fmt);
+  if (M < 0 || N < 0 || K < 0) return fail(HQ_ERR_INVALID_ARG, "negative size");
+  if (M >= k2p31 || N >= k2p31 || K >= k2p31) return fail(HQ_ERR_TOO_LARGE, "M, N and K must be below 2^31");
+  if (block < 32 || block % 32 != 0 || block >= k2p31)
+    return fail(HQ_ERR_INVALID_ARG, "block = %lld must be a positive multiple of 32", (long long)block);
+  if (K % 16 != 0) return fail(HQ_ERR_INVALID_ARG, "K = %lld must be a multiple of 16", (long long)K);
+  if (N % 8 != 0) return fail(HQ_ERR_INVALID_ARG, "N = %lld must be a multiple of 8 (16-byte output rows)", (long long)N);
+  const int64_t nb = (K + block - 1) / block;
+  if (!out || (K > 0 && ((!xq && M > 0) || (!wq && N > 0) || (!x_scales && M > 0) || (!w_scales && N > 0))))
+    return fail(HQ_ERR_INVALID_ARG, "operands, scales and out must not be null");
+  if (!is_aligned(out, 16) || !is_aligned(xq, 16) || !is_aligned(wq, 16) || !is_aligned(bias, 16))
+    return fail(HQ_ERR_MISALIGNED, "A, B, bias and out must be 16-byte aligned");
+  if (!is_aligned(x_scales, 4) || !is_aligned(w_scales, 4)) return fail(HQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  const Range outs[] = {{out, static_cast<size_t>(M) * static_cast<size_t>(N) * 2, "out"}};
+  const Range ins[] = {{xq, static_cast<size_t>(M * K), "A"},
+                       {wq, static_cast<size_t>(N * K), "B"},
+                       {x_scales, static_cast<size_t>(M * nb) * 4, "x_scales"},
+                       {w_scales, static_cast<size_t>(N * nb) * 4, "w_scales"},
+                       {bias, bias ? static_cast<size_t>(N) * 2 : 0, "bias"}};
+  hq_status s = check_overlaps(outs, 1, ins, 5);
+  if (s != HQ_OK) return s;
+  const Range devs[] = {{xq, 0, "A"}, {wq, 0, "B"}, {x_scales, 0, "x_scales"}, {w_scales, 0, "w_scales"},
+                        {bias, 0, "bias"}, {out, 0, "out"}};
+  s = check_device_ptrs(devs, 6);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  if (M == 0 || N == 0) return ok();
+  hq::BlockScaledGemmArgs g;
+  g.fmt = fmt; g.a = xq; g.b = wq; g.x_scales = x_scales; g.w_scales = w_scales; g.block = block; g.bias = bias;
+  g.M = M; g.N = N; g.K = K; g.out = out;
+  g.stream = reinterpret_cast<cudaStream_t>(stream);
+  std::string msg;
+  return launched(hq::launch_gemm_blockscaled(g, &msg), "block-scaled gemm launch", msg);
+}
+
 hq_status hq_grouped_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,
                                int64_t x_scale_len, const float* w_scale, int64_t w_scale_len,
                                const int32_t* offsets, int32_t E, int64_t M_total, int64_t N, int64_t K, void* out,

@@ -1,0 +1,482 @@
+// gemm_bs.cu -- block-scaled FP8 GEMM on sm_100a tensor cores.
+//
+// out[m, n] = bf16_rn( sum_b xs[m, b] * ws[n, b] * S_b[m, n]  (+ bias[n]) ),
+// S_b[m, n] = sum over the K block b of A[m, k] * B[n, k]
+// (hip-quant README "Block-scaled Linear and Adafactor Kernel Helpers": the
+// pre-quantized block-scaled linear consumes the FP8 bytes and FP32 per-block
+// scales of both operands; "Block-wise FP8 Scaling": one dequant scale per
+// block of block_size consecutive elements along the last dimension, scales
+// [..., ceil(K / block_size)], the last block the short remainder).
+//
+// The block scales are arbitrary f32 values.  The tensor cores' block-scaled
+// MMA applies power-of-two scale factors only, so the per-block sums are
+// promoted in software, out of tensor memory:
+//   warp 0      TMA producer: 128-byte K slices of A and B (128 rows each)
+//               into a ring of shared-memory stages (128B swizzle).
+//   warp 1      allocates TMEM: four 128-column FP32 accumulators in two
+//               slots of two.  One thread issues tcgen05.mma kind::f8f6f4, 32
+//               K per instruction; all products of one scale block go to one
+//               accumulator (the first overwrites it); a slot's two blocks
+//               are committed together, so the epilogue hands back a slot
+//               per two blocks while the other slot fills.  Blocks need not
+//               align with the 128-wide stages.
+//   warps 2..9  epilogue, two warps per TMEM lane quadrant, 64 columns each:
+//               per slot, tcgen05.ld of each block's partial sums, then
+//               acc += partial * (xs[m,b] * ws[n,b]) in registers with packed
+//               f32x2 multiplies and fmas, and the slot is handed back;
+//               after the last block, + bias, round to bf16, 16-byte stores.
+// Persistent CTAs, one per SM, tiles in groups of 8 M tiles.  Every wait is
+// bounded: on a stalled barrier the CTA sets the device error word, drains
+// what it has in flight, frees TMEM and exits.
+#include "hq_internal.cuh"
+#include "ptx.cuh"
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+namespace hq {
+namespace {
+
+constexpr int kBsTile = 128;                         // tile rows and columns (MMA M = N = 128)
+constexpr int kBsStages = 6;
+constexpr int kBsAcc = 4;                            // TMEM accumulators (4 x 128 columns)
+constexpr int kBsGroupBlocks = 2;                    // scale blocks per handshake
+constexpr int kBsSlots = kBsAcc / kBsGroupBlocks;    // groups in flight
+constexpr int kBsThreads = 320;                      // TMA, MMA, 8 epilogue warps
+constexpr int kBsOperandBytes = kBsTile * 128;       // one 128 x 128-byte K slice
+constexpr int kBsSmem = kBsStages * 2 * kBsOperandBytes + 8 * 64 * kBsGroupBlocks * 4 + 1024;
+constexpr int kBsGroupM = 8;
+
+struct BsParams {
+  int M, N, K;
+  int nkb;               // 128-wide K stages
+  int nks;               // 32-wide MMA K steps
+  int spb;               // K steps per scale block
+  int nb;                // scale blocks: ceil(K / block)
+  int m_tiles, n_tiles;
+  const float* xs;       // [M, nb]
+  const float* ws;       // [N, nb]
+  const uint16_t* bias;  // bf16 [N] or null
+  uint16_t* out;         // bf16 [M, N]
+  uint32_t idesc;
+  unsigned* err;
+};
+
+using ptx::smem_u32;
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err,
+                                         unsigned long long limit = ptx::kWaitLimitNs) {
+  return ptx::mbar_wait(bar, parity, abort_flag, err, kDevErrTimeout, limit);
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// K-major operand, 128-byte swizzle, 128-byte rows, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// 32 lanes x 32 columns of 32-bit, waited in the same asm block.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// (a0, a1) += (p0, p1) * ((w0, w1) * (x, x)): one packed multiply and one
+// packed fma, each IEEE round-to-nearest per lane.
+__device__ __forceinline__ void promote2(float& a0, float& a1, uint32_t p0, uint32_t p1, float w0, float w1,
+                                         float x) {
+  asm("{\n\t.reg .b64 acc, prt, wsc, xsc;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 prt, {%2, %3};\n\t"
+      "mov.b64 wsc, {%4, %5};\n\t"
+      "mov.b64 xsc, {%6, %6};\n\t"
+      "mul.rn.f32x2 wsc, wsc, xsc;\n\t"
+      "fma.rn.f32x2 acc, prt, wsc, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(p0), "r"(p1), "f"(w0), "f"(w1), "f"(x));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void tile_coords(int t, const BsParams& p, int& m0, int& n0) {
+  const int per_group = kBsGroupM * p.n_tiles;
+  const int g = t / per_group;
+  const int first_m = g * kBsGroupM;
+  const int gsize = min(kBsGroupM, p.m_tiles - first_m);
+  const int r = t - g * per_group;
+  m0 = (first_m + r % gsize) * kBsTile;
+  n0 = (r / gsize) * kBsTile;
+}
+
+__global__ void __launch_bounds__(kBsThreads, 1)
+    k_gemm_bs(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, const BsParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kBsStages];
+  __shared__ __align__(8) uint64_t empty_bar[kBsStages];
+  __shared__ __align__(8) uint64_t afull_bar[kBsSlots];
+  __shared__ __align__(8) uint64_t aempty_bar[kBsSlots];
+  __shared__ __align__(8) uint64_t final_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-byte aligned stages
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kBsStages * kBsOperandBytes;
+  float* sWs = reinterpret_cast<float*>(smem + 2 * kBsStages * kBsOperandBytes);  // per epilogue warp
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kBsStages; ++s) {
+      ptx::mbar_init(&full_bar[s], 1);
+      ptx::mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < kBsSlots; ++a) {
+      ptx::mbar_init(&afull_bar[a], 1);
+      ptx::mbar_init(&aempty_bar[a], 8);  // one arrive per epilogue warp
+    }
+    ptx::mbar_init(&final_bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0 && p.nkb > 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_b) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(kBsAcc * kBsTile)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  const int total = p.m_tiles * p.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed_parity[kBsStages];
+      bool armed[kBsStages];
+#pragma unroll
+      for (int s = 0; s < kBsStages; ++s) { armed[s] = false; armed_parity[s] = 0; }
+      bool stop = false;
+      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+        int m0, n0;
+        tile_coords(t, p, m0, n0);
+        for (int kb = 0; kb < p.nkb; ++kb) {
+          if (!wait_bar(&empty_bar[stage], phase ^ 1u, &abort_flag, p.err)) { stop = true; break; }
+          ptx::mbar_arrive_expect_tx(&full_bar[stage], 2 * kBsOperandBytes);
+          tma_load_2d(sA + stage * kBsOperandBytes, &tm_a, &full_bar[stage], kb * 128, m0);
+          tma_load_2d(sB + stage * kBsOperandBytes, &tm_b, &full_bar[stage], kb * 128, n0);
+#pragma unroll
+          for (int s = 0; s < kBsStages; ++s)
+            if (s == stage) { armed[s] = true; armed_parity[s] = phase; }
+          if (++stage == kBsStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (abort_flag) {  // every armed stage's last transfer lands before exit
+#pragma unroll
+        for (int s = 0; s < kBsStages; ++s) {
+          int dummy = 0;
+          if (armed[s]) wait_bar(&full_bar[s], armed_parity[s], &dummy, nullptr, ptx::kDrainLimitNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    // One thread issues and commits; scale blocks go in groups of
+    // kBsGroupBlocks, each block into its own accumulator of the group's slot.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t jg = 0;  // groups issued so far (the slot ring position)
+      bool issued = false, stop = false;
+      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+        int ks = 0;
+        for (int b0 = 0; b0 < p.nb && !stop; b0 += kBsGroupBlocks, ++jg) {
+          const uint32_t sl = jg % kBsSlots;
+          const uint32_t sph = (jg / kBsSlots) & 1u;
+          if (!wait_bar(&aempty_bar[sl], sph ^ 1u, &abort_flag, p.err)) { stop = true; break; }
+          tc_fence_after();
+          for (int i = 0; i < kBsGroupBlocks && b0 + i < p.nb && !stop; ++i) {
+            const uint32_t d_tmem = tmem_base + (sl * kBsGroupBlocks + i) * kBsTile;
+            const int kfirst = ks;
+            const int kend = min(p.nks, (b0 + i + 1) * p.spb);
+            for (; ks < kend; ++ks) {
+              const int sub = ks & 3;
+              if (sub == 0) {
+                if (!wait_bar(&full_bar[stage], phase, &abort_flag, p.err)) { stop = true; break; }
+                tc_fence_after();
+              }
+              const uint64_t ad = smem_desc(smem_u32(sA + stage * kBsOperandBytes));
+              const uint64_t bd = smem_desc(smem_u32(sB + stage * kBsOperandBytes));
+              mma_f8(d_tmem, ad + 2u * sub, bd + 2u * sub, p.idesc, ks > kfirst ? 1u : 0u);
+              issued = true;
+              if (sub == 3 || ks == p.nks - 1) {  // the stage's last K step: hand the stage back
+                tc_commit(&empty_bar[stage]);
+                if (++stage == kBsStages) { stage = 0; phase ^= 1u; }
+              }
+            }
+          }
+          if (stop) break;
+          tc_commit(&afull_bar[sl]);
+        }
+      }
+      if (abort_flag && issued) {
+        int dummy = 0;
+        tc_commit(&final_bar);
+        wait_bar(&final_bar, 0, &dummy, nullptr, ptx::kDrainLimitNs);
+      }
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------- epilogue
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    const int half = ew >> 2;
+    float* wsh = sWs + ew * 64 * kBsGroupBlocks;  // [block of the group][64 columns]
+    uint32_t jg = 0;
+    bool stop = false;
+    for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+      int m0, n0;
+      tile_coords(t, p, m0, n0);
+      const int row = m0 + quad * 32 + lane;
+      const bool vrow = row < p.M;
+      const int c0 = n0 + half * 64;  // this warp's first column
+      const float* xrow = p.xs + static_cast<int64_t>(vrow ? row : 0) * p.nb;
+      const bool v0 = c0 + lane < p.N, v1 = c0 + 32 + lane < p.N;
+      const float* wcol0 = p.ws + static_cast<int64_t>(v0 ? c0 + lane : 0) * p.nb;
+      const float* wcol1 = p.ws + static_cast<int64_t>(v1 ? c0 + 32 + lane : 0) * p.nb;
+      float acc[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+      // scales of the next group, loaded one group ahead
+      float xn[kBsGroupBlocks], wn0[kBsGroupBlocks], wn1[kBsGroupBlocks];
+#pragma unroll
+      for (int i = 0; i < kBsGroupBlocks; ++i) {
+        const bool in = i < p.nb;
+        xn[i] = in ? __ldg(xrow + i) : 0.0f;
+        wn0[i] = (in && v0) ? __ldg(wcol0 + i) : 0.0f;
+        wn1[i] = (in && v1) ? __ldg(wcol1 + i) : 0.0f;
+      }
+      for (int b0 = 0; b0 < p.nb; b0 += kBsGroupBlocks, ++jg) {
+        float xb[kBsGroupBlocks];
+#pragma unroll
+        for (int i = 0; i < kBsGroupBlocks; ++i) {
+          xb[i] = xn[i];
+          wsh[i * 64 + lane] = wn0[i];
+          wsh[i * 64 + 32 + lane] = wn1[i];
+          const int bn = b0 + kBsGroupBlocks + i;
+          if (bn < p.nb) {
+            xn[i] = __ldg(xrow + bn);
+            wn0[i] = v0 ? __ldg(wcol0 + bn) : 0.0f;
+            wn1[i] = v1 ? __ldg(wcol1 + bn) : 0.0f;
+          }
+        }
+        __syncwarp();
+        const uint32_t sl = jg % kBsSlots;
+        const uint32_t sph = (jg / kBsSlots) & 1u;
+        if (!wait_bar(&afull_bar[sl], sph, &abort_flag, p.err)) { stop = true; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int i = 0; i < kBsGroupBlocks; ++i) {
+          if (b0 + i >= p.nb) break;
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t v[32];
+            tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (sl * kBsGroupBlocks + i) * kBsTile +
+                          static_cast<uint32_t>(half * 64 + ch * 32),
+                      v);
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 w = *reinterpret_cast<const float4*>(wsh + i * 64 + ch * 32 + e);
+              promote2(acc[ch * 32 + e], acc[ch * 32 + e + 1], v[e], v[e + 1], w.x, w.y, xb[i]);
+              promote2(acc[ch * 32 + e + 2], acc[ch * 32 + e + 3], v[e + 2], v[e + 3], w.z, w.w, xb[i]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&aempty_bar[sl]);
+      }
+      if (stop) break;
+      if (vrow) {
+        uint16_t* orow = p.out + static_cast<int64_t>(row) * p.N;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int n = c0 + g * 8;
+          if (n >= p.N) break;  // N % 8 == 0: a group of 8 is inside or outside
+          float o[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) o[k] = acc[g * 8 + k];
+          if (p.bias) {
+            const uint4 bb = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              o[2 * k] = __fadd_rn(o[2 * k], __uint_as_float(bw[k] << 16));
+              o[2 * k + 1] = __fadd_rn(o[2 * k + 1], __uint_as_float(bw[k] & 0xFFFF0000u));
+            }
+          }
+          const uint4 st = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                                      pack_bf16x2(o[6], o[7]));
+          *reinterpret_cast<uint4*>(orow + n) = st;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kBsAcc * kBsTile)
+                 : "memory");
+  }
+}
+
+// --------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// FP8 [rows, cols] row-major, {128-byte, 128-row} boxes, 128B swizzle; out of
+// range elements read as zero codes.
+bool make_fp8_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, std::string* msg) {
+  auto encode = encode_fn();
+  if (!encode) {
+    *msg = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, kBsTile};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[128];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (%d) for [%llu, %llu]", static_cast<int>(r),
+             static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols));
+    *msg = buf;
+    return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_blockscaled(const BlockScaledGemmArgs& a, std::string* msg) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(k_gemm_bs, cudaFuncAttributeMaxDynamicSharedMemorySize, kBsSmem);
+  });
+  if (attr_err != cudaSuccess) {
+    *msg = "cudaFuncSetAttribute failed";
+    return attr_err;
+  }
+  unsigned* err = device_error_word();
+  if (err == nullptr) {
+    *msg = "the device error word is not available";
+    return cudaErrorUnknown;
+  }
+  CUtensorMap ta, tb;
+  memset(&ta, 0, sizeof(ta));
+  memset(&tb, 0, sizeof(tb));
+  if (a.K > 0) {  // K == 0: no loads are issued and the maps are never read
+    if (!make_fp8_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), msg) ||
+        !make_fp8_map(&tb, a.b, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), msg))
+      return cudaErrorInvalidValue;
+  }
+  BsParams p;
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.nkb = static_cast<int>((a.K + 127) / 128);
+  p.nks = static_cast<int>((a.K + 31) / 32);
+  p.spb = static_cast<int>(a.block / 32);
+  p.nb = static_cast<int>((a.K + a.block - 1) / a.block);
+  p.m_tiles = static_cast<int>((a.M + kBsTile - 1) / kBsTile);
+  p.n_tiles = static_cast<int>((a.N + kBsTile - 1) / kBsTile);
+  p.xs = a.x_scales;
+  p.ws = a.w_scales;
+  p.bias = static_cast<const uint16_t*>(a.bias);
+  p.out = static_cast<uint16_t*>(a.out);
+  p.idesc = (1u << 4)                                         // D: FP32
+            | (static_cast<uint32_t>(a.fmt) << 7) | (static_cast<uint32_t>(a.fmt) << 10)  // E4M3 / E5M2
+            | (static_cast<uint32_t>(kBsTile >> 3) << 17)       // N / 8
+            | (static_cast<uint32_t>(kBsTile >> 4) << 24);      // M / 16
+  p.err = err;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  const int sms = device_sm_count(dev);
+  const int grid = static_cast<int>(tiles < sms ? (tiles < 1 ? 1 : tiles) : sms);
+  k_gemm_bs<<<grid, kBsThreads, kBsSmem, a.stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace hq

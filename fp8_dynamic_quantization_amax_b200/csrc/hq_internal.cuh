@@ -1,5 +1,6 @@
 // hq_internal.cuh -- declarations shared by the translation units of
-// libhq.so (api.cu, quantize.cu, gemm.cu).  Not part of the public ABI.
+// libhq.so (api.cu, quantize.cu, gemm.cu, gemm_bs.cu, noalloc.cu).  Not part
+// of the public ABI.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -74,6 +75,23 @@ struct GemmArgs {
 
 // Returns cudaSuccess or the failing call's error; *msg gets a description.
 cudaError_t launch_gemm(const GemmArgs& a, std::string* msg);
+
+// Block-scaled FP8 GEMM: out = bf16(sum_b xs[m,b] ws[n,b] S_b (+ bias[n])),
+// scales [M | N, ceil(K / block)], block % 32 == 0, K % 16 == 0, N % 8 == 0,
+// A, B, out and bias 16-byte aligned.
+struct BlockScaledGemmArgs {
+  int fmt;
+  const void* a;            // FP8 [M, K]
+  const void* b;            // FP8 [N, K]
+  const float* x_scales;    // [M, nb]
+  const float* w_scales;    // [N, nb]
+  int64_t block;
+  const void* bias;         // bf16 [N] or null
+  int64_t M, N, K;
+  void* out;                // bf16 [M, N]
+  cudaStream_t stream;
+};
+cudaError_t launch_gemm_blockscaled(const BlockScaledGemmArgs& a, std::string* msg);
 
 // Device error word (set by bounded waits and by offset validation).
 enum : unsigned { kDevErrTimeout = 1u, kDevErrBadOffsets = 2u };

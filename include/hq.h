@@ -145,6 +145,33 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
                           void* workspace, size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * Block-scaled FP8 GEMM (hip-quant README "Block-scaled Linear and Adafactor
+ * Kernel Helpers": the pre-quantized block-scaled linear consumes FP8 bytes
+ * and FP32 per-block scales of both operands; "Block-wise FP8 Scaling": one
+ * dequant scale per block of `block` elements along K, the last block the
+ * short remainder):
+ *   out[m,n] = bf16_rn( sum_b x_scales[m,b] * w_scales[n,b] * S_b[m,n] + bias[n] )
+ * with S_b = sum over k in block b of dec(xq[m,k]) * dec(wq[n,k]), accumulated
+ * in FP32 on the tensor cores, the block terms summed in FP32.
+ *
+ * Arguments: xq device [M, K] and wq device [N, K] FP8 codes of format fmt
+ *   (K-major: the NT layout), 16-byte aligned; x_scales device f32
+ *   [M, ceil(K / block)], w_scales device f32 [N, ceil(K / block)] (as
+ *   hq_quantize_fp8_blockwise writes them); block a positive multiple of 32;
+ *   K % 16 == 0; bias device bf16 [N] or NULL, 16-byte aligned; out
+ *   caller-owned device bf16 [M, N], N % 8 == 0, 16-byte aligned, overwritten
+ *   (K == 0 writes bf16(bias) or zeros).  M == 0 or N == 0 returns HQ_OK with
+ *   no launch.
+ * Errors: HQ_ERR_INVALID_ARG, HQ_ERR_MISALIGNED, HQ_ERR_OVERLAP,
+ *   HQ_ERR_WRONG_DEVICE, HQ_ERR_UNSUPPORTED_ARCH, HQ_ERR_TOO_LARGE,
+ *   HQ_ERR_CUDA; a stalled kernel reports HQ_ERR_TIMEOUT through
+ *   hq_check_device_error.
+ */
+hq_status hq_gemm_blockscaled(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scales,
+                              const float* w_scales, int64_t block, const void* bias, int64_t M, int64_t N, int64_t K,
+                              void* out, hq_stream_t stream);
+
+/*
  * Block-wise FP8 (hip-quant README "Block-wise FP8 Scaling"): the codes of x
  * [rows, cols] plus one f32 dequant scale per block of `block` consecutive
  * elements along the last dimension, scales [rows, ceil(cols / block)] (the

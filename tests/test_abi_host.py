@@ -248,3 +248,21 @@ def test_blockwise_rejections():
     assert dcall(out=BASE + 0x2000004) == MISALIGNED and dcall(q=BASE + 8) == MISALIGNED
     assert dcall(out=BASE + 0x40) == OVERLAP and dcall(out=BASE + 0x1000000 - 0x100) == OVERLAP
     assert dcall(cols=0, q=None, s=None, out=None) == OK
+
+
+def test_blockscaled_gemm_rejections():
+    g = L.hq_gemm_blockscaled
+
+    def call(xq=BASE, wq=BASE + 0x1000000, fmt=H.E4M3, xs=BASE + 0x2000000, ws=BASE + 0x3000000, block=32,
+             bias=None, M=64, N=128, K=256, out=BASE + 0x4000000):
+        return g(xq, wq, fmt, xs, ws, block, bias, M, N, K, out, None)
+
+    assert call(block=16) == INVALID and call(block=48) == INVALID and call(block=0) == INVALID
+    assert call(K=40) == INVALID and call(N=12) == INVALID and call(fmt=2) == INVALID and call(M=-1) == INVALID
+    assert call(out=None) == INVALID and call(xs=None) == INVALID and call(wq=None) == INVALID
+    assert call(out=BASE + 0x4000008) == MISALIGNED and call(xq=BASE + 4) == MISALIGNED
+    assert call(bias=BASE + 0x5000004) == MISALIGNED and call(ws=BASE + 0x3000002) == MISALIGNED
+    assert call(out=BASE + 0x100) == OVERLAP                 # out over A
+    assert call(out=BASE + 0x2000000 - 0x100) == OVERLAP     # out running into x_scales
+    assert call(bias=BASE + 0x4000000 + 0x40) == OVERLAP     # bias inside out
+    assert call(M=1 << 31) == TOO_LARGE
