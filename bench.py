@@ -58,6 +58,9 @@ def dist_env():
 # sweep: quantize only, bf16 [8192, 8192]; every granularity x format.
 # blockwise: block-wise quantize of the sweep input along its rows (E4M3 at
 #   blocks of 128 and 32, stochastic E5M2 at 128) and the bf16 dequantize.
+# blockscaled, blockscaled32: the large layer with block-wise scales along K
+#   (E4M3, blocks of 128 / 32): X and W quantized block-wise every step, then
+#   the block-scaled GEMM.
 # moe / moe_bf16: per-token quantize of the routed tokens + grouped a8w8 GEMM
 #   over 64 experts (W quantized once); the bf16 grouped GEMM alone.
 WORKLOADS = {
@@ -71,6 +74,8 @@ WORKLOADS = {
     "stack": dict(kind="stack", M=2048, N=4096, K=1024, steps_cycle=200, ring=16),
     "backward": dict(kind="backward", M=16384, N=28672, K=8192, ring=16),
     "blockwise": dict(kind="blockwise", M=8192, N=0, K=8192),
+    "blockscaled": dict(kind="blockscaled", M=16384, N=28672, K=8192, block=128),
+    "blockscaled32": dict(kind="blockscaled", M=16384, N=28672, K=8192, block=32),
     "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
     "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }
@@ -95,6 +100,11 @@ def workload_desc(name, cfg):
     if k == "sweep":
         return ("quantize sweep: bf16 [%d,%d] ~N(0,1), 0.1%% x100 outliers, 0.1%% zeros, one zero row; "
                 "per-tensor / per-token / per-channel x E4M3 / E5M2" % (cfg["M"], cfg["K"]))
+    if k == "blockscaled":
+        return ("block-scaled a8w8 layer: X bf16 [%d,%d] ~N(0,1), W bf16 [%d,%d] ~N(0,0.02), both quantized "
+                "block-wise to E4M3 with one f32 scale per %d elements along K every step, then the block-scaled "
+                "GEMM, out bf16 [%d,%d] (caller-owned)" % (cfg["M"], cfg["K"], cfg["N"], cfg["K"], cfg["block"],
+                                                          cfg["M"], cfg["N"]))
     if k == "blockwise":
         return ("block-wise quantize: bf16 [%d,%d] ~N(0,1) with the sweep's outliers and zeros, scales per block "
                 "along the rows: E4M3 blocks of 128 and 32, stochastic E5M2 blocks of 128, and the bf16 "
@@ -274,6 +284,58 @@ def build(args, cfg, rank, dev, stream, peaks):
         l2 = "inputs larger than L2 (W %d MB, X %d MB, out %d MB); no flush" % (N * K * 2 >> 20, M * K * 2 >> 20,
                                                                                M * N * 2 >> 20)
         return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=h2d, d2h=M * N * 2,
+                    roofline=roofline, extras=extras, l2=l2, flush=None)
+
+    if kind == "blockscaled":
+        blk = cfg["block"]
+        nb = -(-K // blk)
+        x_host = bf16_host(W.large_x(M, K, seed=rank)).view(M, K)
+        w_host = bf16_host(W.large_w(N, K)).view(N, K)
+        x, w = x_host.to(dev), w_host.to(dev)
+        xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        wq = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        xs = torch.empty((M, nb), dtype=torch.float32, device=dev)
+        ws = torch.empty((N, nb), dtype=torch.float32, device=dev)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        out_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        lib, P, st = hq.lib, (lambda t: t.data_ptr()), stream.cuda_stream
+
+        def qb(src, q, sc):
+            rows, cols = src.shape
+            hq.check(lib.hq_quantize_fp8_blockwise(P(src), hq.BF16, rows, cols, hq.E4M3, blk, 0, 0, P(q), P(sc),
+                                                   None, st))
+
+        calls = [("quantize X", lambda: qb(x, xq, xs), 1), ("quantize W", lambda: qb(w, wq, ws), 1),
+                 ("gemm", lambda: hq.check(lib.hq_gemm_blockscaled(P(xq), P(wq), hq.E4M3, P(xs), P(ws), blk, None,
+                                                                   M, N, K, P(out), st)), 1)]
+
+        def e2e():
+            x.copy_(x_host, non_blocking=True)
+            w.copy_(w_host, non_blocking=True)
+            for c in calls:
+                c[1]()
+            out_host.copy_(out, non_blocking=True)
+
+        flops = 2.0 * M * N * K
+
+        def roofline(ms):
+            a = flops / (ms["gemm"] / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": round(a, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(a / fp8_peak, 4), "traffic": None,
+                    "kernel": "k_gemm_bs (tcgen05 kind::f8f6f4 per scale block, f32x2 promotion from TMEM)",
+                    "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal fp8/bf16 dense ratio)" %
+                                   (peaks["_src"], peaks["bf16_tflops"], FP8_OVER_BF16)}
+
+        def extras(ms):
+            d = {}
+            for label, rows in (("quantize X", M), ("quantize W", N)):
+                gb = q_bytes(rows, K, rows * nb) / (ms[label] / 1e3) / 1e9
+                d[label] = {"ms": round(ms[label], 4), "GB/s": round(gb, 1), "frac_hbm": round(gb / peaks["hbm_gbs"], 4)}
+            return {"quantize_blockwise": d, "gemm_ms": round(ms["gemm"], 4), "block": blk}
+
+        l2 = "inputs larger than L2 (W %d MB, X %d MB, out %d MB); no flush" % (N * K * 2 >> 20, M * K * 2 >> 20,
+                                                                               M * N * 2 >> 20)
+        return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=(M * K + N * K) * 2, d2h=M * N * 2,
                     roofline=roofline, extras=extras, l2=l2, flush=None)
 
     if kind == "backward":
@@ -679,6 +741,12 @@ def run_ours(args, rank, local_rank, world):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and cfg["kind"] in ("layer", "decode"):
         mx = min(256, cfg["M"])
         cpu = cpu_baseline(cfg["M"], cfg["N"], cfg["K"], budget_rows=(mx, min(cfg["N"], 4096 * 256 // mx)))
+    elif rank == 0 and world == 1 and not args.no_cpu_baseline and cfg["kind"] == "blockscaled":
+        mx, nw = 256, 4096
+        fl, dt = cpu_blockscaled_sample(cfg["M"], cfg["N"], cfg["K"], cfg["block"], (mx, nw))
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": "X %d rows x W %d rows (K=%d, block %d): block-wise quantize of both + exact block-scaled "
+                         "GEMM, %.1f s" % (mx, nw, cfg["K"], cfg["block"], dt), "seconds": round(dt, 2)}
     elif rank == 0 and world == 1 and not args.no_cpu_baseline and cfg["kind"] in ("sweep", "blockwise"):
         rows = 256
         fn = cpu_sweep_sample if cfg["kind"] == "sweep" else cpu_blockwise_sample
@@ -745,6 +813,24 @@ def cpu_baseline(M, N, K, budget_rows, seed=0):
             "seconds": round(dt, 2)}
 
 
+def cpu_blockscaled_sample(M, N, K, block, budget_rows, seed=0):
+    """The oracle on a bounded sample of the block-scaled layer: block-wise
+    quantize of `mx` rows of X and `nw` rows of W, then the block-scaled GEMM
+    of the sample.  Returns (flops, seconds)."""
+    import oracle as O
+    import workloads as W
+    mx, nw = budget_rows
+    rng = np.random.default_rng(seed)
+    x = W.f32_to_bf16_bits(rng.standard_normal((mx, K), dtype=np.float32))
+    w = W.f32_to_bf16_bits(rng.standard_normal((nw, K), dtype=np.float32) * np.float32(0.02))
+    O.lib()
+    t = time.perf_counter()
+    xq, xs, _ = O.quantize_blockwise(x, O.E4M3, block)
+    wq, ws, _ = O.quantize_blockwise(w, O.E4M3, block)
+    O.gemm_blockscaled(xq, wq, O.E4M3, xs, ws, block)
+    return 2.0 * mx * nw * K, time.perf_counter() - t
+
+
 def cpu_sweep_sample(rows, cols, seed=0):
     """The oracle quantizing a row sample of the sweep input in every mode;
     returns (algorithmic bytes, seconds)."""
@@ -799,6 +885,19 @@ def run_reference(args, rank, world):
         sample = ("per step: %d rows x %d cols of the sweep input, %s" %
                   (rows, K, "all six modes" if cfg["kind"] == "sweep" else "the four block-wise calls"))
         dtype = "fp8 codes from bf16, f64 oracle"
+    elif cfg["kind"] == "blockscaled":
+        rows = (8, 512)
+        for _ in range(args.warmup):
+            cpu_blockscaled_sample(M, N, K, cfg["block"], rows)
+        t = time.perf_counter()
+        fl = 0.0
+        for i in range(args.steps):
+            fl += cpu_blockscaled_sample(M, N, K, cfg["block"], rows, seed=i)[0]
+        dt = time.perf_counter() - t
+        value, unit = fl / dt / 1e12, "TFLOP/s"
+        sample = ("per step: X %d rows x W %d rows (K=%d, block %d), block-wise quantize + exact block-scaled GEMM"
+                  % (rows[0], rows[1], K, cfg["block"]))
+        dtype = "fp8_e4m3 codes, per-block f32 scales, exact block sums, f64"
     else:
         rows = (8, 512)
         for _ in range(args.warmup):
