@@ -7,18 +7,18 @@
 // accumulate; megablocks-hip TODO-gg.md: the grouped per-expert form, output
 // overwritten.)
 //
-// Design (one persistent CTA per SM, 192 threads, 6 warps):
+// Design (persistent CTAs or CTA pairs, one per SM, 320 threads, 10 warps):
 //   warp 0      TMA producer: one elected thread streams 128-byte-wide K
 //               slices of A (128 rows) and B (BN rows) into a ring of shared
 //               memory stages (128B swizzle), signalling mbarriers.
-//   warp 1      allocates TMEM (two BN-column FP32 accumulators) and issues
-//               tcgen05.mma (kind::f8f6f4 for FP8, kind::f16 for bf16) from
-//               one thread; tcgen05.commit frees a stage / publishes an
-//               accumulator.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp owns its
-//               32-lane TMEM quadrant), scale, round to bf16, 16-byte stores.
-//               Two accumulators let the epilogue of tile i overlap the
-//               main loop of tile i+1.
+//   warp 1      allocates TMEM (two FP32 accumulators of up to 256 columns)
+//               and issues tcgen05.mma (kind::f8f6f4 for FP8, kind::f16 for
+//               bf16) from one thread; tcgen05.commit frees a stage /
+//               publishes an accumulator (CTA pairs: cta_group::2).
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (two warps per
+//               32-lane TMEM quadrant), scale, bias, round to bf16 (or FP8),
+//               TMA or 16-byte stores.  Two accumulators let the epilogue of
+//               tile i overlap the main loop of tile i+1.
 // Every wait is bounded: on a stalled barrier the CTA records an error in a
 // device word, drains what it has in flight and exits instead of hanging.
 #include "fp8_cvt.cuh"
