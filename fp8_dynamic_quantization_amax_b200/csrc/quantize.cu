@@ -9,18 +9,27 @@
 //   scale = 1 / m (the dequant scale), amax_out = amax
 //
 // Kernel family (memory bound; every kernel keeps several 16-byte loads or
-// bulk copies in flight per thread and no kernel waits on another CTA):
+// bulk copies in flight per thread; only the single-launch kernels wait on
+// other CTAs, at one bounded grid barrier of a cooperative launch):
 //   per-token   one pass, persistent CTAs: a ring of shared-memory stages is
 //               filled by 1-D bulk copies (TMA), each stage a group of whole
 //               rows; a stage is reduced and cast while the next ones load.
 //               Unaligned or very long rows take a scalar path.
-//   per-tensor  two launches: phase 1 reduces amax with per-CTA partials and
-//               an atomicMax on the f32 bit pattern; the last CTA (threadfence
-//               + counter election) publishes m.  Phase 2 casts, walking the
-//               tensor backwards so its first reads hit what phase 1 left in L2.
-//   per-channel the same two phases on [column strip x row band] tiles.
+//   per-tensor  large aligned inputs: one cooperative launch that keeps the
+//               first part of each CTA's range in shared and tensor memory
+//               across the grid barrier and re-reads the rest from L2.
+//               Otherwise two launches: phase 1 reduces amax with per-CTA
+//               partials and an atomicMax on the f32 bit pattern, the last
+//               CTA (threadfence + counter election) publishes m; phase 2
+//               casts, walking the tensor backwards to reuse L2.
+//   per-channel the same two forms on [column strip x row band] tiles.
 //   delayed     one pass with the multiplier already in the ring; the last
 //               CTA folds amax into hist[idx] and publishes the next scale.
+//   transposed  per-tensor codes written row-major and transposed through
+//               64 x 64 shared-memory tiles (the backward GEMMs' operands).
+//   stochastic  E5M2 with one counter-based SplitMix64 draw per element.
+//   block-wise  one scale per block along the last dimension: the per-token
+//               stage pipeline with warp-level block reductions.
 //
 // Instruction economy (the kernels are ALU-issue bound otherwise):
 //   - amax runs on raw bit patterns: for non-negative floats the unsigned
@@ -2254,8 +2263,10 @@ template <int DT>
 cudaError_t launch_block_typed(const QuantizeArgs& a, int64_t block, bool sr) {
   int dev = 0;
   cudaGetDevice(&dev);
-  // Power-of-two blocks go to the warp-cooperative kernel: block / kVec lanes
-  // per block (2..32), or one block per unit of 2, 4 or 8 warp-wide vectors.
+  // Power-of-two blocks of up to four warp-wide vector spans (W elements)
+  // take the staged kernels when a stage pair of rows fits; otherwise, and
+  // for eight spans, the unstaged warp-cooperative kernel; any other block
+  // (a multiple of 16) one thread per block.
   constexpr int64_t W = 32 * Dt<DT>::kVec;
   const bool pow2 = (block & (block - 1)) == 0;
   int log2_block = 0;
