@@ -76,3 +76,12 @@ def test_every_workload_is_described_and_sized():
                                "moe_bf16")
     # one quantize call's algorithmic bytes: bf16 read + code write + f32 scales
     assert bench.q_bytes(4, 8, 4) == 4 * 8 * 3 + 16
+
+
+def test_blockscaled_reference_leg_reports_tflops():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "blockscaled", "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert "block-scaled" in line["config"]["workload"] and "block 128" in line["cpu_baseline"]["sample"]
