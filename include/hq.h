@@ -12,6 +12,12 @@
  *     amax), commit "finalize fp8 scale rings inside quantize kernels" (the
  *     [hist | scale | counter] ring updated by the last block), mm_fp8 and
  *     linear_forward_fp8 (NT layout: A = XQ[M,K], B = WQ[N,K]).
+ *   - hip-quant 0.6.0 README: "Stochastic E5M2 Backward Gradients" (round
+ *     up or down with probability proportional to the distance, from a
+ *     stateless hash of (seed, element index)), "Block-wise FP8 Scaling"
+ *     (one FP32 dequant scale per block along the last dimension) and
+ *     "Block-scaled Linear and Adafactor Kernel Helpers" (the linear on
+ *     block-wise FP8 bytes and scales of both operands).
  *   - fuel-ir 0.22.4 src/quant_scale.rs: ScaleGranularity, scale_count,
  *     ScalePair.
  *   - ROCm/aiter PR 6437 "Technical Details": an a8w8 GEMM that writes a
