@@ -30,7 +30,7 @@
  *  [GG]  megablocks-hip _dev/TODO-gg.md: per-expert Y_e = X_e . W_e^T, the
  *        output is overwritten, never accumulated.
  *
- * Readings where the pages are silent (each also listed in the design doc):
+ * Readings where the pages are silent:
  *  R1  NaN input encodes to the canonical code 0x7F in both formats.
  *  R2  The cast saturates: |y| >= fmax (including +-Inf) -> sign | max code.
  *  R3  amax skips NaN and +-Inf elements.
