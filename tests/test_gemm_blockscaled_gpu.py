@@ -3,7 +3,7 @@ Linear and Adafactor Kernel Helpers": FP8 bytes plus FP32 per-block scales of
 both operands; "Block-wise FP8 Scaling": scales [..., ceil(K / block_size)])
 against the oracle, through the C ABI.
 
-Tolerance (written here, from the workload statement): |out - ref| <=
+Tolerance (the pass criterion of the scaled GEMM): |out - ref| <=
 8e-3 |ref| + 1e-3 max|ref| with ref the exact block sums, scaled and summed
 in fp64, rounded once to bf16.  Shapes cover several M and N tiles with
 ragged edges, blocks of 32 (four per 128-wide stage) to 256 (two stages per

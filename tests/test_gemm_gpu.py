@@ -5,7 +5,7 @@ rest is untouched; invalid outs raise and leave the buffer untouched; empty
 out is a no-op; operands on the host are rejected; the output is
 overwritten, never accumulated (megablocks-hip TODO-gg.md).
 
-Tolerance (written here, from the workload statement): |out - ref| <=
+Tolerance (the pass criterion of the scaled GEMM): |out - ref| <=
 8e-3 |ref| + 1e-3 max|ref| with ref the exact product rounded to bf16.
 """
 import numpy as np

@@ -5,8 +5,8 @@ This module draws random numbers and lays them out; it holds none of the
 quantization or GEMM arithmetic.  bf16 tensors are returned as uint16 bit
 patterns, rounded from float32 samples to nearest-even by torch's CPU cast.
 
-Workload recipes (sizes and distributions from the workload statement; the
-unstated details are this module's readings):
+Workload recipes (the benchmark configurations' sizes and distributions;
+details they leave open are this module's readings):
   tiny      X f32 [64,256] ~N(0,1), rows 3 and 17 scaled x50;
             W f32 [128,256] ~N(0,0.02); seed 0.
   sweep     bf16 [8192,8192] ~N(0,1); 0.1% of positions x100; a further 0.1%
