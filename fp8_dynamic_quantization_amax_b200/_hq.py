@@ -193,6 +193,16 @@ def hq_gemm_blockscaled(xq, wq, x_scales, w_scales, fmt=E4M3, block=32, bias=Non
     return out
 
 
+def hq_linear_blockwise(x, w, bias=None, fmt=E4M3, block=32, out=None, stream=None):
+    """The block-scaled linear on bf16 / f16 / f32 operands: x [M, K] and
+    w [N, K] quantized block-wise along K (three C-ABI calls: two
+    hq_quantize_fp8_blockwise, one hq_gemm_blockscaled).  Returns bf16
+    out [M, N] = x . w^T (+ bias) within the FP8 error."""
+    xq, xs = hq_quantize_fp8_blockwise(x, fmt, block, stream=stream)
+    wq, ws = hq_quantize_fp8_blockwise(w, fmt, block, stream=stream)
+    return hq_gemm_blockscaled(xq, wq, xs, ws, fmt, block, bias=bias, out=out, stream=stream)
+
+
 def hq_dequantize_fp8_blockwise(q, scales, fmt=E4M3, block=32, out_dtype=torch.float32, stream=None):
     """f32(dec(q) * block scale), as float32 or rounded to bfloat16."""
     rows, cols = q.shape

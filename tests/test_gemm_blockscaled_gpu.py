@@ -135,3 +135,23 @@ def test_blockscaled_gemm_empty_is_a_no_op():
                                      out.data_ptr(), None) == 0
     torch.cuda.synchronize()
     assert (host_bits(out) == 0).all()
+
+
+def test_linear_blockwise_is_quantize_then_gemm():
+    # the convenience path equals the three calls it chains, bit for bit, and
+    # tracks the bf16 product within the FP8 error
+    rng = np.random.default_rng(21)
+    M, N, K, block = 96, 264, 512, 32
+    xb = W.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    wb = W.f32_to_bf16_bits((rng.standard_normal((N, K)) * 0.05).astype(np.float32))
+    bias = W.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32))
+    x, w, b = dev_bf16(xb), dev_bf16(wb), dev_bf16(bias)
+    out = H.hq_linear_blockwise(x, w, bias=b, block=block)
+    xq, xs = H.hq_quantize_fp8_blockwise(x, O.E4M3, block)
+    wq, ws = H.hq_quantize_fp8_blockwise(w, O.E4M3, block)
+    ref = H.hq_gemm_blockscaled(xq, wq, xs, ws, O.E4M3, block, bias=b)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    qx, sx, _ = O.quantize_blockwise(xb, O.E4M3, block)
+    qw, sw, _ = O.quantize_blockwise(wb, O.E4M3, block)
+    assert_gemm_close(host_bits(out), O.gemm_blockscaled(qx, qw, O.E4M3, sx, sw, block, bias))
