@@ -31,6 +31,7 @@
 // what it has in flight, frees TMEM and exits.
 #include "hq_internal.cuh"
 #include "ptx.cuh"
+#include "tc.cuh"
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -68,60 +69,9 @@ struct BsParams {
   unsigned* err;
 };
 
-using ptx::smem_u32;
-
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err,
                                          unsigned long long limit = ptx::kWaitLimitNs) {
   return ptx::mbar_wait(bar, parity, abort_flag, err, kDevErrTimeout, limit);
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-          smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// K-major operand, 128-byte swizzle, 128-byte rows, 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(1) << 16;
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
-  return d;
-}
-
-__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-// 32 lanes x 32 columns of 32-bit, waited in the same asm block.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr)
-      : "memory");
 }
 
 // (a0, a1) += (p0, p1) * ((w0, w1) * (x, x)): one packed multiply and one
@@ -138,11 +88,6 @@ __device__ __forceinline__ void promote2(float& a0, float& a1, uint32_t p0, uint
       "mov.b64 {%0, %1}, acc;\n\t}"
       : "+f"(a0), "+f"(a1)
       : "r"(p0), "r"(p1), "f"(w0), "f"(w1), "f"(x));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __device__ __forceinline__ void tile_coords(int t, const BsParams& p, int& m0, int& n0) {
@@ -268,7 +213,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
                 // K steps past K in the last stage read the zero fill
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                  mma_f8(d_tmem, ad + 2u * k, bd + 2u * k, p.idesc, (kb > kb_first || k > 0) ? 1u : 0u);
+                  mma_issue<0>(d_tmem, ad + 2u * k, bd + 2u * k, p.idesc, (kb > kb_first || k > 0) ? 1u : 0u);
                 tc_commit(&empty_bar[stage]);
                 issued = true;
               }
@@ -313,7 +258,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
             if (q < nsteps) {
               const int kk = ks + q;
               const uint32_t blk = static_cast<uint32_t>(kk / p.spb - b0);  // 0 or 1 within the group
-              mma_f8(d0 + blk * kBsTile, ad + 2u * (kk & 3), bd + 2u * (kk & 3), p.idesc,
+              mma_issue<0>(d0 + blk * kBsTile, ad + 2u * (kk & 3), bd + 2u * (kk & 3), p.idesc,
                      (kk % p.spb != 0) ? 1u : 0u);
             }
           }
@@ -356,7 +301,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
               }
               const uint64_t ad = smem_desc(smem_u32(sA + stage * kBsOperandBytes));
               const uint64_t bd = smem_desc(smem_u32(sB + stage * kBsOperandBytes));
-              mma_f8(d_tmem, ad + 2u * sub, bd + 2u * sub, p.idesc, ks > kfirst ? 1u : 0u);
+              mma_issue<0>(d_tmem, ad + 2u * sub, bd + 2u * sub, p.idesc, ks > kfirst ? 1u : 0u);
               issued = true;
               if (sub == 3 || ks == p.nks - 1) {  // the stage's last K step: hand the stage back
                 tc_commit(&empty_bar[stage]);
@@ -482,44 +427,6 @@ __global__ void __launch_bounds__(kBsThreads, 1)
 }
 
 // --------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// FP8 [rows, cols] row-major, {128-byte, 128-row} boxes, 128B swizzle; out of
-// range elements read as zero codes.
-bool make_fp8_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, std::string* msg) {
-  auto encode = encode_fn();
-  if (!encode) {
-    *msg = "cuTensorMapEncodeTiled is not available from the driver";
-    return false;
-  }
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols};
-  cuuint32_t box[2] = {128, kBsTile};
-  cuuint32_t estr[2] = {1, 1};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    char buf[128];
-    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (%d) for [%llu, %llu]", static_cast<int>(r),
-             static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols));
-    *msg = buf;
-    return false;
-  }
-  return true;
-}
-
 }  // namespace
 
 cudaError_t launch_gemm_blockscaled(const BlockScaledGemmArgs& a, std::string* msg) {
@@ -541,8 +448,8 @@ cudaError_t launch_gemm_blockscaled(const BlockScaledGemmArgs& a, std::string* m
   memset(&ta, 0, sizeof(ta));
   memset(&tb, 0, sizeof(tb));
   if (a.K > 0) {  // K == 0: no loads are issued and the maps are never read
-    if (!make_fp8_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), msg) ||
-        !make_fp8_map(&tb, a.b, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), msg))
+    if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), 1, kBsTile, msg) ||
+        !make_map(&tb, a.b, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K), 1, kBsTile, msg))
       return cudaErrorInvalidValue;
   }
   BsParams p;
