@@ -22,9 +22,10 @@ F32, BF16, F16 = 0, 1, 2
 
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
             "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic",
-            "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_blockscaled", "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8",
-            "hq_grouped_gemm_bf16",
-            "hq_quantize_fp8_noalloc", "hq_check_device_error", "hq_last_error", "hq_version"]
+            "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_blockscaled",
+            "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
+            "hq_quantize_fp8_noalloc", "hq_debug_bounded_wait", "hq_check_device_error", "hq_last_error",
+            "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
 
 
@@ -53,6 +54,8 @@ def _load():
     L.hq_quantize_fp8.restype = ci
     L.hq_quantize_fp8_noalloc.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P]
     L.hq_quantize_fp8_noalloc.restype = ci
+    L.hq_debug_bounded_wait.argtypes = [ctypes.c_uint64, P]
+    L.hq_debug_bounded_wait.restype = ci
     L.hq_gemm_blockscaled.argtypes = [P, P, ci, P, P, i64, P, i64, i64, i64, P, P]
     L.hq_gemm_blockscaled.restype = ci
     L.hq_quantize_fp8_blockwise.argtypes = [P, ci, i64, i64, ci, i64, ci, ctypes.c_uint64, P, P, P, P]

@@ -619,6 +619,15 @@ hq_status hq_grouped_gemm_bf16(const void* x, const void* w, const int32_t* offs
   return gemm_common(1, x, w, 0, nullptr, 0, nullptr, 0, offsets, E, M_total, N, K, out, stream);
 }
 
+hq_status hq_debug_bounded_wait(uint64_t limit_ns, hq_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 2000000000ull)
+    return fail(HQ_ERR_INVALID_ARG, "limit_ns = %llu outside [1 us, 2 s]", (unsigned long long)limit_ns);
+  hq_status s = check_arch();
+  if (s != HQ_OK) return s;
+  return launched(hq::launch_bounded_wait_probe(limit_ns, reinterpret_cast<cudaStream_t>(stream)),
+                  "bounded-wait probe launch");
+}
+
 hq_status hq_check_device_error(void) {
   unsigned w = 0;
   const cudaError_t e = hq::read_and_clear_device_error(&w);

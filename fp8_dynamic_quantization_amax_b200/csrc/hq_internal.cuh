@@ -1,6 +1,6 @@
 // hq_internal.cuh -- declarations shared by the translation units of
-// libhq.so (api.cu, quantize.cu, gemm.cu, gemm_bs.cu, noalloc.cu).  Not part
-// of the public ABI.
+// libhq.so (api.cu, quantize.cu, gemm.cu, gemm_bs.cu, noalloc.cu, probe.cu).
+// Not part of the public ABI.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -100,6 +100,9 @@ cudaError_t read_and_clear_device_error(unsigned* word);
 unsigned* device_error_word();
 
 int device_sm_count(int dev);
+
+// One bounded wait that nothing completes (probe.cu): sets kDevErrTimeout.
+cudaError_t launch_bounded_wait_probe(unsigned long long limit_ns, cudaStream_t stream);
 
 // Records a printf-style message for hq_last_error() and returns s.
 hq_status set_error(hq_status s, const char* fmt, ...);

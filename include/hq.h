@@ -420,6 +420,19 @@ hq_status hq_quantize_fp8_noalloc(const void* x, hq_dtype xt, int64_t rows, int6
                                   float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,
                                   hq_stream_t stream);
 
+/*
+ * Test hook for the failure path of the library's bounded waits: launches
+ * one thread that waits on a shared-memory barrier nothing completes, for
+ * limit_ns nanoseconds (1 us .. 2 s).  The wait then gives up, records a
+ * timeout in the device error word and the kernel returns normally (no trap,
+ * no fault); the next hq_check_device_error() returns HQ_ERR_TIMEOUT and
+ * clears the word.  Every wait in the library's kernels takes this path on a
+ * stalled barrier.
+ * Errors: HQ_ERR_INVALID_ARG (limit outside the range), HQ_ERR_UNSUPPORTED_ARCH,
+ *   HQ_ERR_CUDA.
+ */
+hq_status hq_debug_bounded_wait(uint64_t limit_ns, hq_stream_t stream);
+
 /* Synchronizes the current device, then reads and clears the device error
    word: HQ_OK, HQ_ERR_TIMEOUT (a bounded wait in a kernel gave up; that
    launch's outputs are undefined), HQ_ERR_INVALID_ARG (malformed grouped

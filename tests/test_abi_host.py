@@ -266,3 +266,8 @@ def test_blockscaled_gemm_rejections():
     assert call(out=BASE + 0x2000000 - 0x100) == OVERLAP     # out running into x_scales
     assert call(bias=BASE + 0x4000000 + 0x40) == OVERLAP     # bias inside out
     assert call(M=1 << 31) == TOO_LARGE
+
+
+def test_bounded_wait_probe_rejects_out_of_range_limits():
+    assert L.hq_debug_bounded_wait(10, None) == INVALID             # below 1 us
+    assert L.hq_debug_bounded_wait(3_000_000_000, None) == INVALID  # above 2 s
