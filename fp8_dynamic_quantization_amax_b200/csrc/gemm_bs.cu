@@ -198,14 +198,21 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         for (int b0 = 0; b0 < p.nb && !stop; b0 += kBsGroupBlocks, ++jg) {
           const uint32_t sl = jg % kBsSlots;
           const uint32_t sph = (jg / kBsSlots) & 1u;
-          if (!wait_bar(&aempty_bar[sl], sph ^ 1u, &abort_flag, p.err)) { stop = true; break; }
+          // the warp agrees on giving up, so that no lane is left at a warp-wide step
+          if (__any_sync(0xFFFFFFFFu, !wait_bar(&aempty_bar[sl], sph ^ 1u, &abort_flag, p.err))) {
+            stop = true;
+            break;
+          }
           tc_fence_after();
           for (int i = 0; i < kBsGroupBlocks && b0 + i < p.nb && !stop; ++i) {
             const uint32_t d_tmem = tmem_base + (sl * kBsGroupBlocks + i) * kBsTile;
             const int kb_first = kb;
             const int kb_end = min(p.nkb, (b0 + i + 1) * spbs);
             for (; kb < kb_end; ++kb) {
-              if (!wait_bar(&full_bar[stage], phase, &abort_flag, p.err)) { stop = true; break; }
+              if (__any_sync(0xFFFFFFFFu, !wait_bar(&full_bar[stage], phase, &abort_flag, p.err))) {
+                stop = true;
+                break;
+              }
               tc_fence_after();
               if (lane == 0) {
                 const uint64_t ad = smem_desc(smem_u32(sA + stage * kBsOperandBytes));
@@ -367,7 +374,11 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         __syncwarp();
         const uint32_t sl = jg % kBsSlots;
         const uint32_t sph = (jg / kBsSlots) & 1u;
-        if (!wait_bar(&afull_bar[sl], sph, &abort_flag, p.err)) { stop = true; break; }
+        // the warp agrees on giving up: the TMEM loads below are warp-wide
+        if (__any_sync(0xFFFFFFFFu, !wait_bar(&afull_bar[sl], sph, &abort_flag, p.err))) {
+          stop = true;
+          break;
+        }
         tc_fence_after();
 #pragma unroll
         for (int i = 0; i < kBsGroupBlocks; ++i) {
