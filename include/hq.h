@@ -191,6 +191,8 @@ hq_status hq_gemm_blockscaled(const uint8_t* xq, const uint8_t* wq, hq_fp8_forma
  * Arguments: x device [rows, cols] f32 / bf16 / f16 (xt), q device uint8
  *   [rows, cols], both 16-byte aligned; cols % 16 == 0; block % 16 == 0;
  *   scales device f32 [rows * ceil(cols / block)]; amax_out the same or NULL.
+ *   rows == 0 or cols == 0 returns HQ_OK with no launch once the shape and
+ *   enum checks pass (null buffers allowed then).
  * Errors: HQ_ERR_INVALID_ARG, HQ_ERR_MISALIGNED, HQ_ERR_OVERLAP,
  *   HQ_ERR_WRONG_DEVICE, HQ_ERR_UNSUPPORTED_ARCH, HQ_ERR_TOO_LARGE,
  *   HQ_ERR_CUDA.
@@ -202,8 +204,8 @@ hq_status hq_quantize_fp8_blockwise(const void* x, hq_dtype xt, int64_t rows, in
 /*
  * Block-wise dequantize: out[r, c] = f32(dec(q[r, c]) * scales[r, c / block])
  * (one f32 multiply), written as f32 (out_type HQ_F32) or rounded to bf16
- * (HQ_BF16).  Same layout rules as hq_quantize_fp8_blockwise; out 16-byte
- * aligned.
+ * (HQ_BF16).  Same layout rules, and the same empty-shape rule, as
+ * hq_quantize_fp8_blockwise; out 16-byte aligned.
  */
 hq_status hq_dequantize_fp8_blockwise(const uint8_t* q, hq_fp8_format fmt, int64_t rows, int64_t cols,
                                       int64_t block, const float* scales, hq_dtype out_type, void* out,
