@@ -848,3 +848,20 @@ def test_blockscaled_gemm_entries_equal_the_full_product():
     ms = rng.integers(0, M, 30)
     ns = rng.integers(0, N, 30)
     assert np.array_equal(O.gemm_blockscaled_entries(xq, wq, O.E5M2, xs, ws, block, ms, ns, bias), full[ms, ns])
+
+
+@pytest.mark.parametrize("fmt,rel,sub", [(O.E4M3, 2.0 ** -4, 2.0 ** -10), (O.E5M2, 2.0 ** -3, 2.0 ** -17)])
+def test_blockwise_round_trip_within_half_a_step(fmt, rel, sub):
+    # decode(quantize(x)) * block scale is within half a code step of x:
+    # 2^-(mantissa bits + 1) relative for normal codes, half the subnormal
+    # step (scaled) otherwise; a block index mixed up between the two
+    # functions breaks it at once
+    rng = np.random.default_rng(79)
+    rows, cols, block = 6, 200, 32
+    band = np.exp(rng.uniform(-10, 6, (rows, -(-cols // 8)))).repeat(8, axis=1)[:, :cols]
+    x = (rng.standard_normal((rows, cols)) * band).astype(np.float32)
+    q, s, _ = O.quantize_blockwise(x, fmt, block)
+    back = O.dequantize_blockwise(q, fmt, block, s).astype(np.float64)
+    sc = np.repeat(s, block, axis=1)[:, :cols].astype(np.float64)
+    err = np.abs(back - x.astype(np.float64))
+    assert (err <= np.abs(x) * (rel + 2.0 ** -20) + sc * sub).all()
