@@ -277,7 +277,7 @@ def _parse_ring_golden():
 def test_ring_hand_trace():
     ring = np.array([0, 0, 1, 0], np.float32)
     steps = _parse_ring_golden()
-    assert len(steps) == 6
+    assert len(steps) == 11
     for st in steps:
         x = st["x"].copy()
         q, s, am = O.quantize(x.reshape(1, 4), O.E4M3, O.PER_TENSOR, ring=ring,
