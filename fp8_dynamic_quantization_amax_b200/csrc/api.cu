@@ -180,11 +180,18 @@ size_t hq_quantize_workspace_bytes(hq_granularity g, int64_t rows, int64_t cols,
   return hq::quantize_workspace_bytes(static_cast<int>(g), rows, cols, delayed);
 }
 
-hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
-                          hq_granularity g, uint8_t* q, float* scales, float* amax_out, float* ring,
-                          int32_t ring_len, int32_t ring_idx, int32_t ring_margin, void* workspace,
-                          size_t workspace_bytes, hq_stream_t stream) {
-  // ---- arguments
+}  // extern "C"
+
+namespace hq {
+// The argument checks of hq_quantize_fp8 that do not involve the workspace,
+// in the order that entry point applies them.  *empty is set when the call
+// has no scale group (scale_count == 0): such a call returns HQ_OK without
+// a launch.
+hq_status quantize_check_args(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                              hq_granularity g, const uint8_t* q, const float* scales, const float* amax_out,
+                              const float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,
+                              bool* empty) {
+  *empty = false;
   if (xt != HQ_F32 && xt != HQ_BF16 && xt != HQ_F16) return fail(HQ_ERR_INVALID_ARG, "invalid dtype %d", (int)xt);
   if (fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", (int)fmt);
   if (g != HQ_PER_TENSOR && g != HQ_PER_TOKEN && g != HQ_PER_CHANNEL)
@@ -202,16 +209,42 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
   const int64_t ns = hq_scale_count(g, rows, cols);
   const int64_t n = rows * cols;
   const size_t esize = (xt == HQ_F32) ? 4 : 2;
-  const size_t need = hq::quantize_workspace_bytes(static_cast<int>(g), rows, cols, ring != nullptr);
-  if (ns == 0) return ok();
+  if (ns == 0) {
+    *empty = true;
+    return ok();
+  }
   if (n > 0 && (!x || !q)) return fail(HQ_ERR_INVALID_ARG, "x and q must not be null");
   if (!scales) return fail(HQ_ERR_INVALID_ARG, "scales must not be null");
-  if (need > 0 && !workspace) return fail(HQ_ERR_INVALID_ARG, "this mode needs a workspace of %zu bytes", need);
-  if (need > 0 && workspace_bytes < need)
-    return fail(HQ_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
   if (!is_aligned(x, esize)) return fail(HQ_ERR_MISALIGNED, "x is not aligned to its element size");
   if (!is_aligned(scales, 4) || !is_aligned(amax_out, 4) || !is_aligned(ring, 4))
     return fail(HQ_ERR_MISALIGNED, "scales, amax_out and ring must be 4-byte aligned");
+  const Range outs[] = {{q, static_cast<size_t>(n), "q"},
+                        {scales, static_cast<size_t>(ns) * 4, "scales"},
+                        {amax_out, amax_out ? static_cast<size_t>(ns) * 4 : 0, "amax_out"},
+                        {ring, ring ? static_cast<size_t>(ring_len + 2) * 4 : 0, "ring"}};
+  const Range ins[] = {{x, static_cast<size_t>(n) * esize, "x"}};
+  return check_overlaps(outs, 4, ins, 1);
+}
+}  // namespace hq
+
+extern "C" {
+
+hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                          hq_granularity g, uint8_t* q, float* scales, float* amax_out, float* ring,
+                          int32_t ring_len, int32_t ring_idx, int32_t ring_margin, void* workspace,
+                          size_t workspace_bytes, hq_stream_t stream) {
+  // ---- arguments
+  bool empty = false;
+  hq_status s = hq::quantize_check_args(x, xt, rows, cols, fmt, g, q, scales, amax_out, ring, ring_len, ring_idx,
+                                        ring_margin, &empty);
+  if (s != HQ_OK || empty) return s;
+  const int64_t ns = hq_scale_count(g, rows, cols);
+  const int64_t n = rows * cols;
+  const size_t esize = (xt == HQ_F32) ? 4 : 2;
+  const size_t need = hq::quantize_workspace_bytes(static_cast<int>(g), rows, cols, ring != nullptr);
+  if (need > 0 && !workspace) return fail(HQ_ERR_INVALID_ARG, "this mode needs a workspace of %zu bytes", need);
+  if (need > 0 && workspace_bytes < need)
+    return fail(HQ_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
   if (need > 0 && !is_aligned(workspace, 256)) return fail(HQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
   const Range outs[] = {{q, static_cast<size_t>(n), "q"},
                         {scales, static_cast<size_t>(ns) * 4, "scales"},
@@ -219,7 +252,7 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
                         {ring, ring ? static_cast<size_t>(ring_len + 2) * 4 : 0, "ring"},
                         {workspace, need, "workspace"}};
   const Range ins[] = {{x, static_cast<size_t>(n) * esize, "x"}};
-  hq_status s = check_overlaps(outs, 5, ins, 1);
+  s = check_overlaps(outs, 5, ins, 1);
   if (s != HQ_OK) return s;
   // ---- device
   const Range devs[] = {{n > 0 ? x : nullptr, 0, "x"}, {n > 0 ? q : nullptr, 0, "q"}, {scales, 0, "scales"},
@@ -632,7 +665,11 @@ hq_status hq_check_device_error(void) {
   unsigned w = 0;
   const cudaError_t e = hq::read_and_clear_device_error(&w);
   if (e != cudaSuccess) return fail(HQ_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
-  if (w & hq::kDevErrTimeout) return fail(HQ_ERR_TIMEOUT, "a kernel's bounded wait gave up");
+  if (w & hq::kDevErrTimeout) {
+    // a kernel that gave up may have left its scratch words set
+    hq::noalloc_scratch_invalidate();
+    return fail(HQ_ERR_TIMEOUT, "a kernel's bounded wait gave up");
+  }
   if (w & hq::kDevErrBadOffsets) return fail(HQ_ERR_INVALID_ARG, "grouped GEMM offsets were malformed");
   return ok();
 }

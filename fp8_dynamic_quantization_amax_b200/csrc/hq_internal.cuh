@@ -107,4 +107,15 @@ cudaError_t launch_bounded_wait_probe(unsigned long long limit_ns, cudaStream_t 
 // Records a printf-style message for hq_last_error() and returns s.
 hq_status set_error(hq_status s, const char* fmt, ...);
 
+// The argument checks of hq_quantize_fp8 that do not involve the workspace
+// (api.cu); *empty is set for a call with no scale group.
+hq_status quantize_check_args(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
+                              hq_granularity g, const uint8_t* q, const float* scales, const float* amax_out,
+                              const float* ring, int32_t ring_len, int32_t ring_idx, int32_t ring_margin,
+                              bool* empty);
+
+// Marks the no-allocation entry point's static scratch for clearing on its
+// next call on every device (noalloc.cu).
+void noalloc_scratch_invalidate();
+
 }  // namespace hq

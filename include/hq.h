@@ -121,8 +121,10 @@ size_t hq_quantize_workspace_bytes(hq_granularity g, int64_t rows, int64_t cols,
  * ops.cu ring commit and pack_quantize_params).  The kernel quantizes with
  * m = ring[ring_len], writes scales[0] = 1/m, and its last block then
  * stores this call's amax in hist[ring_idx], takes win = max(hist) and, if
- * win is finite and > 0, publishes ring[ring_len] = (fmax / win) * 2^-margin
- * (kept otherwise).  The counter word must be 0 on entry and is 0 on exit.
+ * win is finite and > 0, forms next = f32(fmax / win) * 2^-margin; next
+ * replaces ring[ring_len] only when it is finite and > 0 (a subnormal win
+ * or a large |margin| can overflow it to +Inf or underflow it to 0; the old
+ * scale then stays).  The counter word must be 0 on entry and is 0 on exit.
  * A fresh ring is hist = 0, scale = 1, counter = 0; the caller passes
  * ring_idx = step mod ring_len.
  *
@@ -373,7 +375,7 @@ hq_status hq_gemm_a8w8_ex(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fm
  * (decreasing, or outside [0, M_total]) never cause an access outside the
  * buffers: offsets are clamped and the device error word records
  * HQ_ERR_INVALID_ARG.
- * Errors as hq_gemm_a8w8, plus E < 1 (HQ_ERR_INVALID_ARG).
+ * Errors as hq_gemm_a8w8, plus E outside [1, 1024] (HQ_ERR_INVALID_ARG).
  */
 hq_status hq_grouped_gemm_a8w8(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt,
                                const float* x_scale, int64_t x_scale_len,
@@ -408,11 +410,15 @@ hq_status hq_grouped_gemm_bf16(const void* x, const void* w,
  * up to 32,764 columns; a larger one returns HQ_ERR_TOO_LARGE before any
  * launch.  The call itself allocates nothing.
  *
- * The first call on a device that needs the array looks up its device
- * address and clears it (a synchronous memset on that device); make that
- * first call before any stream capture.  Every call leaves the array zero
- * again.  All calls share the one array: two calls that may overlap on the
- * GPU (different streams, or different host threads) race on it and must be
+ * The argument checks run first, in hq_quantize_fp8's order; the size limit
+ * and the array's set-up come after them.  The first call on a device that
+ * needs the array looks up its device address and clears it (a synchronous
+ * memset on that device); make that first call before any stream capture.
+ * Every call leaves the array zero again.  After a call that returned
+ * HQ_ERR_CUDA, or after hq_check_device_error() reported HQ_ERR_TIMEOUT, the
+ * next call clears the array again (synchronously) before using it.  All
+ * calls share the one array: two calls that may overlap on the GPU
+ * (different streams, or different host threads) race on it and must be
  * serialised by the caller.
  */
 #define HQ_NOALLOC_SCRATCH_BYTES (256u * 1024u)

@@ -84,6 +84,32 @@ def test_noalloc_matches_workspace_entry_point_twice(gran, shape, dtype, fmt):
     H.hq_check_device_error()
 
 
+@pytest.mark.parametrize("gran,shape,dtype", [
+    (H.PER_TENSOR, (2048, 4096), torch.bfloat16),    # 16 MiB: the single-launch per-tensor kernel
+    (H.PER_CHANNEL, (256, 32760), torch.bfloat16),   # 16 MiB, 16 column strips: the single-launch per-channel kernel
+    (H.PER_CHANNEL, (128, 8192), torch.float32),     # exactly 4 MiB
+])
+def test_noalloc_single_launch_kernels_twice_vs_oracle(gran, shape, dtype):
+    # Inputs of 4 MiB and more take the single-launch kernels, whose grid
+    # barrier counters and departure count live in the scratch and must be
+    # back at zero for the next call.
+    import oracle as O
+    x = _input(shape, dtype, seed=11 + shape[0])
+    xh = x.view(torch.int16).cpu().numpy().view(np.uint16) if dtype == torch.bfloat16 else x.cpu().numpy()
+    q_o, s_o, a_o = O.quantize(xh, O.E4M3, gran)
+    q_ref, s_ref, a_ref = workspace_call(x, H.E4M3, gran)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        st, q, s, a = noalloc_call(x, H.E4M3, gran)
+        assert st == H.HQ_OK, H.lib.hq_last_error().decode()
+        torch.cuda.synchronize()
+        assert _same(q, q_ref) and _same(s, s_ref) and _same(a, a_ref)
+        np.testing.assert_array_equal(q.cpu().numpy(), q_o)
+        np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), s_o.view(np.uint32))
+        np.testing.assert_array_equal(a.cpu().numpy().view(np.uint32), a_o.view(np.uint32))
+    H.hq_check_device_error()
+
+
 def test_noalloc_delayed_ring_two_steps():
     L = 16
     ring_a = torch.zeros(L + 2, dtype=torch.float32, device="cuda")
@@ -98,6 +124,18 @@ def test_noalloc_delayed_ring_two_steps():
         assert _same(q, q_ref) and _same(s, s_ref) and _same(a, a_ref)
         assert _same(ring_b, ring_a)
     H.hq_check_device_error()
+
+
+def test_noalloc_checks_arguments_before_the_size_limit():
+    # an invalid granularity with a shape the scratch could not hold: the
+    # argument error comes first, as hq_quantize_fp8 would report it
+    x = _input((4, 40000), torch.bfloat16, seed=5)
+    st, q, s, a = noalloc_call(x, H.E4M3, H.PER_TENSOR)
+    assert st == H.HQ_OK
+    bad = H.lib.hq_quantize_fp8_noalloc(_p(x), H._DT[x.dtype], 4, 40000, H.E4M3, 7, _p(q), _p(s), _p(a),
+                                        None, 0, 0, 0, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert bad == 1  # HQ_ERR_INVALID_ARG
+    assert "granularity" in H.lib.hq_last_error().decode()
 
 
 def test_noalloc_refuses_a_shape_beyond_its_scratch():
