@@ -132,3 +132,43 @@ def test_fp8_out_empty_steps_the_ring():
     torch.cuda.synchronize()
     assert torch.equal(ring_f, ring_u) and torch.equal(s_f, s_u)
     assert float(host(ring_f)[L - 1]) == 0.0
+
+
+@pytest.mark.parametrize("q_fmt", [O.E4M3, O.E5M2])
+def test_fp8_out_ring_keeps_scale_when_next_not_finite(q_fmt):
+    # The ring publishes next = f32(fmax / win) * 2^-margin only when next is
+    # finite and > 0 (the delayed-scaling step of AstrAI ops.cu, with the
+    # guard of hip-quant's "Training-path numerical guards").  Three ring
+    # states reach the guard, one control publishes:
+    #   a subnormal window (hist holds 2^-140, the result is all zero):
+    #     fmax / 2^-140 overflows to +Inf
+    #   margin -126 on a result of amax 44: next overflows to +Inf
+    #   margin 126 with 2^127 in the window: next underflows to 0
+    M, N, K = 300, 272, 144
+    xq, wq, xs, ws, _ = operands(7, M, N, K, O.E4M3)
+    zeros = np.zeros_like(xq)
+    cases = [("subnormal window", zeros, 2.0 ** -140, 0, False),
+             ("margin -126", xq, 0.0, -126, False),
+             ("margin 126", xq, 2.0 ** 127, 126, False),
+             ("control", xq, 0.0, 0, True)]
+    for name, x_codes, preset, margin, publishes in cases:
+        ring = fresh_ring(0.75)
+        ring[5] = np.float32(preset)
+        ring_f = torch.from_numpy(ring.copy()).cuda()
+        ring_u = ring_f.clone()
+        args = (dev(x_codes), dev(wq), dev(xs), dev(ws), H.E4M3)
+        q_f, s_f = H.hq_gemm_a8w8_ex(*args, q_fmt=q_fmt, ring=ring_f, ring_idx=2, ring_margin=margin)
+        h = H.hq_gemm_a8w8_ex(*args)
+        q_u, s_u = H.hq_quantize_fp8(h, q_fmt, H.PER_TENSOR, ring=ring_u, ring_idx=2, ring_margin=margin)
+        torch.cuda.synchronize()
+        assert torch.equal(q_f, q_u), name
+        assert torch.equal(ring_f.view(torch.int32), ring_u.view(torch.int32)), name
+        # the oracle's delayed quantize of the GPU's own bf16 result
+        ring_o = ring.copy()
+        q_o, s_o, _ = O.quantize(host_bits(h), q_fmt, O.PER_TENSOR, ring=ring_o, ring_idx=2, ring_margin=margin)
+        np.testing.assert_array_equal(host(q_f), q_o)
+        np.testing.assert_array_equal(host(s_f).view(np.uint32), s_o.view(np.uint32))
+        np.testing.assert_array_equal(host(ring_f).view(np.uint32), ring_o.view(np.uint32))
+        kept = host(ring_f)[L] == np.float32(0.75)
+        assert kept != publishes, name
+    H.hq_check_device_error()

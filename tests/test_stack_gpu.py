@@ -3,12 +3,18 @@ quantize X_t, W_up with their rings -> h = GEMM -> quantize h, W_down with
 their rings -> y = GEMM (per-tensor E4M3, ring length 16, margin 0, X_t std
 ramping 0.5 -> 8; AstrAI ops.cu linear_forward_fp8 and the ring commit).
 
-The oracle is never fed a GPU output.  Stages whose inputs come from the
-generator (X_t, W_up, W_down) are compared bit-exactly, rings included, every
-step.  The later stages (h, its ring, y) depend on GEMM outputs that may
-differ from the exact oracle by a bf16 rounding, so they are compared within
-the GEMM tolerance on a reduced-size stack where the oracle runs the whole
-chain, and by properties at full size.
+Stages whose inputs come from the generator (X_t, W_up, W_down) are compared
+bit-exactly, rings included, every step.  The later stages (h, its ring, y)
+depend on GEMM outputs that may differ from the exact oracle by a bf16
+rounding.  They are checked two ways:
+  - chained: on a reduced-size stack the oracle runs the whole chain from
+    generator inputs alone; h and y within the GEMM tolerance, h's ring
+    within a bf16 rounding;
+  - stage-wise, at full size: every 40 steps the oracle's delayed quantize is
+    fed the GPU's bf16 h and a copy of the GPU's h ring taken before the
+    step, so q(h), its scale and the ring after the step must be bit-exact;
+    y is then compared at sampled entries with the oracle's GEMM of the
+    GPU's q(h) and the oracle's q(W_down), within the GEMM tolerance.
 """
 import numpy as np
 import pytest
@@ -96,6 +102,9 @@ def test_stack_full_size():
     for t in range(steps):
         x = W.delayed_x(t, tokens, dim, steps)
         before = {k: r.copy() for k, r in rings_o.items()}
+        stage_check = t % 40 == 0 or t == steps - 1
+        if stage_check:
+            h_ring_before = host(rings_d["h"]).copy()  # synchronises: no launch of this step yet
         xq, xs = q_delayed(dev_bf16(x), rings_d["x"], t)
         wuq, wus = q_delayed(wu_d, rings_d["wu"], t)
         h = H.hq_gemm_a8w8(xq, wuq, xs, wus, H.E4M3)
@@ -112,7 +121,7 @@ def test_stack_full_size():
         # property: h's ring recorded max|h| of the h it quantized, exactly
         hb = host_bits(h)
         assert host(rings_d["h"])[t % L] == np.abs(W.bf16_bits_to_f32(hb)).max()
-        if t % 40 == 0 or t == steps - 1:
+        if stage_check:
             xqo, xso, _ = O.quantize(x, O.E4M3, O.PER_TENSOR, ring=before["x"], ring_idx=t % L)
             wqo, wso, _ = O.quantize(wu, O.E4M3, O.PER_TENSOR, ring=before["wu"], ring_idx=t % L)
             np.testing.assert_array_equal(host(xq), xqo)
@@ -121,5 +130,20 @@ def test_stack_full_size():
             ns = rng.integers(0, hidden, 512)
             ref = O.gemm_a8w8_entries(xqo, wqo, O.E4M3, xso, wso, ms, ns)
             assert_gemm_close(hb[ms, ns], ref)
-            assert np.isfinite(W.bf16_bits_to_f32(host_bits(y))).all()
+            # stage-wise: the oracle's delayed quantize of the GPU's h with the
+            # GPU's h ring as it stood before this step
+            h_ring_o = h_ring_before.copy()
+            hqo, hso, hao = O.quantize(hb, O.E4M3, O.PER_TENSOR, ring=h_ring_o, ring_idx=t % L)
+            hq_g = host(hq_)
+            np.testing.assert_array_equal(hq_g, hqo)
+            np.testing.assert_array_equal(host(hs).view(np.uint32), hso.view(np.uint32))
+            np.testing.assert_array_equal(host(rings_d["h"]).view(np.uint32), h_ring_o.view(np.uint32))
+            wdqo, wdso, _ = O.quantize(wd, O.E4M3, O.PER_TENSOR, ring=before["wd"], ring_idx=t % L)
+            np.testing.assert_array_equal(host(wdq), wdqo)
+            np.testing.assert_array_equal(host(wds).view(np.uint32), wdso.view(np.uint32))
+            # y = GEMM(q(h), q(W_down)) at sampled entries and two full rows
+            ms = np.concatenate([rng.integers(0, tokens, 1024), np.full(dim, 7), np.full(dim, tokens - 1)])
+            ns = np.concatenate([rng.integers(0, dim, 1024), np.arange(dim), np.arange(dim)])
+            ref_y = O.gemm_a8w8_entries(hq_g, wdqo, O.E4M3, hso, wdso, ms, ns)
+            assert_gemm_close(host_bits(y)[ms, ns], ref_y)
     H.hq_check_device_error()
