@@ -48,6 +48,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <type_traits>
+#include <mutex>
 
 namespace hq {
 namespace {
@@ -377,6 +378,77 @@ __global__ void __launch_bounds__(kThreads, 4) k_token_tma(
     for (int s = 0; s < S; ++s)
       if (pend_mask & (1u << s))
         ptx::mbar_wait(&full[s], (pend_parity >> s) & 1u, &dummy, nullptr, 0, ptx::kDrainLimitNs);
+  }
+}
+
+// Register-resident path for rows of up to 32 * VPL 16-byte vectors.  A warp
+// takes RPW whole rows at a time: lane l loads vectors l, l + 32, ... of each
+// row (one warp load instruction covers 512 contiguous bytes) and keeps them
+// in registers; the row's raw maximum is reduced by shuffles, and the codes
+// are cast from the same registers.  x is read from DRAM exactly once, with
+// no shared memory and no block-wide barrier; the persistent warps of other
+// rows keep the loads in flight while one warp reduces and casts.
+constexpr int kRegThreads = 128;
+
+template <int DT>
+__device__ __forceinline__ uint32_t warp_lmax(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = Dt<DT>::lmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+template <int DT, int FMT, int VPL, int RPW>
+__global__ void __launch_bounds__(kRegThreads) k_token_reg(const void* __restrict__ x, int64_t rows, int64_t nv,
+                                                           uint8_t* __restrict__ q, float* __restrict__ scales,
+                                                           float* __restrict__ amax_out) {
+  constexpr int VEC = Dt<DT>::kVec;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kRegThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kRegThreads) >> 5;
+  const uint4* xv = static_cast<const uint4*>(x);
+  for (int64_t r0 = warp0 * RPW; r0 < rows; r0 += nwarps * RPW) {
+    uint4 u[RPW][VPL];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        const int64_t v = lane + 32 * j;
+        u[r][j] = (r0 + r < rows && v < nv) ? ld_stream(xv + (r0 + r) * nv + v) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const int64_t row = r0 + r;
+      if (row >= rows) break;  // warp-uniform
+      uint32_t mraw = 0;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) mraw = Dt<DT>::lmax(mraw, vec_mag<DT>(u[r][j]));
+      mraw = warp_lmax<DT>(mraw);
+      const bool nf = Dt<DT>::nonfinite(mraw);  // the same on every lane
+      float amax;
+      if (!nf) {
+        amax = Dt<DT>::value(mraw);
+      } else {  // rare: finite-only maximum on the exact path
+        amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) amax = vec_amax_exact<DT>(u[r][j], amax);
+        amax = warp_max(amax);
+      }
+      const float m = multiplier(amax, Fmt<FMT>::kMax);
+      if (lane == 0) {
+        scales[row] = __fdiv_rn(1.0f, m);
+        if (amax_out) amax_out[row] = amax;
+      }
+      uint8_t* qr = q + row * nv * VEC;
+      if (!nf) {
+#pragma unroll
+        for (int j = 0; j < VPL; ++j)
+          if (lane + 32 * j < nv) vec_store<DT, FMT, true>(qr + (lane + 32 * j) * VEC, u[r][j], m);
+      } else {
+#pragma unroll
+        for (int j = 0; j < VPL; ++j)
+          if (lane + 32 * j < nv) vec_store<DT, FMT, false>(qr + (lane + 32 * j) * VEC, u[r][j], m);
+      }
+    }
   }
 }
 
@@ -1968,6 +2040,29 @@ cudaError_t launch_tensor_fused(const QuantizeArgs& a, int dev, int64_t n, float
                                      dim3(kFusedThreads), args, smem, a.stream);
 }
 
+// Per-token rows of up to 1024 vectors: the register-resident kernel on a
+// persistent grid of as many resident CTAs as its registers allow.
+template <int DT, int FMT, int VPL, int RPW>
+cudaError_t launch_token_reg(const QuantizeArgs& a, int dev, int64_t nv) {
+  static int per_sm = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_token_reg<DT, FMT, VPL, RPW>, kRegThreads, 0) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      per_sm = 0;
+    }
+  });
+  const int64_t warps_needed = (a.rows + RPW - 1) / RPW;
+  const int64_t ctas_needed = (warps_needed + kRegThreads / 32 - 1) / (kRegThreads / 32);
+  int64_t grid = static_cast<int64_t>(device_sm_count(dev)) * std::max(per_sm, 1);
+  if (grid > ctas_needed) grid = ctas_needed;
+  if (grid < 1) grid = 1;
+  k_token_reg<DT, FMT, VPL, RPW><<<static_cast<unsigned>(grid), kRegThreads, 0, a.stream>>>(a.x, a.rows, nv, a.q,
+                                                                                           a.scales, a.amax_out);
+  return cudaGetLastError();
+}
+
 template <int DT, int FMT>
 cudaError_t launch_typed(const QuantizeArgs& a) {
   constexpr int VEC = Dt<DT>::kVec;
@@ -1991,6 +2086,15 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
   }
 
   if (a.gran == 1) {  // per-token
+    if (row_vec && a.cols > 0 && a.cols / VEC <= 32 * 32) {
+      const int64_t nv = a.cols / VEC;
+      if (nv <= 32) return launch_token_reg<DT, FMT, 1, 16>(a, dev, nv);
+      if (nv <= 64) return launch_token_reg<DT, FMT, 2, 8>(a, dev, nv);
+      if (nv <= 128) return launch_token_reg<DT, FMT, 4, 4>(a, dev, nv);
+      if (nv <= 256) return launch_token_reg<DT, FMT, 8, 2>(a, dev, nv);
+      if (nv <= 512) return launch_token_reg<DT, FMT, 16, 1>(a, dev, nv);
+      return launch_token_reg<DT, FMT, 32, 1>(a, dev, nv);
+    }
     if (row_vec && a.cols > 0) {
       // Stages of at least 32 KB (whole rows), two per CTA, as many CTAs per
       // SM as shared memory and registers allow (a sweep over stage size,

@@ -69,6 +69,27 @@ def test_quantize_bit_exact(dtype, gran, fmt):
     H.hq_check_device_error()
 
 
+# Per-token rows of up to 1024 16-byte vectors take the register-resident
+# kernel: every vectors-per-lane bucket (1, 2, 4, 8, 16, 32) with a ragged
+# vector count, row counts that are not multiples of the rows a warp takes,
+# and more rows than the resident warps (the persistent loop).
+TOKEN_REG_CASES = [((37, 8184), "bf16"), ((45, 4104), "bf16"), ((19, 1544), "bf16"), ((23, 968), "bf16"),
+                   ((11, 264), "bf16"), ((1000, 16), "bf16"), ((29, 4092), "f32"), ((9, 6000), "f16"),
+                   ((20000, 512), "bf16"), ((4000, 8192), "bf16"), ((3001, 2048), "f32")]
+
+
+@pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
+def test_per_token_register_kernel(fmt):
+    for i, (shape, dtype) in enumerate(TOKEN_REG_CASES):
+        xh, xd = make_input(shape, dtype, seed=7000 + 10 * i + fmt)
+        q, s, a = run_gpu(xd, fmt, O.PER_TOKEN)
+        qo, so, ao = O.quantize(xh, fmt, O.PER_TOKEN)
+        np.testing.assert_array_equal(q, qo, err_msg="codes %s %s" % (shape, dtype))
+        np.testing.assert_array_equal(s.view(np.uint32), so.view(np.uint32), err_msg="scales %s" % (shape,))
+        np.testing.assert_array_equal(a.view(np.uint32), ao.view(np.uint32), err_msg="amax %s" % (shape,))
+    H.hq_check_device_error()
+
+
 @pytest.mark.parametrize("gran", [O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL])
 def test_misaligned_input_takes_scalar_path(gran):
     # x starting 2 bytes into an allocation: no 16-byte vectors possible
