@@ -285,7 +285,8 @@ def build(args, cfg, rank, dev, stream, peaks):
         l2 = "inputs larger than L2 (W %d MB, X %d MB, out %d MB); no flush" % (N * K * 2 >> 20, M * K * 2 >> 20,
                                                                                M * N * 2 >> 20)
         return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=h2d, d2h=M * N * 2,
-                    roofline=roofline, extras=extras, l2=l2, flush=None)
+                    roofline=roofline, extras=extras, l2=l2, flush=None,
+                    tensors=dict(xq=xq, wq=wq, xs=xs, ws=ws))
 
     if kind == "blockscaled":
         blk = cfg["block"]
@@ -663,6 +664,111 @@ def build(args, cfg, rank, dev, stream, peaks):
                    (M * K * 2 >> 20, E * N * K * (1 if kind == "moe" else 2) >> 20, M * N * 2 >> 20))
 
 
+def time_workload(wl, steps, warmup, stream, world, dev, hq):
+    """Warm-up, then exactly `steps` steps bracketed by a barrier and a device
+    synchronise, with CUDA events on the launching stream around every call
+    and clocks sampled during the timed region.  Returns the per-call mean
+    times, the timed region's milliseconds (max over ranks) and the clocks."""
+    import torch
+    import torch.distributed as dist
+
+    calls = wl["calls"]
+
+    def step(ev=None):
+        for j, (_, fn, _) in enumerate(calls):
+            if wl["flush"] is not None:
+                wl["flush"]()
+            if ev is not None:
+                ev[2 * j].record(stream)
+            fn()
+            if ev is not None:
+                ev[2 * j + 1].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    hq.hq_check_device_error()
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(calls))] for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    hq.hq_check_device_error()
+    ms_by = {c[0]: statistics.mean(e[2 * j].elapsed_time(e[2 * j + 1]) for e in evs) for j, c in enumerate(calls)}
+    region = t0.elapsed_time(t1)
+    if wl["flush"] is not None:  # flushes sit between the calls: time the calls alone
+        region = sum(sum(e[2 * j].elapsed_time(e[2 * j + 1]) for j in range(len(calls))) for e in evs)
+    return ms_by, max_over_ranks(region, world, dev), clk
+
+
+# Workloads measured beside the default one, in the same process, so that its
+# line carries the whole metric: the quantize sweep, the grouped MoE GEMMs and
+# the delayed-scaling stack step (steps per workload).
+COMPANIONS = (("sweep", 10), ("moe", 20), ("moe_bf16", 20), ("stack", 200))
+
+
+def companion_line(args, name, steps, rank, world, dev, stream, peaks, hq):
+    import torch
+
+    cfg = WORKLOADS[name]
+    sub = argparse.Namespace(**dict(vars(args), workload=name))
+    wl = build(sub, cfg, rank, dev, stream, peaks)
+    ms_by, ms, clk = time_workload(wl, steps, 5, stream, world, dev, hq)
+    scale = 1e12 if wl["unit"] == "TFLOP/s" else 1e9
+    d = {"workload": workload_desc(name, cfg), "value": round(wl["per_step"] * steps * world / (ms / 1e3) / scale, 2),
+         "unit": wl["unit"], "steps": steps, "warmup": 5, "ms_per_step": round(ms / steps, 4),
+         "roofline": wl["roofline"](ms_by), "call_ms": {k: round(v, 4) for k, v in ms_by.items()},
+         "l2": wl["l2"], "gpu_launches": sum(c[2] for c in wl["calls"]) * steps,
+         "clocks": {"sm_mhz": clk.get("sm_mhz"), "reasons": clk.get("reasons")}}
+    d.update(wl["extras"](ms_by))
+    wl.pop("graphs", None)
+    del wl
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return d
+
+
+def scaled_mm_ceiling(t, M, N, K, stream, fp8_peak, reps=10):
+    """torch._scaled_mm (a library FP8 GEMM with row-wise scales) on the same
+    codes and scales, timed with CUDA events: a stated ceiling for the large
+    layer's GEMM, not part of the measured path."""
+    import torch
+
+    try:
+        a = t["xq"].view(torch.float8_e4m3fn)
+        b = t["wq"].view(torch.float8_e4m3fn).t()  # [K, N], column-major
+        sa, sb = t["xs"].view(M, 1), t["ws"].view(1, N)
+        for _ in range(3):
+            out = torch._scaled_mm(a, b, scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            out = torch._scaled_mm(a, b, scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        del out
+        tf = 2.0 * M * N * K / (ms / 1e3) / 1e12
+        return {"op": "torch._scaled_mm, E4M3 row-wise scales, bf16 out (library GEMM; a ceiling, not a target)",
+                "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_of_fp8_peak": round(tf / fp8_peak, 4),
+                "reps": reps}
+    except Exception as exc:  # the ceiling is context only: record why it is missing
+        return {"op": "torch._scaled_mm", "unavailable": "%s: %s" % (type(exc).__name__, str(exc).splitlines()[0])}
+
+
 def run_ours(args, rank, local_rank, world):
     import torch
     import torch.distributed as dist
@@ -680,44 +786,7 @@ def run_ours(args, rank, local_rank, world):
     stream = torch.cuda.current_stream(dev)
     wl = build(args, cfg, rank, dev, stream, peaks)
     calls = wl["calls"]
-
-    def step(ev=None):
-        for j, (_, fn, _) in enumerate(calls):
-            if wl["flush"] is not None:
-                wl["flush"]()
-            if ev is not None:
-                ev[2 * j].record(stream)
-            fn()
-            if ev is not None:
-                ev[2 * j + 1].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    hq.hq_check_device_error()
-
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(calls))] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    hq.hq_check_device_error()
-    ms_by = {c[0]: statistics.mean(e[2 * j].elapsed_time(e[2 * j + 1]) for e in evs) for j, c in enumerate(calls)}
-    region = t0.elapsed_time(t1)
-    if wl["flush"] is not None:  # flushes sit between the calls: time the calls alone
-        region = sum(sum(e[2 * j].elapsed_time(e[2 * j + 1]) for j in range(len(calls))) for e in evs)
-    ms = max_over_ranks(region, world, dev)
+    ms_by, ms, clk = time_workload(wl, args.steps, args.warmup, stream, world, dev, hq)
     scale = 1e12 if wl["unit"] == "TFLOP/s" else 1e9
     value = wl["per_step"] * args.steps * world / (ms / 1e3) / scale
 
@@ -738,6 +807,15 @@ def run_ours(args, rank, local_rank, world):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = wl["per_step"] * e2e_steps * world / (e2e_ms / 1e3) / scale
 
+    # the default workload's line also carries the rest of the metric
+    also = None
+    if args.workload == "large" and not args.no_companions:
+        fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+        also = {"scaled_mm_ceiling": scaled_mm_ceiling(wl["tensors"], cfg["M"], cfg["N"], cfg["K"], stream,
+                                                       fp8_peak)}
+        for name, steps in COMPANIONS:
+            also[name] = companion_line(args, name, steps, rank, world, dev, stream, peaks, hq)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and cfg["kind"] in ("layer", "decode"):
         mx = min(256, cfg["M"])
@@ -755,6 +833,8 @@ def run_ours(args, rank, local_rank, world):
         cpu = {"value": byts / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": "%d rows x %d cols of the workload's input, every call of the step, %.1f s"
                          % (rows, cfg["K"], dt), "seconds": round(dt, 2)}
+    if cpu is not None:
+        cpu["host"] = host_cpu()
 
     wl.pop("graphs", None)  # release captured graphs before the process group goes
     if world > 1:
@@ -787,14 +867,36 @@ def run_ours(args, rank, local_rank, world):
         "cpu_baseline": cpu,
     }
     line.update(wl["extras"](ms_by))
+    if also is not None:
+        line["also"] = also
     print(json.dumps(line))
 
 
+def host_cpu():
+    """The host's logical CPU count, the CPUs this process may use, and the
+    CPU model name."""
+    model = None
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count()
+    return {"nproc": os.cpu_count(), "usable": usable, "model": model}
+
+
 # --------------------------------------------------------------- oracle
-def cpu_baseline(M, N, K, budget_rows, seed=0):
+def cpu_baseline(M, N, K, budget_rows, seed=0, all_cores=True):
     """The oracle, as it stands, on a bounded sample of the workload: per-token
     quantize of `mx` rows of X and `nw` rows of W, then the exact GEMM of the
-    sample.  Returns TFLOP/s of the sample's GEMM flops per oracle time."""
+    sample.  Returns TFLOP/s of the sample's GEMM flops per oracle time: on
+    one core, and (all_cores) on every usable core, each thread running the
+    unchanged single-threaded oracle on its own slice of rows."""
     import oracle as O
     import workloads as W
     mx, nw = budget_rows
@@ -808,10 +910,36 @@ def cpu_baseline(M, N, K, budget_rows, seed=0):
     O.gemm_a8w8(xq, wq, O.E4M3, xs, ws)
     dt = time.perf_counter() - t
     flops = 2.0 * mx * nw * K
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": "X %d rows x W %d rows (K=%d): per-token quantize of both + exact GEMM, %.1f s"
-                      % (mx, nw, K, dt),
-            "seconds": round(dt, 2)}
+    d = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+         "sample": "X %d rows x W %d rows (K=%d): per-token quantize of both + exact GEMM, %.1f s"
+                   % (mx, nw, K, dt),
+         "seconds": round(dt, 2)}
+    if not all_cores:
+        return d
+    import concurrent.futures as cf
+    try:
+        threads = len(os.sched_getaffinity(0))
+    except AttributeError:
+        threads = os.cpu_count() or 1
+
+    def slices(n):
+        step = -(-n // threads)
+        return [(i, min(n, i + step)) for i in range(0, n, step)]
+
+    t = time.perf_counter()
+    with cf.ThreadPoolExecutor(threads) as ex:  # the oracle's C calls release the GIL
+        xp = list(ex.map(lambda r: O.quantize(x[r[0]:r[1]], O.E4M3, O.PER_TOKEN), slices(mx)))
+        wp = list(ex.map(lambda r: O.quantize(w[r[0]:r[1]], O.E4M3, O.PER_TOKEN), slices(nw)))
+        xq2, xs2 = np.concatenate([p[0] for p in xp]), np.concatenate([p[1] for p in xp])
+        wq2, ws2 = np.concatenate([p[0] for p in wp]), np.concatenate([p[1] for p in wp])
+        list(ex.map(lambda r: O.gemm_a8w8(xq2[r[0]:r[1]], wq2, O.E4M3, xs2[r[0]:r[1]], ws2), slices(mx)))
+    dta = time.perf_counter() - t
+    single = dict(d)
+    d.update({"value": flops / dta / 1e12, "cores": threads, "seconds": round(dta, 2),
+              "sample": "the same sample on %d threads (each runs the single-threaded oracle on a slice of rows), "
+                        "%.1f s" % (threads, dta),
+              "single_core": {"value": single["value"], "seconds": single["seconds"], "cores": 1}})
+    return d
 
 
 def cpu_blockscaled_sample(M, N, K, block, budget_rows, seed=0):
@@ -932,6 +1060,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="large")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-companions", action="store_true",
+                    help="default workload only: skip the sweep / MoE / stack lines and the library ceiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
