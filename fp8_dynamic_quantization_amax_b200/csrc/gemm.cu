@@ -23,6 +23,7 @@
 // device word, drains what it has in flight and exits instead of hanging.
 #include "fp8_cvt.cuh"
 #include "hq_internal.cuh"
+#include "launch.cuh"
 #include "ptx.cuh"
 #include "tc.cuh"
 
@@ -89,6 +90,35 @@ __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, ui
   asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// Two columns at once with packed f32x2 arithmetic: (a0, a1) * (x * s0,
+// x * s1), each product rounded once (the same operations, in the same
+// order, as the scalar form), plus the bias pair (b0, b1) by one fused
+// multiply-add each when with_bias.
+__device__ __forceinline__ void scale2(float a0, float a1, float s0, float s1, float x, float& r0, float& r1) {
+  asm("{\n\t.reg .b64 a, s, xx;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 s, {%4, %5};\n\t"
+      "mov.b64 xx, {%6, %6};\n\t"
+      "mul.rn.f32x2 s, s, xx;\n\t"
+      "mul.rn.f32x2 a, a, s;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(s0), "f"(s1), "f"(x));
+}
+__device__ __forceinline__ void scale2_bias(float a0, float a1, float s0, float s1, float x, float b0, float b1,
+                                            float& r0, float& r1) {
+  asm("{\n\t.reg .b64 a, s, xx, b;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 s, {%4, %5};\n\t"
+      "mov.b64 xx, {%6, %6};\n\t"
+      "mov.b64 b, {%7, %8};\n\t"
+      "mul.rn.f32x2 s, s, xx;\n\t"
+      "fma.rn.f32x2 a, a, s, b;\n\t"
+      "mov.b64 {%0, %1}, a;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(s0), "f"(s1), "f"(x), "f"(b0), "f"(b1));
+}
+
 // One chunk's 32 scaled values of a lane's row, plus the bias (bias != null),
 // rounded to bf16 pairs: w[j] holds columns n0 + 2j (low half) and n0 + 2j + 1.
 // has_acc == false (K == 0) reads the accumulator as zero.
@@ -99,7 +129,9 @@ __device__ __forceinline__ void chunk_to_bf16(const uint32_t (&v)[32], bool has_
     for (int j = 0; j < 16; ++j) {
       const float a0 = has_acc ? __uint_as_float(v[2 * j]) : 0.0f;
       const float a1 = has_acc ? __uint_as_float(v[2 * j + 1]) : 0.0f;
-      w[j] = pack_bf16x2(a0 * (xsv * sc[2 * j]), a1 * (xsv * sc[2 * j + 1]));
+      float r0, r1;
+      scale2(a0, a1, sc[2 * j], sc[2 * j + 1], xsv, r0, r1);
+      w[j] = pack_bf16x2(r0, r1);
     }
   } else {
     const uint32_t* bp = reinterpret_cast<const uint32_t*>(bias) + (n0 >> 1);
@@ -108,18 +140,19 @@ __device__ __forceinline__ void chunk_to_bf16(const uint32_t (&v)[32], bool has_
       const float a0 = has_acc ? __uint_as_float(v[2 * j]) : 0.0f;
       const float a1 = has_acc ? __uint_as_float(v[2 * j + 1]) : 0.0f;
       const uint32_t bb = (n0 + 2 * j < N) ? __ldg(bp + j) : 0u;
-      w[j] = pack_bf16x2(__fmaf_rn(a0, xsv * sc[2 * j], __uint_as_float(bb << 16)),
-                         __fmaf_rn(a1, xsv * sc[2 * j + 1], __uint_as_float(bb & 0xFFFF0000u)));
+      float r0, r1;
+      scale2_bias(a0, a1, sc[2 * j], sc[2 * j + 1], xsv, __uint_as_float(bb << 16), __uint_as_float(bb & 0xFFFF0000u),
+                  r0, r1);
+      w[j] = pack_bf16x2(r0, r1);
     }
   }
 }
 
 // FP8 output of one chunk: codes of f32(bf16 value) * m, saturating RNE (NaN
-// -> 0x7F); the lane's finite-only amax is updated over its valid columns
-// and the chunk's codes are stored at the lane's row (qout + row * N + n0).
-__device__ __forceinline__ void chunk_to_fp8(const uint32_t (&w)[16], int qfmt, float qm, bool vrow, uint8_t* qrow,
-                                             int n0, int N, float& qam) {
-  uint32_t c4[8];
+// -> 0x7F), into c4 (the lane's 32 codes, column n0 in the low byte of
+// c4[0]); the lane's finite-only amax is updated over its valid columns.
+__device__ __forceinline__ void chunk_to_fp8(const uint32_t (&w)[16], int qfmt, float qm, bool vrow, int n0, int N,
+                                             float& qam, uint32_t (&c4)[8]) {
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const float lo = __uint_as_float(w[j] << 16);
@@ -128,10 +161,6 @@ __device__ __forceinline__ void chunk_to_fp8(const uint32_t (&w)[16], int qfmt, 
     const uint32_t c2 = (qfmt == 0) ? cvt2_exact<0>(__fmul_rn(lo, qm), __fmul_rn(hi, qm))
                                     : cvt2_exact<1>(__fmul_rn(lo, qm), __fmul_rn(hi, qm));
     c4[j >> 1] = (j & 1) ? (c4[j >> 1] | (c2 << 16)) : c2;
-  }
-  if (vrow) {  // N % 16 == 0 and n0 % 32 == 0: 16 or 32 codes of this chunk lie inside the row
-    st_global_v4(qrow + n0, c4[0], c4[1], c4[2], c4[3]);
-    if (n0 + 32 <= N) st_global_v4(qrow + n0 + 16, c4[4], c4[5], c4[6], c4[7]);
   }
 }
 
@@ -198,6 +227,79 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
+}
+
+// ------------------------------------------------------------ epilogue
+// One epilogue warp's share of a tile: chunks half, half + 2, ... of 32
+// columns (chunk j's scales at wsh + 32 j), read from TMEM at tacc (the
+// warp's lane quadrant and the accumulator's first column).  Per chunk the
+// warp scales (+ bias) and rounds to bf16, then writes either the FP8 codes,
+// or the 32 x 32 chunk through its staging tile with one TMA store (rows
+// inside the tile's valid rows, a whole chunk inside the tile), or masked
+// 16-byte stores.
+template <int KIND, int kChunks>
+__device__ __forceinline__ void epilogue_chunks(uint32_t tacc, int half, int lane, int col0, int col_end, int tile_end,
+                                                int row0, bool vrow, bool tma_ok, bool has_acc, float xsv,
+                                                const float* wsh, const Params& p, const uint16_t* bias, uint16_t* orow,
+                                                uint8_t* qrow, float qm, float& qam, uint8_t* sb,
+                                                const CUtensorMap* tm_out, uint64_t out_pol) {
+  auto process = [&](const uint32_t (&v)[32], int j) {
+    const int n0 = col0 + (half + 2 * j) * 32;
+    if (n0 >= col_end) return;
+    uint32_t w[16];
+    chunk_to_bf16(v, has_acc, xsv, wsh + j * 32, bias, n0, p.N, w);
+    if (KIND == 0 && qrow != nullptr) {
+      uint32_t c4[8];
+      chunk_to_fp8(w, p.qfmt, qm, vrow, n0, p.N, qam, c4);
+      if (tma_ok && n0 + 32 <= tile_end) {
+        // the 32 x 32 codes through the staging tile, 32-byte rows with the
+        // 32-byte swizzle: 16-byte half h of row r sits at h ^ ((r >> 2) & 1)
+        if (lane == 0) bulk_wait_read_le0();
+        __syncwarp();
+        const uint32_t flip = (static_cast<uint32_t>(lane) >> 2) & 1u;
+        st_shared_v4(sb + lane * 32 + (flip << 4), c4[0], c4[1], c4[2], c4[3]);
+        st_shared_v4(sb + lane * 32 + ((flip ^ 1u) << 4), c4[4], c4[5], c4[6], c4[7]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tm_out, sb, n0, row0, out_pol);
+          bulk_commit_group();
+        }
+      } else if (vrow) {  // N % 16 == 0 and n0 % 32 == 0: 16 or 32 codes of this chunk lie inside the row
+        st_global_v4(qrow + n0, c4[0], c4[1], c4[2], c4[3]);
+        if (n0 + 32 <= p.N) st_global_v4(qrow + n0 + 16, c4[4], c4[5], c4[6], c4[7]);
+      }
+      return;
+    }
+    // the tensor map clips at M and N; a 16-column tail chunk inside N is masked
+    if (tma_ok && n0 + 32 <= tile_end) {
+      if (lane == 0) bulk_wait_read_le0();  // the previous chunk's store has read the staging tile
+      __syncwarp();
+      // the staging tile is the 64-byte-swizzled image of the 32 x 32 box:
+      // 16-byte chunk k of row r sits at chunk k ^ ((r >> 1) & 3), which
+      // spreads each quarter-warp's stores over all banks
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        st_shared_v4(sb + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2],
+                     w[4 * k + 3]);
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tm_out, sb, n0, row0, out_pol);
+        bulk_commit_group();
+      }
+    } else if (vrow) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (n0 + 8 * k < col_end) st_global_v4(orow + n0 + 8 * k, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    }
+  };
+#pragma unroll 1
+  for (int j = 0; half + 2 * j < kChunks; ++j) {
+    uint32_t v[32];
+    tmem_ld32(tacc + static_cast<uint32_t>((half + 2 * j) * 32), v);
+    process(v, j);
+  }
 }
 
 // ------------------------------------------------------------ tile schedule
@@ -337,6 +439,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     abort_flag = 0;
     ptx::fence_mbarrier_init();
   }
+  pdl_wait();  // launched with programmatic stream serialization: global memory only after this
   if (threadIdx.x == 32 && p.offsets != nullptr) build_tile_prefix<kBM>(p, tile_prefix, row_start);
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
@@ -407,11 +510,13 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++i) {
       const int acc = i & 1;
       const uint32_t acc_phase = (i >> 1) & 1;
-      if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) break;
+      // the warp agrees on giving up a wait, so that no lane is left at a
+      // warp-wide step after another has left
+      if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag))) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
       for (int kb = 0; kb < p.nkb; kb += KPS) {
-        if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { stop = true; break; }
+        if (__any_sync(0xFFFFFFFFu, !mbar_wait(&full_bar[stage], phase, &abort_flag))) { stop = true; break; }
         tc_fence_after();
         if (lane == 0) {
           const int nsub = min(KPS, p.nkb - kb);
@@ -459,7 +564,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int acc = i & 1;
       const uint32_t acc_phase = (i >> 1) & 1;
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag)) break;
+      // the warp agrees on giving up: the TMEM loads below are warp-wide
+      if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag))) break;
       tc_fence_after();
       const Tile T = decode_tile<kBM, BN>(t, p, tile_prefix, row_start);
       const int row0 = T.row_lo + quad * 32;
@@ -482,41 +588,10 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
-#pragma unroll 1
-      for (int i = 0; half + 2 * i < kChunks; ++i) {
-        const int c = (half + 2 * i) * 32;  // chunk's first column within the tile
-        uint32_t v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride +
-                      static_cast<uint32_t>(c),
-                  v);
-        const int n0 = T.col0 + c;
-        if (n0 >= ncap) continue;
-        const float* sc = wsh + i * 32;
-        uint32_t w[16];
-        chunk_to_bf16(v, has_acc, xsv, sc, bias, n0, p.N, w);
-        if (KIND == 0 && qrow != nullptr) {
-          chunk_to_fp8(w, p.qfmt, qm, vrow, qrow, n0, p.N, qam);
-          continue;
-        }
-        // the tensor map clips at N; a 16-column tail chunk inside N is masked
-        if (tma_ok && (BN % 32 == 0 || n0 + 32 <= T.col0 + BN)) {
-          if (lane == 0) bulk_wait_read_le0();  // the previous chunk's store has read the staging tile
-          __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            st_shared_v4(sb + lane * 64 + k * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tm_out, sb, n0, row0, out_pol);
-            bulk_commit_group();
-          }
-        } else if (vrow) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (n0 + 8 * k < ncap) st_global_v4(orow + n0 + 8 * k, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-        }
-      }
+      epilogue_chunks<KIND, kChunks>(
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride, half, lane,
+          T.col0, ncap, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qam, sb, &tm_out,
+          out_pol);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[acc]);
@@ -536,7 +611,9 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
 }
 
 // --------------------------------------------------------------- host side
-// bf16 out[M, N] for TMA stores: 32 x 32 boxes, no swizzle.
+// bf16 out[M, N] for TMA stores: 32 x 32 boxes (64-byte rows) with the
+// 64-byte swizzle, so that the epilogue's staging stores avoid bank
+// conflicts.
 bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, std::string* msg) {
   auto encode = get_encode_fn();
   if (!encode) {
@@ -548,7 +625,7 @@ bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, st
   cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     char buf[128];
@@ -559,12 +636,34 @@ bool make_out_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, st
   return true;
 }
 
-// The bf16 output's tensor map.  With an FP8 output the kernels store no bf16
-// tile; the map then describes the code buffer (M rows of N bytes) so that it
-// still names memory the call owns.
+// FP8 codes out[M, N] (N % 16 == 0) for TMA stores: 32 x 32 boxes (32-byte
+// rows) with the 32-byte swizzle.
+bool make_codes_map(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, std::string* msg) {
+  auto encode = get_encode_fn();
+  if (!encode) {
+    *msg = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[128];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (%d) for the FP8 output", static_cast<int>(r));
+    *msg = buf;
+    return false;
+  }
+  return true;
+}
+
+// The output's tensor map: the bf16 out, or the FP8 codes with an FP8 output.
 bool make_result_map(CUtensorMap* map, const GemmArgs& a, std::string* msg) {
   if (a.q_out != nullptr)
-    return make_out_map(map, a.q_out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N / 2), msg);
+    return make_codes_map(map, a.q_out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), msg);
   return make_out_map(map, a.out, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), msg);
 }
 
@@ -643,8 +742,8 @@ cudaError_t run(const GemmArgs& a, std::string* msg) {
     tiles_bound = (static_cast<int64_t>(p.m_tiles) + a.E) * p.n_tiles;
   int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
   if (grid < 1) grid = 1;
-  k_gemm<KIND, BN, STAGES, AROWS, KPS><<<grid, kGemm1Threads, kSmem, a.stream>>>(ta, tb, to, p);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm<KIND, BN, STAGES, AROWS, KPS>, dim3(grid), dim3(kGemm1Threads), kSmem, a.stream, false,
+                    ta, tb, to, p);
 }
 
 // ====================================================== 2-CTA pair kernel
@@ -705,26 +804,31 @@ __device__ __forceinline__ void mma_issue_pair(uint32_t d_tmem, uint64_t adesc, 
   }
 }
 
-// BN = 256 * NSUB columns per pair tile.  NSUB = 1: two accumulators, so tile
-// i's epilogue overlaps tile i+1's main loop.  NSUB = 2: each K step issues two
-// N=256 MMAs against the same A stage (a quarter fewer operand bytes per
-// flop) into one 512-column accumulator; the epilogue then does not overlap.
-template <int KIND, int BN, int STAGES>
+// BN = SUBN * NSUB columns per pair tile; one MMA per sub-tile per K step
+// (M = 256 across the pair, N = SUBN), each CTA holding SUBN/2 rows of every
+// sub-tile of B.  When two BN-column accumulators fit in TMEM (BN <= 256),
+// tile i's epilogue overlaps tile i+1's main loop.  NSUB = 2: each K step issues two
+// MMAs against the same A stage (fewer operand bytes per flop) into one
+// accumulator of up to 512 columns; the epilogue then does not overlap.
+template <int KIND, int SUBN, int NSUB, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_gemm2(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
             const __grid_constant__ CUtensorMap tm_out, const Params p) {
-  static_assert(BN == 256 || BN == 512, "pair tile width: 256 or 512 columns");
-  constexpr int NSUB = BN / 256;
-  constexpr int kABytes = 128 * kBKBytes;  // this CTA's 128 rows of A
-  constexpr int kBSub = 128 * kBKBytes;    // this CTA's 128 rows of one 256-column sub-tile of B
+  constexpr int BN = SUBN * NSUB;
+  static_assert(SUBN % 16 == 0 && SUBN >= 32 && SUBN <= 256, "MMA N (M = 256 across the pair): 16 .. 256, step 16");
+  static_assert((SUBN / 2) % 8 == 0, "each CTA's half of a sub-tile keeps whole 1024-byte swizzle atoms");
+  static_assert(BN % 32 == 0 && BN <= 512, "32-column epilogue chunks; at most the 512 TMEM columns");
+  constexpr int kABytes = 128 * kBKBytes;           // this CTA's 128 rows of A
+  constexpr int kBSub = (SUBN / 2) * kBKBytes;      // this CTA's SUBN/2 rows of one sub-tile of B
   constexpr int kBBytes = NSUB * kBSub;
   constexpr int kStageBytes = kABytes + kBBytes;
   constexpr int kKElems = (KIND == 0) ? 128 : 64;
-  constexpr int kAccs = (NSUB == 1) ? 2 : 1;  // accumulators in TMEM
+  constexpr int kAccs = (2 * BN <= 512) ? 2 : 1;  // accumulators in TMEM
   constexpr uint32_t kTmemCols = 512u;
   constexpr uint32_t kAccStride = 256u;
-  constexpr int kPrefetch = 2 * STAGES;  // L2 prefetch distance for B, in K blocks
-  constexpr int kMyChunks = BN / 64;     // 32-column chunks per epilogue warp (two warps per quadrant)
+  constexpr int kPrefetch = 2 * STAGES;           // L2 prefetch distance for B, in K blocks
+  constexpr int kChunks = BN / 32;                // 32-column epilogue chunks
+  constexpr int kMyChunks = (kChunks + 1) / 2;    // per epilogue warp (two warps per quadrant)
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -764,6 +868,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     ptx::fence_mbarrier_init();
   }
   // each CTA of the pair builds the same tile prefix from the device offsets
+  pdl_wait();  // launched with programmatic stream serialization: global memory only after this
   if (threadIdx.x == 32 && p.offsets != nullptr) build_tile_prefix<256>(p, tile_prefix, row_start);
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
@@ -797,7 +902,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // rows past the tile's own (another expert's, or past M) only reach
         // accumulator rows that are never stored
         const int a_row = T.a_row + static_cast<int>(rank) * 128;
-        const int b_row = T.b_row + static_cast<int>(rank) * 128;  // + 256 per sub-tile
+        const int b_row = T.b_row + static_cast<int>(rank) * (SUBN / 2);  // + SUBN per sub-tile
         for (int kb = 0; kb < p.nkb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { stop = true; break; }
           const uint32_t full_leader = mapa_shared(smem_u32(&full_bar[stage]), 0);
@@ -805,13 +910,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tma_load_2d_pair(sA + stage * kABytes, &tm_a, full_leader, kb * kKElems, a_row);
 #pragma unroll
           for (int s = 0; s < NSUB; ++s)
-            tma_load_2d_pair(sB + stage * kBBytes + s * kBSub, &tm_b, full_leader, kb * kKElems, b_row + 256 * s);
+            tma_load_2d_pair(sB + stage * kBBytes + s * kBSub, &tm_b, full_leader, kb * kKElems, b_row + SUBN * s);
           // The clusters that share this B tile run in step, so its DRAM
           // latency would stall all of them at once: ask L2 for the B tile
           // kPrefetch blocks ahead.
           if (kb + kPrefetch < p.nkb) {
 #pragma unroll
-            for (int s = 0; s < NSUB; ++s) tma_prefetch_2d(&tm_b, (kb + kPrefetch) * kKElems, b_row + 256 * s);
+            for (int s = 0; s < NSUB; ++s) tma_prefetch_2d(&tm_b, (kb + kPrefetch) * kKElems, b_row + SUBN * s);
           }
           pend_mask |= 1u << stage;
           pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
@@ -836,11 +941,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int t = cluster; t < total && !stop; t += nclusters, ++i) {
         const int acc = i % kAccs;
         const uint32_t acc_phase = (i / kAccs) & 1;
-        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) break;
+        // the warp agrees on giving up a wait, so that no lane is left at a
+        // warp-wide step after another has left
+        if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc) * kAccStride;
         for (int kb = 0; kb < p.nkb; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { stop = true; break; }
+          if (__any_sync(0xFFFFFFFFu, !mbar_wait(&full_bar[stage], phase, &abort_flag))) { stop = true; break; }
           tc_fence_after();
           if (lane == 0) {
             const uint64_t ad = smem_desc(smem_u32(sA + stage * kABytes));
@@ -849,7 +956,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int s = 0; s < NSUB; ++s) {
                 const uint64_t bd = smem_desc(smem_u32(sB + stage * kBBytes + s * kBSub));
-                mma_issue_pair<KIND>(d_tmem + 256u * s, ad + 2u * k, bd + 2u * k, p.idesc,
+                mma_issue_pair<KIND>(d_tmem + static_cast<uint32_t>(SUBN * s), ad + 2u * k, bd + 2u * k, p.idesc,
                                      (kb > 0 || k > 0) ? 1u : 0u);
               }
             tc_commit_pair(&empty_bar[stage]);
@@ -893,7 +1000,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int t = cluster; t < total; t += nclusters, ++i) {
       const int acc = i % kAccs;
       const uint32_t acc_phase = (i / kAccs) & 1;
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag)) break;
+      // the warp agrees on giving up: the TMEM loads below are warp-wide
+      if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag))) break;
       tc_fence_after();
       const Tile T = decode_tile<256, BN>(t, p, tile_prefix, row_start);
       const int row0 = T.row_lo + static_cast<int>(rank) * 128 + quad * 32;  // this warp's first row
@@ -906,50 +1014,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (KIND == 0) {
         const float* wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
 #pragma unroll 1
-        for (int j = 0; j < kMyChunks; ++j) {
+        for (int j = 0; half + 2 * j < kChunks; ++j) {
           const int n = T.col0 + (half + 2 * j) * 32 + lane;
           wsh[j * 32 + lane] = (n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f;
         }
       } else {
-        for (int j = 0; j < kMyChunks; ++j) wsh[j * 32 + lane] = 1.0f;
+        for (int j = 0; half + 2 * j < kChunks; ++j) wsh[j * 32 + lane] = 1.0f;
       }
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
-#pragma unroll 1
-      for (int j = 0; j < kMyChunks; ++j) {
-        const int c = (half + 2 * j) * 32;  // chunk's first column within the tile
-        uint32_t v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride +
-                      static_cast<uint32_t>(c),
-                  v);
-        const int n0 = T.col0 + c;
-        if (n0 >= p.N) continue;
-        const float* sc = wsh + j * 32;
-        uint32_t w[16];
-        chunk_to_bf16(v, has_acc, xsv, sc, bias, n0, p.N, w);
-        if (KIND == 0 && qrow != nullptr) {
-          chunk_to_fp8(w, p.qfmt, qm, vrow, qrow, n0, p.N, qam);
-          continue;
-        }
-        if (tma_ok) {
-          if (lane == 0) bulk_wait_read_le0();  // the previous chunk's store has read the staging tile
-          __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            st_shared_v4(sb + lane * 64 + k * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tm_out, sb, n0, row0, out_pol);
-            bulk_commit_group();
-          }
-        } else if (vrow) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (n0 + 8 * k < p.N) st_global_v4(orow + n0 + 8 * k, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-        }
-      }
+      epilogue_chunks<KIND, kChunks>(
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride, half, lane,
+          T.col0, p.N, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qam, sb, &tm_out,
+          out_pol);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -969,16 +1047,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-template <int KIND, int BN, int STAGES>
+template <int KIND, int SUBN, int NSUB, int STAGES>
 cudaError_t run2(const GemmArgs& a, std::string* msg) {
+  constexpr int BN = SUBN * NSUB;
   constexpr int kElem = (KIND == 0) ? 1 : 2;
-  constexpr int kSmem = STAGES * (128 + BN / 2) * kBKBytes + 8 * 2048 + 8 * (BN / 64) * 32 * 4 + 1024;
+  constexpr int kSmem =
+      STAGES * (128 + BN / 2) * kBKBytes + 8 * 2048 + 8 * ((BN / 32 + 1) / 2) * 32 * 4 + 1024;
   static_assert(kSmem + 8400 <= 232448, "shared memory over the 227 KB per-CTA limit");
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_clusters = 0;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_gemm2<KIND, BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    attr_err =
+        cudaFuncSetAttribute(k_gemm2<KIND, SUBN, NSUB, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(148, 1, 1);
@@ -991,7 +1072,7 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
     attr.val.clusterDim.z = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, k_gemm2<KIND, BN, STAGES>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, k_gemm2<KIND, SUBN, NSUB, STAGES>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       max_clusters = 0;
     }
@@ -1006,7 +1087,7 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
   if (a.K > 0) {
     if (!make_map(&ta, a.a, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.K), kElem, 128, msg) ||
         !make_map(&tb, a.b, static_cast<uint64_t>(a.E) * static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.K),
-                  kElem, 128, msg))
+                  kElem, SUBN / 2, msg))
       return cudaErrorInvalidValue;
   }
   CUtensorMap to;
@@ -1029,8 +1110,8 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
   p.out = static_cast<uint16_t*>(a.out);
   set_fused_epilogue(a, p);
   const uint32_t ab_fmt = (KIND == 0) ? static_cast<uint32_t>(a.fmt) : 1u;
-  p.idesc = (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
-            (static_cast<uint32_t>(256 >> 4) << 24);  // one MMA: M = 256 across the pair, N = 256
+  p.idesc = (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (static_cast<uint32_t>(SUBN >> 3) << 17) |
+            (static_cast<uint32_t>(256 >> 4) << 24);  // one MMA: M = 256 across the pair, N = SUBN
   int dev = 0;
   cudaGetDevice(&dev);
   int clusters = device_sm_count(dev) / 2;
@@ -1039,8 +1120,8 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
   const int64_t tiles = static_cast<int64_t>(p.m_tiles + (a.offsets != nullptr ? a.E : 0)) * p.n_tiles;
   if (tiles < clusters) clusters = static_cast<int>(tiles);
   if (clusters < 1) clusters = 1;
-  k_gemm2<KIND, BN, STAGES><<<2 * clusters, kGemmThreads, kSmem, a.stream>>>(ta, tb, to, p);
-  return cudaGetLastError();
+  return launch_pdl(k_gemm2<KIND, SUBN, NSUB, STAGES>, dim3(2 * clusters), dim3(kGemmThreads), kSmem, a.stream,
+                    false, ta, tb, to, p);
 }
 
 }  // namespace
@@ -1054,13 +1135,13 @@ cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
   const bool pair = a.offsets == nullptr && a.kind == 0 && (a.N % 256 == 0) && a.N >= 2048 && a.M >= 512;
   // 256 x 512 pair tiles read a quarter fewer operand bytes per flop; with
   // enough M their coarser last round costs little
-  if (pair && a.N % 512 == 0 && a.M >= 8192) return run2<0, 512, 4>(a, msg);
-  if (pair) return run2<0, 256, 6>(a, msg);
+  if (pair && a.N % 512 == 0 && a.M >= 8192) return run2<0, 256, 2, 4>(a, msg);
+  if (pair) return run2<0, 256, 1, 6>(a, msg);
   // Grouped GEMMs with wide experts run on CTA pairs too: 256-row tiles per
   // expert, one third fewer operand bytes per flop than 128 x 256 tiles.
   if (a.offsets != nullptr && a.N >= 1024 && a.M >= 512) {
-    if (a.kind == 0) return run2<0, 256, 6>(a, msg);
-    return run2<1, 256, 6>(a, msg);
+    if (a.kind == 0) return run2<0, 256, 1, 6>(a, msg);
+    return run2<1, 256, 1, 6>(a, msg);
   }
   // Small M (decode): the weight stream from HBM is the bound, and each SM
   // streams at a roughly fixed rate, so the tile width is the narrowest that

@@ -430,12 +430,14 @@ hq_status hq_quantize_fp8_noalloc(const void* x, hq_dtype xt, int64_t rows, int6
 
 /*
  * Test hook for the failure path of the library's bounded waits: launches
- * one thread that waits on a shared-memory barrier nothing completes, for
- * limit_ns nanoseconds (1 us .. 2 s).  The wait then gives up, records a
- * timeout in the device error word and the kernel returns normally (no trap,
- * no fault); the next hq_check_device_error() returns HQ_ERR_TIMEOUT and
- * clears the word.  Every wait in the library's kernels takes this path on a
- * stalled barrier.
+ * one warp whose lanes wait on a shared-memory barrier nothing completes,
+ * lane l for limit_ns * (1 + l/32) nanoseconds (limit_ns in 1 us .. 2 s).
+ * The first lane to give up records a timeout in the device error word and
+ * ends the other lanes' waits; the warp agrees on giving up before a
+ * warp-wide step (as the GEMM warps do before their warp-wide tensor-memory
+ * loads) and the kernel returns normally (no trap, no fault).  The next
+ * hq_check_device_error() returns HQ_ERR_TIMEOUT and clears the word.  Every
+ * wait in the library's kernels takes this path on a stalled barrier.
  * Errors: HQ_ERR_INVALID_ARG (limit outside the range), HQ_ERR_UNSUPPORTED_ARCH,
  *   HQ_ERR_CUDA.
  */

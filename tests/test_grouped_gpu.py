@@ -38,6 +38,8 @@ CASES = [  # (counts per expert, N, K)
     # second-CTA weight rows belong to the next expert, ragged K
     ([3, 0, 300, 1, 0, 257, 40], 1024, 256),
     ([520, 0, 17], 1040, 160),
+    # N = 1408 with a ragged K and a partial 256-row tile in every expert
+    ([520, 0, 17, 700], 1408, 96),
 ]
 
 
