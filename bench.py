@@ -71,7 +71,8 @@ WORKLOADS = {
     "decode16": dict(kind="decode", M=16, N=28672, K=8192),
     "decode128": dict(kind="decode", M=128, N=28672, K=8192),
     "sweep": dict(kind="sweep", M=8192, N=0, K=8192),
-    "stack": dict(kind="stack", M=2048, N=4096, K=1024, steps_cycle=200, ring=16),
+    "stack": dict(kind="stack", M=2048, N=4096, K=1024, steps_cycle=200, ring=16, fused=True),
+    "stack_unfused": dict(kind="stack", M=2048, N=4096, K=1024, steps_cycle=200, ring=16, fused=False),
     "backward": dict(kind="backward", M=16384, N=28672, K=8192, ring=16),
     "blockwise": dict(kind="blockwise", M=8192, N=0, K=8192),
     "blockscaled": dict(kind="blockscaled", M=16384, N=28672, K=8192, block=128),
@@ -97,7 +98,8 @@ def workload_desc(name, cfg):
     if k == "stack":
         return ("delayed-scaling linear stack: X_t bf16 [2048,1024] (std 0.5 -> 8 over 200 steps), W_up bf16 "
                 "[4096,1024], W_down bf16 [1024,4096] ~N(0,0.02); per-tensor E4M3 with four amax-history rings "
-                "(length 16); h = GEMM(q(X), q(W_up)), y = GEMM(q(h), q(W_down)); step replayed as a CUDA graph")
+                "(length 16); h = GEMM(q(X), q(W_up)), y = GEMM(q(h), q(W_down)); step replayed as a CUDA graph; "
+                "q(h) %s" % ("fused into the first GEMM's epilogue" if cfg.get("fused") else "a separate kernel"))
     if k == "sweep":
         return ("quantize sweep: bf16 [%d,%d] ~N(0,1), 0.1%% x100 outliers, 0.1%% zeros, one zero row; "
                 "per-tensor / per-token / per-channel x E4M3 / E5M2" % (cfg["M"], cfg["K"]))
@@ -443,11 +445,15 @@ def build(args, cfg, rank, dev, stream, peaks):
                                    workspace=ws[key], stream=torch.cuda.current_stream(dev))
             q(x_stage, "x", xq, xsc)
             q(wu, "wu", wuq, wusc)
-            # h stays a bf16 round trip through L2: at K = 1024 the GEMM's
-            # epilogue is its critical path, and the separate quantize of the
-            # 16 MB h (an L2 read) costs less than the FP8-output epilogue
-            hq.hq_gemm_a8w8(xq, wuq, xsc, wusc, hq.E4M3, out=h, stream=torch.cuda.current_stream(dev))
-            q(h, "h", hq_, hsc)
+            if cfg["fused"]:
+                # h leaves the GEMM as FP8 codes: its delayed per-tensor
+                # quantize (ring h) runs in the GEMM's epilogue
+                hq.hq_gemm_a8w8_ex(xq, wuq, xsc, wusc, hq.E4M3, q_out=hq_, q_fmt=hq.E4M3, q_scale=hsc,
+                                   ring=rings["h"], ring_idx=idx, workspace=ws["h"],
+                                   stream=torch.cuda.current_stream(dev))
+            else:
+                hq.hq_gemm_a8w8(xq, wuq, xsc, wusc, hq.E4M3, out=h, stream=torch.cuda.current_stream(dev))
+                q(h, "h", hq_, hsc)
             q(wd, "wd", wdq, wdsc)
             hq.hq_gemm_a8w8(hq_, wdq, hsc, wdsc, hq.E4M3, out=y, stream=torch.cuda.current_stream(dev))
 
@@ -501,14 +507,18 @@ def build(args, cfg, rank, dev, stream, peaks):
                     "peak_source": "%s bf16 burst x 2 (nominal fp8/bf16)" % peaks["_src"]}
 
         def extras(ms):
-            d = {"kernels_per_step": 6, "rings": "4 x [16 hist | scale | counter], updated on the device every step"}
+            d = {"kernels_per_step": 5 if cfg["fused"] else 6,
+                 "rings": "4 x [16 hist | scale | counter], updated on the device every step",
+                 "h": "FP8 codes from the GEMM's epilogue (delayed quantize fused)" if cfg["fused"] else
+                      "bf16 from the GEMM, then a separate delayed quantize"}
             if graphs is not None:
                 d["graph_launches_per_step"] = 1
             else:
                 d["graph_capture"] = "failed (%s); eager launches" % graph_error
             return d
 
-        return dict(calls=[("step", step_fn, 6)], per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=T * D * 2,
+        return dict(calls=[("step", step_fn, 5 if cfg["fused"] else 6)], per_step=flops, unit="TFLOP/s", e2e=e2e,
+                    h2d=T * D * 2,
                     d2h=T * D * 2, roofline=roofline, extras=extras, flush=None, graphs=graphs,
                     l2="working set (X 4 MB, W 16 MB, h 16 MB) fits L2: a steady-state layer step")
 

@@ -90,7 +90,11 @@ def test_stack_reduced_size_full_chain():
     H.hq_check_device_error()
 
 
-def test_stack_full_size():
+@pytest.mark.parametrize("fused", [False, True])
+def test_stack_full_size(fused):
+    # fused: h leaves the first GEMM as FP8 codes, its delayed quantize run by
+    # the GEMM's epilogue (hq_gemm_a8w8_ex with q_out); the bf16 h that the
+    # checks need comes from a plain GEMM call on the same operands
     tokens, dim, hidden, steps = 2048, 1024, 4096, 200
     wu, wd = W.delayed_weights(dim, hidden)
     wu_d, wd_d = dev_bf16(wu), dev_bf16(wd)
@@ -107,8 +111,12 @@ def test_stack_full_size():
             h_ring_before = host(rings_d["h"]).copy()  # synchronises: no launch of this step yet
         xq, xs = q_delayed(dev_bf16(x), rings_d["x"], t)
         wuq, wus = q_delayed(wu_d, rings_d["wu"], t)
-        h = H.hq_gemm_a8w8(xq, wuq, xs, wus, H.E4M3)
-        hq_, hs = q_delayed(h, rings_d["h"], t)
+        if fused:
+            hq_, hs = H.hq_gemm_a8w8_ex(xq, wuq, xs, wus, H.E4M3, q_fmt=H.E4M3, ring=rings_d["h"], ring_idx=t % L)
+            h = H.hq_gemm_a8w8(xq, wuq, xs, wus, H.E4M3)
+        else:
+            h = H.hq_gemm_a8w8(xq, wuq, xs, wus, H.E4M3)
+            hq_, hs = q_delayed(h, rings_d["h"], t)
         wdq, wds = q_delayed(wd_d, rings_d["wd"], t)
         y = H.hq_gemm_a8w8(hq_, wdq, hs, wds, H.E4M3)
         # the oracle's ring steps for the generator-fed stages
