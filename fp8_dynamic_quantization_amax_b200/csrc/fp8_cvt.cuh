@@ -24,6 +24,17 @@ __device__ __forceinline__ uint32_t cvt2_exact(float lo, float hi) {
   return v;
 }
 
+// The same for inputs known not to be NaN: the conversion alone.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt2_fast(float lo, float hi) {
+  unsigned short r;
+  if (FMT == 0)
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  else
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 template <int FMT>
 __device__ __forceinline__ uint8_t cvt1_exact(float y) {
   return static_cast<uint8_t>(cvt2_exact<FMT>(y, 0.0f) & 0xFFu);

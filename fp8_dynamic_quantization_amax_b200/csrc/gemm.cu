@@ -148,19 +148,47 @@ __device__ __forceinline__ void chunk_to_bf16(const uint32_t (&v)[32], bool has_
   }
 }
 
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // FP8 output of one chunk: codes of f32(bf16 value) * m, saturating RNE (NaN
 // -> 0x7F), into c4 (the lane's 32 codes, column n0 in the low byte of
-// c4[0]); the lane's finite-only amax is updated over its valid columns.
+// c4[0]); the lane's finite-only amax over its valid columns is kept as the
+// raw bits of the largest bf16 magnitude in qraw (for non-negative bf16
+// values the unsigned order of the bits is the numeric order), or in qam on
+// the exact path.  Columns past N hold zero (their scales are zero), so only
+// rows past the tile's valid rows (vrow false) need excluding.  A chunk
+// without an Inf or NaN takes one max.u16x2 per pair and the plain
+// conversion; otherwise each element is checked.
 __device__ __forceinline__ void chunk_to_fp8(const uint32_t (&w)[16], int qfmt, float qm, bool vrow, int n0, int N,
-                                             float& qam, uint32_t (&c4)[8]) {
+                                             uint32_t& qraw, float& qam, uint32_t (&c4)[8]) {
+  uint32_t mx = 0;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float lo = __uint_as_float(w[j] << 16);
-    const float hi = __uint_as_float(w[j] & 0xFFFF0000u);
-    if (vrow && n0 + 2 * j < N) qam = fmaxf(qam, fmaxf(finite_abs(lo), finite_abs(hi)));
-    const uint32_t c2 = (qfmt == 0) ? cvt2_exact<0>(__fmul_rn(lo, qm), __fmul_rn(hi, qm))
-                                    : cvt2_exact<1>(__fmul_rn(lo, qm), __fmul_rn(hi, qm));
-    c4[j >> 1] = (j & 1) ? (c4[j >> 1] | (c2 << 16)) : c2;
+  for (int j = 0; j < 16; ++j) mx = max_u16x2(mx, w[j] & 0x7FFF7FFFu);
+  const uint32_t mmax = max(mx & 0xFFFFu, mx >> 16);
+  if (mmax < 0x7F80u) {  // no Inf or NaN in this lane's chunk
+    if (vrow) qraw = max(qraw, mmax);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float lo = __uint_as_float(w[j] << 16);
+      const float hi = __uint_as_float(w[j] & 0xFFFF0000u);
+      const uint32_t c2 = (qfmt == 0) ? cvt2_fast<0>(__fmul_rn(lo, qm), __fmul_rn(hi, qm))
+                                      : cvt2_fast<1>(__fmul_rn(lo, qm), __fmul_rn(hi, qm));
+      c4[j >> 1] = (j & 1) ? (c4[j >> 1] | (c2 << 16)) : c2;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float lo = __uint_as_float(w[j] << 16);
+      const float hi = __uint_as_float(w[j] & 0xFFFF0000u);
+      if (vrow && n0 + 2 * j < N) qam = fmaxf(qam, fmaxf(finite_abs(lo), finite_abs(hi)));
+      const uint32_t c2 = (qfmt == 0) ? cvt2_exact<0>(__fmul_rn(lo, qm), __fmul_rn(hi, qm))
+                                      : cvt2_exact<1>(__fmul_rn(lo, qm), __fmul_rn(hi, qm));
+      c4[j >> 1] = (j & 1) ? (c4[j >> 1] | (c2 << 16)) : c2;
+    }
   }
 }
 
@@ -241,7 +269,7 @@ template <int KIND, int kChunks>
 __device__ __forceinline__ void epilogue_chunks(uint32_t tacc, int half, int lane, int col0, int col_end, int tile_end,
                                                 int row0, bool vrow, bool tma_ok, bool has_acc, float xsv,
                                                 const float* wsh, const Params& p, const uint16_t* bias, uint16_t* orow,
-                                                uint8_t* qrow, float qm, float& qam, uint8_t* sb,
+                                                uint8_t* qrow, float qm, uint32_t& qraw, float& qam, uint8_t* sb,
                                                 const CUtensorMap* tm_out, uint64_t out_pol) {
   auto process = [&](const uint32_t (&v)[32], int j) {
     const int n0 = col0 + (half + 2 * j) * 32;
@@ -250,7 +278,7 @@ __device__ __forceinline__ void epilogue_chunks(uint32_t tacc, int half, int lan
     chunk_to_bf16(v, has_acc, xsv, wsh + j * 32, bias, n0, p.N, w);
     if (KIND == 0 && qrow != nullptr) {
       uint32_t c4[8];
-      chunk_to_fp8(w, p.qfmt, qm, vrow, n0, p.N, qam, c4);
+      chunk_to_fp8(w, p.qfmt, qm, vrow, n0, p.N, qraw, qam, c4);
       if (tma_ok && n0 + 32 <= tile_end) {
         // the 32 x 32 codes through the staging tile, 32-byte rows with the
         // 32-byte swizzle: 16-byte half h of row r sits at h ^ ((r >> 2) & 1)
@@ -457,7 +485,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
   const int total = (p.offsets != nullptr) ? tile_prefix[p.E] : p.m_tiles * p.n_tiles;
-  float qam = 0.0f;  // FP8 output: this thread's finite-only amax of the bf16 result
+  float qam = 0.0f;    // FP8 output: this thread's finite-only amax of the bf16 result (exact path)
+  uint32_t qraw = 0;   // the same as the raw bits of the largest bf16 magnitude (fast path)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -590,7 +619,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
       epilogue_chunks<KIND, kChunks>(
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride, half, lane,
-          T.col0, ncap, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qam, sb, &tm_out,
+          T.col0, ncap, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qraw, qam, sb, &tm_out,
           out_pol);
       tc_fence_before();
       __syncwarp();
@@ -602,7 +631,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemm1Threads / 32>(p, qam);
+  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemm1Threads / 32>(p, fmaxf(qam, __uint_as_float(qraw << 16)));
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
@@ -888,7 +917,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
   const int total = (p.offsets != nullptr) ? tile_prefix[p.E] : p.m_tiles * p.n_tiles;  // tiles of 256 x BN
-  float qam = 0.0f;  // FP8 output: this thread's finite-only amax of the bf16 result
+  float qam = 0.0f;    // FP8 output: this thread's finite-only amax of the bf16 result (exact path)
+  uint32_t qraw = 0;   // the same as the raw bits of the largest bf16 magnitude (fast path)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -1026,7 +1056,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
       epilogue_chunks<KIND, kChunks>(
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride, half, lane,
-          T.col0, p.N, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qam, sb, &tm_out,
+          T.col0, p.N, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qraw, qam, sb, &tm_out,
           out_pol);
       tc_fence_before();
       __syncwarp();
@@ -1038,7 +1068,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemmThreads / 32>(p, qam);
+  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemmThreads / 32>(p, fmaxf(qam, __uint_as_float(qraw << 16)));
   cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
   if (warp == 1) {
     tc_fence_after();
