@@ -99,7 +99,8 @@ def workload_desc(name, cfg):
         return ("delayed-scaling linear stack: X_t bf16 [2048,1024] (std 0.5 -> 8 over 200 steps), W_up bf16 "
                 "[4096,1024], W_down bf16 [1024,4096] ~N(0,0.02); per-tensor E4M3 with four amax-history rings "
                 "(length 16); h = GEMM(q(X), q(W_up)), y = GEMM(q(h), q(W_down)); step replayed as a CUDA graph; "
-                "q(h) %s" % ("fused into the first GEMM's epilogue" if cfg.get("fused") else "a separate kernel"))
+                "%s" % ("q(X), q(W_up), q(W_down) in one batched launch, q(h) in the first GEMM's epilogue"
+                        if cfg.get("fused") else "four separate delayed quantizes"))
     if k == "sweep":
         return ("quantize sweep: bf16 [%d,%d] ~N(0,1), 0.1%% x100 outliers, 0.1%% zeros, one zero row; "
                 "per-tensor / per-token / per-channel x E4M3 / E5M2" % (cfg["M"], cfg["K"]))
@@ -443,18 +444,24 @@ def build(args, cfg, rank, dev, stream, peaks):
             def q(x, key, qo, so):
                 hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TENSOR, q=qo, scales=so, ring=rings[key], ring_idx=idx,
                                    workspace=ws[key], stream=torch.cuda.current_stream(dev))
-            q(x_stage, "x", xq, xsc)
-            q(wu, "wu", wuq, wusc)
             if cfg["fused"]:
-                # h leaves the GEMM as FP8 codes: its delayed per-tensor
-                # quantize (ring h) runs in the GEMM's epilogue
+                # X, W_up and W_down quantized with their rings in one launch;
+                # h leaves the first GEMM as FP8 codes, its delayed quantize
+                # (ring h) run by the GEMM's epilogue: three kernels per step
+                hq.hq_quantize_fp8_delayed_batch(
+                    [dict(x=x_stage, ring=rings["x"], ring_idx=idx, q=xq, scale=xsc, workspace=ws["x"]),
+                     dict(x=wu, ring=rings["wu"], ring_idx=idx, q=wuq, scale=wusc, workspace=ws["wu"]),
+                     dict(x=wd, ring=rings["wd"], ring_idx=idx, q=wdq, scale=wdsc, workspace=ws["wd"])],
+                    hq.E4M3, stream=torch.cuda.current_stream(dev))
                 hq.hq_gemm_a8w8_ex(xq, wuq, xsc, wusc, hq.E4M3, q_out=hq_, q_fmt=hq.E4M3, q_scale=hsc,
                                    ring=rings["h"], ring_idx=idx, workspace=ws["h"],
                                    stream=torch.cuda.current_stream(dev))
             else:
+                q(x_stage, "x", xq, xsc)
+                q(wu, "wu", wuq, wusc)
                 hq.hq_gemm_a8w8(xq, wuq, xsc, wusc, hq.E4M3, out=h, stream=torch.cuda.current_stream(dev))
                 q(h, "h", hq_, hsc)
-            q(wd, "wd", wdq, wdsc)
+                q(wd, "wd", wdq, wdsc)
             hq.hq_gemm_a8w8(hq_, wdq, hsc, wdsc, hq.E4M3, out=y, stream=torch.cuda.current_stream(dev))
 
         # one graph per ring slot (the slot index is a launch argument)
@@ -507,17 +514,17 @@ def build(args, cfg, rank, dev, stream, peaks):
                     "peak_source": "%s bf16 burst x 2 (nominal fp8/bf16)" % peaks["_src"]}
 
         def extras(ms):
-            d = {"kernels_per_step": 5 if cfg["fused"] else 6,
+            d = {"kernels_per_step": 3 if cfg["fused"] else 6,
                  "rings": "4 x [16 hist | scale | counter], updated on the device every step",
-                 "h": "FP8 codes from the GEMM's epilogue (delayed quantize fused)" if cfg["fused"] else
-                      "bf16 from the GEMM, then a separate delayed quantize"}
+                 "quantize": ("X, W_up, W_down in one batched launch; h in the first GEMM's epilogue"
+                              if cfg["fused"] else "four separate delayed quantizes (h from a bf16 round trip)")}
             if graphs is not None:
                 d["graph_launches_per_step"] = 1
             else:
                 d["graph_capture"] = "failed (%s); eager launches" % graph_error
             return d
 
-        return dict(calls=[("step", step_fn, 5 if cfg["fused"] else 6)], per_step=flops, unit="TFLOP/s", e2e=e2e,
+        return dict(calls=[("step", step_fn, 3 if cfg["fused"] else 6)], per_step=flops, unit="TFLOP/s", e2e=e2e,
                     h2d=T * D * 2,
                     d2h=T * D * 2, roofline=roofline, extras=extras, flush=None, graphs=graphs,
                     l2="working set (X 4 MB, W 16 MB, h 16 MB) fits L2: a steady-state layer step")

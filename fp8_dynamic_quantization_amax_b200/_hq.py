@@ -24,9 +24,17 @@ EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_q
             "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic",
             "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_blockscaled",
             "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
-            "hq_quantize_fp8_noalloc", "hq_debug_bounded_wait", "hq_check_device_error", "hq_last_error",
-            "hq_version"]
+            "hq_quantize_fp8_noalloc", "hq_quantize_fp8_delayed_batch", "hq_debug_bounded_wait",
+            "hq_check_device_error", "hq_last_error", "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
+
+
+class DelayedTensor(ctypes.Structure):
+    """hq_delayed_tensor: one tensor of a batched delayed quantize."""
+    _fields_ = [("x", ctypes.c_void_p), ("n", ctypes.c_int64), ("q", ctypes.c_void_p),
+                ("scale", ctypes.c_void_p), ("amax_out", ctypes.c_void_p), ("ring", ctypes.c_void_p),
+                ("ring_len", ctypes.c_int32), ("ring_idx", ctypes.c_int32), ("ring_margin", ctypes.c_int32),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
 
 
 class HQError(RuntimeError):
@@ -54,6 +62,8 @@ def _load():
     L.hq_quantize_fp8.restype = ci
     L.hq_quantize_fp8_noalloc.argtypes = [P, ci, i64, i64, ci, ci, P, P, P, P, i32, i32, i32, P]
     L.hq_quantize_fp8_noalloc.restype = ci
+    L.hq_quantize_fp8_delayed_batch.argtypes = [ctypes.POINTER(DelayedTensor), i32, ci, ci, P]
+    L.hq_quantize_fp8_delayed_batch.restype = ci
     L.hq_debug_bounded_wait.argtypes = [ctypes.c_uint64, P]
     L.hq_debug_bounded_wait.restype = ci
     L.hq_gemm_blockscaled.argtypes = [P, P, ci, P, P, i64, P, i64, i64, i64, P, P]
@@ -106,13 +116,14 @@ _DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
 _ws_cache = {}
 
 
-def _workspace(device, nbytes):
-    """A zero-filled workspace per (device, size).  The library returns its
-    accumulator words to zero after each call, so calls that run one after
-    another on one stream can share it."""
+def _workspace(device, nbytes, slot=0):
+    """A zero-filled workspace per (device, size, slot).  The library returns
+    its accumulator words to zero after each call, so calls that run one
+    after another on one stream can share it; tensors of one batched call run
+    at once and take different slots."""
     if nbytes == 0:
         return None
-    key = (device, nbytes)
+    key = (device, nbytes, slot)
     ws = _ws_cache.get(key)
     if ws is None:
         ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
@@ -166,6 +177,41 @@ def hq_quantize_fp8(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=N
                               _ptr(workspace), 0 if workspace is None else workspace.numel(),
                               _stream(stream)))
     return q, scales
+
+
+def hq_quantize_fp8_delayed_batch(items, fmt=E4M3, stream=None):
+    """Delayed per-tensor quantize of up to 8 CUDA tensors of one dtype in one
+    launch.  items: list of dicts with x (any shape, contiguous), ring (f32
+    [len+2]), ring_idx, and optionally ring_margin, q, scale, amax_out,
+    workspace.  Returns [(q, scale)] in order; each ring is stepped in place."""
+    if not 1 <= len(items) <= 8:
+        raise ValueError("1 to 8 tensors")
+    dt = items[0]["x"].dtype
+    if dt not in _DT or any(it["x"].dtype != dt for it in items):
+        raise ValueError("all tensors must share one of float32, bfloat16, float16")
+    arr = (DelayedTensor * len(items))()
+    keep, outs = [], []
+    for i, it in enumerate(items):
+        x = it["x"].contiguous()
+        n = x.numel()
+        q = it.get("q")
+        if q is None:
+            q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+        scale = it.get("scale")
+        if scale is None:
+            scale = torch.empty((1,), dtype=torch.float32, device=x.device)
+        ring = it["ring"]
+        ws = it.get("workspace")
+        if ws is None:
+            ws = _workspace(x.device, hq_quantize_workspace_bytes(PER_TENSOR, 1, n, True), slot=1 + i)
+        am = it.get("amax_out")
+        arr[i] = DelayedTensor(x.data_ptr(), n, q.data_ptr(), scale.data_ptr(), None if am is None else am.data_ptr(),
+                               ring.data_ptr(), ring.numel() - 2, it["ring_idx"], it.get("ring_margin", 0),
+                               None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel())
+        keep += [x, ws]
+        outs.append((q, scale))
+    check(lib.hq_quantize_fp8_delayed_batch(arr, len(items), _DT[dt], fmt, _stream(stream)))
+    return outs
 
 
 def hq_quantize_fp8_blockwise(x, fmt=E4M3, block=32, stochastic=False, seed=0, amax_out=None, stream=None):

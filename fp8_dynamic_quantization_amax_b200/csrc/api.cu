@@ -271,6 +271,71 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
   return launched(hq::launch_quantize(a), "quantize launch");
 }
 
+hq_status hq_quantize_fp8_delayed_batch(const hq_delayed_tensor* tensors, int32_t count, hq_dtype xt,
+                                        hq_fp8_format fmt, hq_stream_t stream) {
+  // ---- arguments
+  if (!tensors) return fail(HQ_ERR_INVALID_ARG, "tensors must not be null");
+  if (count < 1 || count > 8) return fail(HQ_ERR_INVALID_ARG, "count = %d outside [1, 8]", count);
+  const size_t esize = (xt == HQ_F32) ? 4 : 2;
+  Range all[8][6];  // per tensor: x, q, scale, amax_out, ring, workspace
+  for (int i = 0; i < count; ++i) {
+    const hq_delayed_tensor& t = tensors[i];
+    bool empty = false;
+    hq_status s = hq::quantize_check_args(t.x, xt, 1, t.n, fmt, HQ_PER_TENSOR, t.q, t.scale, t.amax_out, t.ring,
+                                          t.ring_len, t.ring_idx, t.ring_margin, &empty);
+    if (s != HQ_OK) return fail(s, "tensor %d: %s", i, hq_last_error());
+    if (!t.ring) return fail(HQ_ERR_INVALID_ARG, "tensor %d: a delayed quantize needs a ring", i);
+    const size_t need = hq::quantize_workspace_bytes(HQ_PER_TENSOR, 1, t.n, 1);
+    if (need > 0 && !t.workspace) return fail(HQ_ERR_INVALID_ARG, "tensor %d: a workspace of %zu bytes is needed", i, need);
+    if (need > 0 && t.workspace_bytes < need)
+      return fail(HQ_ERR_INVALID_ARG, "tensor %d: workspace of %zu bytes is smaller than the %zu needed", i,
+                  t.workspace_bytes, need);
+    if (need > 0 && !is_aligned(t.workspace, 256))
+      return fail(HQ_ERR_MISALIGNED, "tensor %d: workspace must be 256-byte aligned", i);
+    all[i][0] = {t.x, static_cast<size_t>(t.n) * esize, "x"};
+    all[i][1] = {t.q, static_cast<size_t>(t.n), "q"};
+    all[i][2] = {t.scale, 4, "scale"};
+    all[i][3] = {t.amax_out, t.amax_out ? 4u : 0u, "amax_out"};
+    all[i][4] = {t.ring, static_cast<size_t>(t.ring_len + 2) * 4, "ring"};
+    all[i][5] = {t.workspace, need, "workspace"};
+    // the workspace against this tensor's other buffers
+    for (int k = 0; k < 5; ++k)
+      if (overlaps(all[i][5], all[i][k]))
+        return fail(HQ_ERR_OVERLAP, "tensor %d: workspace overlaps %s", i, all[i][k].name);
+  }
+  // tensors run at once: no output of one may overlap any buffer of another
+  for (int i = 0; i < count; ++i)
+    for (int j = 0; j < count; ++j) {
+      if (i == j) continue;
+      for (int a = 1; a < 6; ++a)
+        for (int b = 0; b < 6; ++b)
+          if (overlaps(all[i][a], all[j][b]))
+            return fail(HQ_ERR_OVERLAP, "tensor %d's %s overlaps tensor %d's %s", i, all[i][a].name, j,
+                        all[j][b].name);
+    }
+  // ---- device
+  for (int i = 0; i < count; ++i) {
+    const hq_delayed_tensor& t = tensors[i];
+    const Range devs[] = {{t.n > 0 ? t.x : nullptr, 0, "x"}, {t.n > 0 ? t.q : nullptr, 0, "q"}, {t.scale, 0, "scale"},
+                          {t.amax_out, 0, "amax_out"}, {t.ring, 0, "ring"}, {t.workspace, 0, "workspace"}};
+    hq_status s = check_device_ptrs(devs, 6);
+    if (s != HQ_OK) return fail(s, "tensor %d: %s", i, hq_last_error());
+  }
+  hq_status s = check_arch();
+  if (s != HQ_OK) return s;
+  // ---- launch
+  hq::DelayedTensorArgs a[8];
+  for (int i = 0; i < count; ++i) {
+    const hq_delayed_tensor& t = tensors[i];
+    a[i].x = t.x; a[i].n = t.n; a[i].q = t.q; a[i].scale = t.scale; a[i].amax_out = t.amax_out;
+    a[i].ring = t.ring; a[i].ring_len = t.ring_len; a[i].ring_idx = t.ring_idx; a[i].ring_margin = t.ring_margin;
+    a[i].ws = t.workspace;
+  }
+  return launched(hq::launch_quantize_delayed_batch(static_cast<int>(xt), static_cast<int>(fmt), a, count,
+                                                    reinterpret_cast<cudaStream_t>(stream)),
+                  "batched delayed quantize launch");
+}
+
 hq_status hq_quantize_fp8_blockwise(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_fp8_format fmt,
                                     int64_t block, int stochastic, uint64_t seed, uint8_t* q, float* scales,
                                     float* amax_out, hq_stream_t stream) {

@@ -36,6 +36,21 @@ struct QuantizeArgs {
 
 size_t quantize_workspace_bytes(int gran, int64_t rows, int64_t cols, int delayed);
 cudaError_t launch_quantize(const QuantizeArgs& a);
+
+// One tensor of a batched delayed (ring) per-tensor quantize.
+struct DelayedTensorArgs {
+  const void* x;
+  int64_t n;          // elements
+  uint8_t* q;
+  float* scale;       // f32[1]: 1/m
+  float* amax_out;    // nullable
+  float* ring;        // [ring_len | scale | counter]
+  int ring_len, ring_idx, ring_margin;
+  void* ws;           // the delayed workspace (one amax word), zero between calls
+};
+// Up to 8 tensors of one dtype (xt) and format in one launch.
+cudaError_t launch_quantize_delayed_batch(int xt, int fmt, const DelayedTensorArgs* t, int count,
+                                          cudaStream_t stream);
 // Per-tensor quantize writing the codes row-major (a.q, nullable) and
 // transposed (a.qt); rows % 16 == 0, cols % 16 == 0, x 16-byte aligned.
 cudaError_t launch_quantize_transpose(const QuantizeArgs& a);
@@ -92,6 +107,9 @@ struct BlockScaledGemmArgs {
   cudaStream_t stream;
 };
 cudaError_t launch_gemm_blockscaled(const BlockScaledGemmArgs& a, std::string* msg);
+// The same GEMM with the block scales applied while converting the codes to
+// bf16 MMA operands (gemm.cu): no per-block round trip through TMEM.
+cudaError_t launch_gemm_blockscaled_bf16(const BlockScaledGemmArgs& a, std::string* msg);
 
 // Device error word (set by bounded waits and by offset validation).
 enum : unsigned { kDevErrTimeout = 1u, kDevErrBadOffsets = 2u };

@@ -41,9 +41,11 @@
 //   - the cast is one FMUL per element plus one cvt.rn.satfinite per pair.
 #include "fp8_cvt.cuh"
 #include "hq_internal.cuh"
+#include "launch.cuh"
 #include "ptx.cuh"
 
 #include <algorithm>
+#include <cstring>
 #include <cfloat>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -402,6 +404,7 @@ __global__ void __launch_bounds__(kRegThreads) k_token_reg(const void* __restric
                                                            uint8_t* __restrict__ q, float* __restrict__ scales,
                                                            float* __restrict__ amax_out) {
   constexpr int VEC = Dt<DT>::kVec;
+  pdl_wait();  // launched with programmatic stream serialization
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kRegThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kRegThreads) >> 5;
@@ -635,6 +638,20 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   return v;
 }
 
+// Arrival at the grid barrier by one thread after a CTA-wide barrier: the
+// release fence orders every write the CTA made before it (the maxima
+// folded in with relaxed atomics) ahead of the arrival.
+__device__ __forceinline__ void grid_arrive(uint32_t* arrivals) {
+  asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(arrivals) : "memory");
+}
+// Departure counter: returns the count before this CTA's increment, with
+// acquire-release order (the last CTA sees every other CTA's earlier reads
+// of the workspace as done before it clears it).
+__device__ __forceinline__ uint32_t grid_depart(uint32_t* departures) {
+  uint32_t v;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(v) : "l"(departures) : "memory");
+  return v;
+}
 __device__ __forceinline__ bool grid_barrier(uint32_t* arrivals, unsigned* err_word) {
   const unsigned long long t0 = ptx::globaltimer();
   for (uint32_t it = 0;; ++it) {
@@ -643,7 +660,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* arrivals, unsigned* err_w
       atomicOr(err_word, kDevErrTimeout);
       return false;
     }
-    __nanosleep(100);
+    __nanosleep(32);
   }
 }
 
@@ -711,6 +728,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
   const int64_t s0 = b0 + nheld;                               // TMEM part [s0, s1)
   const int64_t s1 = min(b1, s0 + static_cast<int64_t>(kTmemVecs) * T);  // L2 part [s1, b1)
   const bool tail_cta = blockIdx.x == gridDim.x - 1;
+  pdl_wait();  // launched with programmatic stream serialization
 
   if (tid == 0) {
     abort_flag = 0;
@@ -792,20 +810,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
     if (tid == 0) {
       if (nf) atomicOr(&ws[3], 1u);
       atomicMax(&ws[0], __float_as_uint(r));
-      __threadfence();
-      atomicAdd(&ws[1], 1u);
+      grid_arrive(&ws[1]);
       // grid barrier: every CTA has published its amax
       const bool ok = !abort_flag && grid_barrier(&ws[1], err_word);
       s_amax = __uint_as_float(__ldcg(&ws[0]));
       s_flags = (__ldcg(&ws[3]) != 0u ? 1 : 0) | (ok ? 0 : 2);
-      __threadfence();
-      // departure: the last CTA to leave clears the workspace
-      if (atomicAdd(&ws[2], 1u) == gridDim.x - 1) {
-        atomicExch(&ws[0], 0u);
-        atomicExch(&ws[3], 0u);
-        atomicExch(&ws[1], 0u);
-        atomicExch(&ws[2], 0u);
-      }
     }
   }
   __syncthreads();
@@ -851,6 +860,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
   tc_before_sync();
   __syncthreads();
   tc_after_sync();
+  // departure, off the critical path: the last CTA to leave clears the
+  // workspace (every CTA read it right after the barrier)
+  if (tid == 0 && grid_depart(&ws[2]) == gridDim.x - 1) {
+    atomicExch(&ws[0], 0u);
+    atomicExch(&ws[3], 0u);
+    atomicExch(&ws[1], 0u);
+    atomicExch(&ws[2], 0u);
+  }
+  __syncwarp();
   if (tid < 32) tmem_dealloc_warp(tmem_slot);
 }
 
@@ -1075,16 +1093,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
   float* red = reinterpret_cast<float*>(fsm);  // [RL][SC] row-lane maxima; later the strip's multipliers
   uint4* held = reinterpret_cast<uint4*>(fsm + RL * SC * 4);  // [nh][sv]
   const uint4* xv = static_cast<const uint4*>(x);  // row r, column vector c: xv[r * nvc + c]
+  pdl_wait();  // launched with programmatic stream serialization
 
-  if (tid == 0) {
-    abort_flag = 0;
-    ptx::mbar_init(&bar, 1);
-    ptx::fence_mbarrier_init();
+  if (tid < 32) {  // warp 0: the held rows' bulk copies, one per row, spread over the lanes
+    if (tid == 0) {
+      abort_flag = 0;
+      ptx::mbar_init(&bar, 1);
+      ptx::fence_mbarrier_init();
+      if (nh > 0 && sv > 0) ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nh * sv * 16));
+    }
+    __syncwarp();
     if (nh > 0 && sv > 0) {
       const uint64_t pol = policy_evict_first();
       const uint32_t row_bytes = static_cast<uint32_t>(sv * 16);
-      ptx::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nh) * row_bytes);
-      for (int64_t i = 0; i < nh; ++i) bulk_load_hint(held + i * sv, xv + (r0 + i) * nvc + c0, row_bytes, &bar, pol);
+      for (int64_t i = tid; i < nh; i += 32) bulk_load_hint(held + i * sv, xv + (r0 + i) * nvc + c0, row_bytes, &bar, pol);
     }
   }
   if (tid < 32) tmem_alloc_warp(&tmem_slot);
@@ -1179,12 +1201,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
     for (int l = 1; l < RL; ++l) a = fmaxf(a, red[l * SC + e]);
     atomicMax(&ws_amax[c0 * VEC + e], __float_as_uint(a));
   }
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
     if (nf) atomicOr(&header[1], 1u);
-    __threadfence();
-    atomicAdd(&header[0], 1u);
+    grid_arrive(&header[0]);
     const bool ok = !abort_flag && grid_barrier(&header[0], err_word);
     s_flags = (__ldcg(&header[1]) != 0u ? 1 : 0) | (ok ? 0 : 2);
   }
@@ -1204,22 +1224,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
       }
     }
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const bool last = atomicAdd(&header[2], 1u) == gridDim.x - 1;
-    s_flags |= last ? 4 : 0;
-  }
-  __syncthreads();
-  if (s_flags & 4) {  // every CTA has read the maxima: clear them and the header
-    for (int64_t col = tid; col < cols; col += T) ws_amax[col] = 0u;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      atomicExch(&header[1], 0u);
-      atomicExch(&header[0], 0u);
-      atomicExch(&header[2], 0u);
-    }
-  }
   if (ok) {
     // ---- phase 2: cast the tile: this lane's L2 rows from the end backwards,
     // then its TMEM rows, then the held rows
@@ -1261,6 +1265,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
   tc_before_sync();
   __syncthreads();
   tc_after_sync();
+  // departure, off the critical path: the last CTA to leave clears the
+  // maxima and the header (every CTA read them right after the barrier)
+  if (tid == 0) s_flags = (grid_depart(&header[2]) == gridDim.x - 1) ? 4 : 0;
+  __syncthreads();
+  if (s_flags & 4) {
+    for (int64_t col = tid; col < cols; col += T) ws_amax[col] = 0u;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      atomicExch(&header[1], 0u);
+      atomicExch(&header[0], 0u);
+      atomicExch(&header[2], 0u);
+    }
+  }
   if (tid < 32) tmem_dealloc_warp(tmem_slot);
 }
 
@@ -1268,19 +1286,28 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
 // Ring: [hist[len] | scale | counter].  Workspace word [0]: amax accumulator.
 // One pass: cast with the ring's multiplier while reducing amax.  A thread
 // whose raw maximum shows a non-finite element redoes its vectors on the
-// exact path (finite-only amax, canonical NaN codes).
+// exact path (finite-only amax, canonical NaN codes).  The body runs as CTA
+// `cta` of `ncta` CTAs given one tensor (the single launch, or one tensor's
+// share of a batched launch); the last of them to finish steps the ring.
+// The ring's history is read at the start (only the last CTA writes it, at
+// the end), so the last CTA's tail is one acquire-release increment and one
+// exchange.
+constexpr int kRingPrefetch = 64;  // history words read ahead into shared memory
+
 template <int DT, int FMT, bool VECP>
-__global__ void __launch_bounds__(kThreads) k_delayed(
-    const void* __restrict__ x, int64_t n, uint8_t* __restrict__ q, float* __restrict__ ring,
-    int len, int idx, int margin, uint32_t* __restrict__ ws, float* __restrict__ scales,
-    float* __restrict__ amax_out) {
+__device__ __forceinline__ void delayed_body(const void* __restrict__ x, int64_t n, uint8_t* __restrict__ q,
+                                             float* __restrict__ ring, int len, int idx, int margin,
+                                             uint32_t* __restrict__ ws, float* __restrict__ scales,
+                                             float* __restrict__ amax_out, int64_t cta, int64_t ncta) {
   constexpr int VEC = VECP ? Dt<DT>::kVec : 1;
   __shared__ float sh[kThreads / 32];
   __shared__ bool is_last;
+  __shared__ float hist_sh[kRingPrefetch];
   const float m = __ldcg(&ring[len]);
   const bool m_finite = fabsf(m) <= FLT_MAX;
-  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
-  const int64_t gstride = static_cast<int64_t>(gridDim.x) * kThreads;
+  if (threadIdx.x < kRingPrefetch && static_cast<int>(threadIdx.x) < len) hist_sh[threadIdx.x] = __ldcg(&ring[threadIdx.x]);
+  const int64_t gtid = cta * kThreads + threadIdx.x;
+  const int64_t gstride = ncta * kThreads;
   float amax = 0.0f;
   int64_t done = 0;
   if (VECP) {
@@ -1325,33 +1352,80 @@ __global__ void __launch_bounds__(kThreads) k_delayed(
   uint32_t* counter = reinterpret_cast<uint32_t*>(ring + len + 1);
   if (threadIdx.x == 0) {
     atomicMax(&ws[0], __float_as_uint(amax));
-    __threadfence();
-    is_last = atomicAdd(counter, 1u) == gridDim.x - 1;
+    uint32_t prev;  // release: this CTA's maximum is in before the count; acquire for the last CTA
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
+    is_last = prev == static_cast<uint32_t>(ncta - 1);
   }
   __syncthreads();
   if (!is_last) return;
-  __threadfence();
   __shared__ float a_sh;
-  if (threadIdx.x == 0) {
-    const float a = __uint_as_float(atomicExch(&ws[0], 0u));
-    a_sh = a;
-    ring[idx] = a;  // fold this step's amax into the history slot
-    __threadfence_block();
-  }
+  if (threadIdx.x == 0) a_sh = __uint_as_float(atomicExch(&ws[0], 0u));
   __syncthreads();
-  float win = 0.0f;
-  for (int i = threadIdx.x; i < len; i += kThreads) win = fmaxf(win, __ldcg(&ring[i]));
-  win = block_max(win, sh);
-  if (threadIdx.x == 0) {
-    const float a = a_sh;
-    if (win <= FLT_MAX && win > 0.0f) {
-      const float next = ldexpf(__fdiv_rn(Fmt<FMT>::kMax, win), -margin);
-      if (next <= FLT_MAX && next > 0.0f) ring[len] = next;
-    }
-    scales[0] = __fdiv_rn(1.0f, m);
-    if (amax_out) amax_out[0] = a;
-    atomicExch(counter, 0u);
+  const float a = a_sh;
+  // the window: max of the history with this step's slot replaced by a
+  float win;
+  if (len <= kRingPrefetch) {  // from the history read at the start
+    if (threadIdx.x != 0) return;
+    win = a;
+    for (int i = 0; i < len; ++i)
+      if (i != idx) win = fmaxf(win, hist_sh[i]);
+  } else {
+    float w = (threadIdx.x == 0) ? a : 0.0f;
+    for (int i = threadIdx.x; i < len; i += kThreads)
+      if (i != idx) w = fmaxf(w, __ldcg(&ring[i]));
+    win = block_max(w, sh);
+    if (threadIdx.x != 0) return;
   }
+  ring[idx] = a;
+  if (win <= FLT_MAX && win > 0.0f) {
+    const float next = ldexpf(__fdiv_rn(Fmt<FMT>::kMax, win), -margin);
+    if (next <= FLT_MAX && next > 0.0f) ring[len] = next;
+  }
+  scales[0] = __fdiv_rn(1.0f, m);
+  if (amax_out) amax_out[0] = a;
+  atomicExch(counter, 0u);
+}
+
+template <int DT, int FMT, bool VECP>
+__global__ void __launch_bounds__(kThreads) k_delayed(
+    const void* __restrict__ x, int64_t n, uint8_t* __restrict__ q, float* __restrict__ ring,
+    int len, int idx, int margin, uint32_t* __restrict__ ws, float* __restrict__ scales,
+    float* __restrict__ amax_out) {
+  pdl_wait();  // launched with programmatic stream serialization
+  delayed_body<DT, FMT, VECP>(x, n, q, ring, len, idx, margin, ws, scales, amax_out, blockIdx.x, gridDim.x);
+}
+
+// Batched delayed quantize: up to kBatchMax tensors of one dtype and format in
+// one launch.  Tensor t owns CTAs [cta0[t], cta0[t + 1]); each tensor's CTAs
+// run the single-tensor body with their own ring, workspace and counter.
+constexpr int kBatchMax = 8;
+struct DelayedBatch {
+  int count;
+  int cta0[kBatchMax + 1];
+  const void* x[kBatchMax];
+  int64_t n[kBatchMax];
+  uint8_t* q[kBatchMax];
+  float* scales[kBatchMax];
+  float* amax_out[kBatchMax];
+  float* ring[kBatchMax];
+  int len[kBatchMax], idx[kBatchMax], margin[kBatchMax];
+  uint32_t* ws[kBatchMax];
+  int vec[kBatchMax];  // 1: 16-byte vector path
+};
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kThreads) k_delayed_batch(const __grid_constant__ DelayedBatch b) {
+  pdl_wait();  // launched with programmatic stream serialization
+  int t = 0;
+  while (t + 1 < b.count && static_cast<int>(blockIdx.x) >= b.cta0[t + 1]) ++t;
+  const int64_t cta = static_cast<int64_t>(blockIdx.x) - b.cta0[t];
+  const int64_t ncta = b.cta0[t + 1] - b.cta0[t];
+  if (b.vec[t])
+    delayed_body<DT, FMT, true>(b.x[t], b.n[t], b.q[t], b.ring[t], b.len[t], b.idx[t], b.margin[t], b.ws[t],
+                                b.scales[t], b.amax_out[t], cta, ncta);
+  else
+    delayed_body<DT, FMT, false>(b.x[t], b.n[t], b.q[t], b.ring[t], b.len[t], b.idx[t], b.margin[t], b.ws[t],
+                                 b.scales[t], b.amax_out[t], cta, ncta);
 }
 
 // ----------------------------------------- per-tensor with a transposed copy
@@ -2034,10 +2108,8 @@ cudaError_t launch_tensor_fused(const QuantizeArgs& a, int dev, int64_t n, float
   float* scales = a.scales;
   float* amax_out = a.amax_out;
   unsigned* err = device_error_word();
-  void* args[] = {(void*)&x, (void*)&n, (void*)&per, (void*)&held_max, (void*)&q, (void*)&ws,
-                  (void*)&fmax, (void*)&scales, (void*)&amax_out, (void*)&err};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_tensor_fused<DT, FMT>), dim3(grid),
-                                     dim3(kFusedThreads), args, smem, a.stream);
+  return launch_pdl(k_tensor_fused<DT, FMT>, dim3(grid), dim3(kFusedThreads), smem, a.stream, true, x, n, per,
+                    held_max, q, ws, fmax, scales, amax_out, err);
 }
 
 // Per-token rows of up to 1024 vectors: the register-resident kernel on a
@@ -2058,9 +2130,8 @@ cudaError_t launch_token_reg(const QuantizeArgs& a, int dev, int64_t nv) {
   int64_t grid = static_cast<int64_t>(device_sm_count(dev)) * std::max(per_sm, 1);
   if (grid > ctas_needed) grid = ctas_needed;
   if (grid < 1) grid = 1;
-  k_token_reg<DT, FMT, VPL, RPW><<<static_cast<unsigned>(grid), kRegThreads, 0, a.stream>>>(a.x, a.rows, nv, a.q,
-                                                                                           a.scales, a.amax_out);
-  return cudaGetLastError();
+  return launch_pdl(k_token_reg<DT, FMT, VPL, RPW>, dim3(static_cast<unsigned>(grid)), dim3(kRegThreads), 0,
+                    a.stream, false, a.x, a.rows, nv, a.q, a.scales, a.amax_out);
 }
 
 template <int DT, int FMT>
@@ -2077,12 +2148,10 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
     uint32_t* ws = static_cast<uint32_t*>(a.ws);
     const int grid = flat_grid(flat_vec ? n / VEC : n, dev, kUnroll);
     if (flat_vec)
-      k_delayed<DT, FMT, true><<<grid, kThreads, 0, a.stream>>>(a.x, n, a.q, a.ring, a.ring_len, a.ring_idx,
-                                                                a.ring_margin, ws, a.scales, a.amax_out);
-    else
-      k_delayed<DT, FMT, false><<<grid, kThreads, 0, a.stream>>>(a.x, n, a.q, a.ring, a.ring_len, a.ring_idx,
-                                                                 a.ring_margin, ws, a.scales, a.amax_out);
-    return cudaGetLastError();
+      return launch_pdl(k_delayed<DT, FMT, true>, dim3(grid), dim3(kThreads), 0, a.stream, false, a.x, n, a.q, a.ring,
+                        a.ring_len, a.ring_idx, a.ring_margin, ws, a.scales, a.amax_out);
+    return launch_pdl(k_delayed<DT, FMT, false>, dim3(grid), dim3(kThreads), 0, a.stream, false, a.x, n, a.q, a.ring,
+                      a.ring_len, a.ring_idx, a.ring_margin, ws, a.scales, a.amax_out);
   }
 
   if (a.gran == 1) {  // per-token
@@ -2170,12 +2239,9 @@ cudaError_t launch_typed(const QuantizeArgs& a) {
       float* scales = a.scales;
       float* amax_out = a.amax_out;
       unsigned* err = device_error_word();
-      void* args[] = {(void*)&x, (void*)&rows, (void*)&cols, (void*)&nstrips, (void*)&band, (void*)&held,
-                      (void*)&q, (void*)&header, (void*)&ws_amax, (void*)&f, (void*)&scales, (void*)&amax_out,
-                      (void*)&err};
-      return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_channel_fused<DT, FMT>),
-                                         dim3(static_cast<unsigned>(strips * bands)), dim3(kFusedThreads), args, smem,
-                                         a.stream);
+      return launch_pdl(k_channel_fused<DT, FMT>, dim3(static_cast<unsigned>(strips * bands)), dim3(kFusedThreads),
+                        smem, a.stream, true, x, rows, cols, nstrips, band, held, q, header, ws_amax, f, scales,
+                        amax_out, err);
     }
   }
 
@@ -2455,6 +2521,49 @@ size_t quantize_workspace_bytes(int gran, int64_t rows, int64_t cols, int delaye
   const size_t c4 = static_cast<size_t>((cols + 3) / 4) * 4;
   size_t b = 16 + c4 * 4 + static_cast<size_t>(cols) * 4;
   return (b + 255) / 256 * 256;
+}
+
+template <int DT, int FMT>
+cudaError_t launch_delayed_batch_typed(const DelayedTensorArgs* t, int count, cudaStream_t stream) {
+  constexpr int VEC = Dt<DT>::kVec;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  DelayedBatch b;
+  memset(&b, 0, sizeof(b));
+  b.count = count;
+  int total = 0;
+  for (int i = 0; i < count; ++i) {
+    const bool vec = aligned(t[i].x, 16) && aligned(t[i].q, VEC);
+    b.cta0[i] = total;
+    total += flat_grid(vec ? t[i].n / VEC : t[i].n, dev, kUnroll);
+    b.x[i] = t[i].x;
+    b.n[i] = t[i].n;
+    b.q[i] = t[i].q;
+    b.scales[i] = t[i].scale;
+    b.amax_out[i] = t[i].amax_out;
+    b.ring[i] = t[i].ring;
+    b.len[i] = t[i].ring_len;
+    b.idx[i] = t[i].ring_idx;
+    b.margin[i] = t[i].ring_margin;
+    b.ws[i] = static_cast<uint32_t*>(t[i].ws);
+    b.vec[i] = vec ? 1 : 0;
+  }
+  b.cta0[count] = total;
+  return launch_pdl(k_delayed_batch<DT, FMT>, dim3(static_cast<unsigned>(total)), dim3(kThreads), 0, stream, false, b);
+}
+
+cudaError_t launch_quantize_delayed_batch(int xt, int fmt, const DelayedTensorArgs* t, int count,
+                                          cudaStream_t stream) {
+  if (count < 1 || count > kBatchMax) return cudaErrorInvalidValue;
+  switch (xt * 2 + fmt) {
+    case 0: return launch_delayed_batch_typed<0, 0>(t, count, stream);
+    case 1: return launch_delayed_batch_typed<0, 1>(t, count, stream);
+    case 2: return launch_delayed_batch_typed<1, 0>(t, count, stream);
+    case 3: return launch_delayed_batch_typed<1, 1>(t, count, stream);
+    case 4: return launch_delayed_batch_typed<2, 0>(t, count, stream);
+    case 5: return launch_delayed_batch_typed<2, 1>(t, count, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_quantize(const QuantizeArgs& a) {

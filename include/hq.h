@@ -153,6 +153,46 @@ hq_status hq_quantize_fp8(const void* x, hq_dtype xt, int64_t rows, int64_t cols
                           void* workspace, size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * Delayed (amax-history ring) per-tensor quantize of several tensors in one
+ * launch: each tensor gets exactly what hq_quantize_fp8 in delayed mode
+ * (ring != NULL, HQ_PER_TENSOR) would give it -- codes of f32(x) * m with
+ * m = ring[ring_len], scale[0] = 1/m, amax_out[0] = the finite-only amax,
+ * and the ring stepped (AstrAI ops.cu ring commit: every operand's ring is
+ * finalized by the kernel that quantizes it; a layer quantizes its input
+ * and weights this way every step).  One launch instead of `count` saves
+ * the launch gaps of small tensors.
+ *
+ * tensors: host array of `count` descriptors (1 <= count <= 8); every
+ *   tensor has element type xt and FP8 format fmt:
+ *     x          device, n elements (rows*cols flattened), aligned to xt
+ *     n          elements (>= 0; n == 0 steps the ring with amax 0)
+ *     q          device, n bytes
+ *     scale      device f32[1]
+ *     amax_out   device f32[1] or NULL
+ *     ring       device f32[ring_len + 2], counter word 0 on entry
+ *     ring_len, ring_idx, ring_margin   as hq_quantize_fp8
+ *     workspace  device, >= hq_quantize_workspace_bytes(HQ_PER_TENSOR, 1,
+ *                n, 1) bytes, 256-byte aligned, zero on entry (left zero)
+ * The tensors' buffers must not overlap each other (they run at once).
+ * Errors: as hq_quantize_fp8 for each tensor (the message names it), plus
+ *   HQ_ERR_INVALID_ARG for count outside [1, 8] or a NULL tensors array,
+ *   and HQ_ERR_OVERLAP between tensors.  Nothing is launched on any error.
+ */
+typedef struct {
+  const void* x;
+  int64_t n;
+  uint8_t* q;
+  float* scale;
+  float* amax_out;
+  float* ring;
+  int32_t ring_len, ring_idx, ring_margin;
+  void* workspace;
+  size_t workspace_bytes;
+} hq_delayed_tensor;
+hq_status hq_quantize_fp8_delayed_batch(const hq_delayed_tensor* tensors, int32_t count, hq_dtype xt,
+                                        hq_fp8_format fmt, hq_stream_t stream);
+
+/*
  * Block-scaled FP8 GEMM (hip-quant README "Block-scaled Linear and Adafactor
  * Kernel Helpers": the pre-quantized block-scaled linear consumes FP8 bytes
  * and FP32 per-block scales of both operands; "Block-wise FP8 Scaling": one

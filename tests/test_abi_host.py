@@ -271,3 +271,31 @@ def test_blockscaled_gemm_rejections():
 def test_bounded_wait_probe_rejects_out_of_range_limits():
     assert L.hq_debug_bounded_wait(10, None) == INVALID             # below 1 us
     assert L.hq_debug_bounded_wait(3_000_000_000, None) == INVALID  # above 2 s
+
+
+def test_delayed_batch_rejections():
+    # argument checks of the batched delayed quantize, before any CUDA call
+    L = H.lib
+
+    def tensor(i, n=4096, ring_len=16, idx=0, margin=0, ring=True, ws=True, x=None):
+        base = BASE + i * 0x10000000
+        return H.DelayedTensor(base if x is None else x, n, base + 0x1000000, base + 0x2000000, None,
+                               (base + 0x3000000) if ring else None, ring_len, idx, margin,
+                               (base + 0x4000000) if ws else None, 256 if ws else 0)
+
+    def call(ts, count=None, xt=H.BF16, fmt=H.E4M3):
+        arr = (H.DelayedTensor * max(1, len(ts)))(*ts)
+        return L.hq_quantize_fp8_delayed_batch(arr, len(ts) if count is None else count, xt, fmt, None)
+
+    assert L.hq_quantize_fp8_delayed_batch(None, 1, H.BF16, H.E4M3, None) == INVALID
+    assert call([tensor(0)], count=0) == INVALID and call([tensor(0)] * 9) == INVALID
+    assert call([tensor(0)], xt=7) == INVALID and call([tensor(0)], fmt=5) == INVALID
+    assert call([tensor(0), tensor(1, ring=False)]) == INVALID          # a delayed quantize needs a ring
+    assert call([tensor(0, idx=16)]) == INVALID                         # ring_idx outside [0, len)
+    assert call([tensor(0, margin=127)]) == INVALID
+    assert call([tensor(0), tensor(1, ws=False)]) == INVALID            # no workspace
+    assert call([tensor(0, x=BASE + 2 + 1)]) == MISALIGNED              # x not aligned to bf16
+    t1 = tensor(1)
+    t1.q = BASE + 0x1000000 + 64                                        # tensor 1's codes over tensor 0's
+    assert call([tensor(0), t1]) == OVERLAP
+    assert "tensor 1" in L.hq_last_error().decode()

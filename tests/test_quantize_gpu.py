@@ -90,6 +90,28 @@ def test_per_token_register_kernel(fmt):
     H.hq_check_device_error()
 
 
+# Wide per-channel inputs of 4 MB and more on the single-launch kernel: a
+# ragged last column strip, row bands whose rows land in tensor memory,
+# shared memory and L2, NaN/Inf rows (exact path) and a finite input (fast
+# path).
+STRIP_CASES = [((4099, 4744), "bf16"), ((2000, 2400), "f32"), ((1100, 6000), "f16"), ((700, 9000), "bf16")]
+
+
+@pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
+def test_per_channel_wide(fmt):
+    cases = [make_input(shape, dtype, seed=8000 + i) for i, (shape, dtype) in enumerate(STRIP_CASES)]
+    rng = np.random.default_rng(8100 + fmt)
+    b = W.f32_to_bf16_bits((rng.standard_normal((2600, 8200)) * 2.0).astype(np.float32))
+    cases.append((b, dev_bf16(b)))
+    for xh, xd in cases:
+        q, s, a = run_gpu(xd, fmt, O.PER_CHANNEL)
+        qo, so, ao = O.quantize(xh, fmt, O.PER_CHANNEL)
+        np.testing.assert_array_equal(q, qo, err_msg="codes %s %s" % (xd.shape, xd.dtype))
+        np.testing.assert_array_equal(s.view(np.uint32), so.view(np.uint32))
+        np.testing.assert_array_equal(a.view(np.uint32), ao.view(np.uint32))
+    H.hq_check_device_error()
+
+
 @pytest.mark.parametrize("gran", [O.PER_TENSOR, O.PER_TOKEN, O.PER_CHANNEL])
 def test_misaligned_input_takes_scalar_path(gran):
     # x starting 2 bytes into an allocation: no 16-byte vectors possible
@@ -147,6 +169,38 @@ FUSED_CASES = {
     O.PER_TENSOR: [((1025, 2051), "f32"), ((2048, 1100), "bf16"), ((1501, 1401), "f16")],
     O.PER_CHANNEL: [((1025, 2052), "f32"), ((2048, 1104), "bf16"), ((1501, 1400), "f16"), ((130, 32768), "bf16")],
 }
+
+
+# Per-tensor inputs larger than every CTA's on-chip share (148 x 464 KB), so
+# that part of each CTA's range streams through L2 between the phases.
+# Ragged element tails, non-finite values in the streamed part (the exact
+# path) and in a CTA's on-chip part, and a finite input.
+@pytest.mark.parametrize("fmt", [O.E4M3, O.E5M2])
+def test_per_tensor_beyond_on_chip(fmt):
+    rng = np.random.default_rng(8200 + fmt)
+    cases = []
+    xf = (rng.standard_normal((4001, 5003)) * 3.0).astype(np.float32)  # 80 MB, n % 4 == 3
+    xf.reshape(-1)[[5, 77_000_000 // 4, xf.size - 3_000_000, xf.size - 2]] = [np.inf, np.nan, -np.inf, np.nan]
+    cases.append((xf, torch.from_numpy(xf).cuda()))
+    xb = W.f32_to_bf16_bits((rng.standard_normal((9001, 8191)) * 2.0).astype(np.float32))  # 147 MB, n % 8 == 7
+    cases.append((xb, dev_bf16(xb)))
+    xb2 = xb.copy()
+    xb2.reshape(-1)[xb2.size - 5_000_000] = 0x7FC0  # a NaN in the L2-streamed part
+    cases.append((xb2, dev_bf16(xb2)))
+    for xh, xd in cases:
+        rows, cols = xd.shape
+        ws = torch.zeros(H.hq_quantize_workspace_bytes(O.PER_TENSOR, rows, cols), dtype=torch.uint8, device="cuda")
+        qo, so, ao = O.quantize(xh, fmt, O.PER_TENSOR)
+        for _ in range(2):
+            a = torch.full((1,), -7.0, dtype=torch.float32, device="cuda")
+            q, s = H.hq_quantize_fp8(xd, fmt, O.PER_TENSOR, amax_out=a, workspace=ws)
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(host(q), qo, err_msg="codes %s %s" % (xd.shape, xd.dtype))
+            np.testing.assert_array_equal(host(s).view(np.uint32), so.view(np.uint32))
+            np.testing.assert_array_equal(host(a).view(np.uint32), ao.view(np.uint32))
+            assert (host(ws) == 0).all()
+        del xd, q
+    H.hq_check_device_error()
 
 
 @pytest.mark.parametrize("gran", [O.PER_TENSOR, O.PER_CHANNEL])
@@ -232,4 +286,46 @@ def test_quantize_sweep_full_size(sweep_input, gran, fmt):
     assert np.array_equal(q, qo)
     if gran == O.PER_TOKEN:
         assert s[4321] == 1.0 and (q[4321] == 0).all()   # the all-zero row
+    H.hq_check_device_error()
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_delayed_batch_equals_separate_calls(dtype):
+    # hq_quantize_fp8_delayed_batch: several tensors' delayed quantizes in one
+    # launch give exactly the separate delayed calls' codes, scales, amax and
+    # rings, step after step, and the oracle's
+    L = 16
+    shapes = [(64, 1000), (3, 5), (0, 8), (257, 4104), (1, 8)]
+    rings_b = [torch.from_numpy(np.r_[np.zeros(L, np.float32), 1.0, 0.0].astype(np.float32)).cuda() for _ in shapes]
+    rings_s = [r.clone() for r in rings_b]
+    rings_o = [np.r_[np.zeros(L, np.float32), 1.0, 0.0].astype(np.float32) for _ in shapes]
+    for step in range(5):
+        items, hosts, devs = [], [], []
+        for i, shape in enumerate(shapes):
+            xh, xd = make_input(shape, dtype, seed=9000 + 100 * step + i)
+            if i == 3 and xd.numel() > 1:  # a view one element in: not 16-byte aligned
+                buf = torch.empty(xd.numel() + 1, dtype=xd.dtype, device="cuda")
+                buf[1:] = xd.reshape(-1)
+                xd = buf[1:].view(shape)
+            hosts.append(xh)
+            devs.append(xd)
+            items.append(dict(x=xd, ring=rings_b[i], ring_idx=(step + i) % L, ring_margin=step % 3,
+                              amax_out=torch.full((1,), -7.0, device="cuda")))
+        outs = H.hq_quantize_fp8_delayed_batch(items, H.E5M2 if step % 2 else H.E4M3)
+        fmt = O.E5M2 if step % 2 else O.E4M3
+        for i, shape in enumerate(shapes):
+            a_s = torch.full((1,), -7.0, device="cuda")
+            q_s, s_s = H.hq_quantize_fp8(devs[i], fmt, H.PER_TENSOR, amax_out=a_s, ring=rings_s[i],
+                                         ring_idx=(step + i) % L, ring_margin=step % 3)
+            torch.cuda.synchronize()
+            q_b, s_b = outs[i]
+            assert torch.equal(q_b.reshape(q_s.shape), q_s), (step, shape)
+            assert torch.equal(s_b.view(torch.int32), s_s.view(torch.int32))
+            assert torch.equal(items[i]["amax_out"].view(torch.int32), a_s.view(torch.int32))
+            assert torch.equal(rings_b[i].view(torch.int32), rings_s[i].view(torch.int32))
+            qo, so, ao = O.quantize(hosts[i].reshape(shape), fmt, O.PER_TENSOR, ring=rings_o[i],
+                                    ring_idx=(step + i) % L, ring_margin=step % 3)
+            np.testing.assert_array_equal(host(q_b).reshape(qo.shape), qo)
+            np.testing.assert_array_equal(host(s_b).view(np.uint32), so.view(np.uint32))
+            np.testing.assert_array_equal(host(rings_b[i]).view(np.uint32), rings_o[i].view(np.uint32))
     H.hq_check_device_error()
