@@ -60,7 +60,8 @@ def dist_env():
 #   blocks of 128 and 32, stochastic E5M2 at 128) and the bf16 dequantize.
 # blockscaled, blockscaled32: the large layer with block-wise scales along K
 #   (E4M3, blocks of 128 / 32): X and W quantized block-wise every step, then
-#   the block-scaled GEMM; blockscaled_mid: M=4096, N=8192 (the ncu capture).
+#   the block-scaled GEMM; blockscaled_mid / blockscaled32_mid: M=4096,
+#   N=8192 at blocks of 128 / 32 (the ncu captures).
 # moe / moe_bf16: per-token quantize of the routed tokens + grouped a8w8 GEMM
 #   over 64 experts (W quantized once); the bf16 grouped GEMM alone.
 WORKLOADS = {
@@ -78,6 +79,7 @@ WORKLOADS = {
     "blockscaled": dict(kind="blockscaled", M=16384, N=28672, K=8192, block=128),
     "blockscaled32": dict(kind="blockscaled", M=16384, N=28672, K=8192, block=32),
     "blockscaled_mid": dict(kind="blockscaled", M=4096, N=8192, K=8192, block=128),
+    "blockscaled32_mid": dict(kind="blockscaled", M=4096, N=8192, K=8192, block=32),
     "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
     "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }

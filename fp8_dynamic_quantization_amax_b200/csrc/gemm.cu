@@ -1161,8 +1161,13 @@ cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
   // 256-wide tiles halve the A bytes per MMA cycle; worth a ragged last N
   // tile once N is large enough
   const bool wide = ((a.N % 256 == 0) && a.N >= 2048 && a.M >= 256) || (a.offsets != nullptr && a.N >= 1024);
-  // Large dense GEMMs run on CTA pairs (256 x 256 tiles).
-  const bool pair = a.offsets == nullptr && a.kind == 0 && (a.N % 256 == 0) && a.N >= 2048 && a.M >= 512;
+  // Large dense GEMMs run on CTA pairs (256 x 256 tiles).  Below M = 4096
+  // only with much work: for M = 1024 .. 3072 at K = 1024 .. 4096 the 1-CTA
+  // 128 x 256 tiles measured 2-7 % faster (the pair's set-up and coarser
+  // last round weigh more in a 15-40 us GEMM); at M = 2048, N = 28672,
+  // K = 8192 the pair was 3 % faster.
+  const bool pair = a.offsets == nullptr && a.kind == 0 && (a.N % 256 == 0) && a.N >= 2048 &&
+                    (a.M >= 4096 || (a.M >= 512 && static_cast<double>(a.M) * a.N * a.K >= 137438953472.0));  // 2^37
   // 256 x 512 pair tiles read a quarter fewer operand bytes per flop; with
   // enough M their coarser last round costs little
   if (pair && a.N % 512 == 0 && a.M >= 8192) return run2<0, 256, 2, 4>(a, msg);

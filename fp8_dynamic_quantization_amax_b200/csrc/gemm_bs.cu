@@ -26,6 +26,14 @@
 //               acc += partial * (xs[m,b] * ws[n,b]) in registers with packed
 //               f32x2 multiplies and fmas, and the slot is handed back;
 //               after the last block, + bias, round to bf16, 16-byte stores.
+//   warp 10     block-scale loader: per tile and chunk of 4 blocks, the
+//               tile's 128 xs rows and 128 ws rows (one 16-byte load per row
+//               when nb % 4 == 0), written transposed ([block][row]) into a
+//               ring of shared-memory slots.  The scales of a row are strided
+//               by nb in memory, so a warp-wide load of one block's scales
+//               touches 32 cache lines; loading 4 blocks per row once per CTA
+//               (instead of per epilogue warp and block) keeps the L1 load
+//               pipe, which the per-warp loads saturated, out of the way.
 // Persistent CTAs, one per SM, tiles in groups of 8 M tiles.  Every wait is
 // bounded: on a stalled barrier the CTA sets the device error word, drains
 // what it has in flight, frees TMEM and exits.
@@ -49,9 +57,12 @@ constexpr int kBsStages = 6;
 constexpr int kBsAcc = 4;                            // TMEM accumulators (4 x 128 columns)
 constexpr int kBsGroupBlocks = 2;                    // scale blocks per handshake
 constexpr int kBsSlots = kBsAcc / kBsGroupBlocks;    // groups in flight
-constexpr int kBsThreads = 320;                      // TMA, MMA, 8 epilogue warps
+constexpr int kBsThreads = 352;                      // TMA, MMA, 8 epilogue warps, scale loader
 constexpr int kBsOperandBytes = kBsTile * 128;       // one 128 x 128-byte K slice
-constexpr int kBsSmem = kBsStages * 2 * kBsOperandBytes + 8 * 64 * kBsGroupBlocks * 4 + 1024;
+constexpr int kBsChunk = 4;                          // scale blocks per loader slot
+constexpr int kBsScSlots = 4;                        // loader slots in flight
+constexpr int kBsScBytes = 2 * kBsChunk * kBsTile * 4;  // xs and ws of one chunk: [2][kBsChunk][128] f32
+constexpr int kBsSmem = kBsStages * 2 * kBsOperandBytes + kBsScSlots * kBsScBytes + 1024;
 constexpr int kBsGroupM = 8;
 
 struct BsParams {
@@ -63,6 +74,7 @@ struct BsParams {
   int m_tiles, n_tiles;
   const float* xs;       // [M, nb]
   const float* ws;       // [N, nb]
+  int sc_vec;            // 1: nb % 4 == 0 and both scale arrays 16-byte aligned (16-byte scale loads)
   const uint16_t* bias;  // bf16 [N] or null
   uint16_t* out;         // bf16 [M, N]
   uint32_t idesc;
@@ -75,19 +87,36 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 }
 
 // (a0, a1) += (p0, p1) * ((w0, w1) * (x, x)): one packed multiply and one
-// packed fma, each IEEE round-to-nearest per lane.
+// packed fma (FMUL2 / FFMA2), each IEEE round-to-nearest per lane.
 __device__ __forceinline__ void promote2(float& a0, float& a1, uint32_t p0, uint32_t p1, float w0, float w1,
                                          float x) {
-  asm("{\n\t.reg .b64 acc, prt, wsc, xsc;\n\t"
-      "mov.b64 acc, {%0, %1};\n\t"
-      "mov.b64 prt, {%2, %3};\n\t"
-      "mov.b64 wsc, {%4, %5};\n\t"
-      "mov.b64 xsc, {%6, %6};\n\t"
-      "mul.rn.f32x2 wsc, wsc, xsc;\n\t"
-      "fma.rn.f32x2 acc, prt, wsc, acc;\n\t"
-      "mov.b64 {%0, %1}, acc;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "r"(p0), "r"(p1), "f"(w0), "f"(w1), "f"(x));
+  const float2 r = __ffma2_rn(make_float2(__uint_as_float(p0), __uint_as_float(p1)),
+                              __fmul2_rn(make_float2(w0, w1), make_float2(x, x)), make_float2(a0, a1));
+  a0 = r.x;
+  a1 = r.y;
+}
+
+// 32 TMEM lanes x 64 columns of 32-bit in one load and its wait.  No memory
+// clobber: TMEM is not memory the compiler sees, so shared-memory loads may
+// move across it; the volatile asm keeps its order against the tcgen05
+// fences, which are volatile asm too.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]),
+        "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]),
+        "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]),
+        "=r"(v[48]), "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]),
+        "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]), "=r"(v[63])
+      : "r"(taddr));
 }
 
 __device__ __forceinline__ void tile_coords(int t, const BsParams& p, int& m0, int& n0) {
@@ -107,6 +136,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   __shared__ __align__(8) uint64_t empty_bar[kBsStages];
   __shared__ __align__(8) uint64_t afull_bar[kBsSlots];
   __shared__ __align__(8) uint64_t aempty_bar[kBsSlots];
+  __shared__ __align__(8) uint64_t sfull_bar[kBsScSlots];
+  __shared__ __align__(8) uint64_t sempty_bar[kBsScSlots];
   __shared__ __align__(8) uint64_t final_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -115,7 +146,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-byte aligned stages
   uint8_t* sA = smem;
   uint8_t* sB = smem + kBsStages * kBsOperandBytes;
-  float* sWs = reinterpret_cast<float*>(smem + 2 * kBsStages * kBsOperandBytes);  // per epilogue warp
+  // scale slots: [slot][xs | ws][block of the chunk][128 rows]
+  float* sSc = reinterpret_cast<float*>(smem + 2 * kBsStages * kBsOperandBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -127,6 +159,10 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     for (int a = 0; a < kBsSlots; ++a) {
       ptx::mbar_init(&afull_bar[a], 1);
       ptx::mbar_init(&aempty_bar[a], 8);  // one arrive per epilogue warp
+    }
+    for (int a = 0; a < kBsScSlots; ++a) {
+      ptx::mbar_init(&sfull_bar[a], 1);   // the loader's lane 0
+      ptx::mbar_init(&sempty_bar[a], 8);  // one arrive per epilogue warp
     }
     ptx::mbar_init(&final_bar, 1);
     abort_flag = 0;
@@ -327,13 +363,13 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 10) {
     // -------------------------------------------------------- epilogue
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int half = ew >> 2;
-    float* wsh = sWs + ew * 64 * kBsGroupBlocks;  // [block of the group][64 columns]
     uint32_t jg = 0;
+    uint32_t cs = 0, cph = 0;  // scale slot ring position
     bool stop = false;
     for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
       int m0, n0;
@@ -341,37 +377,11 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       const int row = m0 + quad * 32 + lane;
       const bool vrow = row < p.M;
       const int c0 = n0 + half * 64;  // this warp's first column
-      const float* xrow = p.xs + static_cast<int64_t>(vrow ? row : 0) * p.nb;
-      const bool v0 = c0 + lane < p.N, v1 = c0 + 32 + lane < p.N;
-      const float* wcol0 = p.ws + static_cast<int64_t>(v0 ? c0 + lane : 0) * p.nb;
-      const float* wcol1 = p.ws + static_cast<int64_t>(v1 ? c0 + 32 + lane : 0) * p.nb;
       float acc[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
-      // scales of the next group, loaded one group ahead
-      float xn[kBsGroupBlocks], wn0[kBsGroupBlocks], wn1[kBsGroupBlocks];
-#pragma unroll
-      for (int i = 0; i < kBsGroupBlocks; ++i) {
-        const bool in = i < p.nb;
-        xn[i] = in ? __ldg(xrow + i) : 0.0f;
-        wn0[i] = (in && v0) ? __ldg(wcol0 + i) : 0.0f;
-        wn1[i] = (in && v1) ? __ldg(wcol1 + i) : 0.0f;
-      }
-      for (int b0 = 0; b0 < p.nb; b0 += kBsGroupBlocks, ++jg) {
-        float xb[kBsGroupBlocks];
-#pragma unroll
-        for (int i = 0; i < kBsGroupBlocks; ++i) {
-          xb[i] = xn[i];
-          wsh[i * 64 + lane] = wn0[i];
-          wsh[i * 64 + 32 + lane] = wn1[i];
-          const int bn = b0 + kBsGroupBlocks + i;
-          if (bn < p.nb) {
-            xn[i] = __ldg(xrow + bn);
-            wn0[i] = v0 ? __ldg(wcol0 + bn) : 0.0f;
-            wn1[i] = v1 ? __ldg(wcol1 + bn) : 0.0f;
-          }
-        }
-        __syncwarp();
+      const float* sc = sSc;  // the current chunk's slot
+      for (int b0 = 0; b0 < p.nb && !stop; b0 += kBsGroupBlocks, ++jg) {
         const uint32_t sl = jg % kBsSlots;
         const uint32_t sph = (jg / kBsSlots) & 1u;
         // the warp agrees on giving up: the TMEM loads below are warp-wide
@@ -382,21 +392,35 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int i = 0; i < kBsGroupBlocks; ++i) {
-          if (b0 + i >= p.nb) break;
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            uint32_t v[32];
-            tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (sl * kBsGroupBlocks + i) * kBsTile +
-                          static_cast<uint32_t>(half * 64 + ch * 32),
-                      v);
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 w = *reinterpret_cast<const float4*>(wsh + i * 64 + ch * 32 + e);
-              promote2(acc[ch * 32 + e], acc[ch * 32 + e + 1], v[e], v[e + 1], w.x, w.y, xb[i]);
-              promote2(acc[ch * 32 + e + 2], acc[ch * 32 + e + 3], v[e + 2], v[e + 3], w.z, w.w, xb[i]);
+          const int b = b0 + i;
+          if (b >= p.nb) break;
+          const int bi = b % kBsChunk;
+          if (bi == 0) {  // a chunk opens: its scales are in slot cs
+            if (__any_sync(0xFFFFFFFFu, !wait_bar(&sfull_bar[cs], cph, &abort_flag, p.err))) {
+              stop = true;
+              break;
             }
+            sc = sSc + cs * (2 * kBsChunk * kBsTile);
+          }
+          const float xb = sc[bi * kBsTile + quad * 32 + lane];
+          const float* wrow = sc + (kBsChunk + bi) * kBsTile + half * 64;
+          uint32_t v[64];
+          tmem_ld64(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (sl * kBsGroupBlocks + i) * kBsTile +
+                        static_cast<uint32_t>(half * 64),
+                    v);
+#pragma unroll
+          for (int e = 0; e < 64; e += 4) {
+            const float4 w = *reinterpret_cast<const float4*>(wrow + e);
+            promote2(acc[e], acc[e + 1], v[e], v[e + 1], w.x, w.y, xb);
+            promote2(acc[e + 2], acc[e + 3], v[e + 2], v[e + 3], w.z, w.w, xb);
+          }
+          if (bi == kBsChunk - 1 || b == p.nb - 1) {  // the chunk's last block: hand its slot back
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sempty_bar[cs]);
+            if (++cs == kBsScSlots) { cs = 0; cph ^= 1u; }
           }
         }
+        if (stop) break;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&aempty_bar[sl]);
@@ -424,6 +448,53 @@ __global__ void __launch_bounds__(kBsThreads, 1)
                                       pack_bf16x2(o[6], o[7]));
           *reinterpret_cast<uint4*>(orow + n) = st;
         }
+      }
+    }
+  } else {
+    // ------------------------------------------------------ scale loader
+    // Lane l fills rows l, l + 32, l + 64, l + 96 of the tile: xs of those
+    // rows and ws of those columns, kBsChunk blocks each; rows past M or N
+    // and blocks past nb read as zero.
+    uint32_t cs = 0, cph = 0;
+    bool stop = false;
+    for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
+      int m0, n0;
+      tile_coords(t, p, m0, n0);
+      for (int b0 = 0; b0 < p.nb; b0 += kBsChunk) {
+        if (__any_sync(0xFFFFFFFFu, !wait_bar(&sempty_bar[cs], cph ^ 1u, &abort_flag, p.err))) {
+          stop = true;
+          break;
+        }
+        float* sx = sSc + cs * (2 * kBsChunk * kBsTile);
+        float* sw = sx + kBsChunk * kBsTile;
+#pragma unroll
+        for (int j = 0; j < kBsTile / 32; ++j) {
+          const int r = lane + 32 * j;
+          float xv[kBsChunk], wv[kBsChunk];
+          const bool xin = m0 + r < p.M, win = n0 + r < p.N;
+          const float* xp = p.xs + static_cast<int64_t>(xin ? m0 + r : 0) * p.nb + b0;
+          const float* wp = p.ws + static_cast<int64_t>(win ? n0 + r : 0) * p.nb + b0;
+          if (p.sc_vec) {  // b0 + 4 <= nb
+            const float4 x4 = __ldg(reinterpret_cast<const float4*>(xp));
+            const float4 w4 = __ldg(reinterpret_cast<const float4*>(wp));
+            xv[0] = x4.x; xv[1] = x4.y; xv[2] = x4.z; xv[3] = x4.w;
+            wv[0] = w4.x; wv[1] = w4.y; wv[2] = w4.z; wv[3] = w4.w;
+          } else {
+#pragma unroll
+            for (int i = 0; i < kBsChunk; ++i) {
+              xv[i] = (b0 + i < p.nb) ? __ldg(xp + i) : 0.0f;
+              wv[i] = (b0 + i < p.nb) ? __ldg(wp + i) : 0.0f;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < kBsChunk; ++i) {
+            sx[i * kBsTile + r] = xin ? xv[i] : 0.0f;
+            sw[i * kBsTile + r] = win ? wv[i] : 0.0f;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sfull_bar[cs]);  // releases the lanes' stores to the epilogue
+        if (++cs == kBsScSlots) { cs = 0; cph ^= 1u; }
       }
     }
   }
@@ -475,6 +546,10 @@ cudaError_t launch_gemm_blockscaled(const BlockScaledGemmArgs& a, std::string* m
   p.n_tiles = static_cast<int>((a.N + kBsTile - 1) / kBsTile);
   p.xs = a.x_scales;
   p.ws = a.w_scales;
+  p.sc_vec = (p.nb % 4 == 0 && reinterpret_cast<uintptr_t>(a.x_scales) % 16 == 0 &&
+              reinterpret_cast<uintptr_t>(a.w_scales) % 16 == 0)
+                 ? 1
+                 : 0;
   p.bias = static_cast<const uint16_t*>(a.bias);
   p.out = static_cast<uint16_t*>(a.out);
   p.idesc = (1u << 4)                                         // D: FP32

@@ -22,7 +22,11 @@ pytestmark = pytest.mark.gpu
 
 # (M, N, K, block)
 SHAPES = [(1, 8, 16, 32), (7, 24, 80, 32), (130, 136, 256, 32), (200, 264, 384, 64), (128, 128, 512, 128),
-          (257, 392, 1040, 256), (64, 128, 4096, 32), (300, 520, 272, 96), (129, 256, 2048, 128)]
+          (257, 392, 1040, 256), (64, 128, 4096, 32), (300, 520, 272, 96), (129, 256, 2048, 128),
+          # more 128 x 128 tiles than SMs: CTAs walk several tiles, so the
+          # accumulator and scale rings wrap across tile boundaries (nb = 8:
+          # 16-byte scale loads; nb = 7: a partial last chunk of scales)
+          (1280, 2048, 256, 32), (1300, 2056, 208, 32)]
 
 
 def rand_codes(rng, shape, fmt):

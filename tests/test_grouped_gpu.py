@@ -40,6 +40,8 @@ CASES = [  # (counts per expert, N, K)
     ([520, 0, 17], 1040, 160),
     # N = 1408 with a ragged K and a partial 256-row tile in every expert
     ([520, 0, 17, 700], 1408, 96),
+    # N = 1032: a last column tile of 8 columns (N % 16 = 8)
+    ([300, 5, 260], 1032, 64),
 ]
 
 
