@@ -187,6 +187,11 @@ def test_per_tensor_beyond_on_chip(fmt):
     xb2 = xb.copy()
     xb2.reshape(-1)[xb2.size - 5_000_000] = 0x7FC0  # a NaN in the L2-streamed part
     cases.append((xb2, dev_bf16(xb2)))
+    # the largest finite value and a NaN both in the last CTA's streamed part
+    xb3 = xb.copy()
+    big = int(W.f32_to_bf16_bits(np.float32(1.0e4)).reshape(-1)[0])
+    xb3.reshape(-1)[[xb3.size - 1000, xb3.size - 2_000_000]] = [big, 0x7FC0]
+    cases.append((xb3, dev_bf16(xb3)))
     for xh, xd in cases:
         rows, cols = xd.shape
         ws = torch.zeros(H.hq_quantize_workspace_bytes(O.PER_TENSOR, rows, cols), dtype=torch.uint8, device="cuda")
