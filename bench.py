@@ -95,8 +95,10 @@ def workload_desc(name, cfg):
     if k == "backward":
         return ("backward of the large a8w8 layer: grad g bf16 [%d,%d] ~N(0,1e-3) quantized per tensor with a "
                 "delayed ring into row-major and transposed codes; W bf16 [%d,%d] and X bf16 [%d,%d] re-quantized "
-                "transposed with their forward multipliers; dX = g W [%d,%d], dW = g^T X [%d,%d] on the NT GEMM" %
-                (cfg["M"], cfg["N"], cfg["N"], cfg["K"], cfg["M"], cfg["K"], cfg["M"], cfg["K"], cfg["N"], cfg["K"]))
+                "transposed with their forward multipliers; grad_bias = g summed over rows, bf16 [%d]; "
+                "dX = g W [%d,%d], dW = g^T X [%d,%d] on the NT GEMM" %
+                (cfg["M"], cfg["N"], cfg["N"], cfg["K"], cfg["M"], cfg["K"], cfg["N"], cfg["M"], cfg["K"], cfg["N"],
+                 cfg["K"]))
     if k == "stack":
         return ("delayed-scaling linear stack: X_t bf16 [2048,1024] (std 0.5 -> 8 over 200 steps), W_up bf16 "
                 "[4096,1024], W_down bf16 [1024,4096] ~N(0,0.02); per-tensor E4M3 with four amax-history rings "
@@ -364,9 +366,12 @@ def build(args, cfg, rank, dev, stream, peaks):
         sg, sw, sx = (torch.empty((1,), dtype=torch.float32, device=dev) for _ in range(3))
         dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
         dW = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        db = torch.empty((N,), dtype=torch.bfloat16, device=dev)
         dX_host = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
         dW_host = torch.empty((N, K), dtype=torch.bfloat16).pin_memory()
+        db_host = torch.empty((N,), dtype=torch.bfloat16).pin_memory()
         wsg, wsw, wsx = (torch.zeros(256, dtype=torch.uint8, device=dev) for _ in range(3))
+        wsb = torch.zeros(hq.hq_grad_bias_workspace_bytes(M, N), dtype=torch.uint8, device=dev)
         lib, P = hq.lib, (lambda t: None if t is None else t.data_ptr())
         st = stream.cuda_stream
         counter = [0]
@@ -387,15 +392,20 @@ def build(args, cfg, rank, dev, stream, peaks):
             hq.hq_gemm_a8w8(g8, wT8, sg, sw, hq.E4M3, out=dX, stream=stream)
             hq.hq_gemm_a8w8(gT8, xT8, sg, sx, hq.E4M3, out=dW, stream=stream)
 
-        calls = [("quantize g, W^T, X^T", quant, 3), ("dX and dW GEMMs", gemms, 2)]
+        def grad_bias():
+            hq.check(lib.hq_grad_bias(P(g), hq.BF16, M, N, P(db), P(wsb), wsb.numel(), st))
+
+        calls = [("quantize g, W^T, X^T", quant, 3), ("grad_bias", grad_bias, 1), ("dX and dW GEMMs", gemms, 2)]
 
         def e2e():
             g.copy_(g_host, non_blocking=True)
             x.copy_(x_host, non_blocking=True)
             quant()
+            grad_bias()
             gemms()
             dX_host.copy_(dX, non_blocking=True)
             dW_host.copy_(dW, non_blocking=True)
+            db_host.copy_(db, non_blocking=True)
 
         flops = 2.0 * 2 * M * N * K
 
@@ -409,13 +419,17 @@ def build(args, cfg, rank, dev, stream, peaks):
         def extras(ms):
             qbytes = (M * N * 2 + 2 * M * N) + (N * K * 2 + N * K) + (M * K * 2 + M * K)
             gb = qbytes / (ms["quantize g, W^T, X^T"] / 1e3) / 1e9
+            bb = (M * N * 2 + N * 2) / (ms["grad_bias"] / 1e3) / 1e9
             return {"quantize_transpose": {"ms": round(ms["quantize g, W^T, X^T"], 4), "GB/s": round(gb, 1),
                                            "frac_hbm": round(gb / peaks["hbm_gbs"], 4),
                                            "bytes": "g: 2 B read + 2 x 1 B codes; W, X: 2 B read + 1 B codes"},
+                    "grad_bias": {"ms": round(ms["grad_bias"], 4), "GB/s": round(bb, 1),
+                                  "frac_hbm": round(bb / peaks["hbm_gbs"], 4),
+                                  "bytes": "g: 2 B read per element + 2 B per column"},
                     "gemm_ms": round(ms["dX and dW GEMMs"], 4)}
 
         return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=(M * N + M * K) * 2,
-                    d2h=(M * K + N * K) * 2, roofline=roofline, extras=extras, flush=None,
+                    d2h=(M * K + N * K + N) * 2, roofline=roofline, extras=extras, flush=None,
                     l2="inputs larger than L2 (g %d MB, X %d MB, W %d MB); no flush" %
                        (M * N * 2 >> 20, M * K * 2 >> 20, N * K * 2 >> 20))
 

@@ -24,7 +24,8 @@ EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_q
             "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic",
             "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_blockscaled",
             "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
-            "hq_quantize_fp8_noalloc", "hq_quantize_fp8_delayed_batch", "hq_debug_bounded_wait",
+            "hq_quantize_fp8_noalloc", "hq_quantize_fp8_delayed_batch", "hq_grad_bias",
+            "hq_grad_bias_workspace_bytes", "hq_debug_bounded_wait",
             "hq_check_device_error", "hq_last_error", "hq_version"]
 NOALLOC_SCRATCH_BYTES = 256 * 1024
 
@@ -76,6 +77,10 @@ def _load():
     L.hq_quantize_e5m2_stochastic.restype = ci
     L.hq_quantize_fp8_transpose.argtypes = [P, ci, i64, i64, ci, P, P, P, P, P, P, i32, i32, i32, P, sz, P]
     L.hq_quantize_fp8_transpose.restype = ci
+    L.hq_grad_bias_workspace_bytes.argtypes = [i64, i64]
+    L.hq_grad_bias_workspace_bytes.restype = sz
+    L.hq_grad_bias.argtypes = [P, ci, i64, i64, P, P, sz, P]
+    L.hq_grad_bias.restype = ci
     L.hq_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, i64, i64, i64, P, P]
     L.hq_gemm_a8w8.restype = ci
     L.hq_gemm_a8w8_ex.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P, P, ci, P, P, P, i32, i32, i32, P,
@@ -304,6 +309,28 @@ def hq_quantize_fp8_transpose(x, fmt=E4M3, q=False, multiplier=None, amax_out=No
                                         _ptr(amax_out), _ptr(multiplier), _ptr(ring), ring_len, ring_idx,
                                         ring_margin, _ptr(workspace), workspace.numel(), _stream(stream)))
     return qo, qt, scales
+
+
+def hq_grad_bias_workspace_bytes(rows, cols):
+    return lib.hq_grad_bias_workspace_bytes(rows, cols)
+
+
+def hq_grad_bias(g, out=None, workspace=None, stream=None):
+    """Bias gradient of a 2-D CUDA tensor g [rows, cols]: the column sums,
+    accumulated in f32, in g's dtype ([cols]).  Returns out."""
+    if g.dim() != 2:
+        raise ValueError("g must be 2-D")
+    if g.dtype not in _DT:
+        raise ValueError("g must be float32, bfloat16 or float16")
+    g = g.contiguous()
+    rows, cols = g.shape
+    if out is None:
+        out = torch.empty((cols,), dtype=g.dtype, device=g.device)
+    if workspace is None:
+        workspace = _workspace(g.device, hq_grad_bias_workspace_bytes(rows, cols), slot="grad_bias")
+    check(lib.hq_grad_bias(_ptr(g), _DT[g.dtype], rows, cols, _ptr(out), _ptr(workspace),
+                           0 if workspace is None else workspace.numel(), _stream(stream)))
+    return out
 
 
 def hq_quantize_fp8_noalloc(x, fmt=E4M3, gran=PER_TOKEN, q=None, scales=None, amax_out=None, ring=None,

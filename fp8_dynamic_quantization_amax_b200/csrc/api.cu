@@ -409,6 +409,40 @@ hq_status hq_dequantize_fp8_blockwise(const uint8_t* q, hq_fp8_format fmt, int64
                   "block-wise dequantize launch");
 }
 
+size_t hq_grad_bias_workspace_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return 0;
+  return hq::grad_bias_workspace_bytes(rows, cols);
+}
+
+hq_status hq_grad_bias(const void* g, hq_dtype gt, int64_t rows, int64_t cols, void* out, void* workspace,
+                       size_t workspace_bytes, hq_stream_t stream) {
+  if (gt != HQ_F32 && gt != HQ_BF16 && gt != HQ_F16) return fail(HQ_ERR_INVALID_ARG, "invalid dtype %d", (int)gt);
+  if (rows < 0 || cols < 0) return fail(HQ_ERR_INVALID_ARG, "negative shape [%lld, %lld]", (long long)rows, (long long)cols);
+  if (rows >= k2p31 || cols >= k2p31 || (cols > 0 && rows > (k2p40 - 1) / cols))
+    return fail(HQ_ERR_TOO_LARGE, "shape [%lld, %lld] is beyond the supported range", (long long)rows, (long long)cols);
+  if (cols == 0) return ok();
+  const size_t esize = (gt == HQ_F32) ? 4 : 2;
+  const size_t need = hq::grad_bias_workspace_bytes(rows, cols);
+  if (!out || !workspace || (rows > 0 && !g)) return fail(HQ_ERR_INVALID_ARG, "g, out and workspace must not be null");
+  if (workspace_bytes < need)
+    return fail(HQ_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+  if ((g && !is_aligned(g, esize)) || !is_aligned(out, esize))
+    return fail(HQ_ERR_MISALIGNED, "g and out must be aligned to their element size");
+  if (!is_aligned(workspace, 256)) return fail(HQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  const Range outs[] = {{out, static_cast<size_t>(cols) * esize, "out"}, {workspace, need, "workspace"}};
+  const Range ins[] = {{g, static_cast<size_t>(rows) * static_cast<size_t>(cols) * esize, "g"}};
+  hq_status s = check_overlaps(outs, 2, ins, 1);
+  if (s != HQ_OK) return s;
+  const Range devs[] = {{g, 0, "g"}, {out, 0, "out"}, {workspace, 0, "workspace"}};
+  s = check_device_ptrs(devs, 3);
+  if (s != HQ_OK) return s;
+  s = check_arch();
+  if (s != HQ_OK) return s;
+  return launched(hq::launch_grad_bias(g, static_cast<int>(gt), rows, cols, out, workspace,
+                                       reinterpret_cast<cudaStream_t>(stream)),
+                  "bias gradient launch");
+}
+
 hq_status hq_quantize_e5m2_stochastic(const void* x, hq_dtype xt, int64_t rows, int64_t cols, hq_granularity g,
                                       uint64_t seed, uint8_t* q, float* scales, float* amax_out, void* workspace,
                                       size_t workspace_bytes, hq_stream_t stream) {

@@ -60,6 +60,12 @@ cudaError_t launch_quantize_sr(const QuantizeArgs& a);
 // Block-wise quantize (scales [rows, ceil(cols / block)]) and dequantize;
 // block % 16 == 0, cols % 16 == 0, 16-byte aligned buffers.
 cudaError_t launch_quantize_blockwise(const QuantizeArgs& a, int64_t block, bool stochastic);
+// Bias gradient: column sums of g [rows, cols] (xt 0 f32, 1 bf16, 2 f16) in
+// f32, written in g's dtype; ws as grad_bias_workspace_bytes, its counters
+// zero between calls.
+size_t grad_bias_workspace_bytes(int64_t rows, int64_t cols);
+cudaError_t launch_grad_bias(const void* g, int xt, int64_t rows, int64_t cols, void* out, void* ws,
+                             cudaStream_t stream);
 cudaError_t launch_dequantize_blockwise(const uint8_t* q, int fmt, int64_t rows, int64_t cols, int64_t block,
                                         const float* scales, bool bf16_out, void* out, cudaStream_t stream);
 

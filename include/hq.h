@@ -319,6 +319,35 @@ hq_status hq_quantize_fp8_transpose(const void* x, hq_dtype xt, int64_t rows, in
                                     void* workspace, size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * Bias gradient of a linear layer's backward pass (AstrAI
+ * csrc/kernels/fp8/ops.cu linear_backward_fp8: the bias gradient is g
+ * summed over dim 0 and cast back to g's dtype):
+ *   out[c] = dtype( sum over r of g[r, c] ),  c in [0, cols)
+ * The sum is accumulated in f32 in a fixed order (the rows of fixed bands
+ * in order, then the bands in order), so repeated calls give identical
+ * bits; it is rounded once to g's dtype (bf16 / f16 round-to-nearest-even,
+ * or f32).  NaN and Inf propagate as in an f32 sum.  rows == 0 gives zeros.
+ *
+ * Arguments:
+ *   g          device, [rows, cols] row-major, f32 / bf16 / f16 (gt),
+ *              aligned to its element size (16-byte alignment of g and
+ *              of every row takes the vector path)
+ *   out        device, [cols] of gt, aligned to its element size
+ *   workspace  device, >= hq_grad_bias_workspace_bytes(rows, cols) bytes,
+ *              256-byte aligned, zero on entry and zero again on return (a
+ *              counter per column strip; the rest holds per-band partial
+ *              sums and need not be zero)
+ * Errors: HQ_ERR_INVALID_ARG (null, negative shape, bad dtype, workspace
+ *   too small), HQ_ERR_MISALIGNED, HQ_ERR_OVERLAP (out or workspace
+ *   overlapping g or each other), HQ_ERR_WRONG_DEVICE,
+ *   HQ_ERR_UNSUPPORTED_ARCH, HQ_ERR_TOO_LARGE (rows or cols >= 2^31, or
+ *   rows * cols >= 2^40), HQ_ERR_CUDA.  cols == 0 is a no-op.
+ */
+size_t hq_grad_bias_workspace_bytes(int64_t rows, int64_t cols);
+hq_status hq_grad_bias(const void* g, hq_dtype gt, int64_t rows, int64_t cols, void* out, void* workspace,
+                       size_t workspace_bytes, hq_stream_t stream);
+
+/*
  * Scaled FP8 GEMM, NT layout, into a caller-owned bf16 buffer:
  *   out[m, n] = bf16_rn( acc[m, n] * x_scale[m'] * w_scale[n'] ),
  *   acc[m, n] = sum_k dec(xq[m, k]) * dec(wq[n, k])   (FP32 accumulation)

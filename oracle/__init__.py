@@ -80,6 +80,10 @@ def lib():
         L.hqo_decode_array.restype = None
         L.hqo_ring_update.argtypes = [ctypes.c_float, ci, P, ci, ci, ci]
         L.hqo_ring_update.restype = None
+        L.hqo_double_to_f16.argtypes = [ctypes.c_double]
+        L.hqo_double_to_f16.restype = ctypes.c_uint16
+        L.hqo_grad_bias.argtypes = [P, ci, i64, i64, P, P]
+        L.hqo_grad_bias.restype = None
         _lib = L
     return _lib
 
@@ -337,6 +341,22 @@ def grouped_gemm_bf16(x, w, offsets, out=None):
     if rc != 0:
         raise ValueError("oracle grouped gemm: malformed offsets")
     return out
+
+
+def double_to_f16(v: float) -> int:
+    return lib().hqo_double_to_f16(v)
+
+
+def grad_bias(g: np.ndarray, return_ref: bool = False):
+    """Bias gradient: column sums of g [rows, cols] (fp64, rows in order),
+    rounded once to g's dtype (bf16 bit patterns, float16 or float32)."""
+    g = np.ascontiguousarray(g)
+    rows, cols = g.shape
+    dt = _dtype_code(g)
+    out = np.empty(cols, {F32: np.float32, BF16: np.uint16, F16: np.float16}[dt])
+    ref = np.empty(cols, np.float64) if return_ref else None
+    lib().hqo_grad_bias(_p(g), dt, rows, cols, _p(out), _p(ref))
+    return (out, ref) if return_ref else out
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -21,7 +21,9 @@
  *        hist[idx], reduces the window, publishes the next scale; ring
  *        packs [hist | scale | counter]), pack_quantize_params (len =
  *        numel-2, idx = caller's slot, margin from the recipe), mm_fp8
- *        (out = a @ b^T * (sa*sb), FP32 accumulate).
+ *        (out = a @ b^T * (sa*sb), FP32 accumulate), linear_backward_fp8
+ *        (the bias gradient is the sum of g over its rows, cast back to
+ *        g's dtype).
  *  [QS]  fuel-ir 0.22.4 src/quant_scale.rs: ScaleGranularity (PerTensor
  *        f32[1], PerToken f32[n_rows], PerChannel f32[n_cols]) and
  *        scale_count.
@@ -665,4 +667,49 @@ void hqo_encode_sat_array(const float* y, int64_t n, int fmt, uint8_t* out) {
 void hqo_decode_array(const uint8_t* c, int64_t n, int fmt, double* out) {
   int64_t i;
   for (i = 0; i < n; ++i) out[i] = hqo_decode(c[i], fmt);
+}
+
+/* ---------------------------------------------------------- bias gradient */
+
+/* Round a double to the nearest f16 (ties to even), once: 10 fraction bits,
+   exponent bias 15, subnormal step 2^-24, values from 65520 up to Inf. */
+uint16_t hqo_double_to_f16(double v) {
+  double a, q, r;
+  int e;
+  uint16_t sign = (v < 0 || (v == 0.0 && signbit(v))) ? 0x8000 : 0;
+  if (isnan(v)) return 0x7E00;
+  a = fabs(v);
+  if (isinf(v)) return (uint16_t)(sign | 0x7C00);
+  if (a == 0.0) return sign;
+  if (a < ldexp(1.0, -14)) {
+    q = ldexp(1.0, -24);
+  } else {
+    frexp(a, &e);
+    q = ldexp(1.0, (e - 1) - 10);
+  }
+  r = nearbyint(a / q) * q;
+  if (r > 65504.0) return (uint16_t)(sign | 0x7C00);
+  if (r < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)(r / ldexp(1.0, -24)));
+  frexp(r, &e); /* r = f * 2^e, f in [0.5, 1): leading bit 2^(e-1) */
+  return (uint16_t)(sign | (uint16_t)((e - 1 + 15) << 10) |
+                    (uint16_t)(r / ldexp(1.0, e - 1) * 1024.0 - 1024.0));
+}
+
+/* Bias gradient ([AS] linear_backward_fp8: the sum of g over dim 0, cast
+   to g's dtype): sum[c] = sum over r of g[r, c] in fp64, rows in order,
+   then rounded once to g's dtype (bf16 or f16 ties-to-even, or f32).
+   out holds dtype elements [cols]; ref (optional) the fp64 sums. */
+void hqo_grad_bias(const void* g, int dtype, int64_t rows, int64_t cols, void* out, double* ref) {
+  int64_t r, c;
+  double* s = (double*)calloc((size_t)(cols > 0 ? cols : 1), sizeof(double));
+  if (!s) return;
+  for (r = 0; r < rows; ++r) /* row by row: each column's terms still added in row order */
+    for (c = 0; c < cols; ++c) s[c] += (double)load_elem(g, dtype, r * cols + c);
+  for (c = 0; c < cols; ++c) {
+    if (ref) ref[c] = s[c];
+    if (dtype == 0) ((float*)out)[c] = (float)s[c];
+    else if (dtype == 1) ((uint16_t*)out)[c] = hqo_double_to_bf16(s[c]);
+    else ((uint16_t*)out)[c] = hqo_double_to_f16(s[c]);
+  }
+  free(s);
 }

@@ -299,3 +299,25 @@ def test_delayed_batch_rejections():
     t1.q = BASE + 0x1000000 + 64                                        # tensor 1's codes over tensor 0's
     assert call([tensor(0), t1]) == OVERLAP
     assert "tensor 1" in L.hq_last_error().decode()
+
+
+def test_grad_bias_rejections():
+    # argument checks of the bias gradient, before any CUDA call
+    L = H.lib
+    need = H.hq_grad_bias_workspace_bytes(100, 64)
+    assert need == 256 + 4 * 64 * 4  # four bands (32 rows and more each) of partials, one strip counter (padded)
+    assert H.hq_grad_bias_workspace_bytes(16384, 28672) == 256 * ((28672 // 256 * 4 + 255) // 256) + 64 * 28672 * 4
+    assert H.hq_grad_bias_workspace_bytes(-1, 4) == 0
+    g, out, ws = BASE, BASE + 0x1000000, BASE + 0x2000000
+    assert L.hq_grad_bias(g, 9, 100, 64, out, ws, need, None) == INVALID            # dtype
+    assert L.hq_grad_bias(g, H.BF16, -1, 64, out, ws, need, None) == INVALID        # shape
+    assert L.hq_grad_bias(g, H.BF16, 1 << 31, 64, out, ws, need, None) == TOO_LARGE
+    assert L.hq_grad_bias(g, H.BF16, 100, 64, None, ws, need, None) == INVALID      # no out
+    assert L.hq_grad_bias(g, H.BF16, 100, 64, out, None, need, None) == INVALID     # no workspace
+    assert L.hq_grad_bias(g, H.BF16, 100, 64, out, ws, need - 4, None) == INVALID   # workspace too small
+    assert L.hq_grad_bias(g + 1, H.BF16, 100, 64, out, ws, need, None) == MISALIGNED
+    assert L.hq_grad_bias(g, H.F32, 100, 64, out + 2, ws, need, None) == MISALIGNED
+    assert L.hq_grad_bias(g, H.BF16, 100, 64, out, ws + 64, need, None) == MISALIGNED
+    assert L.hq_grad_bias(g, H.BF16, 100, 64, g + 64, ws, need, None) == OVERLAP     # out inside g
+    assert L.hq_grad_bias(g, H.BF16, 100, 64, out, g + 256, need, None) == OVERLAP   # workspace inside g
+    assert L.hq_grad_bias(g, H.BF16, 100, 0, out, ws, need, None) == OK              # cols == 0: nothing to do

@@ -117,3 +117,93 @@ def test_backward_gemms_vs_oracle(fmt):
                                                  gso, xso))
     np.testing.assert_array_equal(host(ring_d).view(np.uint32), ring.view(np.uint32))
     H.hq_check_device_error()
+
+
+# ------------------------------------------------------------ bias gradient
+# AstrAI ops.cu linear_backward_fp8: grad_bias = g summed over dim 0, in g's
+# dtype.  The GPU sums in f32 in a fixed order, the oracle in fp64; the
+# tolerance is the f32 summation bound (rows * 2^-24 * sum |g|, doubled for
+# the two levels of the kernel's sum) plus one step of the output dtype at
+# the result (a value near a rounding boundary may round either way).
+GB_SHAPES = [  # (rows, cols, dtype): vector and element paths, ragged strips and bands, one band and many
+    (1, 8, "bf16"), (7, 24, "f16"), (300, 1001, "f32"), (1000, 2056, "bf16"), (130, 36, "f16"),
+    (129, 4100, "f32"), (5000, 520, "bf16"), (9000, 264, "f16"), (0, 40, "bf16"),
+]
+
+
+def _as_f64(a, dtype):
+    if dtype == "bf16":
+        return O.bf16_bits_to_f32(a).astype(np.float64)
+    return np.asarray(a).astype(np.float64)
+
+
+def _step(v, dtype):
+    mant = {"bf16": 7, "f16": 10, "f32": 23}[dtype]
+    low = {"bf16": -133, "f16": -24, "f32": -149}[dtype]
+    e = np.floor(np.log2(np.maximum(np.abs(v), 1e-300)))
+    return np.maximum(2.0 ** (e - mant), 2.0 ** low)
+
+
+def _abs_col_sums(gh, dtype):
+    out = np.zeros(gh.shape[1], np.float64)
+    for i in range(0, gh.shape[0], 1024):  # in row chunks: the full-size g would not fit as fp64
+        v = _as_f64(gh[i:i + 1024], dtype)
+        out += np.abs(np.where(np.isfinite(v), v, 0.0)).sum(axis=0)
+    return out
+
+
+def _check_grad_bias(got, gh, dtype):
+    """got: the GPU result as bf16 bit patterns, f16 or f32 values."""
+    want, ref = O.grad_bias(gh, return_ref=True)
+    rows = gh.shape[0]
+    got64, want64 = _as_f64(got, dtype), _as_f64(want, dtype)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got64), nan)
+    inf = np.isinf(ref)
+    assert np.array_equal(got64[inf], ref[inf])
+    fin = ~(nan | inf)
+    bound = 2.0 * rows * 2.0 ** -24 * _abs_col_sums(gh, dtype)[fin]
+    err = np.abs(got64[fin] - ref[fin])
+    assert (err <= bound + _step(ref[fin], dtype)).all(), np.max(err - bound - _step(ref[fin], dtype))
+    # and never further than one output step from the oracle's own rounding
+    assert (np.abs(got64[fin] - want64[fin]) <= _step(want64[fin], dtype) + bound).all()
+
+
+def _fetch(t, dtype):
+    return host_bits(t) if dtype == "bf16" else host(t)
+
+
+@pytest.mark.parametrize("case", range(len(GB_SHAPES)))
+def test_grad_bias_vs_oracle(case):
+    rows, cols, dtype = GB_SHAPES[case]
+    gh, gd = make((rows, cols), dtype, seed=600 + case, specials=rows * cols >= 5000)
+    ws = torch.zeros(H.hq_grad_bias_workspace_bytes(rows, cols), dtype=torch.uint8, device="cuda")
+    got = [H.hq_grad_bias(gd, workspace=ws) for _ in range(2)]
+    torch.cuda.synchronize()
+    a, b = _fetch(got[0], dtype), _fetch(got[1], dtype)
+    assert np.array_equal(a.view(np.uint8), b.view(np.uint8))  # fixed order: identical bits
+    _check_grad_bias(a, gh, dtype)
+    assert (host(ws)[:256] == 0).all()  # the strip counters are back to zero
+    H.hq_check_device_error()
+
+
+def test_grad_bias_unaligned_rows_and_view():
+    # g a view whose rows start off the 16-byte grid: the element path
+    rows, cols = 777, 1029
+    gh, gd = make((rows, cols + 3), "bf16", seed=650, specials=False)
+    view = gd[:, 3:]  # not contiguous; the binding makes it contiguous
+    got = H.hq_grad_bias(view)
+    torch.cuda.synchronize()
+    _check_grad_bias(host_bits(got), np.ascontiguousarray(gh[:, 3:]), "bf16")
+
+
+def test_grad_bias_full_backward_shape():
+    # g of the large layer's backward ([16384, 28672] bf16, ~N(0, 1)):
+    # every column against the oracle
+    rows, cols = 16384, 28672
+    rng = np.random.default_rng(660)
+    gh = W.f32_to_bf16_bits(rng.standard_normal((rows, cols), dtype=np.float32))
+    got = H.hq_grad_bias(dev_bf16(gh))
+    torch.cuda.synchronize()
+    _check_grad_bias(host_bits(got), gh, "bf16")
+    H.hq_check_device_error()

@@ -865,3 +865,67 @@ def test_blockwise_round_trip_within_half_a_step(fmt, rel, sub):
     sc = np.repeat(s, block, axis=1)[:, :cols].astype(np.float64)
     err = np.abs(back - x.astype(np.float64))
     assert (err <= np.abs(x) * (rel + 2.0 ** -20) + sc * sub).all()
+
+
+# ------------------------------------------------------------ bias gradient
+# AstrAI ops.cu linear_backward_fp8: the bias gradient is g summed over dim 0
+# and cast back to g's dtype.
+
+
+def test_double_to_f16_matches_numpy():
+    # the oracle's own f16 rounding against numpy's double -> half cast (an
+    # independent implementation), over 12 decades and the edges: the largest
+    # finite value, the overflow threshold 65520, subnormals, signed zero, Inf
+    rng = np.random.default_rng(91)
+    v = rng.standard_normal(20000) * np.exp(rng.uniform(-25, 12, 20000))
+    v = np.concatenate([v, [65504.0, 65519.99, 65520.0, -65520.0, 1e-8, 6e-8, 2.98e-8, -0.0, 0.0,
+                            np.inf, -np.inf, 2.0 ** -24 * 1.5, 2.0 ** -14 * (1 - 2.0 ** -11)]])
+    mine = np.array([O.double_to_f16(float(x)) for x in v], np.uint16)
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16).view(np.uint16)
+    assert np.array_equal(mine, ref)
+    assert O.double_to_f16(float("nan")) & 0x7C00 == 0x7C00 and O.double_to_f16(float("nan")) & 0x3FF
+
+
+def test_grad_bias_closed_form():
+    # g[r, c] = (r + 1) * (c % 5 - 2): the column sums are (c % 5 - 2) * R(R+1)/2,
+    # exact in every dtype for R = 15 (120 * 2 = 240 < 256); a transposed or
+    # shifted index changes them
+    R, C = 15, 37
+    r = np.arange(1, R + 1, dtype=np.float64)[:, None]
+    c = (np.arange(C) % 5 - 2).astype(np.float64)[None, :]
+    g = r * c
+    want = (np.arange(C) % 5 - 2) * (R * (R + 1) // 2)
+    out32 = O.grad_bias(g.astype(np.float32))
+    assert np.array_equal(out32, want.astype(np.float32))
+    out16 = O.grad_bias(g.astype(np.float16))
+    assert np.array_equal(out16.astype(np.float64), want)
+    outb = O.grad_bias(W.f32_to_bf16_bits(g.astype(np.float32)))
+    assert np.array_equal(O.bf16_bits_to_f32(outb).astype(np.float64), want)
+    assert O.grad_bias(np.zeros((0, 4), np.float32)).tolist() == [0.0] * 4
+
+
+def test_grad_bias_is_the_rounded_exact_sum():
+    # random bf16 g: the fp64 sums (exact here: 300 terms of 8-bit
+    # significands within 2^40 of each other) against an exact integer
+    # re-summation, and the output is that sum rounded once to bf16
+    rng = np.random.default_rng(92)
+    R, C = 300, 41
+    x = (rng.standard_normal((R, C)) * 3).astype(np.float32)
+    x[np.abs(x) < 2.0 ** -30] = 0.0  # every value a multiple of 2^-40 after bf16 rounding
+    gb = W.f32_to_bf16_bits(x)
+    out, ref = O.grad_bias(gb, return_ref=True)
+    vals = O.bf16_bits_to_f32(gb).astype(np.float64)
+    scale = 2.0 ** 40
+    exact = (vals * scale).astype(np.int64).sum(axis=0) / scale  # integers: exact
+    assert np.array_equal(ref, exact)
+    assert np.array_equal(out, np.array([O.double_to_bf16(v) for v in exact], np.uint16))
+
+
+def test_grad_bias_non_finite():
+    g = np.ones((6, 4), np.float32)
+    g[2, 1] = np.nan
+    g[3, 2] = np.inf
+    g[1, 3], g[4, 3] = np.inf, -np.inf
+    out = O.grad_bias(g)
+    assert out[0] == 6.0 and np.isnan(out[1]) and out[2] == np.inf and np.isnan(out[3])
