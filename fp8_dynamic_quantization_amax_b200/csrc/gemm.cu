@@ -593,9 +593,9 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int acc = i & 1;
       const uint32_t acc_phase = (i >> 1) & 1;
-      // the warp agrees on giving up: the TMEM loads below are warp-wide
-      if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag))) break;
-      tc_fence_after();
+      // The tile's row and column scales do not depend on the accumulator:
+      // they are loaded before the wait, so their latency overlaps the
+      // tile's main loop instead of adding to the epilogue.
       const Tile T = decode_tile<kBM, BN>(t, p, tile_prefix, row_start);
       const int row0 = T.row_lo + quad * 32;
       const int row = row0 + lane;
@@ -605,15 +605,22 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       const int ncap = min(p.N, T.col0 + BN);  // end of this tile's columns
       float xsv = 0.0f;
       if (vrow) xsv = (KIND == 0) ? __ldg(p.xs + (p.xs_bcast ? 0 : row)) : 1.0f;
-      if (KIND == 0) {
+      float wpre[kMyChunks];
+      {
         const float* wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
-        for (int i = 0; half + 2 * i < kChunks; ++i) {
-          const int n = T.col0 + (half + 2 * i) * 32 + lane;
-          wsh[i * 32 + lane] = (n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < kMyChunks; ++j) {
+          const int ch = half + 2 * j;
+          const int n = T.col0 + ch * 32 + lane;
+          wpre[j] = (KIND != 0) ? 1.0f
+                                : ((ch < kChunks && n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f);
         }
-      } else {
-        for (int i = 0; half + 2 * i < kChunks; ++i) wsh[i * 32 + lane] = 1.0f;
       }
+      // the warp agrees on giving up: the TMEM loads below are warp-wide
+      if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int j = 0; j < kMyChunks; ++j) wsh[j * 32 + lane] = wpre[j];
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
@@ -1030,9 +1037,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int t = cluster; t < total; t += nclusters, ++i) {
       const int acc = i % kAccs;
       const uint32_t acc_phase = (i / kAccs) & 1;
-      // the warp agrees on giving up: the TMEM loads below are warp-wide
-      if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag))) break;
-      tc_fence_after();
+      // The tile's row and column scales do not depend on the accumulator:
+      // they are loaded before the wait, so their latency overlaps the
+      // tile's main loop instead of adding to the epilogue (with one
+      // 512-column accumulator the epilogue does not overlap the next tile).
       const Tile T = decode_tile<256, BN>(t, p, tile_prefix, row_start);
       const int row0 = T.row_lo + static_cast<int>(rank) * 128 + quad * 32;  // this warp's first row
       const int row = row0 + lane;
@@ -1041,16 +1049,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const bool tma_ok = row0 < T.row_hi && (p.offsets == nullptr || row0 + 32 <= T.row_hi);
       float xsv = 0.0f;
       if (vrow) xsv = (KIND == 0) ? __ldg(p.xs + (p.xs_bcast ? 0 : row)) : 1.0f;
-      if (KIND == 0) {
+      float wpre[kMyChunks];
+      {
         const float* wsp = p.ws + (p.ws_bcast ? 0 : static_cast<int64_t>(T.expert) * p.N);
-#pragma unroll 1
-        for (int j = 0; half + 2 * j < kChunks; ++j) {
-          const int n = T.col0 + (half + 2 * j) * 32 + lane;
-          wsh[j * 32 + lane] = (n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < kMyChunks; ++j) {
+          const int ch = half + 2 * j;
+          const int n = T.col0 + ch * 32 + lane;
+          wpre[j] = (KIND != 0) ? 1.0f
+                                : ((ch < kChunks && n < p.N) ? __ldg(wsp + (p.ws_bcast ? 0 : n)) : 0.0f);
         }
-      } else {
-        for (int j = 0; half + 2 * j < kChunks; ++j) wsh[j * 32 + lane] = 1.0f;
       }
+      // the warp agrees on giving up: the TMEM loads below are warp-wide
+      if (__any_sync(0xFFFFFFFFu, !mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int j = 0; j < kMyChunks; ++j) wsh[j * 32 + lane] = wpre[j];
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
