@@ -252,6 +252,46 @@ def build(args, cfg, rank, dev, stream, peaks):
                 c[1]()
             out_host.copy_(out, non_blocking=True)
 
+        e2e_pipelined = None
+        if kind == "layer":
+            # a second set of step inputs and outputs, for a double-buffered run
+            sets = [(x, w, out), (torch.empty_like(x), torch.empty_like(w), torch.empty_like(out))]
+            s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+            def e2e_pipelined(n, e0, e1):
+                """n steps through the public API, double-buffered: step i+1's
+                host-to-device copies (one copy stream) and step i-1's
+                device-to-host copy (another) overlap step i's kernels.  Every
+                step still copies its inputs in and its result out."""
+                h2d_done = [torch.cuda.Event() for _ in range(2)]
+                comp_done = [torch.cuda.Event() for _ in range(2)]
+                d2h_done = [torch.cuda.Event() for _ in range(2)]
+                s_in.wait_stream(stream)
+                e0.record(s_in)
+                for i in range(n):
+                    b = i % 2
+                    xb, wb, ob = sets[b]
+                    if i >= 2:
+                        s_in.wait_event(comp_done[b])  # the kernels of step i-2 are done with these inputs
+                    with torch.cuda.stream(s_in):
+                        xb.copy_(x_host, non_blocking=True)
+                        wb.copy_(w_host, non_blocking=True)
+                    h2d_done[b].record(s_in)
+                    stream.wait_event(h2d_done[b])
+                    if i >= 2:
+                        stream.wait_event(d2h_done[b])  # step i-2's result has been read back
+                    hq.hq_quantize_fp8(xb, hq.E4M3, hq.PER_TOKEN, q=xq, scales=xs, stream=stream)
+                    hq.hq_quantize_fp8(wb, hq.E4M3, hq.PER_TOKEN, q=wq, scales=ws, stream=stream)
+                    hq.hq_gemm_a8w8(xq, wq, xs, ws, hq.E4M3, out=ob, stream=stream)
+                    comp_done[b].record(stream)
+                    s_out.wait_event(comp_done[b])
+                    with torch.cuda.stream(s_out):
+                        out_host.copy_(ob, non_blocking=True)
+                    d2h_done[b].record(s_out)
+                stream.wait_stream(s_in)
+                stream.wait_stream(s_out)
+                e1.record(stream)
+
         flops = 2.0 * M * N * K
         h2d = (M * K + (N * K if kind == "layer" else 0)) * 2
 
@@ -291,7 +331,8 @@ def build(args, cfg, rank, dev, stream, peaks):
 
         l2 = "inputs larger than L2 (W %d MB, X %d MB, out %d MB); no flush" % (N * K * 2 >> 20, M * K * 2 >> 20,
                                                                                M * N * 2 >> 20)
-        return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=h2d, d2h=M * N * 2,
+        return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, e2e_pipelined=e2e_pipelined, h2d=h2d,
+                    d2h=M * N * 2,
                     roofline=roofline, extras=extras, l2=l2, flush=None,
                     tensors=dict(xq=xq, wq=wq, xs=xs, ws=ws))
 
@@ -824,18 +865,28 @@ def run_ours(args, rank, local_rank, world):
     value = wl["per_step"] * args.steps * world / (ms / 1e3) / scale
 
     # end to end through the C ABI with host buffers: the step's H2D copies,
-    # its kernels and the D2H of its results, every step
-    e2e_steps = max(1, min(args.steps, 5))
-    wl["e2e"]()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    # its kernels and the D2H of its results, every step (double-buffered
+    # across steps where the workload provides it)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
+    pipelined = wl.get("e2e_pipelined")
+    if pipelined is not None:
+        e2e_steps = max(1, min(args.steps, 8))
+        pipelined(2, e0, e1)  # warm-up
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        pipelined(e2e_steps, e0, e1)
+    else:
+        e2e_steps = max(1, min(args.steps, 5))
         wl["e2e"]()
-    e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            wl["e2e"]()
+        e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = wl["per_step"] * e2e_steps * world / (e2e_ms / 1e3) / scale
@@ -894,8 +945,12 @@ def run_ours(args, rank, local_rank, world):
         "roofline": wl["roofline"](ms_by),
         "call_ms": {k: round(v, 4) for k, v in ms_by.items()},
         "clocks": clk,
-        "e2e": {"value": round(e2e_value, 2), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
-                "d2h_bytes_per_step": wl["d2h"], "steps": e2e_steps},
+        "e2e": dict({"value": round(e2e_value, 2), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
+                     "d2h_bytes_per_step": wl["d2h"], "steps": e2e_steps},
+                    **({"pipelined": "double-buffered: step i+1's host-to-device copies and step i-1's "
+                                     "device-to-host copy run on two copy streams while step i's kernels run; "
+                                     "the timed region spans the first copy in to the last copy out"}
+                       if pipelined is not None else {})),
         "gpu_launches": sum(c[2] for c in calls) * args.steps,
         "cpu_baseline": cpu,
     }
