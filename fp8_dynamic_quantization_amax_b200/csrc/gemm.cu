@@ -1144,7 +1144,12 @@ cudaError_t run2(const GemmArgs& a, std::string* msg) {
   p.nkb = static_cast<int>((a.K + (kBKBytes / kElem) - 1) / (kBKBytes / kElem));
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.m_tiles = static_cast<int>((a.M + 255) / 256);
-  p.group_m = 8;
+  // Groups of 16 M-tiles (4096 rows): the group's A rows (32 MB at K = 8192)
+  // stay in L2 while B streams past, so B is read once per 4096 rows.  At
+  // M = 8192, N = 28672, K = 8192: DRAM 1371 MB per launch against 1780 MB
+  // with groups of 8 and 2075 MB with groups of 32 (whose 64 MB of A no
+  // longer stays), and 1-2 % faster.
+  p.group_m = 16;
   p.E = a.E;
   p.offsets = a.offsets;
   p.xs = a.x_scale;
