@@ -468,6 +468,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     ptx::fence_mbarrier_init();
   }
   pdl_wait();  // launched with programmatic stream serialization: global memory only after this
+  pdl_launch_dependents();
   if (threadIdx.x == 32 && p.offsets != nullptr) build_tile_prefix<kBM>(p, tile_prefix, row_start);
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");
@@ -905,6 +906,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
   // each CTA of the pair builds the same tile prefix from the device offsets
   pdl_wait();  // launched with programmatic stream serialization: global memory only after this
+  // No early pdl_launch_dependents() here: this grid runs for milliseconds,
+  // and the next kernel's CTAs parked beside it for that long cost the
+  // power-capped large GEMM 1-3 % (measured); the next launch waits for
+  // this grid's CTAs to exit, as without the trigger.
   if (threadIdx.x == 32 && p.offsets != nullptr) build_tile_prefix<256>(p, tile_prefix, row_start);
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_a) : "memory");

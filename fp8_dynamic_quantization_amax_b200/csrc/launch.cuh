@@ -16,6 +16,16 @@ namespace hq {
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Lets the next kernel in the stream launch now rather than when this grid's
+// CTAs exit: its CTAs are dispatched as this grid's leave the SMs (or into
+// room they leave free) and run their set-up up to their own pdl_wait(),
+// which still returns only once this grid has completed.  Every kernel calls
+// it right after its pdl_wait(), so once all of a grid's CTAs have started
+// the next launch is already in flight.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                               bool cooperative, Args... args) {

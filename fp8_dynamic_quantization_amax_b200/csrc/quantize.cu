@@ -405,6 +405,7 @@ __global__ void __launch_bounds__(kRegThreads) k_token_reg(const void* __restric
                                                            float* __restrict__ amax_out) {
   constexpr int VEC = Dt<DT>::kVec;
   pdl_wait();  // launched with programmatic stream serialization
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kRegThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kRegThreads) >> 5;
@@ -729,6 +730,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_tensor_fused(
   const int64_t s1 = min(b1, s0 + static_cast<int64_t>(kTmemVecs) * T);  // L2 part [s1, b1)
   const bool tail_cta = blockIdx.x == gridDim.x - 1;
   pdl_wait();  // launched with programmatic stream serialization
+  pdl_launch_dependents();
 
   if (tid == 0) {
     abort_flag = 0;
@@ -1094,6 +1096,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_channel_fused(
   uint4* held = reinterpret_cast<uint4*>(fsm + RL * SC * 4);  // [nh][sv]
   const uint4* xv = static_cast<const uint4*>(x);  // row r, column vector c: xv[r * nvc + c]
   pdl_wait();  // launched with programmatic stream serialization
+  pdl_launch_dependents();
 
   if (tid < 32) {  // warp 0: the held rows' bulk copies, one per row, spread over the lanes
     if (tid == 0) {
@@ -1392,6 +1395,7 @@ __global__ void __launch_bounds__(kThreads) k_delayed(
     int len, int idx, int margin, uint32_t* __restrict__ ws, float* __restrict__ scales,
     float* __restrict__ amax_out) {
   pdl_wait();  // launched with programmatic stream serialization
+  pdl_launch_dependents();
   delayed_body<DT, FMT, VECP>(x, n, q, ring, len, idx, margin, ws, scales, amax_out, blockIdx.x, gridDim.x);
 }
 
@@ -1416,6 +1420,7 @@ struct DelayedBatch {
 template <int DT, int FMT>
 __global__ void __launch_bounds__(kThreads) k_delayed_batch(const __grid_constant__ DelayedBatch b) {
   pdl_wait();  // launched with programmatic stream serialization
+  pdl_launch_dependents();
   int t = 0;
   while (t + 1 < b.count && static_cast<int>(blockIdx.x) >= b.cta0[t + 1]) ++t;
   const int64_t cta = static_cast<int64_t>(blockIdx.x) - b.cta0[t];
