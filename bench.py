@@ -488,44 +488,69 @@ def build(args, cfg, rank, dev, stream, peaks):
             return torch.empty((r, c), dtype=torch.uint8, device=dev)
         def f1():
             return torch.empty((1,), dtype=torch.float32, device=dev)
-        xq, wuq, hq_, wdq = u8(T, D), u8(H, D), u8(T, H), u8(D, H)
+        pipe = cfg["fused"]
+        nb = 2 if pipe else 1  # code / scale buffers of X, W_up, W_down: one per step parity when pipelined
+        xq, wuq, wdq = [u8(T, D) for _ in range(nb)], [u8(H, D) for _ in range(nb)], [u8(D, H) for _ in range(nb)]
+        xsc, wusc, wdsc = [f1() for _ in range(nb)], [f1() for _ in range(nb)], [f1() for _ in range(nb)]
+        hq_, hsc = u8(T, H), f1()
         h = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-        xsc, wusc, hsc, wdsc = f1(), f1(), f1(), f1()
         y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
         y_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
         ws = {k: torch.zeros(hq.hq_quantize_workspace_bytes(hq.PER_TENSOR, 1, 1, True), dtype=torch.uint8, device=dev)
               for k in rings}
+        side = torch.cuda.Stream(dev) if pipe else None
+        assert cyc % 2 == 0  # buffer parity stays aligned with the step index across the cycle
+
+        def quantize_batch(t, b, st):
+            # X_t (resident), W_up and W_down with their rings, slot t mod L, in one launch
+            idx = t % L
+            hq.hq_quantize_fp8_delayed_batch(
+                [dict(x=xs_dev[t], ring=rings["x"], ring_idx=idx, q=xq[b], scale=xsc[b], workspace=ws["x"]),
+                 dict(x=wu, ring=rings["wu"], ring_idx=idx, q=wuq[b], scale=wusc[b], workspace=ws["wu"]),
+                 dict(x=wd, ring=rings["wd"], ring_idx=idx, q=wdq[b], scale=wdsc[b], workspace=ws["wd"])],
+                hq.E4M3, stream=st)
 
         def body(t):
-            # step t quantizes its own resident X_t with ring slot t mod L
+            st = torch.cuda.current_stream(dev)
             idx = t % L
-            x_t = xs_dev[t]
+            if pipe:
+                # step t's two GEMMs read the codes that step t-1 quantized into
+                # buffer t mod 2; step t+1's batched quantize writes the other
+                # buffer on a side stream beside the second GEMM, whose 128
+                # tiles leave 20 SMs free (each ring still sees its updates
+                # in step order).  h leaves the first GEMM as FP8 codes, its
+                # delayed quantize (ring h) run by the epilogue.
+                b = t % 2
+                hq.hq_gemm_a8w8_ex(xq[b], wuq[b], xsc[b], wusc[b], hq.E4M3, q_out=hq_, q_fmt=hq.E4M3, q_scale=hsc,
+                                   ring=rings["h"], ring_idx=idx, workspace=ws["h"], stream=st)
+                side.wait_stream(st)
+                hq.hq_gemm_a8w8(hq_, wdq[b], hsc, wdsc[b], hq.E4M3, out=y, stream=st)
+                with torch.cuda.stream(side):
+                    quantize_batch((t + 1) % cyc, 1 - b, side)
+                st.wait_stream(side)
+                return
 
             def q(x, key, qo, so):
                 hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TENSOR, q=qo, scales=so, ring=rings[key], ring_idx=idx,
-                                   workspace=ws[key], stream=torch.cuda.current_stream(dev))
-            if cfg["fused"]:
-                # X, W_up and W_down quantized with their rings in one launch;
-                # h leaves the first GEMM as FP8 codes, its delayed quantize
-                # (ring h) run by the GEMM's epilogue: three kernels per step
-                hq.hq_quantize_fp8_delayed_batch(
-                    [dict(x=x_t, ring=rings["x"], ring_idx=idx, q=xq, scale=xsc, workspace=ws["x"]),
-                     dict(x=wu, ring=rings["wu"], ring_idx=idx, q=wuq, scale=wusc, workspace=ws["wu"]),
-                     dict(x=wd, ring=rings["wd"], ring_idx=idx, q=wdq, scale=wdsc, workspace=ws["wd"])],
-                    hq.E4M3, stream=torch.cuda.current_stream(dev))
-                hq.hq_gemm_a8w8_ex(xq, wuq, xsc, wusc, hq.E4M3, q_out=hq_, q_fmt=hq.E4M3, q_scale=hsc,
-                                   ring=rings["h"], ring_idx=idx, workspace=ws["h"],
-                                   stream=torch.cuda.current_stream(dev))
-            else:
-                q(x_t, "x", xq, xsc)
-                q(wu, "wu", wuq, wusc)
-                hq.hq_gemm_a8w8(xq, wuq, xsc, wusc, hq.E4M3, out=h, stream=torch.cuda.current_stream(dev))
-                q(h, "h", hq_, hsc)
-                q(wd, "wd", wdq, wdsc)
-            hq.hq_gemm_a8w8(hq_, wdq, hsc, wdsc, hq.E4M3, out=y, stream=torch.cuda.current_stream(dev))
+                                   workspace=ws[key], stream=st)
+            q(xs_dev[t], "x", xq[0], xsc[0])
+            q(wu, "wu", wuq[0], wusc[0])
+            hq.hq_gemm_a8w8(xq[0], wuq[0], xsc[0], wusc[0], hq.E4M3, out=h, stream=st)
+            q(h, "h", hq_, hsc)
+            q(wd, "wd", wdq[0], wdsc[0])
+            hq.hq_gemm_a8w8(hq_, wdq[0], hsc, wdsc[0], hq.E4M3, out=y, stream=st)
 
-        # one graph per step of the cycle: X_t's address and the ring slot are
-        # launch arguments, so no copy into a fixed input buffer is needed
+        def reset():
+            # fresh rings; when pipelined, step 0's quantize runs here, ahead of step 0
+            for r in rings.values():
+                r.zero_()
+                r[L] = 1.0
+            if pipe:
+                quantize_batch(0, 0, torch.cuda.current_stream(dev))
+
+        # one graph per step of the cycle: X_t's address, the ring slot and
+        # the buffer parity are launch arguments, so no input copy is needed
+        reset()
         for t in range(L):
             body(t)
         torch.cuda.synchronize()
@@ -541,9 +566,7 @@ def build(args, cfg, rank, dev, stream, peaks):
             graphs = None
             graph_error = "%s: %s" % (type(exc).__name__, str(exc).splitlines()[0] if str(exc) else "")
             torch.cuda.synchronize()
-        for r in rings.values():  # the warm-up and capture passes ran the rings: start fresh
-            r.zero_()
-            r[L] = 1.0
+        reset()  # the warm-up and capture passes ran the rings: start fresh
         counter = [0]
 
         def step_fn():
@@ -557,7 +580,8 @@ def build(args, cfg, rank, dev, stream, peaks):
         def e2e():
             t = counter[0] % cyc
             counter[0] += 1
-            xs_dev[t].copy_(xs_host[t], non_blocking=True)
+            tin = (t + 1) % cyc if pipe else t  # the X this step's quantize reads
+            xs_dev[tin].copy_(xs_host[tin], non_blocking=True)
             if graphs is not None:
                 graphs[t].replay()
             else:
@@ -576,7 +600,9 @@ def build(args, cfg, rank, dev, stream, peaks):
         def extras(ms):
             d = {"kernels_per_step": 3 if cfg["fused"] else 6,
                  "rings": "4 x [16 hist | scale | counter], updated on the device every step",
-                 "quantize": ("X, W_up, W_down in one batched launch; h in the first GEMM's epilogue"
+                 "quantize": ("X, W_up, W_down in one batched launch; h in the first GEMM's epilogue; step t+1's "
+                              "batched quantize runs on a second stream inside step t's graph, beside step t's "
+                              "GEMMs (codes and scales double-buffered by step parity)"
                               if cfg["fused"] else "four separate delayed quantizes (h from a bf16 round trip)")}
             if graphs is not None:
                 d["graph_launches_per_step"] = 1
@@ -587,6 +613,7 @@ def build(args, cfg, rank, dev, stream, peaks):
         return dict(calls=[("step", step_fn, 3 if cfg["fused"] else 6)], per_step=flops, unit="TFLOP/s", e2e=e2e,
                     h2d=T * D * 2,
                     d2h=T * D * 2, roofline=roofline, extras=extras, flush=None, graphs=graphs,
+                    tensors=dict(y=y, rings=rings),
                     l2="working set (X 4 MB, W 16 MB, h 16 MB) fits L2: a steady-state layer step")
 
     if kind == "sweep":
