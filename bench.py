@@ -1,7 +1,7 @@
 """Benchmark of the dynamic-FP8 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload large|large4096|large8192|decode1|decode16|decode128|sweep|stack|backward|moe|moe_bf16]
+                    [--workload large|large4096|large8192|decode1|decode16|decode128|sweep|stack|backward|blockq|moe|...]
 
 Default workload (the large a8w8 GEMM layer): X bf16 [16384, 8192] ~N(0,1),
 W bf16 [28672, 8192] ~N(0,0.02).  One step = per-token E4M3 quantize of X,
@@ -62,6 +62,9 @@ def dist_env():
 #   (E4M3, blocks of 128 / 32): X and W quantized block-wise every step, then
 #   the block-scaled GEMM; blockscaled_mid / blockscaled32_mid: M=4096,
 #   N=8192 at blocks of 128 / 32 (the ncu captures).
+# blockq / blockq_unfused: the large layer whose result leaves as block-wise
+#   E4M3 codes with one f32 scale per 32 columns of a row: written by the
+#   GEMM's epilogue, or by a block-wise quantize of the bf16 result.
 # moe / moe_bf16: per-token quantize of the routed tokens + grouped a8w8 GEMM
 #   over 64 experts (W quantized once); the bf16 grouped GEMM alone.
 WORKLOADS = {
@@ -80,6 +83,8 @@ WORKLOADS = {
     "blockscaled32": dict(kind="blockscaled", M=16384, N=28672, K=8192, block=32),
     "blockscaled_mid": dict(kind="blockscaled", M=4096, N=8192, K=8192, block=128),
     "blockscaled32_mid": dict(kind="blockscaled", M=4096, N=8192, K=8192, block=32),
+    "blockq": dict(kind="blockq", M=16384, N=28672, K=8192, fused=True),
+    "blockq_unfused": dict(kind="blockq", M=16384, N=28672, K=8192, fused=False),
     "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
     "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }
@@ -113,6 +118,12 @@ def workload_desc(name, cfg):
                 "block-wise to E4M3 with one f32 scale per %d elements along K every step, then the block-scaled "
                 "GEMM, out bf16 [%d,%d] (caller-owned)" % (cfg["M"], cfg["K"], cfg["N"], cfg["K"], cfg["block"],
                                                           cfg["M"], cfg["N"]))
+    if k == "blockq":
+        return ("large a8w8 layer with a block-wise FP8 result: X bf16 [%d,%d] ~N(0,1) per-token E4M3, W bf16 "
+                "[%d,%d] ~N(0,0.02) per-output-channel E4M3, result E4M3 [%d,%d] with one f32 scale per 32 columns "
+                "of a row, %s" % (cfg["M"], cfg["K"], cfg["N"], cfg["K"], cfg["M"], cfg["N"],
+                                  "quantized in the GEMM's epilogue" if cfg["fused"] else
+                                  "from a bf16 result and a block-wise quantize"))
     if k == "blockwise":
         return ("block-wise quantize: bf16 [%d,%d] ~N(0,1) with the sweep's outliers and zeros, scales per block "
                 "along the rows: E4M3 blocks of 128 and 32, stochastic E5M2 blocks of 128, and the bf16 "
@@ -335,6 +346,61 @@ def build(args, cfg, rank, dev, stream, peaks):
                     d2h=M * N * 2,
                     roofline=roofline, extras=extras, l2=l2, flush=None,
                     tensors=dict(xq=xq, wq=wq, xs=xs, ws=ws))
+
+    if kind == "blockq":
+        x_host = bf16_host(W.large_x(M, K, seed=rank)).view(M, K)
+        w_host = bf16_host(W.large_w(N, K)).view(N, K)
+        x, w = x_host.to(dev), w_host.to(dev)
+        xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        wq = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        xs = torch.empty((M,), dtype=torch.float32, device=dev)
+        ws = torch.empty((N,), dtype=torch.float32, device=dev)
+        hq8 = torch.empty((M, N), dtype=torch.uint8, device=dev)
+        hs = torch.empty((M, N // 32), dtype=torch.float32, device=dev)
+        q_host = torch.empty((M, N), dtype=torch.uint8).pin_memory()
+        s_host = torch.empty((M, N // 32), dtype=torch.float32).pin_memory()
+        lib, P, st = hq.lib, (lambda t: t.data_ptr()), stream.cuda_stream
+        calls = [("quantize X", lambda: hq.hq_quantize_fp8(x, hq.E4M3, hq.PER_TOKEN, q=xq, scales=xs, stream=stream), 1),
+                 ("quantize W", lambda: hq.hq_quantize_fp8(w, hq.E4M3, hq.PER_TOKEN, q=wq, scales=ws, stream=stream), 1)]
+        if cfg["fused"]:
+            calls.append(("gemm", lambda: hq.check(lib.hq_gemm_a8w8_blockq(
+                P(xq), P(wq), hq.E4M3, P(xs), M, P(ws), N, None, M, N, K, P(hq8), hq.E4M3, 32, P(hs), st)), 1))
+        else:
+            h = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            calls.append(("gemm", lambda: hq.hq_gemm_a8w8(xq, wq, xs, ws, hq.E4M3, out=h, stream=stream), 1))
+            calls.append(("quantize h", lambda: hq.check(lib.hq_quantize_fp8_blockwise(
+                P(h), hq.BF16, M, N, hq.E4M3, 32, 0, 0, P(hq8), P(hs), None, st)), 1))
+
+        def e2e():
+            x.copy_(x_host, non_blocking=True)
+            w.copy_(w_host, non_blocking=True)
+            for c in calls:
+                c[1]()
+            q_host.copy_(hq8, non_blocking=True)
+            s_host.copy_(hs, non_blocking=True)
+
+        flops = 2.0 * M * N * K
+
+        def roofline(ms):
+            t = ms["gemm"] + ms.get("quantize h", 0.0)
+            a = flops / (t / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": round(a, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(a / fp8_peak, 4), "traffic": None,
+                    "kernel": ("k_gemm2<fp8, 256x512 CTA-pair tile> with the block-wise FP8 epilogue" if cfg["fused"]
+                               else "k_gemm2<fp8, 256x512 CTA-pair tile> + the block-wise quantize of its bf16 result"),
+                    "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal fp8/bf16 dense ratio)" %
+                                   (peaks["_src"], peaks["bf16_tflops"], FP8_OVER_BF16)}
+
+        def extras(ms):
+            d = {"gemm_ms": round(ms["gemm"], 4), "result": "E4M3 [M, N] + f32 scales [M, N/32]"}
+            if "quantize h" in ms:
+                d["quantize_h_ms"] = round(ms["quantize h"], 4)
+            return d
+
+        l2 = "inputs larger than L2 (W %d MB, X %d MB, codes %d MB); no flush" % (N * K * 2 >> 20, M * K * 2 >> 20,
+                                                                                 M * N >> 20)
+        return dict(calls=calls, per_step=flops, unit="TFLOP/s", e2e=e2e, h2d=(M * K + N * K) * 2,
+                    d2h=M * N + M * (N // 32) * 4, roofline=roofline, extras=extras, l2=l2, flush=None)
 
     if kind == "blockscaled":
         blk = cfg["block"]
@@ -968,6 +1034,7 @@ def run_ours(args, rank, local_rank, world):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": ("bf16 -> fp8 codes + f32 scales" if cfg["kind"] in ("sweep", "blockwise") else
+                  "fp8_e4m3 (fp32 accumulate, block-wise E4M3 out)" if cfg["kind"] == "blockq" else
                   "fp8_e4m3 (fp32 accumulate, bf16 out)" if cfg["kind"] != "moe_bf16" else "bf16 (fp32 accumulate)"),
         "data": "synthetic (seeded host generators; X seed = rank)",
         "config": {"workload": workload_desc(args.workload, cfg), "M": cfg["M"], "N": cfg["N"], "K": cfg["K"],

@@ -23,7 +23,7 @@ F32, BF16, F16 = 0, 1, 2
 EXPORTED = ["hq_scale_count", "hq_granularity_name", "hq_scale_pair_name", "hq_quantize_workspace_bytes",
             "hq_quantize_fp8", "hq_quantize_fp8_transpose", "hq_quantize_e5m2_stochastic",
             "hq_quantize_fp8_blockwise", "hq_dequantize_fp8_blockwise", "hq_gemm_blockscaled",
-            "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
+            "hq_gemm_a8w8", "hq_gemm_a8w8_ex", "hq_gemm_a8w8_blockq", "hq_grouped_gemm_a8w8", "hq_grouped_gemm_bf16",
             "hq_quantize_fp8_noalloc", "hq_quantize_fp8_delayed_batch", "hq_grad_bias",
             "hq_grad_bias_workspace_bytes", "hq_debug_bounded_wait",
             "hq_check_device_error", "hq_last_error", "hq_version"]
@@ -86,6 +86,8 @@ def _load():
     L.hq_gemm_a8w8_ex.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P, P, ci, P, P, P, i32, i32, i32, P,
                                   sz, P]
     L.hq_gemm_a8w8_ex.restype = ci
+    L.hq_gemm_a8w8_blockq.argtypes = [P, P, ci, P, i64, P, i64, P, i64, i64, i64, P, ci, i64, P, P]
+    L.hq_gemm_a8w8_blockq.restype = ci
     L.hq_grouped_gemm_a8w8.argtypes = [P, P, ci, P, i64, P, i64, P, i32, i64, i64, i64, P, P]
     L.hq_grouped_gemm_a8w8.restype = ci
     L.hq_grouped_gemm_bf16.argtypes = [P, P, P, i32, i64, i64, i64, P, P]
@@ -397,6 +399,26 @@ def hq_gemm_a8w8_ex(xq, wq, x_scale, w_scale, fmt=E4M3, bias=None, out=None, q_o
                               _ptr(q_amax), _ptr(ring), ring_len, ring_idx, ring_margin, _ptr(workspace),
                               0 if workspace is None else workspace.numel(), _stream(stream)))
     return (q_out, q_scale) if ring is not None else out
+
+
+def hq_gemm_a8w8_blockq(xq, wq, x_scale, w_scale, fmt=E4M3, bias=None, q_fmt=E4M3, block=32, q_out=None,
+                        q_scales=None, stream=None):
+    """The a8w8 GEMM (optional bf16 bias) with its bf16 result quantized
+    block-wise in the epilogue: FP8 codes [M, N] and dequant scales
+    [M, N / block] per 32-column block of a row (bit-identical to
+    hq_gemm_a8w8_ex + hq_quantize_fp8_blockwise).  Returns (q_out, q_scales)."""
+    xq, wq = xq.contiguous(), wq.contiguous()
+    x_scale, w_scale = x_scale.contiguous(), w_scale.contiguous()
+    M, K = xq.shape
+    N = wq.shape[0]
+    if q_out is None:
+        q_out = torch.empty((M, N), dtype=torch.uint8, device=xq.device)
+    if q_scales is None:
+        q_scales = torch.empty((M, N // block if block > 0 else 0), dtype=torch.float32, device=xq.device)
+    check(lib.hq_gemm_a8w8_blockq(_ptr(xq), _ptr(wq), fmt, _ptr(x_scale), x_scale.numel(), _ptr(w_scale),
+                                  w_scale.numel(), _ptr(bias), M, N, K, _ptr(q_out), q_fmt, block, _ptr(q_scales),
+                                  _stream(stream)))
+    return q_out, q_scales
 
 
 def hq_grouped_gemm_a8w8(xq, wq, x_scale, w_scale, offsets, fmt=E4M3, out=None, stream=None):

@@ -563,6 +563,9 @@ struct GemmEx {
   int32_t ring_len, ring_idx, ring_margin;
   void* workspace;
   size_t workspace_bytes;
+  bool blockq = false;         // block-wise FP8 output (no ring) into q_out and q_bscales
+  float* q_bscales = nullptr;  // dequant scales [M, N / q_block]
+  int64_t q_block = 0;
 };
 
 hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const float* xs, int64_t xs_len,
@@ -571,7 +574,8 @@ hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const flo
   // FP8 output: q_out given, or (an empty result has no codes to point at)
   // a ring with no bf16 out
   const bool empty = M == 0 || N == 0;
-  const bool fp8o = ex != nullptr && (ex->q_out != nullptr || (empty && ex->ring != nullptr && out == nullptr));
+  const bool bq = ex != nullptr && ex->blockq;  // block-wise FP8 output
+  const bool fp8o = ex != nullptr && (ex->q_out != nullptr || (empty && (ex->ring != nullptr || bq) && out == nullptr));
   const bool grouped = offsets != nullptr || E != 1 || kind == 1;
   if (kind == 0 && fmt != HQ_E4M3 && fmt != HQ_E5M2) return fail(HQ_ERR_INVALID_ARG, "invalid fp8 format %d", fmt);
   if (M < 0 || N < 0 || K < 0) return fail(HQ_ERR_INVALID_ARG, "negative size");
@@ -599,7 +603,15 @@ hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const flo
     if (grouped) return fail(HQ_ERR_INVALID_ARG, "fused epilogues are for the dense GEMM");
     if (fp8o == (out != nullptr)) return fail(HQ_ERR_INVALID_ARG, "exactly one of out and q_out must be given");
     if (ex->bias && !is_aligned(ex->bias, 4)) return fail(HQ_ERR_MISALIGNED, "bias must be 4-byte aligned");
-    if (fp8o) {
+    if (fp8o && bq) {
+      if (ex->q_fmt != HQ_E4M3 && ex->q_fmt != HQ_E5M2)
+        return fail(HQ_ERR_INVALID_ARG, "invalid q_fmt %d", ex->q_fmt);
+      if (ex->q_block != 32) return fail(HQ_ERR_INVALID_ARG, "block = %lld: only 32 is supported", (long long)ex->q_block);
+      if (N % 32 != 0) return fail(HQ_ERR_INVALID_ARG, "N = %lld must be a multiple of the block (32)", (long long)N);
+      if (!empty && !ex->q_bscales) return fail(HQ_ERR_INVALID_ARG, "q_scales must not be null");
+      if (!is_aligned(ex->q_out, 16)) return fail(HQ_ERR_MISALIGNED, "q_out must start on a 16-byte boundary");
+      if (!is_aligned(ex->q_bscales, 4)) return fail(HQ_ERR_MISALIGNED, "q_scales must be 4-byte aligned");
+    } else if (fp8o) {
       if (ex->q_fmt != HQ_E4M3 && ex->q_fmt != HQ_E5M2)
         return fail(HQ_ERR_INVALID_ARG, "invalid q_fmt %d", ex->q_fmt);
       if (!ex->ring) return fail(HQ_ERR_INVALID_ARG, "q_out needs a delayed-scaling ring");
@@ -627,28 +639,32 @@ hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const flo
   if (!is_aligned(a, 16) || !is_aligned(b, 16)) return fail(HQ_ERR_MISALIGNED, "A and B must be 16-byte aligned");
   if (offsets && !is_aligned(offsets, 4)) return fail(HQ_ERR_MISALIGNED, "offsets must be 4-byte aligned");
   const int64_t ebatch = grouped ? E : 1;
+  const bool dq = fp8o && !bq;  // delayed per-tensor FP8 output
   const Range outs[] = {{dst, static_cast<size_t>(M) * static_cast<size_t>(N) * (fp8o ? 1 : 2), fp8o ? "q_out" : "out"},
-                        {fp8o ? ex->q_scale : nullptr, 4, "q_scale"},
-                        {fp8o ? ex->q_amax : nullptr, 4, "q_amax"},
-                        {fp8o ? ex->ring : nullptr, fp8o ? static_cast<size_t>(ex->ring_len + 2) * 4 : 0, "ring"},
-                        {fp8o ? ex->workspace : nullptr, need, "workspace"}};
+                        {dq ? ex->q_scale : nullptr, 4, "q_scale"},
+                        {dq ? ex->q_amax : nullptr, 4, "q_amax"},
+                        {dq ? ex->ring : nullptr, dq ? static_cast<size_t>(ex->ring_len + 2) * 4 : 0, "ring"},
+                        {dq ? ex->workspace : nullptr, need, "workspace"},
+                        {bq ? ex->q_bscales : nullptr, bq ? static_cast<size_t>(M) * static_cast<size_t>(N / 32) * 4 : 0,
+                         "q_scales"}};
   const Range ins[] = {{a, static_cast<size_t>(M * K * esize), "A"},
                        {b, static_cast<size_t>(ebatch * N * K * esize), "B"},
                        {xs, kind == 0 ? static_cast<size_t>(xs_len) * 4 : 0, "x_scale"},
                        {ws, kind == 0 ? static_cast<size_t>(ws_len) * 4 : 0, "w_scale"},
                        {offsets, offsets ? static_cast<size_t>(E + 1) * 4 : 0, "offsets"},
                        {ex ? ex->bias : nullptr, static_cast<size_t>(N) * 2, "bias"}};
-  hq_status s = check_overlaps(outs, 5, ins, 6);
+  hq_status s = check_overlaps(outs, 6, ins, 6);
   if (s != HQ_OK) return s;
   const Range devs[] = {{a, 0, "A"}, {b, 0, "B"}, {xs, 0, "x_scale"}, {ws, 0, "w_scale"},
                         {offsets, 0, "offsets"}, {dst, 0, "out"}, {ex ? ex->bias : nullptr, 0, "bias"},
-                        {fp8o ? ex->q_scale : nullptr, 0, "q_scale"}, {fp8o ? ex->q_amax : nullptr, 0, "q_amax"},
-                        {fp8o ? ex->ring : nullptr, 0, "ring"}, {fp8o ? ex->workspace : nullptr, 0, "workspace"}};
-  s = check_device_ptrs(devs, 11);
+                        {dq ? ex->q_scale : nullptr, 0, "q_scale"}, {dq ? ex->q_amax : nullptr, 0, "q_amax"},
+                        {dq ? ex->ring : nullptr, 0, "ring"}, {dq ? ex->workspace : nullptr, 0, "workspace"},
+                        {bq ? ex->q_bscales : nullptr, 0, "q_scales"}};
+  s = check_device_ptrs(devs, 12);
   if (s != HQ_OK) return s;
   s = check_arch();
   if (s != HQ_OK) return s;
-  if ((M == 0 || N == 0) && fp8o) {
+  if ((M == 0 || N == 0) && dq) {
     // the delayed quantize of the empty result: amax 0, the ring still steps
     hq::QuantizeArgs qa;
     qa.x = ex->workspace; qa.xt = HQ_BF16; qa.rows = M; qa.cols = N; qa.fmt = ex->q_fmt; qa.gran = HQ_PER_TENSOR;
@@ -667,7 +683,10 @@ hq_status gemm_common(int kind, const void* a, const void* b, int fmt, const flo
   g.stream = reinterpret_cast<cudaStream_t>(stream);
   if (ex) {
     g.bias = ex->bias;
-    if (fp8o) {
+    if (bq) {
+      g.out = nullptr;
+      g.q_out = ex->q_out; g.q_fmt = ex->q_fmt; g.q_bscales = ex->q_bscales;
+    } else if (fp8o) {
       g.out = nullptr;
       g.q_out = ex->q_out; g.q_fmt = ex->q_fmt; g.q_scale = ex->q_scale; g.q_amax = ex->q_amax;
       g.ring = ex->ring; g.ring_len = ex->ring_len; g.ring_idx = ex->ring_idx; g.ring_margin = ex->ring_margin;
@@ -694,6 +713,18 @@ hq_status hq_gemm_a8w8_ex(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fm
   const GemmEx ex{bias, q_out, static_cast<int>(q_fmt), q_scale, q_amax, ring, ring_len, ring_idx, ring_margin,
                   workspace, workspace_bytes};
   return gemm_common(0, xq, wq, fmt, x_scale, x_scale_len, w_scale, w_scale_len, nullptr, 1, M, N, K, out, stream,
+                     &ex);
+}
+
+hq_status hq_gemm_a8w8_blockq(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,
+                              int64_t x_scale_len, const float* w_scale, int64_t w_scale_len, const void* bias,
+                              int64_t M, int64_t N, int64_t K, uint8_t* q_out, hq_fp8_format q_fmt, int64_t block,
+                              float* q_scales, hq_stream_t stream) {
+  GemmEx ex{bias, q_out, static_cast<int>(q_fmt), nullptr, nullptr, nullptr, 0, 0, 0, nullptr, 0};
+  ex.blockq = true;
+  ex.q_bscales = q_scales;
+  ex.q_block = block;
+  return gemm_common(0, xq, wq, fmt, x_scale, x_scale_len, w_scale, w_scale_len, nullptr, 1, M, N, K, nullptr, stream,
                      &ex);
 }
 

@@ -72,6 +72,9 @@ struct Params {
   float* ring;
   int ring_len, ring_idx, ring_margin;
   uint32_t* qws;         // amax accumulator word
+  // block-wise FP8 output instead of the ring: each row's 32-column blocks
+  // quantized on their own, dequant scales [M, N / 32]
+  float* qbs;
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -163,6 +166,24 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
 // rows past the tile's valid rows (vrow false) need excluding.  A chunk
 // without an Inf or NaN takes one max.u16x2 per pair and the plain
 // conversion; otherwise each element is checked.
+// Block-wise FP8 output: the multiplier of one 32-column block of a row
+// (this lane's chunk of bf16 results), as the block-wise quantize derives it:
+// amax over the finite |h|, m = fmax / amax, 1 when amax is 0 or the quotient
+// is not finite.
+__device__ __forceinline__ float chunk_block_multiplier(const uint32_t (&w)[16], int qfmt) {
+  uint32_t mx = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
+    if (lo < 0x7F80u) mx = max(mx, lo);  // bf16 magnitudes below Inf: bit order = value order
+    if (hi < 0x7F80u) mx = max(mx, hi);
+  }
+  const float a = __uint_as_float(mx << 16);
+  if (!(a > 0.0f)) return 1.0f;
+  const float m = __fdiv_rn(qfmt == 0 ? kFmaxE4M3 : kFmaxE5M2, a);
+  return (m <= FLT_MAX) ? m : 1.0f;
+}
+
 __device__ __forceinline__ void chunk_to_fp8(const uint32_t (&w)[16], int qfmt, float qm, bool vrow, int n0, int N,
                                              uint32_t& qraw, float& qam, uint32_t (&c4)[8]) {
   uint32_t mx = 0;
@@ -269,8 +290,8 @@ template <int KIND, int kChunks>
 __device__ __forceinline__ void epilogue_chunks(uint32_t tacc, int half, int lane, int col0, int col_end, int tile_end,
                                                 int row0, bool vrow, bool tma_ok, bool has_acc, float xsv,
                                                 const float* wsh, const Params& p, const uint16_t* bias, uint16_t* orow,
-                                                uint8_t* qrow, float qm, uint32_t& qraw, float& qam, uint8_t* sb,
-                                                const CUtensorMap* tm_out, uint64_t out_pol) {
+                                                uint8_t* qrow, float* qsrow, float qm, uint32_t& qraw, float& qam,
+                                                uint8_t* sb, const CUtensorMap* tm_out, uint64_t out_pol) {
   auto process = [&](const uint32_t (&v)[32], int j) {
     const int n0 = col0 + (half + 2 * j) * 32;
     if (n0 >= col_end) return;
@@ -278,7 +299,12 @@ __device__ __forceinline__ void epilogue_chunks(uint32_t tacc, int half, int lan
     chunk_to_bf16(v, has_acc, xsv, wsh + j * 32, bias, n0, p.N, w);
     if (KIND == 0 && qrow != nullptr) {
       uint32_t c4[8];
-      chunk_to_fp8(w, p.qfmt, qm, vrow, n0, p.N, qraw, qam, c4);
+      float qmc = qm;
+      if (p.qbs != nullptr) {  // block-wise: this chunk is one whole block of the row (N % 32 == 0)
+        qmc = chunk_block_multiplier(w, p.qfmt);
+        if (vrow) qsrow[n0 >> 5] = __fdiv_rn(1.0f, qmc);
+      }
+      chunk_to_fp8(w, p.qfmt, qmc, vrow, n0, p.N, qraw, qam, c4);
       if (tma_ok && n0 + 32 <= tile_end) {
         // the 32 x 32 codes through the staging tile, 32-byte rows with the
         // 32-byte swizzle: 16-byte half h of row r sits at h ^ ((r >> 2) & 1)
@@ -587,7 +613,7 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
     uint8_t* sb = sOut + ew * 2048;
     float* wsh = sWs + ew * kMyChunks * 32;
     const uint64_t out_pol = l2_evict_first_policy();
-    const float qm = (p.qout != nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
+    const float qm = (p.qout != nullptr && p.qbs == nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
     const bool has_acc = p.nkb > 0;
     const uint16_t* bias = (KIND == 0) ? p.bias : nullptr;
     int i = 0;
@@ -625,9 +651,10 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
+      float* qsrow = (KIND == 0 && p.qbs != nullptr) ? p.qbs + static_cast<int64_t>(vrow ? row : 0) * (p.N >> 5) : nullptr;
       epilogue_chunks<KIND, kChunks>(
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride, half, lane,
-          T.col0, ncap, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qraw, qam, sb, &tm_out,
+          T.col0, ncap, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qsrow, qm, qraw, qam, sb, &tm_out,
           out_pol);
       tc_fence_before();
       __syncwarp();
@@ -639,7 +666,8 @@ __global__ void __launch_bounds__(kGemm1Threads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemm1Threads / 32>(p, fmaxf(qam, __uint_as_float(qraw << 16)));
+  if (KIND == 0 && p.qout != nullptr && p.qbs == nullptr)
+    finalize_fp8_out<kGemm1Threads / 32>(p, fmaxf(qam, __uint_as_float(qraw << 16)));
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
@@ -715,6 +743,7 @@ void set_fused_epilogue(const GemmArgs& a, Params& p) {
   p.ring_idx = a.ring_idx;
   p.ring_margin = a.ring_margin;
   p.qws = a.q_ws;
+  p.qbs = a.q_bscales;
 }
 
 template <int KIND, int BN, int STAGES, int AROWS = kBM, int KPS = 1>
@@ -1032,7 +1061,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint8_t* sb = sOut + ew * 2048;
     float* wsh = sWs + ew * kMyChunks * 32;
     const uint64_t out_pol = l2_evict_first_policy();
-    const float qm = (p.qout != nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
+    const float qm = (p.qout != nullptr && p.qbs == nullptr) ? __ldcg(p.ring + p.ring_len) : 0.0f;  // the delayed multiplier
     const bool has_acc = p.nkb > 0;
     const uint16_t* bias = (KIND == 0) ? p.bias : nullptr;
     uint32_t tempty_leader[kAccs];
@@ -1073,9 +1102,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       uint16_t* orow = p.out + static_cast<int64_t>(vrow ? row : 0) * p.N;
       uint8_t* qrow = (KIND == 0 && p.qout != nullptr) ? p.qout + static_cast<int64_t>(vrow ? row : 0) * p.N : nullptr;
+      float* qsrow = (KIND == 0 && p.qbs != nullptr) ? p.qbs + static_cast<int64_t>(vrow ? row : 0) * (p.N >> 5) : nullptr;
       epilogue_chunks<KIND, kChunks>(
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc) * kAccStride, half, lane,
-          T.col0, p.N, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qm, qraw, qam, sb, &tm_out,
+          T.col0, p.N, T.col0 + BN, row0, vrow, tma_ok, has_acc, xsv, wsh, p, bias, orow, qrow, qsrow, qm, qraw, qam, sb, &tm_out,
           out_pol);
       tc_fence_before();
       __syncwarp();
@@ -1087,7 +1117,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (KIND == 0 && p.qout != nullptr) finalize_fp8_out<kGemmThreads / 32>(p, fmaxf(qam, __uint_as_float(qraw << 16)));
+  if (KIND == 0 && p.qout != nullptr && p.qbs == nullptr)
+    finalize_fp8_out<kGemmThreads / 32>(p, fmaxf(qam, __uint_as_float(qraw << 16)));
   cluster_sync();  // no CTA leaves while its peer may still touch its shared memory
   if (warp == 1) {
     tc_fence_after();
@@ -1212,10 +1243,12 @@ cudaError_t launch_gemm(const GemmArgs& a, std::string* msg) {
     int dev = 0;
     cudaGetDevice(&dev);
     const int64_t sms = device_sm_count(dev);
-    const int bn = ((a.N + 63) / 64 <= sms)     ? 64
-                   : ((a.N + 127) / 128 <= sms) ? 128
-                   : ((a.N + 207) / 208 <= sms) ? 208
-                                                : 256;
+    // (a block-wise FP8 output needs tiles that start on its 32-column
+    // blocks: 256 instead of 208)
+    const int bn = ((a.N + 63) / 64 <= sms)                              ? 64
+                   : ((a.N + 127) / 128 <= sms)                          ? 128
+                   : ((a.N + 207) / 208 <= sms && a.q_bscales == nullptr) ? 208
+                                                                          : 256;
     if (a.M <= 16) {
       if (bn == 64) return run<0, 64, 2, 16, 8>(a, msg);
       if (bn == 128) return run<0, 128, 3, 16, 3>(a, msg);

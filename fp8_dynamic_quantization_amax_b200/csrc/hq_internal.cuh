@@ -92,6 +92,7 @@ struct GemmArgs {
   float* ring = nullptr;
   int ring_len = 0, ring_idx = 0, ring_margin = 0;
   uint32_t* q_ws = nullptr;     // amax accumulator word (zero between calls)
+  float* q_bscales = nullptr;   // set: q_out holds block-wise codes (32-column blocks, no ring), scales [M, N/32]
 };
 
 // Returns cudaSuccess or the failing call's error; *msg gets a description.

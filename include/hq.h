@@ -427,6 +427,40 @@ hq_status hq_gemm_a8w8_ex(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fm
                           int32_t ring_margin, void* workspace, size_t workspace_bytes, hq_stream_t stream);
 
 /*
+ * Scaled FP8 GEMM whose epilogue writes its result as block-wise FP8
+ * (hip-quant README "Block-wise FP8 Scaling", with the output step of
+ * AstrAI ops.cu mm_fp8 "out_dtype" 1): the bf16 result
+ *
+ *   h[m, n] = bf16_rn( acc[m, n] * (x_scale[m'] * w_scale[n']) + bias[n] )
+ *
+ * is quantized in blocks of 32 consecutive columns of a row, exactly as
+ * hq_quantize_fp8_blockwise(h, HQ_BF16, M, N, q_fmt, 32, 0, 0, q_out,
+ * q_scales, NULL) would quantize it: per block, amax over the finite |h|,
+ * m = fmax / amax (1 when amax is 0 or the quotient is not finite),
+ * q_scales[m, b] = 1/m, codes of f32(h) * m rounded to nearest even with
+ * saturation (NaN -> 0x7F).  The result is bit-identical to the two calls;
+ * the bf16 h never reaches memory.  The codes and scales are the operand
+ * layout of hq_gemm_blockscaled with block 32 (K = this N), so the next
+ * layer's GEMM can read them directly.  Dense GEMMs only; no ring, no
+ * workspace.
+ *
+ * Arguments as hq_gemm_a8w8_ex, and:
+ *   q_out     device uint8 [M, N] FP8 codes, 16-byte aligned, caller-owned
+ *   q_fmt     format of the output codes
+ *   block     the column block: 32 (the only supported value)
+ *   q_scales  device f32 [M, N / 32] dequant scales, 4-byte aligned
+ *   N % 32 == 0.  M == 0 or N == 0 returns HQ_OK with no launch (q_out and
+ *   q_scales may then be NULL).
+ * Errors: those of hq_gemm_a8w8, plus HQ_ERR_INVALID_ARG (block != 32,
+ *   N % 32 != 0, null q_out / q_scales, bad q_fmt), HQ_ERR_MISALIGNED
+ *   (q_out, q_scales, bias) and HQ_ERR_OVERLAP among all buffers.
+ */
+hq_status hq_gemm_a8w8_blockq(const uint8_t* xq, const uint8_t* wq, hq_fp8_format fmt, const float* x_scale,
+                              int64_t x_scale_len, const float* w_scale, int64_t w_scale_len, const void* bias,
+                              int64_t M, int64_t N, int64_t K, uint8_t* q_out, hq_fp8_format q_fmt, int64_t block,
+                              float* q_scales, hq_stream_t stream);
+
+/*
  * Grouped (per-expert) scaled FP8 GEMM (megablocks-hip TODO-gg.md gmm):
  * for each expert e and each row r in [offsets[e], offsets[e+1]):
  *   out[r, n] = bf16_rn( x_scale[r'] * w_scale[e*N + n'] *

@@ -154,6 +154,28 @@ def test_fused_epilogue_rejections():
     assert gx(out=BASE + 0x6000002, q_out=None, ring=None, ws=None, bias=BASE + 0x5200000) == MISALIGNED
 
 
+def gbq(q_out=BASE + 0x4000000, q_fmt=H.E4M3, block=32, q_scales=BASE + 0x5000000, bias=None, M=64, N=128, K=256):
+    return L.hq_gemm_a8w8_blockq(BASE, BASE + 0x1000000, H.E4M3, BASE + 0x2000000, 1, BASE + 0x3000000, 1, bias,
+                                 M, N, K, q_out, q_fmt, block, q_scales, None)
+
+
+def test_blockwise_output_rejections():
+    # hq_gemm_a8w8_blockq: 32-column blocks only, whole blocks per row, codes
+    # and scales caller-owned and apart from every input
+    assert gbq(block=64) == INVALID and gbq(block=16) == INVALID and gbq(block=0) == INVALID
+    assert gbq(N=112) == INVALID                               # 112 % 32 != 0
+    assert gbq(q_out=None) == INVALID and gbq(q_scales=None) == INVALID
+    assert gbq(q_fmt=3) == INVALID
+    assert gbq(q_out=BASE + 0x4000008) == MISALIGNED
+    assert gbq(q_scales=BASE + 0x5000002) == MISALIGNED
+    assert gbq(bias=BASE + 0x5200001) == MISALIGNED
+    assert gbq(q_out=BASE + 0x10) == OVERLAP                   # codes over XQ
+    assert gbq(q_scales=BASE + 0x4000000 + 64 * 128 - 4) == OVERLAP   # scales run into the codes
+    assert gbq(q_scales=BASE + 0x2000000) == OVERLAP           # scales over x_scale
+    # the shape checks still apply to an empty result
+    assert gbq(M=0, N=112, q_out=None, q_scales=None) == INVALID
+
+
 def qtr(x=BASE, xt=H.BF16, rows=64, cols=128, fmt=H.E4M3, q=None, qt=BASE + 0x1000000, scales=BASE + 0x2000000,
         amax=None, mult=None, ring=None, ring_len=16, ring_idx=0, margin=0, ws=BASE + 0x3000000, wsb=256):
     return L.hq_quantize_fp8_transpose(x, xt, rows, cols, fmt, q, qt, scales, amax, mult, ring, ring_len, ring_idx,

@@ -72,7 +72,7 @@ def test_every_workload_is_described_and_sized():
     for name, cfg in bench.WORKLOADS.items():
         d = bench.workload_desc(name, cfg)
         assert isinstance(d, str) and len(d) > 20
-        assert cfg["kind"] in ("layer", "decode", "sweep", "stack", "backward", "blockwise", "blockscaled", "moe",
+        assert cfg["kind"] in ("layer", "decode", "sweep", "stack", "backward", "blockwise", "blockscaled", "blockq", "moe",
                                "moe_bf16")
     # one quantize call's algorithmic bytes: bf16 read + code write + f32 scales
     assert bench.q_bytes(4, 8, 4) == 4 * 8 * 3 + 16

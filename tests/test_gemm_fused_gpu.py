@@ -172,3 +172,87 @@ def test_fp8_out_ring_keeps_scale_when_next_not_finite(q_fmt):
         kept = host(ring_f)[L] == np.float32(0.75)
         assert kept != publishes, name
     H.hq_check_device_error()
+
+
+# ---------------------------------------------------------------- block-wise FP8 output
+# hq_gemm_a8w8_blockq: the bf16 result quantized in 32-column blocks of a row
+# by the epilogue (hip-quant README "Block-wise FP8 Scaling" on the output of
+# mm_fp8).  Shapes with N % 32 == 0: the 1-CTA tiles, the 256 x 256 CTA pair
+# (M >= 4096, N % 512 != 0), the 256 x 512 pair tile, a 256-wide 1-CTA tile
+# and a decode tile; ragged M everywhere.
+BQ_SHAPES = [(300, 288, 144), (700, 2048, 128), (4200, 1280, 64), (8200, 2048, 32), (260, 2304, 96),
+             (16, 2080, 256)]
+
+
+def _blockq_pair(i, M, N, K, q_fmt, with_bias, big_rows=()):
+    """The fused call and the two calls it fuses, on the same operands."""
+    xq, wq, xs, ws, bias = operands(40 + i, M, N, K, O.E4M3)
+    for r in big_rows:  # rows whose bf16 result overflows to +-Inf in places
+        xs[r] = np.float32(3e38)
+    xq_d, wq_d, xs_d, ws_d = dev(xq), dev(wq), dev(xs), dev(ws)
+    b_d = dev(bias) if with_bias else None
+    q, s = H.hq_gemm_a8w8_blockq(xq_d, wq_d, xs_d, ws_d, H.E4M3, bias=b_d, q_fmt=q_fmt)
+    h = H.hq_gemm_a8w8_ex(xq_d, wq_d, xs_d, ws_d, H.E4M3, bias=b_d)
+    q2, s2 = H.hq_quantize_fp8_blockwise(h, q_fmt, 32)
+    torch.cuda.synchronize()
+    return (xq, wq, xs, ws, bias), q, s, h, q2, s2
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("q_fmt", [H.E4M3, H.E5M2])
+def test_blockwise_out_equals_gemm_then_blockwise_quantize(q_fmt, with_bias):
+    for i, (M, N, K) in enumerate(BQ_SHAPES):
+        _, q, s, _, q2, s2 = _blockq_pair(i, M, N, K, q_fmt, with_bias)
+        assert s.shape == (M, N // 32)
+        assert np.array_equal(host(q), host(q2)), (M, N, K)
+        assert np.array_equal(host(s).view(np.uint32), host(s2).view(np.uint32)), (M, N, K)
+    H.hq_check_device_error()
+
+
+@pytest.mark.parametrize("q_fmt", [H.E4M3, H.E5M2])
+def test_blockwise_out_vs_oracle(q_fmt):
+    # stage-wise: the oracle's GEMM within the GEMM tolerance, then the
+    # oracle's block-wise quantize of the GPU's bf16 result bit for bit
+    for i, (M, N, K) in enumerate(BQ_SHAPES[:3] + BQ_SHAPES[4:]):
+        (xq, wq, xs, ws, bias), q, s, h, _, _ = _blockq_pair(i, M, N, K, q_fmt, True)
+        hb = host_bits(h)
+        assert_gemm_close(hb, O.gemm_a8w8_bias(xq, wq, O.E4M3, xs, ws, bias))
+        qo, so, _ = O.quantize_blockwise(hb, q_fmt, 32)
+        assert np.array_equal(host(q), qo), (M, N, K)
+        assert np.array_equal(host(s).view(np.uint32), so.view(np.uint32)), (M, N, K)
+    H.hq_check_device_error()
+
+
+def test_blockwise_out_non_finite_results():
+    # rows whose scaled result overflows: +-Inf entries leave the block
+    # maxima (finite-only amax) and saturate; an all-Inf block keeps m = 1
+    for i, (M, N, K) in enumerate([(300, 288, 144), (4200, 1280, 64)]):
+        _, q, s, h, q2, s2 = _blockq_pair(i, M, N, K, H.E4M3, False, big_rows=(0, 5, 131))
+        hb = host_bits(h)
+        assert (np.abs(W.bf16_bits_to_f32(hb[[0, 5, 131]])) == np.inf).any()
+        assert np.array_equal(host(q), host(q2))
+        assert np.array_equal(host(s).view(np.uint32), host(s2).view(np.uint32))
+        qo, so, _ = O.quantize_blockwise(hb, H.E4M3, 32)
+        assert np.array_equal(host(q), qo) and np.array_equal(host(s).view(np.uint32), so.view(np.uint32))
+    H.hq_check_device_error()
+
+
+def test_blockwise_out_feeds_the_blockscaled_gemm():
+    # h's codes and scales are the next layer's block-scaled A operand (K = N)
+    M, N, K, N2 = 700, 2048, 128, 384
+    (xq, wq, xs, ws, bias), q, s, h, _, _ = _blockq_pair(2, M, N, K, H.E4M3, True)
+    rng = np.random.default_rng(77)
+    w2 = W.f32_to_bf16_bits(rng.standard_normal((N2, N)).astype(np.float32) * np.float32(0.02))
+    w2q, w2s = H.hq_quantize_fp8_blockwise(dev_bf16(w2), H.E4M3, 32)
+    y = H.hq_gemm_blockscaled(q, w2q, s, w2s, H.E4M3, 32)
+    torch.cuda.synchronize()
+    assert_gemm_close(host_bits(y), O.gemm_blockscaled(host(q), host(w2q), H.E4M3, host(s), host(w2s), 32))
+    H.hq_check_device_error()
+
+
+def test_blockwise_out_empty():
+    xq = torch.zeros((0, 64), dtype=torch.uint8, device="cuda")
+    wq = torch.zeros((64, 64), dtype=torch.uint8, device="cuda")
+    xs = torch.ones(1, device="cuda")
+    q, s = H.hq_gemm_a8w8_blockq(xq, wq, xs, torch.ones(64, device="cuda"), H.E4M3)
+    assert q.shape == (0, 64) and s.shape == (0, 2)
