@@ -64,7 +64,8 @@ def dist_env():
 #   N=8192 at blocks of 128 / 32 (the ncu captures).
 # blockq / blockq_unfused: the large layer whose result leaves as block-wise
 #   E4M3 codes with one f32 scale per 32 columns of a row: written by the
-#   GEMM's epilogue, or by a block-wise quantize of the bf16 result.
+#   GEMM's epilogue, or by a block-wise quantize of the bf16 result;
+#   blockq8192: the fused form at M=8192 (the ncu capture).
 # moe / moe_bf16: per-token quantize of the routed tokens + grouped a8w8 GEMM
 #   over 64 experts (W quantized once); the bf16 grouped GEMM alone.
 WORKLOADS = {
@@ -85,6 +86,7 @@ WORKLOADS = {
     "blockscaled32_mid": dict(kind="blockscaled", M=4096, N=8192, K=8192, block=32),
     "blockq": dict(kind="blockq", M=16384, N=28672, K=8192, fused=True),
     "blockq_unfused": dict(kind="blockq", M=16384, N=28672, K=8192, fused=False),
+    "blockq8192": dict(kind="blockq", M=8192, N=28672, K=8192, fused=True),
     "moe": dict(kind="moe", M=32768, N=1408, K=2048, E=64),
     "moe_bf16": dict(kind="moe_bf16", M=32768, N=1408, K=2048, E=64),
 }
